@@ -1,0 +1,339 @@
+/*
+ * ep_oracle.c -- plain, slow CPU statement of MoE token dispatch and combine.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark load this file's library.  The CUDA library
+ * never includes, links or calls it, and this file includes nothing of the
+ * CUDA library: the two share no code.
+ *
+ * What is computed, and where it comes from:
+ *
+ *  - Dispatch sends every token's hidden vector to each expert it is routed
+ *    to; combine gathers the expert outputs back to the token and merges them
+ *    in BF16.  Pages: "DeepSeek 开源周第二弹：DeepEP —— 首个 MoE 模型训练和推理的
+ *    EP 通信库" (m.youleyou.com), sections "DeepEP 的核心功能" (native FP8
+ *    support) and "DeepEP 的常规内核和低延迟内核" (FP8 dispatch, BF16 result
+ *    merge); deepseek.csdn.net/67bd3eb22e30c863900615cc, section "使用示例"
+ *    (dispatch returns recv_x, recv_topk_idx, recv_topk_weights, handle).
+ *  - The pages do not fix the FP8 format.  This library's reading: OCP FP8
+ *    E4M3 (bias 7, largest finite 448, no infinities, NaN = S.1111.111), one
+ *    fp32 scale per 1x128 block of channels, scale = max(amax, 1e-4) / 448 in
+ *    fp32, q = e4m3(x / scale) with the fp32 quotient rounded to nearest-even
+ *    and saturated to +-448.
+ *  - The receive buffer is expert-major: expert ids ascending, then token
+ *    index ascending, then top-k slot ascending (a stable counting sort of the
+ *    (token, slot) pairs by expert id).  Logical partition p owns experts
+ *    [p*E/P, (p+1)*E/P), so each partition's rows are one contiguous slice.
+ *  - Combine: acc = +0.0f; for k = 0..K-1 with a valid row,
+ *    acc = fmaf(w[t][k], float(expert_out[row][i]), acc); y = bf16_rne(acc).
+ *  - Low-latency dispatch writes the same payload into a padded
+ *    [E, capacity, H] tensor: slot j of (t, k) inside expert e is its stable
+ *    rank among e's rows.  deepseek.csdn.net/67bd3eb22e30c863900615cc,
+ *    section "推理解码阶段的应用": the buffer holds
+ *    num_max_tokens * hidden * num_experts elements, so the capacity per
+ *    expert is num_max_tokens.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fexcess-precision=standard
+ * (no fast-math), so every float operation is a single IEEE-754 binary32
+ * operation rounded to nearest-even, and fmaf is the fused multiply-add.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_INDEX_RANGE 1u /* a topk_idx / row outside its range was skipped */
+#define ORACLE_CAPACITY 4u    /* a low-latency row did not fit its expert's capacity */
+
+/* ---------------------------------------------------------------- BF16 -- */
+
+/* BF16 is the upper half of a binary32 word: sign, 8 exponent bits, 7
+ * mantissa bits.  Widening is exact. */
+float oracle_bf16_to_f32(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* Round binary32 to the nearest BF16, ties to the even mantissa.  For one
+ * sign the magnitude order is the bit order, so the candidates are the
+ * truncated pattern and the next pattern up; the dropped 16 bits decide. */
+uint16_t oracle_bf16_from_f32(float v) {
+    uint32_t u;
+    memcpy(&u, &v, 4);
+    if (isnan(v)) return (uint16_t)((u >> 16) | 0x0040u); /* quiet NaN */
+    uint32_t hi = u >> 16;
+    uint32_t lo = u & 0xFFFFu;
+    if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u))) hi += 1u; /* may carry to inf */
+    return (uint16_t)hi;
+}
+
+/* ---------------------------------------------------------------- E4M3 -- */
+
+/* Decode an OCP E4M3 code: exponent field 0 is subnormal (m * 2^-9),
+ * otherwise (1 + m/8) * 2^(E-7); S.1111.111 is NaN. */
+float oracle_e4m3_to_f32(uint8_t c) {
+    int sign = (c >> 7) & 1;
+    int E = (c >> 3) & 0xF;
+    int m = c & 7;
+    double v;
+    if (E == 15 && m == 7) return sign ? -NAN : NAN;
+    if (E == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp((double)(8 + m), E - 10);
+    return (float)(sign ? -v : v);
+}
+
+/* Round a binary32 value to the nearest E4M3 value, ties to the even
+ * mantissa, magnitudes above 448 saturated to 448 (no infinities in E4M3).
+ * The sign of zero is kept.  All arithmetic is on exact binary64 values:
+ * scaling by a power of two is exact and nearbyint() rounds to nearest-even
+ * in the default rounding mode. */
+uint8_t oracle_e4m3_from_f32(float v) {
+    uint32_t u;
+    memcpy(&u, &v, 4);
+    uint8_t sign = (u >> 31) ? 0x80 : 0x00;
+    if (isnan(v)) return (uint8_t)(sign | 0x7F);
+    double a = fabs((double)v);
+    if (a > 448.0) return (uint8_t)(sign | 0x7E); /* 0x7E = 1.75 * 2^8 = 448 */
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal binade (and zero): spacing 2^-9; m = 8 lands on the
+         * smallest normal 2^-6, whose code is also 8 (E = 1, mantissa 0). */
+        double m = nearbyint(ldexp(a, 9));
+        return (uint8_t)(sign | (uint8_t)m);
+    }
+    int e2;
+    (void)frexp(a, &e2);      /* a = f * 2^e2, f in [0.5, 1) */
+    int unb = e2 - 1;         /* a in [2^unb, 2^(unb+1)) */
+    double m = nearbyint(ldexp(a, 3 - unb)); /* 8 + mantissa, in [8, 16] */
+    int E = unb + 7;
+    if (m == 16.0) { /* rounded up into the next binade */
+        m = 8.0;
+        E += 1;
+    }
+    return (uint8_t)(sign | (uint8_t)(E << 3) | (uint8_t)((int)m - 8));
+}
+
+/* Elementwise loops over the two encoders above (for exhaustive tests). */
+void oracle_e4m3_from_f32_n(int64_t n, const float* v, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_from_f32(v[i]);
+}
+
+void oracle_bf16_from_f32_n(int64_t n, const float* v, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_from_f32(v[i]);
+}
+
+/* ------------------------------------------------------------ quantise -- */
+
+/* Scale of one 1x128 block: max(amax, 1e-4) / 448, one binary32 division. */
+float oracle_block_scale(float amax) {
+    float a = fmaxf(amax, 1e-4f);
+    return a / 448.0f;
+}
+
+/* Quantise one BF16 row of H channels (H a multiple of 128) into E4M3 codes
+ * and H/128 fp32 scales. */
+void oracle_quantize_row(int64_t H, const uint16_t* x, uint8_t* q, float* scales) {
+    int64_t nb = H / 128;
+    for (int64_t b = 0; b < nb; ++b) {
+        float amax = 0.0f;
+        for (int i = 0; i < 128; ++i) amax = fmaxf(amax, fabsf(oracle_bf16_to_f32(x[b * 128 + i])));
+        float s = oracle_block_scale(amax);
+        for (int i = 0; i < 128; ++i) {
+            float xv = oracle_bf16_to_f32(x[b * 128 + i]);
+            q[b * 128 + i] = oracle_e4m3_from_f32(xv / s);
+        }
+        scales[b] = s;
+    }
+}
+
+/* -------------------------------------------------------------- layout -- */
+
+/* Routing layout of topk_idx[T][K] (-1 = masked slot).
+ *   num_tokens_per_expert[e]     rows routed to expert e
+ *   is_token_in_partition[t][p]  1 if token t names any expert of partition p
+ *   num_tokens_per_partition[p]  number of distinct tokens with is_token_in_partition = 1
+ *   expert_offset[E+1]           exclusive prefix sum of num_tokens_per_expert
+ *   row_of[t][k]                 receive row of (t, k), -1 if masked
+ *   src_of[row]                  t*K + k for each of the num_recv rows
+ * An index outside [-1, E) is skipped like a masked slot and reported. */
+uint32_t oracle_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int64_t* topk_idx,
+                       int32_t* num_tokens_per_expert, int32_t* num_tokens_per_partition,
+                       uint8_t* is_token_in_partition, int32_t* expert_offset, int32_t* row_of,
+                       int32_t* src_of, int32_t* num_recv) {
+    uint32_t status = 0;
+    int32_t epp = E / P;
+    int32_t* seen = (int32_t*)calloc((size_t)E, sizeof(int32_t));
+    for (int32_t e = 0; e < E; ++e) num_tokens_per_expert[e] = 0;
+    for (int32_t p = 0; p < P; ++p) num_tokens_per_partition[p] = 0;
+    for (int64_t i = 0; i < T * P; ++i) is_token_in_partition[i] = 0;
+
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t k = 0; k < K; ++k) {
+            int64_t e = topk_idx[t * K + k];
+            if (e == -1) continue;
+            if (e < 0 || e >= E) {
+                status |= ORACLE_INDEX_RANGE;
+                continue;
+            }
+            num_tokens_per_expert[e] += 1;
+            is_token_in_partition[t * P + e / epp] = 1;
+        }
+    }
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t p = 0; p < P; ++p) num_tokens_per_partition[p] += is_token_in_partition[t * P + p];
+
+    expert_offset[0] = 0;
+    for (int32_t e = 0; e < E; ++e) expert_offset[e + 1] = expert_offset[e] + num_tokens_per_expert[e];
+    *num_recv = expert_offset[E];
+
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t k = 0; k < K; ++k) {
+            int64_t e = topk_idx[t * K + k];
+            if (e < 0 || e >= E) {
+                row_of[t * K + k] = -1;
+                continue;
+            }
+            int32_t row = expert_offset[e] + seen[e];
+            seen[e] += 1;
+            row_of[t * K + k] = row;
+            src_of[row] = (int32_t)(t * K + k);
+        }
+    }
+    free(seen);
+    return status;
+}
+
+/* ------------------------------------------------------------ dispatch -- */
+
+/* Copy every token to the rows the layout gave it.
+ *   quant = 1: recv_x is E4M3 [rows][H], recv_scales fp32 [rows][H/128]
+ *   quant = 0: recv_x is the BF16 row, bit for bit [rows][H]; recv_scales unused
+ *   recv_topk_idx[row]     = local expert id e - p*E/P of the row's expert
+ *   recv_topk_weights[row] = topk_weights[t][k]                              */
+uint32_t oracle_dispatch(int64_t T, int64_t H, int32_t K, int32_t E, int32_t P, int32_t quant,
+                         const uint16_t* x, const int64_t* topk_idx, const float* topk_weights,
+                         const int32_t* row_of, uint8_t* recv_x, float* recv_scales,
+                         int32_t* recv_topk_idx, float* recv_topk_weights) {
+    int32_t epp = E / P;
+    int64_t nb = H / 128;
+    uint8_t* q = (uint8_t*)malloc((size_t)H);
+    float* s = (float*)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    for (int64_t t = 0; t < T; ++t) {
+        if (quant == 1) oracle_quantize_row(H, x + t * H, q, s);
+        for (int32_t k = 0; k < K; ++k) {
+            int32_t row = row_of[t * K + k];
+            if (row < 0) continue;
+            int64_t e = topk_idx[t * K + k];
+            if (quant == 1) {
+                memcpy(recv_x + (int64_t)row * H, q, (size_t)H);
+                memcpy(recv_scales + (int64_t)row * nb, s, sizeof(float) * (size_t)nb);
+            } else {
+                memcpy(recv_x + (int64_t)row * H * 2, x + t * H, (size_t)H * 2);
+            }
+            recv_topk_idx[row] = (int32_t)(e - (e / epp) * epp);
+            recv_topk_weights[row] = topk_weights[t * K + k];
+        }
+    }
+    free(q);
+    free(s);
+    return 0;
+}
+
+/* Stand-in for the expert computation in tests and benchmarks: the expert
+ * returns its input.  FP8 rows are dequantised with one binary32 multiply
+ * q * scale and rounded to BF16; BF16 rows are passed through. */
+void oracle_identity_expert(int64_t R, int64_t H, int32_t quant, const uint8_t* recv_x,
+                            const float* recv_scales, uint16_t* expert_out) {
+    int64_t nb = H / 128;
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t i = 0; i < H; ++i) {
+            if (quant == 1) {
+                float v = oracle_e4m3_to_f32(recv_x[r * H + i]) * recv_scales[r * nb + i / 128];
+                expert_out[r * H + i] = oracle_bf16_from_f32(v);
+            } else {
+                uint16_t b;
+                memcpy(&b, recv_x + (r * H + i) * 2, 2);
+                expert_out[r * H + i] = b;
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------- combine -- */
+
+/* y[t][i] = bf16_rne( fmaf chain over k = 0..K-1 of w[t][k] * expert_out[row_of[t][k]][i] ),
+ * starting from +0.0f and skipping masked slots (row -1).  A row outside
+ * [0, expert_rows) is skipped and reported. */
+uint32_t oracle_combine(int64_t T, int64_t H, int32_t K, const uint16_t* expert_out,
+                        int64_t expert_rows, const int32_t* row_of, const float* topk_weights,
+                        uint16_t* y) {
+    uint32_t status = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t i = 0; i < H; ++i) {
+            float acc = 0.0f;
+            for (int32_t k = 0; k < K; ++k) {
+                int32_t row = row_of[t * K + k];
+                if (row < 0) continue;
+                if ((int64_t)row >= expert_rows) {
+                    status |= ORACLE_INDEX_RANGE;
+                    continue;
+                }
+                float v = oracle_bf16_to_f32(expert_out[(int64_t)row * H + i]);
+                acc = fmaf(topk_weights[t * K + k], v, acc);
+            }
+            y[t * H + i] = oracle_bf16_from_f32(acc);
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------ low latency ----- */
+
+/* Low-latency dispatch into a padded [E][cap][H] E4M3 tensor with
+ * [E][cap][H/128] scales.  The slot of (t, k) inside expert e is the number
+ * of earlier (t', k') routed to e (token-major, then k), the same order as the
+ * normal layout.  A row that would land at slot >= cap is dropped and
+ * reported.  recv_expert_count[e] = rows written to expert e.
+ * ll_row_of[t][k] = e*cap + slot (-1 if masked or dropped);
+ * ll_src_of[e*cap + slot] = t*K + k.  Unused slots are not written. */
+uint32_t oracle_ll_dispatch(int64_t T, int64_t H, int32_t K, int32_t E, int32_t cap,
+                            const uint16_t* x, const int64_t* topk_idx, uint8_t* recv_x,
+                            float* recv_scales, int32_t* recv_expert_count, int32_t* ll_row_of,
+                            int32_t* ll_src_of) {
+    uint32_t status = 0;
+    int64_t nb = H / 128;
+    int32_t* seen = (int32_t*)calloc((size_t)E, sizeof(int32_t));
+    uint8_t* q = (uint8_t*)malloc((size_t)H);
+    float* s = (float*)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    for (int64_t t = 0; t < T; ++t) {
+        oracle_quantize_row(H, x + t * H, q, s);
+        for (int32_t k = 0; k < K; ++k) {
+            int64_t e = topk_idx[t * K + k];
+            ll_row_of[t * K + k] = -1;
+            if (e == -1) continue;
+            if (e < 0 || e >= E) {
+                status |= ORACLE_INDEX_RANGE;
+                continue;
+            }
+            int32_t j = seen[e];
+            seen[e] += 1;
+            if (j >= cap) {
+                status |= ORACLE_CAPACITY;
+                continue;
+            }
+            int64_t row = e * (int64_t)cap + j;
+            memcpy(recv_x + row * H, q, (size_t)H);
+            memcpy(recv_scales + row * nb, s, sizeof(float) * (size_t)nb);
+            ll_row_of[t * K + k] = (int32_t)row;
+            ll_src_of[row] = (int32_t)(t * K + k);
+        }
+    }
+    for (int32_t e = 0; e < E; ++e) recv_expert_count[e] = seen[e] < cap ? seen[e] : cap;
+    free(seen);
+    free(q);
+    free(s);
+    return status;
+}
