@@ -1,0 +1,621 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE dispatch / combine hot path on B200.
+
+One step = one pass of the whole path over one batch of the "normal" workload
+(4096 tokens x hidden 7168, top-8 of 256 experts in 8 logical partitions with
+top-4-group routing): routing layout + FP8 dispatch (3 kernels, one call) and
+BF16 combine (1 kernel, one call).  The expert computation between them is out
+of scope; combine reads expert outputs prepared once before timing (the
+dispatched rows dequantised, i.e. identity experts).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  `value` is algorithmic HBM GB/s of the whole
+step (bytes the method must move / device time, summed over ranks' batches,
+max time over ranks).  Each step is captured as two CUDA graphs (dispatch,
+combine) and timed with CUDA events on the launching stream; L2 (126 MB) is
+flushed by a 256 MiB write before every timed step, outside the events.
+`--impl reference` times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dispatch/combine HBM GB/s (% of B200 peak) at 4096x7168 top-8; LL latency µs"
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ helpers --
+
+def env_rank():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        try:
+            d = json.load(open(p))
+            return float(d["hbm_gbs"]), "measured"
+        except Exception:
+            pass
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(T, H, K, E, P, R, fp8: bool):
+    """Bytes the method must move: reads of inputs and writes of outputs,
+    once each; no padding, no unwritten worst-case rows."""
+    payload = R * H * (1 if fp8 else 2)
+    scales = R * (H // 128) * 4 if fp8 else 0
+    meta = (T * K * 8 + T * K * 4          # topk_idx, topk_weights read
+            + R * 4 + R * 4                # recv_topk_idx, recv_topk_weights
+            + R * 4 + T * K * 4            # src_of, row_of
+            + (E + 1) * 4 + E * 4 + P * 4  # offsets, counts
+            + T * P)                       # is_token_in_partition
+    dispatch = T * H * 2 + payload + scales + meta
+    combine = R * H * 2 + T * H * 2 + T * K * 8
+    return dispatch, combine
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the benchmark runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = vis.split(",")[local_rank] if vis else str(local_rank)
+        self.idx = idx.strip()
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", self.idx], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        self.start_time = time.time()
+
+    def mark(self, t0, t1):
+        self.t0, self.t1 = t0, t1
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        end = time.time()
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        if not rows:
+            return None
+        # samples are evenly spaced over [start_time, end]: keep those inside the timed window
+        n = len(rows)
+        ts = [self.start_time + (end - self.start_time) * (i + 0.5) / n for i in range(n)]
+        sel = [r for r, t in zip(rows, ts) if self.t0 is not None and self.t0 <= t <= self.t1]
+        window = "timed region"
+        if not sel:
+            sel, window = rows, "whole run (timed region shorter than the sampling period)"
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        mhz, maxmhz = [], []
+        for r in sel:
+            try:
+                mhz.append(float(r[1]))
+                maxmhz.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxmhz),
+                "reasons": sorted(reasons), "samples": len(mhz), "window": window}
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()[:16]
+
+
+COMBINE_SOURCES = ["combine_get_dispatch_05_b200/csrc/combine.cu",
+                   "combine_get_dispatch_05_b200/csrc/ep_device.cuh"]
+
+
+def profiled_traffic(summary: str, sources):
+    """dram bytes per launch from a committed ncu summary, if it was taken on the
+    current source of the kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    for line in open(p):
+        if ":" in line and line.startswith("- "):
+            k, v = line[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    try:
+        if vals.get("source_sha256") != source_hash(sources):
+            return None
+        return int(float(vals["dram_bytes_per_full_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------- our path -----
+
+class PathRunner:
+    """Device buffers and CUDA graphs for one workload's dispatch + combine."""
+
+    def __init__(self, ep, w, dev, use_graphs=True):
+        import numpy as np
+        import torch
+
+        self.ep, self.w, self.dev = ep, w, dev
+        T, H, K, E, P = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
+        self.T, self.H, self.K, self.E, self.P = T, H, K, E, P
+        self.fp8 = w.quant == "fp8"
+        self.quant = ep.EP_QUANT_FP8_E4M3_1X128 if self.fp8 else ep.EP_QUANT_NONE
+        self.x = torch.from_numpy(w.x.view(np.int16)).to(dev).view(torch.bfloat16)
+        self.idx = torch.from_numpy(w.topk_idx).to(dev)
+        self.wts = torch.from_numpy(w.topk_weights).to(dev)
+        rows = max(T * K, 1)
+        self.recv_q = torch.empty((rows, H), dtype=torch.uint8 if self.fp8 else torch.bfloat16,
+                                  device=dev)
+        self.recv_s = torch.empty((rows, H // 128), dtype=torch.float32, device=dev) \
+            if self.fp8 else None
+        self.recv_i = torch.empty(rows, dtype=torch.int32, device=dev)
+        self.recv_w = torch.empty(rows, dtype=torch.float32, device=dev)
+        self.lay = ep.Layout.empty(T, K, E, P, dev)
+        self.ws = torch.empty(ep.ep_workspace_bytes(T, E, P), dtype=torch.uint8, device=dev)
+        ep.ep_workspace_init(self.ws)
+        self.y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.dispatch()
+        torch.cuda.synchronize()
+        self.R = int(self.lay.num_recv.item())
+        if self.fp8:
+            q = self.recv_q.view(torch.float8_e4m3fn).to(torch.float32)
+            self.eo = (q * self.recv_s.repeat_interleave(128, dim=1)).to(torch.bfloat16)
+            del q
+        else:
+            self.eo = self.recv_q.clone()
+        self.combine()
+        torch.cuda.synchronize()
+        if ep.ep_read_status(self.ws) != 0:
+            raise RuntimeError("device status set during setup")
+        self.bytes_dispatch, self.bytes_combine = algorithmic_bytes(T, H, K, E, P, self.R, self.fp8)
+        self.graphs = None
+        if use_graphs:
+            self.graphs = self._capture()
+
+    def dispatch(self, stream=None):
+        self.ep.ep_dispatch(self.x, self.idx, self.wts, self.E, self.P, self.quant, self.recv_q,
+                            self.recv_s, self.recv_i, self.recv_w, self.lay, self.ws, stream)
+
+    def combine(self, stream=None):
+        self.ep.ep_combine(self.eo, self.lay, self.wts, self.y, self.ws, stream)
+
+    def _capture(self):
+        import torch
+
+        s = torch.cuda.Stream(device=self.dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for _ in range(2):
+                self.dispatch()
+                self.combine()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        gd, gc = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gd):
+            self.dispatch()
+        with torch.cuda.graph(gc):
+            self.combine()
+        torch.cuda.synchronize()
+        return gd, gc
+
+    def run_dispatch(self):
+        if self.graphs:
+            self.graphs[0].replay()
+        else:
+            self.dispatch()
+
+    def run_combine(self):
+        if self.graphs:
+            self.graphs[1].replay()
+        else:
+            self.combine()
+
+    def time_steps(self, steps, warmup, flush):
+        """Per-step (dispatch ms, combine ms) with an L2 flush before each step."""
+        import torch
+
+        for _ in range(warmup):
+            flush.zero_()
+            self.run_dispatch()
+            self.run_combine()
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            evs[i][0].record()
+            self.run_dispatch()
+            evs[i][1].record()
+            self.run_combine()
+            evs[i][2].record()
+        torch.cuda.synchronize()
+        return ([e[0].elapsed_time(e[1]) for e in evs], [e[1].elapsed_time(e[2]) for e in evs])
+
+
+def time_low_latency(ep, w, dev, reps=200):
+    """LL dispatch / combine: CUDA-graph replay median (kernel-only, back to back, L2
+    warm as in decode) and eager call + synchronize wall time (launch-inclusive)."""
+    import numpy as np
+    import torch
+
+    T, H, K, E = w.num_tokens, w.hidden, w.num_topk, w.num_experts
+    cap = w.num_max_tokens
+    x = torch.from_numpy(w.x.view(np.int16)).to(dev).view(torch.bfloat16)
+    idx = torch.from_numpy(w.topk_idx).to(dev)
+    wts = torch.from_numpy(w.topk_weights).to(dev)
+    rq = torch.empty((E, cap, H), dtype=torch.uint8, device=dev)
+    rs = torch.empty((E, cap, H // 128), dtype=torch.float32, device=dev)
+    cnt = torch.empty(E, dtype=torch.int32, device=dev)
+    h = ep.LowLatencyHandle.empty(T, K, E, cap, dev)
+    ws = torch.empty(ep.ep_workspace_bytes(1, E, 1), dtype=torch.uint8, device=dev)
+    ep.ep_workspace_init(ws)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+
+    def disp():
+        ep.ep_low_latency_dispatch(x, idx, cap, E, rq, rs, cnt, h, ws)
+
+    disp()
+    torch.cuda.synchronize()
+    q = rq.view(torch.float8_e4m3fn).to(torch.float32)
+    eo = (q * rs.repeat_interleave(128, dim=-1)).to(torch.bfloat16)
+    del q
+
+    def comb():
+        ep.ep_low_latency_combine(eo, h, wts, y, ws)
+
+    out = {}
+    for name, fn in (("dispatch", disp), ("combine", comb)):
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            fn()
+            fn()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(20):
+            g.replay()
+        torch.cuda.synchronize()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        evs[0].record()
+        for i in range(reps):
+            g.replay()
+            evs[i + 1].record()
+        torch.cuda.synchronize()
+        graph_us = statistics.median(evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(reps))
+        walls = []
+        for _ in range(50):
+            t0 = time.perf_counter()
+            fn()
+            torch.cuda.synchronize()
+            walls.append((time.perf_counter() - t0) * 1e6)
+        out[name] = {"graph_replay_us": round(graph_us, 2),
+                     "eager_call_us": round(statistics.median(walls), 2)}
+    if ep.ep_read_status(ws) != 0:
+        raise RuntimeError("device status set in the low-latency run")
+    out["config"] = f"{T} tokens x hidden {H}, top-{K} of {E} experts, capacity {cap}, FP8"
+    return out
+
+
+def time_e2e(ep, runner, steps):
+    """The same step through the public API with host buffers: pinned host ->
+    device copies of x / topk_idx / topk_weights, dispatch, combine, device -> host
+    copy of y, all inside the device-timed region."""
+    import torch
+
+    hx = runner.x.cpu().pin_memory()
+    hi = runner.idx.cpu().pin_memory()
+    hw = runner.wts.cpu().pin_memory()
+    hy = torch.empty(runner.y.shape, dtype=runner.y.dtype).pin_memory()
+    h2d = hx.numel() * 2 + hi.numel() * 8 + hw.numel() * 4
+    d2h = hy.numel() * 2
+
+    def step():
+        runner.x.copy_(hx, non_blocking=True)
+        runner.idx.copy_(hi, non_blocking=True)
+        runner.wts.copy_(hw, non_blocking=True)
+        runner.dispatch()
+        runner.combine()
+        hy.copy_(runner.y, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    evs[0].record()
+    for _ in range(steps):
+        step()
+    evs[1].record()
+    torch.cuda.synchronize()
+    ms = evs[0].elapsed_time(evs[1]) / steps
+    return ms, h2d, d2h
+
+
+def cpu_baseline(w, min_seconds=10.0):
+    """The oracle, as it stands (single-threaded C), on the same batch."""
+    import oracle
+
+    T, H, K, E, P = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
+    d = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, E, P)
+    eo = oracle.identity_expert(d["recv_x"], d["recv_scales"])
+    bd, bc = algorithmic_bytes(T, H, K, E, P, int(d["num_recv"][0]), True)
+    passes, t = 0, 0.0
+    while t < min_seconds and passes < 50:
+        t0 = time.perf_counter()
+        dd = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, E, P)
+        oracle.combine(eo, dd["row_of"], w.topk_weights)
+        t += time.perf_counter() - t0
+        passes += 1
+    return {"value": round((bd + bc) * passes / t / 1e9, 3), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"the full {T}-token batch (layout + FP8 dispatch + combine), {passes} passes, "
+                      f"{t:.1f} s, single-threaded C"}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import combine_get_dispatch_05_b200 as ep
+    from workloads import make_workload
+
+    rank, world, local = env_rank()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    w = make_workload("normal", seed=args.seed + rank)
+    runner = PathRunner(ep, w, dev, use_graphs=not args.eager)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    d_ms, c_ms = runner.time_steps(args.steps, args.warmup, flush)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t1 = time.time()
+    sampler.mark(t0, t1)
+    status = ep.ep_read_status(runner.ws)
+
+    total_ms = sum(d_ms) + sum(c_ms)
+    tot = torch.tensor([total_ms, sum(c_ms), sum(d_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
+    total_ms = float(tot[0])
+    ms_step = total_ms / args.steps
+    step_bytes = runner.bytes_dispatch + runner.bytes_combine
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = time_e2e(ep, runner, max(5, min(args.steps, 50)))
+        e2e = {"value": round(world * step_bytes / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "ms_per_step": round(e_ms, 4), "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h,
+               "path": "ep_dispatch + ep_combine (Python binding -> C ABI), pinned host buffers"}
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak, peak_kind = measured_peaks()
+    comb_us = float(tot[1]) / args.steps * 1e3
+    disp_us = float(tot[2]) / args.steps * 1e3
+    comb_gbs = runner.bytes_combine / (comb_us * 1e-6) / 1e9
+    disp_gbs = runner.bytes_dispatch / (disp_us * 1e-6) / 1e9
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32 arithmetic; fp8-e4m3 dispatch payload, bf16 combine",
+        "data": "synthetic",
+        "config": {
+            "workload": "normal: 4096 tokens x hidden 7168 BF16, top-8 of 256 experts in 8 "
+                        "logical partitions, top-4-of-8-group routing, FP8 (E4M3, 1x128 scales) "
+                        "dispatch + BF16 combine",
+            "tokens_per_gpu": w.num_tokens, "hidden": w.hidden, "topk": w.num_topk,
+            "experts": w.num_experts, "partitions": w.num_partitions, "recv_rows": runner.R,
+            "bytes_per_step": step_bytes, "seed": args.seed,
+            "l2": "flushed before every timed step (256 MiB write, outside the events)",
+            "launch": "CUDA graphs (dispatch: 3 kernels with programmatic dependent launch; "
+                      "combine: 1 kernel)" if not args.eager else "eager",
+            "parallelism": f"replicas x{world} (independent batches, no exchange)",
+        },
+        "breakdown": {
+            "dispatch": {"us": round(disp_us, 2), "bytes": runner.bytes_dispatch,
+                         "gbs": round(disp_gbs, 1), "frac": round(disp_gbs / peak, 4),
+                         "kernels": "layout_count + layout_rank + dispatch_fp8"},
+            "combine": {"us": round(comb_us, 2), "bytes": runner.bytes_combine,
+                        "gbs": round(comb_gbs, 1), "frac": round(comb_gbs / peak, 4),
+                        "kernels": "combine"},
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": "combine_kernel", "achieved": round(comb_gbs, 1),
+            "peak": peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+            if peak_kind == "measured" else "fallback 6.65 TB/s",
+            "unit": "GB/s", "frac": round(comb_gbs / peak, 4),
+            "traffic": profiled_traffic("combine_kernel_normal_4096x7168.md", COMBINE_SOURCES),
+        },
+        "gpu_launches": 4 * args.steps,
+        "device_status": status,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        result["e2e"] = e2e
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        result["cpu_baseline"] = cpu_baseline(w)
+    if not args.no_extra:
+        extra = {}
+        try:
+            extra["ll"] = time_low_latency(ep, make_workload("ll", seed=args.seed), dev)
+        except Exception as exc:  # report, do not hide
+            extra["ll"] = {"error": repr(exc)}
+        for name in ("skew", "bf16", "stress"):
+            try:
+                wx = make_workload(name, seed=args.seed)
+                r = PathRunner(ep, wx, dev, use_graphs=not args.eager)
+                dd, cc = r.time_steps(args.extra_steps, 3, flush)
+                du, cu = statistics.mean(dd) * 1e3, statistics.mean(cc) * 1e3
+                extra[name] = {
+                    "tokens": wx.num_tokens, "hidden": wx.hidden, "topk": wx.num_topk,
+                    "experts": wx.num_experts, "partitions": wx.num_partitions,
+                    "quant": wx.quant, "recv_rows": r.R,
+                    "dispatch_us": round(du, 2),
+                    "dispatch_gbs": round(r.bytes_dispatch / (du * 1e-6) / 1e9, 1),
+                    "combine_us": round(cu, 2),
+                    "combine_gbs": round(r.bytes_combine / (cu * 1e-6) / 1e9, 1),
+                    "status": ep.ep_read_status(r.ws)}
+                del r
+                torch.cuda.empty_cache()
+            except Exception as exc:
+                extra[name] = {"error": repr(exc)}
+        result["configs"] = extra
+    print(json.dumps(result), flush=True)
+
+
+# -------------------------------------------------------- reference arm -----
+
+def run_reference(args):
+    """The CPU oracle as it stands, on bounded samples of the same workload."""
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return
+    import oracle
+    from workloads import make_workload
+
+    w = make_workload("normal", seed=args.seed)
+    T, H, K, E, P = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
+
+    def make_step(n):
+        xs, idxs, wts = w.x[:n], w.topk_idx[:n], w.topk_weights[:n]
+        ds = oracle.dispatch(xs, idxs, wts, E, P)
+        eos = oracle.identity_expert(ds["recv_x"], ds["recv_scales"])
+
+        def step():
+            dx = oracle.dispatch(xs, idxs, wts, E, P)
+            oracle.combine(eos, dx["row_of"], wts)
+        return step, int(ds["num_recv"][0])
+
+    # calibrate seconds per token, then size each step's sample so the whole run
+    # stays near two minutes
+    n_cal = 64
+    cal, _ = make_step(n_cal)
+    t0 = time.perf_counter()
+    cal()
+    per_tok = (time.perf_counter() - t0) / n_cal
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    S = int(max(1, min(T, budget / per_tok)))
+    step, R = make_step(S)
+    bd, bc = algorithmic_bytes(S, H, K, E, P, R, True)
+
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        step()
+        times.append(time.perf_counter() - t)
+    ms = statistics.mean(times) * 1e3
+    value = (bd + bc) / (ms * 1e-3) / 1e9
+    sample = (f"first {S} of {T} tokens of the normal workload per step (layout + FP8 dispatch + "
+              f"combine), single-threaded C oracle")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 arithmetic; fp8-e4m3 dispatch payload, bf16 combine",
+        "data": "synthetic",
+        "config": {"workload": "normal: 4096 tokens x hidden 7168, top-8 of 256 experts, 8 "
+                               "partitions, FP8 dispatch + BF16 combine", "sample_tokens": S},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--extra-steps", type=int, default=50)
+    ap.add_argument("--eager", action="store_true", help="launch eagerly instead of CUDA graphs")
+    ap.add_argument("--no-extra", action="store_true", help="skip the ll/skew/bf16/stress configs")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, _ = env_rank()
+    if world != args.gpus and not (world == 1 and args.gpus == 1):
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus N > 1 must be launched with torch.distributed.run (one rank per GPU)")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

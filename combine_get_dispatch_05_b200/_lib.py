@@ -1,0 +1,303 @@
+"""ctypes binding of ``libep_b200.so`` (declared in ``include/ep_b200.h``).
+
+Argument marshalling only: each function checks tensor dtypes, shapes and
+devices, passes raw pointers and the current CUDA stream to the C entry point of
+the same name, and raises :class:`EpError` on a non-zero status.  Every step of
+the computation runs in the library's CUDA kernels; there is no fallback.  If
+the library has not been built, importing this module raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libep_b200.so")
+
+EP_OK, EP_ERR_INVALID_ARG, EP_ERR_SHAPE, EP_ERR_WORKSPACE, EP_ERR_CUDA = 0, 1, 2, 3, 4
+EP_DEV_INDEX_RANGE, EP_DEV_TIMEOUT, EP_DEV_CAPACITY = 0x1, 0x2, 0x4
+EP_QUANT_NONE, EP_QUANT_FP8_E4M3_1X128 = 0, 1
+
+EXPORTED = (
+    "ep_abi_version", "ep_status_string", "ep_workspace_bytes", "ep_workspace_init",
+    "ep_read_status", "ep_get_dispatch_layout", "ep_dispatch", "ep_combine",
+    "ep_low_latency_dispatch", "ep_low_latency_combine", "ep_debug_wait_probe",
+)
+
+
+class EpError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+        self.status = status
+
+
+class ep_layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "num_tokens_per_expert", "num_tokens_per_partition", "is_token_in_partition",
+        "expert_offset", "row_of", "src_of", "num_recv")]
+
+
+class ep_ll_handle(ctypes.Structure):
+    _fields_ = [("row_of", ctypes.c_void_p), ("src_of", ctypes.c_void_p)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m combine_get_dispatch_05_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    i64, i32, sz, vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t, ctypes.c_void_p
+    st = ctypes.c_int32
+    L.ep_abi_version.argtypes, L.ep_abi_version.restype = [], i32
+    L.ep_status_string.argtypes, L.ep_status_string.restype = [i32], ctypes.c_char_p
+    L.ep_workspace_bytes.argtypes, L.ep_workspace_bytes.restype = [i64, i32, i32], sz
+    L.ep_workspace_init.argtypes, L.ep_workspace_init.restype = [vp, sz, vp], st
+    L.ep_read_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)]
+    L.ep_read_status.restype = st
+    L.ep_get_dispatch_layout.argtypes = [i64, i32, i32, i32, vp, ctypes.POINTER(ep_layout), vp, sz,
+                                         vp]
+    L.ep_get_dispatch_layout.restype = st
+    L.ep_dispatch.argtypes = [i64, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp,
+                              ctypes.POINTER(ep_layout), vp, sz, vp]
+    L.ep_dispatch.restype = st
+    L.ep_combine.argtypes = [i64, i64, i32, vp, i64, ctypes.POINTER(ep_layout), vp, vp, vp, sz, vp]
+    L.ep_combine.restype = st
+    L.ep_low_latency_dispatch.argtypes = [i64, i64, i32, i32, i32, vp, vp, vp, vp, vp,
+                                          ctypes.POINTER(ep_ll_handle), vp, sz, vp]
+    L.ep_low_latency_dispatch.restype = st
+    L.ep_low_latency_combine.argtypes = [i64, i64, i32, i32, i32, vp,
+                                         ctypes.POINTER(ep_ll_handle), vp, vp, vp, sz, vp]
+    L.ep_low_latency_combine.restype = st
+    L.ep_debug_wait_probe.argtypes, L.ep_debug_wait_probe.restype = [ctypes.c_uint64, vp, sz, vp], st
+    return L
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.ep_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != EP_OK:
+        raise EpError(fn, status)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape=None, numel_at_least=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if numel_at_least is not None and t.numel() < numel_at_least:
+        raise ValueError(f"{name} needs at least {numel_at_least} elements, has {t.numel()}")
+
+
+# ----------------------------------------------------------------- handles --
+
+@dataclass
+class Layout:
+    """Device arrays of one batch's routing layout -- the `handle` that dispatch
+    returns and combine consumes (see ``ep_layout`` in ep_b200.h)."""
+
+    num_tokens_per_expert: torch.Tensor  # int32 [E]
+    num_tokens_per_partition: torch.Tensor  # int32 [P]
+    is_token_in_partition: torch.Tensor  # uint8 [T, P]
+    expert_offset: torch.Tensor  # int32 [E + 1]
+    row_of: torch.Tensor  # int32 [T, K]
+    src_of: torch.Tensor  # int32 [T * K]
+    num_recv: torch.Tensor  # int32 [1]
+
+    @staticmethod
+    def empty(num_tokens: int, num_topk: int, num_experts: int, num_partitions: int,
+              device) -> "Layout":
+        i32 = dict(dtype=torch.int32, device=device)
+        return Layout(
+            torch.empty(num_experts, **i32), torch.empty(num_partitions, **i32),
+            torch.empty((num_tokens, num_partitions), dtype=torch.uint8, device=device),
+            torch.empty(num_experts + 1, **i32), torch.empty((num_tokens, num_topk), **i32),
+            torch.empty(max(num_tokens * num_topk, 1), **i32), torch.empty(1, **i32))
+
+    def c(self) -> ep_layout:
+        return ep_layout(*(t.data_ptr() for t in (
+            self.num_tokens_per_expert, self.num_tokens_per_partition,
+            self.is_token_in_partition, self.expert_offset, self.row_of, self.src_of,
+            self.num_recv)))
+
+
+@dataclass
+class LowLatencyHandle:
+    """Device arrays of a low-latency dispatch (see ``ep_ll_handle``)."""
+
+    row_of: torch.Tensor  # int32 [T, K]: e * num_max_tokens + slot, or -1
+    src_of: torch.Tensor  # int32 [E, num_max_tokens]
+    num_max_tokens: int
+    num_experts: int
+
+    @staticmethod
+    def empty(num_tokens: int, num_topk: int, num_experts: int, num_max_tokens: int,
+              device) -> "LowLatencyHandle":
+        return LowLatencyHandle(
+            torch.empty((num_tokens, num_topk), dtype=torch.int32, device=device),
+            torch.empty((num_experts, num_max_tokens), dtype=torch.int32, device=device),
+            num_max_tokens, num_experts)
+
+    def c(self) -> ep_ll_handle:
+        return ep_ll_handle(self.row_of.data_ptr(), self.src_of.data_ptr())
+
+
+# --------------------------------------------------------------- workspace --
+
+def ep_workspace_bytes(num_tokens: int, num_experts: int, num_partitions: int) -> int:
+    return int(lib.ep_workspace_bytes(num_tokens, num_experts, num_partitions))
+
+
+def ep_workspace_init(workspace: torch.Tensor, stream=None) -> None:
+    _need(workspace, "workspace", torch.uint8)
+    _check("ep_workspace_init",
+           lib.ep_workspace_init(workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_read_status(workspace: torch.Tensor, stream=None) -> int:
+    _need(workspace, "workspace", torch.uint8)
+    bits = ctypes.c_uint32(0)
+    _check("ep_read_status", lib.ep_read_status(workspace.data_ptr(), workspace.numel(),
+                                                _stream(stream), ctypes.byref(bits)))
+    return int(bits.value)
+
+
+# ---------------------------------------------------------------- calls -----
+
+def ep_get_dispatch_layout(topk_idx: torch.Tensor, num_experts: int, num_partitions: int,
+                           layout: Layout, workspace: torch.Tensor, stream=None) -> None:
+    _need(topk_idx, "topk_idx", torch.int64)
+    T, K = topk_idx.shape
+    _need(layout.row_of, "layout.row_of", torch.int32, shape=(T, K))
+    _need(layout.num_tokens_per_expert, "layout.num_tokens_per_expert", torch.int32,
+          shape=(num_experts,))
+    _need(layout.num_tokens_per_partition, "layout.num_tokens_per_partition", torch.int32,
+          shape=(num_partitions,))
+    _need(layout.is_token_in_partition, "layout.is_token_in_partition", torch.uint8,
+          shape=(T, num_partitions))
+    _need(layout.expert_offset, "layout.expert_offset", torch.int32, shape=(num_experts + 1,))
+    _need(layout.src_of, "layout.src_of", torch.int32, numel_at_least=T * K)
+    _need(workspace, "workspace", torch.uint8)
+    c = layout.c()
+    _check("ep_get_dispatch_layout", lib.ep_get_dispatch_layout(
+        T, K, num_experts, num_partitions, topk_idx.data_ptr(), ctypes.byref(c),
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
+                num_experts: int, num_partitions: int, quant: int, recv_x: torch.Tensor,
+                recv_scales: Optional[torch.Tensor], recv_topk_idx: torch.Tensor,
+                recv_topk_weights: torch.Tensor, handle: Layout, workspace: torch.Tensor,
+                stream=None) -> None:
+    _need(x, "x", torch.bfloat16)
+    T, H = x.shape
+    K = topk_idx.shape[1]
+    _need(topk_idx, "topk_idx", torch.int64, shape=(T, K))
+    _need(topk_weights, "topk_weights", torch.float32, shape=(T, K))
+    if quant == EP_QUANT_FP8_E4M3_1X128:
+        _need(recv_x, "recv_x", (torch.uint8, torch.float8_e4m3fn), numel_at_least=T * K * H)
+        _need(recv_scales, "recv_scales", torch.float32, numel_at_least=T * K * (H // 128))
+    else:
+        _need(recv_x, "recv_x", torch.bfloat16, numel_at_least=T * K * H)
+    _need(recv_topk_idx, "recv_topk_idx", torch.int32, numel_at_least=T * K)
+    _need(recv_topk_weights, "recv_topk_weights", torch.float32, numel_at_least=T * K)
+    _need(handle.row_of, "handle.row_of", torch.int32, shape=(T, K))
+    _need(handle.src_of, "handle.src_of", torch.int32, numel_at_least=T * K)
+    _need(handle.is_token_in_partition, "handle.is_token_in_partition", torch.uint8,
+          shape=(T, num_partitions))
+    _need(handle.num_tokens_per_expert, "handle.num_tokens_per_expert", torch.int32,
+          shape=(num_experts,))
+    _need(handle.expert_offset, "handle.expert_offset", torch.int32, shape=(num_experts + 1,))
+    _need(workspace, "workspace", torch.uint8)
+    c = handle.c()
+    _check("ep_dispatch", lib.ep_dispatch(
+        T, H, K, num_experts, num_partitions, quant, x.data_ptr(), topk_idx.data_ptr(),
+        topk_weights.data_ptr(), recv_x.data_ptr(), _ptr(recv_scales), recv_topk_idx.data_ptr(),
+        recv_topk_weights.data_ptr(), ctypes.byref(c), workspace.data_ptr(), workspace.numel(),
+        _stream(stream)))
+
+
+def ep_combine(expert_out: torch.Tensor, handle: Layout, topk_weights: torch.Tensor,
+               y: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
+    _need(expert_out, "expert_out", torch.bfloat16)
+    H = expert_out.shape[-1]
+    rows = expert_out.numel() // H if H else 0
+    T, K = topk_weights.shape
+    _need(topk_weights, "topk_weights", torch.float32)
+    _need(handle.row_of, "handle.row_of", torch.int32, shape=(T, K))
+    _need(y, "y", torch.bfloat16, shape=(T, H))
+    _need(workspace, "workspace", torch.uint8)
+    c = ep_layout(row_of=handle.row_of.data_ptr())
+    _check("ep_combine", lib.ep_combine(
+        T, H, K, expert_out.data_ptr(), rows, ctypes.byref(c), topk_weights.data_ptr(),
+        y.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_low_latency_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, num_max_tokens: int,
+                            num_experts: int, recv_x: torch.Tensor, recv_scales: torch.Tensor,
+                            recv_expert_count: torch.Tensor, handle: LowLatencyHandle,
+                            workspace: torch.Tensor, stream=None) -> None:
+    _need(x, "x", torch.bfloat16)
+    T, H = x.shape
+    K = topk_idx.shape[1]
+    _need(topk_idx, "topk_idx", torch.int64, shape=(T, K))
+    _need(recv_x, "recv_x", (torch.uint8, torch.float8_e4m3fn),
+          shape=(num_experts, num_max_tokens, H))
+    _need(recv_scales, "recv_scales", torch.float32,
+          shape=(num_experts, num_max_tokens, H // 128))
+    _need(recv_expert_count, "recv_expert_count", torch.int32, shape=(num_experts,))
+    _need(handle.row_of, "handle.row_of", torch.int32, shape=(T, K))
+    _need(handle.src_of, "handle.src_of", torch.int32, shape=(num_experts, num_max_tokens))
+    _need(workspace, "workspace", torch.uint8)
+    c = handle.c()
+    _check("ep_low_latency_dispatch", lib.ep_low_latency_dispatch(
+        T, H, K, num_experts, num_max_tokens, x.data_ptr(), topk_idx.data_ptr(),
+        recv_x.data_ptr(), recv_scales.data_ptr(), recv_expert_count.data_ptr(), ctypes.byref(c),
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_low_latency_combine(expert_out: torch.Tensor, handle: LowLatencyHandle,
+                           topk_weights: torch.Tensor, y: torch.Tensor, workspace: torch.Tensor,
+                           stream=None) -> None:
+    _need(expert_out, "expert_out", torch.bfloat16)
+    E, cap, H = expert_out.shape
+    T, K = topk_weights.shape
+    _need(topk_weights, "topk_weights", torch.float32)
+    _need(handle.row_of, "handle.row_of", torch.int32, shape=(T, K))
+    _need(y, "y", torch.bfloat16, shape=(T, H))
+    _need(workspace, "workspace", torch.uint8)
+    c = handle.c()
+    _check("ep_low_latency_combine", lib.ep_low_latency_combine(
+        T, H, K, E, cap, expert_out.data_ptr(), ctypes.byref(c), topk_weights.data_ptr(),
+        y.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_debug_wait_probe(timeout_ns: int, workspace: torch.Tensor, stream=None) -> None:
+    _need(workspace, "workspace", torch.uint8)
+    _check("ep_debug_wait_probe", lib.ep_debug_wait_probe(
+        int(timeout_ns), workspace.data_ptr(), workspace.numel(), _stream(stream)))

@@ -1,0 +1,165 @@
+"""DeepEP-style ``Buffer`` on top of the C ABI.
+
+Shapes of the calls follow the DeepEP pages:
+
+* deepseek.csdn.net/67bd3eb22e30c863900615cc, section "使用示例 / MoE 训练中的应用":
+  ``recv_x, recv_topk_idx, recv_topk_weights, handle, event =
+  buffer.dispatch(x, topk_idx, topk_weights, num_experts)``;
+* same page, section "推理解码阶段的应用":
+  ``recv_hidden_states, recv_expert_count, handle, event, hook =
+  buffer.low_latency_dispatch(hidden_states, topk_idx, num_max_tokens, num_experts)``
+  with a buffer of ``num_max_tokens * hidden * num_experts`` elements;
+* "deepseek-ai/DeepEP" (agentlenshq.com), section "典型工作流程": dispatch, expert
+  GEMM, ``buffer.combine(...)`` reduces the expert outputs back.
+
+Everything runs on one GPU: the ``num_partitions`` logical partitions stand for
+the EP ranks, so there is no process group.  torch provides device memory and
+the stream; every step runs in the library's kernels.  ``event`` is a
+``torch.cuda.Event`` recorded after the launches.  The low-latency ``hook`` is
+a no-op callable: on one GPU there is no receive phase to defer.
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple, Union
+
+import torch
+
+from . import _lib
+from ._lib import EP_QUANT_FP8_E4M3_1X128, EP_QUANT_NONE, Layout, LowLatencyHandle
+
+__all__ = ["Buffer"]
+
+
+def _noop_hook():
+    return None
+
+
+class Buffer:
+    """Dispatch / combine buffer for one GPU.
+
+    ``num_partitions`` logical partitions (the EP ranks of a multi-GPU run)
+    split ``num_experts`` experts into equal contiguous ranges.
+    ``max_tokens`` bounds the batch size the workspace is sized for.
+    """
+
+    def __init__(self, num_experts: int, num_partitions: int = 1, max_tokens: int = 4096,
+                 device: Optional[Union[int, str, torch.device]] = None):
+        if num_experts % num_partitions:
+            raise ValueError("num_experts must be a multiple of num_partitions")
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
+            else torch.device(device)
+        self.num_experts = num_experts
+        self.num_partitions = num_partitions
+        self.max_tokens = max_tokens
+        nbytes = _lib.ep_workspace_bytes(max_tokens, num_experts, num_partitions)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        _lib.ep_workspace_init(self.workspace)
+
+    # ------------------------------------------------------------ helpers --
+    def _check_tokens(self, n: int) -> None:
+        if n > self.max_tokens:
+            raise ValueError(f"{n} tokens exceed this buffer's max_tokens={self.max_tokens}")
+
+    def _event(self) -> torch.cuda.Event:
+        ev = torch.cuda.Event()
+        ev.record()
+        return ev
+
+    def read_status(self) -> int:
+        """Synchronise and return (then clear) the sticky device status bits."""
+        return _lib.ep_read_status(self.workspace)
+
+    # ------------------------------------------------------------- layout --
+    def get_dispatch_layout(self, topk_idx: torch.Tensor):
+        """Returns ``(num_tokens_per_expert, num_tokens_per_partition,
+        is_token_in_partition, handle, event)``."""
+        T, K = topk_idx.shape
+        self._check_tokens(T)
+        lay = Layout.empty(T, K, self.num_experts, self.num_partitions, self.device)
+        _lib.ep_get_dispatch_layout(topk_idx, self.num_experts, self.num_partitions, lay,
+                                    self.workspace)
+        return (lay.num_tokens_per_expert, lay.num_tokens_per_partition,
+                lay.is_token_in_partition, lay, self._event())
+
+    # ----------------------------------------------------------- dispatch --
+    def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
+                 num_experts: Optional[int] = None, use_fp8: bool = True, exact: bool = True):
+        """Returns ``(recv_x, recv_topk_idx, recv_topk_weights, handle, event)``.
+
+        With ``use_fp8`` recv_x is ``(payload float8_e4m3fn [R, H], scales float32
+        [R, H/128])``; otherwise a BF16 ``[R, H]`` tensor.  ``exact`` trims the
+        worst-case (T*K-row) buffers to the R received rows, which reads R back to
+        the host once; ``exact=False`` returns the untrimmed buffers and never
+        synchronises (R is then ``handle.num_recv`` on the device).
+        """
+        if num_experts is not None and num_experts != self.num_experts:
+            raise ValueError("num_experts differs from the buffer's")
+        T, H = x.shape
+        K = topk_idx.shape[1]
+        self._check_tokens(T)
+        rows = max(T * K, 1)
+        dev = self.device
+        handle = Layout.empty(T, K, self.num_experts, self.num_partitions, dev)
+        recv_topk_idx = torch.empty(rows, dtype=torch.int32, device=dev)
+        recv_topk_weights = torch.empty(rows, dtype=torch.float32, device=dev)
+        if use_fp8:
+            recv_q = torch.empty((rows, H), dtype=torch.float8_e4m3fn, device=dev)
+            recv_s = torch.empty((rows, H // 128), dtype=torch.float32, device=dev)
+            _lib.ep_dispatch(x, topk_idx, topk_weights, self.num_experts, self.num_partitions,
+                             EP_QUANT_FP8_E4M3_1X128, recv_q, recv_s, recv_topk_idx,
+                             recv_topk_weights, handle, self.workspace)
+        else:
+            recv_q = torch.empty((rows, H), dtype=torch.bfloat16, device=dev)
+            recv_s = None
+            _lib.ep_dispatch(x, topk_idx, topk_weights, self.num_experts, self.num_partitions,
+                             EP_QUANT_NONE, recv_q, None, recv_topk_idx, recv_topk_weights,
+                             handle, self.workspace)
+        event = self._event()
+        if exact:
+            R = int(handle.num_recv.item())
+            recv_q, recv_topk_idx, recv_topk_weights = recv_q[:R], recv_topk_idx[:R], \
+                recv_topk_weights[:R]
+            if recv_s is not None:
+                recv_s = recv_s[:R]
+        recv_x = (recv_q, recv_s) if use_fp8 else recv_q
+        return recv_x, recv_topk_idx, recv_topk_weights, handle, event
+
+    # ------------------------------------------------------------ combine --
+    def combine(self, expert_out: torch.Tensor, handle: Layout, topk_weights: torch.Tensor):
+        """Returns ``(y, event)``: y[t] = bf16(sum_k w[t,k] * expert_out[row_of[t,k]])."""
+        T = topk_weights.shape[0]
+        H = expert_out.shape[-1]
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=self.device)
+        _lib.ep_combine(expert_out, handle, topk_weights, y, self.workspace)
+        return y, self._event()
+
+    # -------------------------------------------------------- low latency --
+    def low_latency_dispatch(self, hidden_states: torch.Tensor, topk_idx: torch.Tensor,
+                             num_max_tokens: int, num_experts: Optional[int] = None):
+        """Returns ``(recv_hidden_states, recv_expert_count, handle, event, hook)``.
+
+        recv_hidden_states is ``(payload float8_e4m3fn [E, num_max_tokens, H],
+        scales float32 [E, num_max_tokens, H/128])``; slots at or beyond
+        recv_expert_count[e] are not written.
+        """
+        E = self.num_experts if num_experts is None else num_experts
+        T, H = hidden_states.shape
+        K = topk_idx.shape[1]
+        dev = self.device
+        recv_q = torch.empty((E, num_max_tokens, H), dtype=torch.float8_e4m3fn, device=dev)
+        recv_s = torch.empty((E, num_max_tokens, H // 128), dtype=torch.float32, device=dev)
+        count = torch.empty(E, dtype=torch.int32, device=dev)
+        handle = LowLatencyHandle.empty(T, K, E, num_max_tokens, dev)
+        _lib.ep_low_latency_dispatch(hidden_states, topk_idx, num_max_tokens, E, recv_q, recv_s,
+                                     count, handle, self.workspace)
+        return (recv_q, recv_s), count, handle, self._event(), _noop_hook
+
+    def low_latency_combine(self, expert_out: torch.Tensor, topk_idx: Optional[torch.Tensor],
+                            topk_weights: torch.Tensor, handle: LowLatencyHandle):
+        """Returns ``(y, event, hook)``.  ``topk_idx`` is accepted for call-shape
+        compatibility; the rows come from the handle."""
+        T = topk_weights.shape[0]
+        H = expert_out.shape[-1]
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=self.device)
+        _lib.ep_low_latency_combine(expert_out, handle, topk_weights, y, self.workspace)
+        return y, self._event(), _noop_hook

@@ -1,0 +1,139 @@
+// combine.cu -- top-k weighted gather-reduce of expert outputs back into token order.
+//
+// "DeepSeek 开源周第二弹：DeepEP", section "DeepEP 的常规内核和低延迟内核": BF16 result
+// merge; "deepseek-ai/DeepEP", section "典型工作流程": combine reduces the expert
+// outputs back to where the tokens came from.  For token t, channel i:
+//     acc = +0.0f;  for k = 0..K-1 with row_of[t, k] >= 0:
+//         acc = fmaf(w[t, k], float(expert_out[row_of[t, k], i]), acc)
+//     y[t, i] = bf16_rne(acc)
+// The k order is fixed, so the result is bit-reproducible.
+//
+// Layout of the work: a CTA owns a slice of a token's row (blockIdx.y) and walks
+// tokens t = blockIdx.x, blockIdx.x + gridDim.x, ...; each thread owns 8 channels
+// (one 16-byte vector) and issues the K vector loads of its channels before it
+// uses any, so K * 16 bytes per thread (128 B at K = 8) are in flight.  The K
+// source rows are contiguous 14 KB rows (hidden 7168), so every warp reads whole
+// 512-byte runs: the reads are coalesced and the traffic is the algorithmic
+// minimum (K rows read once, one row written).  The rows and weights of the
+// next token are prefetched while the current one is reduced.
+#include "ep_device.cuh"
+#include "ep_internal.h"
+
+namespace ep {
+
+namespace {
+
+constexpr int kCombineMaxThreads = 512;
+constexpr int kLoadBatch = 8;  // vector loads issued before the first FMA
+
+__global__ void __launch_bounds__(kCombineMaxThreads) combine_kernel(CombineParams p,
+                                                                    int64_t vec_per_slice) {
+    __shared__ int rows_sm[2][32];
+    __shared__ float w_sm[2][32];
+    const int tid = threadIdx.x;
+    const int K = p.K;
+    const int64_t T = p.T, V = p.H / 8;
+    const int64_t v0 = static_cast<int64_t>(blockIdx.y) * vec_per_slice;
+    const int64_t v1 = min(V, v0 + vec_per_slice);
+    const uint4* eo = static_cast<const uint4*>(p.expert_out);
+    uint4* y = static_cast<uint4*>(p.y);
+
+    int nrow = -1;
+    float nw = 0.0f;
+    if (tid < K && static_cast<int64_t>(blockIdx.x) < T) {
+        nrow = p.row_of[static_cast<int64_t>(blockIdx.x) * K + tid];
+        nw = p.topk_weights[static_cast<int64_t>(blockIdx.x) * K + tid];
+    }
+    int buf = 0;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x, buf ^= 1) {
+        if (tid < K) {
+            int r = nrow;
+            if (r >= 0 && static_cast<int64_t>(r) >= p.expert_out_rows) {
+                raise_status(p.status, kDevIndexRange);
+                r = -1;
+            }
+            rows_sm[buf][tid] = r;
+            w_sm[buf][tid] = nw;
+            const int64_t tn = t + gridDim.x;
+            if (tn < T) {
+                nrow = p.row_of[tn * K + tid];
+                nw = p.topk_weights[tn * K + tid];
+            }
+        }
+        __syncthreads();
+        const int* rows = rows_sm[buf];
+        const float* ws = w_sm[buf];
+        for (int64_t v = v0 + tid; v < v1; v += blockDim.x) {
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+            for (int k0 = 0; k0 < K; k0 += kLoadBatch) {
+                uint4 d[kLoadBatch];
+#pragma unroll
+                for (int u = 0; u < kLoadBatch; ++u) {
+                    const int k = k0 + u;
+                    const int r = k < K ? rows[k] : -1;
+                    d[u] = r >= 0 ? ld_stream_v4(eo + static_cast<int64_t>(r) * V + v)
+                                  : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int u = 0; u < kLoadBatch; ++u) {
+                    const int k = k0 + u;
+                    if (k < K && rows[k] >= 0) {
+                        const float w = ws[k];
+                        acc[0] = __fmaf_rn(w, bf16_lo(d[u].x), acc[0]);
+                        acc[1] = __fmaf_rn(w, bf16_hi(d[u].x), acc[1]);
+                        acc[2] = __fmaf_rn(w, bf16_lo(d[u].y), acc[2]);
+                        acc[3] = __fmaf_rn(w, bf16_hi(d[u].y), acc[3]);
+                        acc[4] = __fmaf_rn(w, bf16_lo(d[u].z), acc[4]);
+                        acc[5] = __fmaf_rn(w, bf16_hi(d[u].z), acc[5]);
+                        acc[6] = __fmaf_rn(w, bf16_lo(d[u].w), acc[6]);
+                        acc[7] = __fmaf_rn(w, bf16_hi(d[u].w), acc[7]);
+                    }
+                }
+            }
+            uint4 out;
+            out.x = bf16x2_rn(acc[0], acc[1]);
+            out.y = bf16x2_rn(acc[2], acc[3]);
+            out.z = bf16x2_rn(acc[4], acc[5]);
+            out.w = bf16x2_rn(acc[6], acc[7]);
+            y[t * V + v] = out;
+        }
+        // rows_sm[buf] is rewritten two tokens later, after the next barrier
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
+    if (p.T == 0) return cudaSuccess;
+    DeviceInfo dev;
+    cudaError_t err = device_info(&dev);
+    if (err != cudaSuccess) return err;
+    const int64_t V = p.H / 8;
+    // slices of a row: at most kCombineMaxThreads vectors each, and enough
+    // (token, slice) CTAs to cover every SM twice on small batches
+    int64_t slices = (V + kCombineMaxThreads - 1) / kCombineMaxThreads;
+    const int64_t want = (2LL * dev.num_sms + p.T - 1) / p.T;
+    if (slices < want) slices = want;
+    if (slices > V) slices = V;
+    if (slices > 65535) slices = 65535;
+    const int64_t per_slice = (V + slices - 1) / slices;
+    slices = (V + per_slice - 1) / per_slice;
+    int threads = static_cast<int>((per_slice + 31) / 32 * 32);
+    if (threads > kCombineMaxThreads) threads = kCombineMaxThreads;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_kernel, threads, 0) !=
+            cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    int64_t gx = (static_cast<int64_t>(per_sm) * dev.num_sms + slices - 1) / slices;
+    if (gx > p.T) gx = p.T;
+    if (gx < 1) gx = 1;
+    if (gx > 2147483647LL) gx = 2147483647LL;
+    combine_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(slices)), threads, 0,
+                     stream>>>(p, per_slice);
+    return cudaGetLastError();
+}
+
+}  // namespace ep

@@ -1,0 +1,261 @@
+// ep_api.cu -- the exported C ABI (include/ep_b200.h): host-side argument checks,
+// workspace handling and kernel launches.  No allocation, no host synchronisation
+// except in ep_read_status().
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "ep_b200.h"
+#include "ep_device.cuh"
+#include "ep_internal.h"
+
+namespace ep {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_have_info[kMaxDevices];
+DeviceInfo g_info[kMaxDevices];
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ep_status check_routing(int64_t T, int32_t K, int32_t E, int32_t P) {
+    if (T < 0 || K < 1 || K > 32 || E < 1 || E > 4096 || P < 1 || P > 64 || E % P != 0)
+        return EP_ERR_SHAPE;
+    if (T * static_cast<int64_t>(K) >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    return EP_OK;
+}
+
+ep_status check_hidden(int64_t H, bool fp8) {
+    if (H <= 0 || H > 16384) return EP_ERR_SHAPE;
+    if (fp8 ? (H % 128 != 0) : (H % 8 != 0)) return EP_ERR_SHAPE;
+    return EP_OK;
+}
+
+ep_status check_layout_ptrs(const ep_layout* lay, int64_t T) {
+    if (!lay || !lay->num_tokens_per_expert || !lay->num_tokens_per_partition ||
+        !lay->expert_offset || !lay->num_recv)
+        return EP_ERR_INVALID_ARG;
+    if (T > 0 && (!lay->is_token_in_partition || !lay->row_of || !lay->src_of))
+        return EP_ERR_INVALID_ARG;
+    return EP_OK;
+}
+
+inline ep_status cuda_status(cudaError_t e) { return e == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
+
+}  // namespace
+
+cudaError_t device_info(DeviceInfo* out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev >= 0 && dev < kMaxDevices && g_have_info[dev].load(std::memory_order_acquire)) {
+        *out = g_info[dev];
+        return cudaSuccess;
+    }
+    DeviceInfo d;
+    d.device = dev;
+    err = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    int optin = 0;
+    err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (err != cudaSuccess) return err;
+    d.max_smem_optin = static_cast<size_t>(optin);
+    if (dev >= 0 && dev < kMaxDevices) {
+        g_info[dev] = d;
+        g_have_info[dev].store(1, std::memory_order_release);
+    }
+    *out = d;
+    return cudaSuccess;
+}
+
+}  // namespace ep
+
+using namespace ep;
+
+extern "C" {
+
+int32_t ep_abi_version(void) { return 1; }
+
+const char* ep_status_string(int32_t status) {
+    switch (status) {
+        case EP_OK: return "ok";
+        case EP_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, unknown enum)";
+        case EP_ERR_SHAPE: return "unsupported size";
+        case EP_ERR_WORKSPACE: return "workspace too small";
+        case EP_ERR_CUDA: return "CUDA runtime error";
+        default: return "unknown status";
+    }
+}
+
+size_t ep_workspace_bytes(int64_t num_tokens, int32_t num_experts, int32_t num_partitions) {
+    if (num_tokens < 0 || num_experts < 1 || num_partitions < 1) return 0;
+    const size_t body = sizeof(int32_t) * static_cast<size_t>(chunk_stride(num_tokens)) *
+                        (static_cast<size_t>(num_experts) + static_cast<size_t>(num_partitions));
+    return (kWsHeader + body + 255) / 256 * 256;
+}
+
+ep_status ep_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+    if (!workspace || workspace_bytes < kWsHeader) return EP_ERR_INVALID_ARG;
+    return cuda_status(
+        cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_read_status(void* workspace, size_t workspace_bytes, void* stream, uint32_t* bits_out) {
+    if (!workspace || !bits_out || workspace_bytes < kWsHeader) return EP_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t bits = 0;
+    cudaError_t err = cudaMemcpyAsync(&bits, static_cast<uint8_t*>(workspace) + kWsStatus,
+                                      sizeof(bits), cudaMemcpyDeviceToHost, s);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+    if (err == cudaSuccess)
+        err = cudaMemsetAsync(static_cast<uint8_t*>(workspace) + kWsStatus, 0, sizeof(uint32_t), s);
+    if (err != cudaSuccess) return EP_ERR_CUDA;
+    *bits_out = bits;
+    return EP_OK;
+}
+
+ep_status ep_get_dispatch_layout(int64_t num_tokens, int32_t num_topk, int32_t num_experts,
+                                 int32_t num_partitions, const int64_t* topk_idx,
+                                 const ep_layout* layout, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+    ep_status st = check_routing(num_tokens, num_topk, num_experts, num_partitions);
+    if (st != EP_OK) return st;
+    if ((st = check_layout_ptrs(layout, num_tokens)) != EP_OK) return st;
+    if (!workspace || (num_tokens > 0 && !topk_idx)) return EP_ERR_INVALID_ARG;
+    if (workspace_bytes < ep_workspace_bytes(num_tokens, num_experts, num_partitions))
+        return EP_ERR_WORKSPACE;
+    const Workspace ws = carve_workspace(workspace, num_tokens, num_experts);
+    return cuda_status(launch_layout(num_tokens, num_topk, num_experts, num_partitions, topk_idx,
+                                     *layout, ws, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk, int32_t num_experts,
+                      int32_t num_partitions, int32_t quant, const void* x, const int64_t* topk_idx,
+                      const float* topk_weights, void* recv_x, float* recv_scales,
+                      int32_t* recv_topk_idx, float* recv_topk_weights, const ep_layout* handle,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    if (quant != EP_QUANT_NONE && quant != EP_QUANT_FP8_E4M3_1X128) return EP_ERR_INVALID_ARG;
+    const bool fp8 = quant == EP_QUANT_FP8_E4M3_1X128;
+    ep_status st = check_routing(num_tokens, num_topk, num_experts, num_partitions);
+    if (st != EP_OK) return st;
+    if ((st = check_hidden(hidden, fp8)) != EP_OK) return st;
+    if ((st = check_layout_ptrs(handle, num_tokens)) != EP_OK) return st;
+    if (!workspace) return EP_ERR_INVALID_ARG;
+    if (num_tokens > 0) {
+        if (!x || !topk_idx || !topk_weights || !recv_x || !recv_topk_idx || !recv_topk_weights)
+            return EP_ERR_INVALID_ARG;
+        if (fp8 && !recv_scales) return EP_ERR_INVALID_ARG;
+        if (!aligned16(x) || !aligned16(recv_x) || (fp8 && !aligned16(recv_scales)))
+            return EP_ERR_INVALID_ARG;
+    }
+    if (workspace_bytes < ep_workspace_bytes(num_tokens, num_experts, num_partitions))
+        return EP_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Workspace ws = carve_workspace(workspace, num_tokens, num_experts);
+    cudaError_t err =
+        launch_layout(num_tokens, num_topk, num_experts, num_partitions, topk_idx, *handle, ws, s);
+    if (err != cudaSuccess) return EP_ERR_CUDA;
+    DispatchParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = num_topk;
+    p.experts_per_partition = num_experts / num_partitions;
+    p.x = x;
+    p.topk_idx = topk_idx;
+    p.topk_weights = topk_weights;
+    p.row_of = handle->row_of;
+    p.recv_x = recv_x;
+    p.recv_scales = recv_scales;
+    p.recv_topk_idx = recv_topk_idx;
+    p.recv_topk_weights = recv_topk_weights;
+    p.status = ws.status;
+    p.timeout_ns = kDefaultTimeoutNs;
+    return cuda_status(fp8 ? launch_dispatch_fp8(p, s) : launch_dispatch_bf16(p, s));
+}
+
+ep_status ep_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk, const void* expert_out,
+                     int64_t expert_out_rows, const ep_layout* handle, const float* topk_weights,
+                     void* y, void* workspace, size_t workspace_bytes, void* stream) {
+    if (num_tokens < 0 || num_topk < 1 || num_topk > 32 || expert_out_rows < 0) return EP_ERR_SHAPE;
+    if (num_tokens * static_cast<int64_t>(num_topk) >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    ep_status st = check_hidden(hidden, false);
+    if (st != EP_OK) return st;
+    if (!handle || !workspace || workspace_bytes < kWsHeader) return EP_ERR_INVALID_ARG;
+    if (num_tokens == 0) return EP_OK;
+    if (!handle->row_of || !topk_weights || !y || (!expert_out && expert_out_rows > 0))
+        return EP_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(expert_out)) return EP_ERR_INVALID_ARG;
+    CombineParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = num_topk;
+    p.expert_out = expert_out;
+    p.expert_out_rows = expert_out_rows;
+    p.row_of = handle->row_of;
+    p.topk_weights = topk_weights;
+    p.y = y;
+    p.status = carve_workspace(workspace, 0, 1).status;
+    return cuda_status(launch_combine(p, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_low_latency_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                  int32_t num_experts, int32_t num_max_tokens, const void* x,
+                                  const int64_t* topk_idx, void* recv_x, float* recv_scales,
+                                  int32_t* recv_expert_count, const ep_ll_handle* handle,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+    ep_status st = check_routing(num_tokens, num_topk, num_experts, 1);
+    if (st != EP_OK) return st;
+    if ((st = check_hidden(hidden, true)) != EP_OK) return st;
+    if (num_max_tokens < 1 || num_tokens > num_max_tokens) return EP_ERR_SHAPE;
+    if (static_cast<int64_t>(num_experts) * num_max_tokens >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    if (!handle || !workspace || !recv_expert_count || workspace_bytes < kWsHeader)
+        return EP_ERR_INVALID_ARG;
+    if (num_tokens > 0) {
+        if (!x || !topk_idx || !recv_x || !recv_scales || !handle->row_of || !handle->src_of)
+            return EP_ERR_INVALID_ARG;
+        if (!aligned16(x) || !aligned16(recv_x) || !aligned16(recv_scales))
+            return EP_ERR_INVALID_ARG;
+    }
+    LowLatencyDispatchParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = num_topk;
+    p.E = num_experts;
+    p.cap = num_max_tokens;
+    p.x = x;
+    p.topk_idx = topk_idx;
+    p.recv_x = recv_x;
+    p.recv_scales = recv_scales;
+    p.recv_expert_count = recv_expert_count;
+    p.row_of = handle->row_of;
+    p.src_of = handle->src_of;
+    p.status = carve_workspace(workspace, 0, 1).status;
+    p.timeout_ns = kDefaultTimeoutNs;
+    return cuda_status(launch_ll_dispatch(p, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_low_latency_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                 int32_t num_experts, int32_t num_max_tokens,
+                                 const void* expert_out, const ep_ll_handle* handle,
+                                 const float* topk_weights, void* y, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    if (num_experts < 1 || num_max_tokens < 1) return EP_ERR_SHAPE;
+    if (!handle) return EP_ERR_INVALID_ARG;
+    ep_layout lay = {};
+    lay.row_of = handle->row_of;
+    return ep_combine(num_tokens, hidden, num_topk, expert_out,
+                      static_cast<int64_t>(num_experts) * num_max_tokens, &lay, topk_weights, y,
+                      workspace, workspace_bytes, stream);
+}
+
+ep_status ep_debug_wait_probe(uint64_t timeout_ns, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+    if (!workspace || workspace_bytes < kWsHeader) return EP_ERR_INVALID_ARG;
+    const Workspace ws = carve_workspace(workspace, 0, 1);
+    return cuda_status(
+        launch_wait_probe(ws.status, ws.probe_flag, timeout_ns, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+// ep_internal.h -- host-side launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ep_b200.h"
+
+namespace ep {
+
+// Per-device facts the launchers size grids with.
+struct DeviceInfo {
+    int device;
+    int num_sms;
+    size_t max_smem_optin;
+};
+cudaError_t device_info(DeviceInfo* out);
+
+// Number of layout chunks (kChunkTokens tokens each) and their padded stride.
+int64_t num_chunks(int64_t num_tokens);
+int64_t chunk_stride(int64_t num_tokens);
+
+struct Workspace {
+    uint32_t* status;
+    uint32_t* ticket;
+    uint32_t* probe_flag;
+    int32_t* chunk_expert;     // [E][chunk_stride]
+    int32_t* chunk_partition;  // [P][chunk_stride]
+};
+Workspace carve_workspace(void* ws, int64_t num_tokens, int32_t num_experts);
+
+// Launch the layout kernels (count + rank) on `stream`.  The first launch waits
+// for all earlier work in the stream; the rank launch is programmatically
+// dependent on the count launch.
+cudaError_t launch_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int64_t* topk_idx,
+                          const ep_layout& lay, const Workspace& ws, cudaStream_t stream);
+
+struct DispatchParams {
+    int64_t T;
+    int64_t H;
+    int32_t K;
+    int32_t experts_per_partition;
+    const void* x;
+    const int64_t* topk_idx;
+    const float* topk_weights;
+    const int32_t* row_of;
+    void* recv_x;
+    float* recv_scales;
+    int32_t* recv_topk_idx;
+    float* recv_topk_weights;
+    uint32_t* status;
+    uint64_t timeout_ns;
+};
+// Launched programmatically dependent on the preceding (layout) kernel.
+cudaError_t launch_dispatch_fp8(const DispatchParams& p, cudaStream_t stream);
+cudaError_t launch_dispatch_bf16(const DispatchParams& p, cudaStream_t stream);
+
+struct CombineParams {
+    int64_t T;
+    int64_t H;
+    int32_t K;
+    const void* expert_out;
+    int64_t expert_out_rows;
+    const int32_t* row_of;
+    const float* topk_weights;
+    void* y;
+    uint32_t* status;
+};
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+
+struct LowLatencyDispatchParams {
+    int64_t T;
+    int64_t H;
+    int32_t K;
+    int32_t E;
+    int32_t cap;
+    const void* x;
+    const int64_t* topk_idx;
+    void* recv_x;
+    float* recv_scales;
+    int32_t* recv_expert_count;
+    int32_t* row_of;
+    int32_t* src_of;
+    uint32_t* status;
+    uint64_t timeout_ns;
+};
+cudaError_t launch_ll_dispatch(const LowLatencyDispatchParams& p, cudaStream_t stream);
+
+cudaError_t launch_wait_probe(uint32_t* status, uint32_t* flag, uint64_t timeout_ns,
+                              cudaStream_t stream);
+
+// Default bound on any device-side wait (device time).
+constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;
+
+}  // namespace ep

@@ -1,0 +1,50 @@
+// ep_quant.cuh -- the FP8 quantiser shared by the normal and low-latency dispatch kernels.
+//
+// Per 128-channel block of a BF16 row: amax = max |x|, s = max(amax, 1e-4) / 448
+// (one IEEE fp32 division), q = e4m3(x / s) with the fp32 quotient rounded to
+// nearest-even and saturated to +-448 (cvt.rn.satfinite).  The pages fix only
+// "FP8 dispatch" ("DeepSeek 开源周第二弹：DeepEP", section "DeepEP 的常规内核和低延迟
+// 内核"); E4M3 with 1x128 fp32 scales is this library's reading.
+#pragma once
+
+#include "ep_device.cuh"
+
+namespace ep {
+
+// Quantise one BF16 row held in shared memory.  A warp takes two 128-channel
+// blocks at a time: lanes 0-15 the even block, lanes 16-31 the odd one, 8
+// channels (16 bytes) per lane; the block amax is a 16-lane xor-shuffle max.
+__device__ __forceinline__ void quantize_row_fp8(const uint8_t* __restrict__ in,
+                                             uint8_t* __restrict__ out_q,
+                                             float* __restrict__ out_s, int nb, int warp,
+                                             int nwarps, int lane) {
+    const int half = lane >> 4, l16 = lane & 15;
+    for (int bp = warp; 2 * bp < nb; bp += nwarps) {
+        const int b = 2 * bp + half;
+        const bool act = b < nb;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (act) v = reinterpret_cast<const uint4*>(in)[b * 16 + l16];
+        float f[8];
+        f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
+        f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+        f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
+        f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 8));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        const float s = fmaxf(amax, 1e-4f) / 448.0f;  // IEEE division (no fast-math)
+        uint2 q;
+        q.x = e4m3x2(f[0] / s, f[1] / s) | (e4m3x2(f[2] / s, f[3] / s) << 16);
+        q.y = e4m3x2(f[4] / s, f[5] / s) | (e4m3x2(f[6] / s, f[7] / s) << 16);
+        if (act) {
+            reinterpret_cast<uint2*>(out_q)[b * 16 + l16] = q;
+            if (l16 == 0) out_s[b] = s;
+        }
+    }
+}
+
+}  // namespace ep

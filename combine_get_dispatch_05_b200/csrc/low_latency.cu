@@ -1,0 +1,191 @@
+// low_latency.cu -- low-latency dispatch for small decode batches, one fused kernel.
+//
+// deepseek.csdn.net/67bd3eb22e30c863900615cc, section "推理解码阶段的应用":
+// low_latency_dispatch(hidden_states, topk_idx, num_max_tokens, num_experts) returns
+// recv_hidden_states and recv_expert_count; the buffer holds
+// num_max_tokens * hidden * num_experts elements, i.e. num_max_tokens rows per
+// expert.  "DeepSeek 开源周第二弹：DeepEP", section "DeepEP 的常规内核和低延迟内核":
+// 128-token decode batches, FP8 dispatch.
+//
+// One CTA per token does everything the normal path does in three kernels:
+//   - its row's bulk load is issued first, so HBM latency overlaps the rest;
+//   - slot of (t, k) in expert e = number of earlier (t', k') routed to e, counted
+//     directly over the topk_idx prefix (the batch is small, the prefix is L2-hot);
+//     the order is the normal layout's, so slot j of e holds normal row
+//     expert_offset[e] + j;
+//   - CTA 0 also histograms all T*K ids into recv_expert_count;
+//   - quantise (same arithmetic as the normal FP8 path) and bulk-store the row
+//     into slot e * num_max_tokens + j of each destination expert.
+#include "ep_device.cuh"
+#include "ep_internal.h"
+#include "ep_quant.cuh"
+
+namespace ep {
+
+namespace {
+
+constexpr int kLLThreads = 256;
+
+struct LLSmem {
+    uint32_t in_bytes, q_bytes, s_bytes;
+    uint32_t off_q, off_s, off_bar, off_rows, off_cnt, off_eid, off_hist, total;
+};
+
+__host__ __device__ inline LLSmem ll_smem(int64_t H, int32_t E) {
+    LLSmem s;
+    const uint32_t nb = static_cast<uint32_t>(H / 128);
+    s.in_bytes = static_cast<uint32_t>(H) * 2u;
+    s.q_bytes = static_cast<uint32_t>(H);
+    s.s_bytes = (nb * 4u + 15u) & ~15u;
+    s.off_q = s.in_bytes;
+    s.off_s = s.off_q + s.q_bytes;
+    s.off_bar = s.off_s + s.s_bytes;
+    s.off_rows = s.off_bar + 16u;
+    s.off_cnt = s.off_rows + 4u * 32u;
+    s.off_eid = s.off_cnt + 4u * 32u;
+    s.off_hist = s.off_eid + 8u * 32u;
+    s.total = s.off_hist + 4u * static_cast<uint32_t>(E);
+    return s;
+}
+
+__global__ void __launch_bounds__(kLLThreads) ll_dispatch_kernel(LowLatencyDispatchParams p) {
+    extern __shared__ __align__(128) uint8_t sm[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    const int64_t H = p.H;
+    const int K = p.K, E = p.E, cap = p.cap, nb = static_cast<int>(H >> 7);
+    const LLSmem L = ll_smem(H, E);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.off_bar);
+    int* rows_sm = reinterpret_cast<int*>(sm + L.off_rows);
+    int* cnt_sm = reinterpret_cast<int*>(sm + L.off_cnt);
+    int64_t* eid_sm = reinterpret_cast<int64_t*>(sm + L.off_eid);
+    int* hist = reinterpret_cast<int*>(sm + L.off_hist);
+    uint8_t* out_q = sm + L.off_q;
+    float* out_s = reinterpret_cast<float*>(sm + L.off_s);
+    const bool scale_bulk = (static_cast<uint32_t>(nb) * 4u) == L.s_bytes;
+    const int64_t t = blockIdx.x;
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar, L.in_bytes);
+        bulk_load(sm, static_cast<const uint8_t*>(p.x) + t * H * 2, L.in_bytes, bar);
+    }
+    if (tid < K) {
+        eid_sm[tid] = p.topk_idx[t * K + tid];
+        cnt_sm[tid] = 0;
+    }
+    if (blockIdx.x == 0)
+        for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+
+    // slot of (t, k): pairs (t', k') < (t, k) in (token, k) order with the same expert
+    const int64_t base = t * K;
+    for (int64_t j = tid; j < base + K; j += blockDim.x) {
+        const int64_t ej = p.topk_idx[j];
+        for (int k = 0; k < K; ++k)
+            if (j < base + k && ej == eid_sm[k]) atomicAdd(&cnt_sm[k], 1);
+    }
+    if (blockIdx.x == 0) {
+        for (int64_t j = tid; j < p.T * K; j += blockDim.x) {
+            const int64_t ej = p.topk_idx[j];
+            if (ej >= 0 && ej < E) atomicAdd(&hist[ej], 1);
+        }
+    }
+    __syncthreads();
+    if (tid < K) {
+        const int64_t e = eid_sm[tid];
+        int row = -1;
+        if (e != -1 && (e < 0 || e >= E)) {
+            raise_status(p.status, kDevIndexRange);
+        } else if (e >= 0) {
+            const int j = cnt_sm[tid];
+            if (j < cap)
+                row = static_cast<int>(e * cap + j);
+            else
+                raise_status(p.status, kDevCapacity);
+        }
+        rows_sm[tid] = row;
+        p.row_of[base + tid] = row;
+        if (row >= 0) p.src_of[row] = static_cast<int32_t>(base + tid);
+    }
+    if (blockIdx.x == 0)
+        for (int e = tid; e < E; e += blockDim.x) p.recv_expert_count[e] = min(hist[e], cap);
+
+    const bool ok = mbar_wait_bounded(bar, 0, p.timeout_ns);
+    if (!__syncthreads_and(ok)) {
+        if (tid == 0) {
+            raise_status(p.status, kDevTimeout);
+            mbar_wait_bounded(bar, 0, kDefaultTimeoutNs);  // let the load land before exiting
+        }
+        return;
+    }
+    quantize_row_fp8(sm, out_q, out_s, nb, warp, nwarps, lane);
+    fence_proxy_async_smem();
+    __syncthreads();
+    uint8_t* recv_x = static_cast<uint8_t*>(p.recv_x);
+    if (warp == 0 && lane < K) {
+        const int row = rows_sm[lane];
+        if (row >= 0) {
+            bulk_store(recv_x + static_cast<int64_t>(row) * H, out_q, L.q_bytes);
+            if (scale_bulk)
+                bulk_store(p.recv_scales + static_cast<int64_t>(row) * nb, out_s,
+                           static_cast<uint32_t>(nb) * 4u);
+        }
+        bulk_commit();
+    }
+    if (!scale_bulk) {
+        for (int idx = tid; idx < K * nb; idx += blockDim.x) {
+            const int k = idx / nb, b = idx - k * nb;
+            const int r = rows_sm[k];
+            if (r >= 0) p.recv_scales[static_cast<int64_t>(r) * nb + b] = out_s[b];
+        }
+    }
+    if (warp == 0 && lane < K) bulk_wait_all<0>();
+}
+
+__global__ void wait_probe_kernel(uint32_t* status, const volatile uint32_t* flag,
+                                  uint64_t timeout_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    // (1) a flag nothing sets
+    const uint64_t t0 = globaltimer_ns();
+    bool seen = false;
+    while (!(seen = (*flag != 0u))) {
+        if (globaltimer_ns() - t0 > timeout_ns) break;
+    }
+    if (!seen) raise_status(status, kDevTimeout);
+    // (2) an mbarrier waiting for 16 transaction bytes no copy will deliver
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&bar, 16u);
+    if (!mbar_wait_bounded(&bar, 0, timeout_ns)) raise_status(status, kDevTimeout);
+}
+
+}  // namespace
+
+cudaError_t launch_ll_dispatch(const LowLatencyDispatchParams& p, cudaStream_t stream) {
+    if (p.T == 0) {
+        // no tokens: every expert received nothing
+        return cudaMemsetAsync(p.recv_expert_count, 0, sizeof(int32_t) * p.E, stream);
+    }
+    DeviceInfo dev;
+    cudaError_t err = device_info(&dev);
+    if (err != cudaSuccess) return err;
+    const LLSmem L = ll_smem(p.H, p.E);
+    if (L.total > dev.max_smem_optin) return cudaErrorInvalidValue;
+    err = cudaFuncSetAttribute(ll_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(L.total));
+    if (err != cudaSuccess) return err;
+    ll_dispatch_kernel<<<dim3(static_cast<unsigned>(p.T)), kLLThreads, L.total, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_wait_probe(uint32_t* status, uint32_t* flag, uint64_t timeout_ns,
+                              cudaStream_t stream) {
+    wait_probe_kernel<<<1, 1, 0, stream>>>(status, flag, timeout_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace ep

@@ -1,0 +1,235 @@
+/*
+ * ep_b200.h -- C ABI of the B200 (sm_100a) MoE token dispatch / combine library.
+ *
+ * The library is the single-GPU hot path of an expert-parallel (EP)
+ * communication layer in the style of DeepEP:
+ *
+ *   - layout:   from topk_idx, count rows per expert and tokens per logical
+ *               partition, and give every (token, top-k slot) a stable row in an
+ *               expert-contiguous receive buffer;
+ *   - dispatch: quantise each token's BF16 hidden vector to FP8 (or copy it as
+ *               BF16) and write it to each of its rows;
+ *   - combine:  gather the expert outputs of a token's rows and reduce them,
+ *               weighted by topk_weights, back into token order in BF16;
+ *   - low-latency dispatch / combine: the same for small decode batches, into a
+ *               padded [num_experts, num_max_tokens, hidden] receive tensor.
+ *
+ * Sources (the DeepEP pages):
+ *   "DeepSeek 开源周第二弹：DeepEP —— 首个 MoE 模型训练和推理的 EP 通信库"
+ *   (m.youleyou.com), sections "DeepEP 的核心功能" and
+ *   "DeepEP 的常规内核和低延迟内核": normal kernels for training / prefill,
+ *   low-latency kernels for decode, FP8 dispatch, BF16 result merge.
+ *   deepseek.csdn.net/67bd3eb22e30c863900615cc, sections "使用示例 / MoE 训练中的
+ *   应用" (dispatch(x, topk_idx, topk_weights, num_experts) returning recv_x,
+ *   recv_topk_idx, recv_topk_weights, handle, event) and "推理解码阶段的应用"
+ *   (low_latency_dispatch(hidden_states, topk_idx, num_max_tokens,
+ *   num_experts) returning recv_hidden_states, recv_expert_count, handle,
+ *   event, hook; buffer of num_max_tokens * hidden * num_experts elements).
+ *   "deepseek-ai/DeepEP" (agentlenshq.com), section "典型工作流程": dispatch,
+ *   expert GEMM, combine reduces the expert outputs back.
+ *
+ * On one GPU the EP "ranks" are logical partitions of one HBM buffer:
+ * partition p owns experts [p*E/P, (p+1)*E/P) and, because the receive buffer
+ * is expert-major, one contiguous slice of rows.  The exchange is a
+ * device-local permutation; there is no inter-GPU traffic.
+ *
+ * Conventions (every entry point):
+ *   - Pointers named as device memory must be device (or managed) memory of
+ *     the current CUDA device.  Every buffer is owned and allocated by the
+ *     caller; the library allocates nothing and keeps no state between calls
+ *     apart from a per-device cache of the SM count and kernel attributes.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every call is asynchronous on that stream; host-side argument checks
+ *     run before anything is enqueued and return an error synchronously.
+ *   - Device-side problems (an out-of-range expert id, a full low-latency
+ *     expert, a bounded wait that gave up) never trap: the offending row is
+ *     skipped and a sticky bit is set in the workspace's status word, read
+ *     and cleared by ep_read_status().
+ *   - A workspace may be used by one stream at a time; calls that share a
+ *     workspace on different streams race.
+ *   - Layouts: row-major, contiguous.  x / expert_out / y are BF16 bit
+ *     patterns; FP8 payload is OCP E4M3 (one byte per element).  topk_idx is
+ *     int64 (the dtype torch.topk returns), -1 marks a masked slot.
+ *   - Sizes: T = num_tokens >= 0, K = num_topk in [1, 32], E = num_experts in
+ *     [1, 4096], P = num_partitions in [1, 64] dividing E, H = hidden > 0 with
+ *     H % 8 == 0 (BF16) or H % 128 == 0 (FP8), H <= 16384; T * K < 2^31.
+ *     Base pointers of x, recv_x, recv_scales, expert_out, y must be 16-byte
+ *     aligned (the rows move by 16-byte vectors and bulk copies).
+ */
+#ifndef EP_B200_H
+#define EP_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define EP_API __attribute__((visibility("default")))
+#else
+#define EP_API
+#endif
+
+/* Host-side return codes. */
+typedef enum ep_status {
+    EP_OK = 0,
+    EP_ERR_INVALID_ARG = 1, /* a required pointer is NULL, misaligned, or an enum is unknown */
+    EP_ERR_SHAPE = 2,       /* a size is outside the supported range (see Conventions) */
+    EP_ERR_WORKSPACE = 3,   /* workspace smaller than ep_workspace_bytes() */
+    EP_ERR_CUDA = 4         /* the CUDA runtime reported an error (launch / copy) */
+} ep_status;
+
+/* Sticky device status bits (ep_read_status). */
+#define EP_DEV_INDEX_RANGE 0x1u /* an expert id outside [-1, E) or a row outside the buffer: skipped */
+#define EP_DEV_TIMEOUT 0x2u     /* a bounded device wait gave up; the kernel stopped early */
+#define EP_DEV_CAPACITY 0x4u    /* a low-latency row did not fit num_max_tokens: dropped */
+
+/* Dispatch payload format. */
+typedef enum ep_quant {
+    EP_QUANT_NONE = 0,           /* BF16 rows copied bit for bit */
+    EP_QUANT_FP8_E4M3_1X128 = 1  /* E4M3 codes + one fp32 scale per 128 channels */
+} ep_quant;
+
+/*
+ * The layout of one batch, and the `handle` that dispatch returns and combine
+ * consumes (deepseek.csdn.net/67bd3eb22e30c863900615cc, "使用示例": dispatch
+ * returns a handle).  A struct of caller-owned device pointers:
+ *   num_tokens_per_expert[E]     rows routed to expert e
+ *   num_tokens_per_partition[P]  distinct tokens that name >= 1 expert of partition p
+ *   is_token_in_partition[T*P]   uint8 0/1
+ *   expert_offset[E+1]           exclusive prefix sum of num_tokens_per_expert
+ *   row_of[T*K]                  receive row of (t, k); -1 for a masked / skipped slot
+ *   src_of[T*K]                  inverse of row_of: t*K + k for rows [0, num_recv)
+ *   num_recv[1]                  R = number of receive rows
+ * Row order: expert id ascending, then token ascending, then k ascending.
+ */
+typedef struct ep_layout {
+    int32_t* num_tokens_per_expert;
+    int32_t* num_tokens_per_partition;
+    uint8_t* is_token_in_partition;
+    int32_t* expert_offset;
+    int32_t* row_of;
+    int32_t* src_of;
+    int32_t* num_recv;
+} ep_layout;
+
+/*
+ * Handle of a low-latency dispatch (caller-owned device pointers):
+ *   row_of[T*K]   e * num_max_tokens + slot, or -1 (masked, skipped or dropped)
+ *   src_of[E*num_max_tokens]   t*K + k for slots [0, recv_expert_count[e]); other slots unwritten
+ */
+typedef struct ep_ll_handle {
+    int32_t* row_of;
+    int32_t* src_of;
+} ep_ll_handle;
+
+/* Version of this ABI (incremented on any signature change). */
+EP_API int32_t ep_abi_version(void);
+
+/* Human-readable name of an ep_status value. */
+EP_API const char* ep_status_string(int32_t status);
+
+/* Bytes of device workspace the calls need for a batch of num_tokens tokens
+ * (status word, scan counters, per-chunk expert counts).  The same workspace
+ * serves every entry point for batches up to that size. */
+EP_API size_t ep_workspace_bytes(int64_t num_tokens, int32_t num_experts, int32_t num_partitions);
+
+/* Zero a workspace (once, after allocating it) on `stream`. */
+EP_API ep_status ep_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, return the sticky device status bits in *bits_out and
+ * clear them.  The only call that blocks the host. */
+EP_API ep_status ep_read_status(void* workspace, size_t workspace_bytes, void* stream, uint32_t* bits_out);
+
+/*
+ * Routing layout of topk_idx[T*K] (device, int64) into *layout (all seven
+ * arrays written).  Per-expert counts, per-partition distinct-token counts and
+ * flags, expert offsets, and the stable row of every (t, k).  An id outside
+ * [-1, E) is treated as masked and sets EP_DEV_INDEX_RANGE.
+ */
+EP_API ep_status ep_get_dispatch_layout(int64_t num_tokens, int32_t num_topk, int32_t num_experts,
+                                 int32_t num_partitions, const int64_t* topk_idx,
+                                 const ep_layout* layout, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/*
+ * Dispatch (deepseek.csdn.net/67bd3eb22e30c863900615cc, "使用示例":
+ * dispatch(x, topk_idx, topk_weights, num_experts) -> recv_x, recv_topk_idx,
+ * recv_topk_weights, handle, event).  Computes the layout into *handle, then
+ * writes token t to every row row_of[t, k]:
+ *   quant = EP_QUANT_FP8_E4M3_1X128: recv_x (uint8 [T*K, H]) gets E4M3 codes
+ *     q = e4m3_rne_satfinite(x / s) and recv_scales (fp32 [T*K, H/128]) gets
+ *     s = max(amax, 1e-4) / 448 of each 128-channel block (fp32 division);
+ *   quant = EP_QUANT_NONE: recv_x (BF16 [T*K, H]) gets the row bit for bit;
+ *     recv_scales may be NULL.
+ *   recv_topk_idx[row] = e - p*E/P (expert id local to its partition, int32),
+ *   recv_topk_weights[row] = topk_weights[t, k].
+ * Receive buffers are sized for the worst case (T*K rows) so no host sync is
+ * needed; the first *handle->num_recv rows are valid.
+ * x: BF16 [T, H]; topk_idx: int64 [T, K]; topk_weights: fp32 [T, K] (device).
+ */
+EP_API ep_status ep_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk, int32_t num_experts,
+                      int32_t num_partitions, int32_t quant, const void* x, const int64_t* topk_idx,
+                      const float* topk_weights, void* recv_x, float* recv_scales,
+                      int32_t* recv_topk_idx, float* recv_topk_weights, const ep_layout* handle,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Combine ("DeepSeek 开源周第二弹：DeepEP", "DeepEP 的常规内核和低延迟内核": BF16
+ * result merge; "deepseek-ai/DeepEP", "典型工作流程": combine reduces the
+ * expert outputs back).  For every token t and channel i:
+ *   acc = +0.0f; for k = 0..K-1 with row = handle->row_of[t, k] >= 0:
+ *       acc = fmaf(topk_weights[t, k], float(expert_out[row, i]), acc)
+ *   y[t, i] = bf16_round_to_nearest_even(acc)
+ * expert_out: BF16 [expert_out_rows, H]; a row >= expert_out_rows is skipped
+ * and sets EP_DEV_INDEX_RANGE.  y: BF16 [T, H].  Only handle->row_of is read.
+ */
+EP_API ep_status ep_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk, const void* expert_out,
+                     int64_t expert_out_rows, const ep_layout* handle, const float* topk_weights,
+                     void* y, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Low-latency dispatch (deepseek.csdn.net/67bd3eb22e30c863900615cc,
+ * "推理解码阶段的应用").  One fused kernel: layout, FP8 quantisation and
+ * scatter into the padded tensors
+ *   recv_x      uint8 [E, num_max_tokens, H]      (E4M3 codes)
+ *   recv_scales fp32  [E, num_max_tokens, H/128]
+ * Slot j of (t, k) inside expert e is its rank among e's rows in
+ * (token, k) order -- the same order as the normal layout, so slot j of
+ * expert e holds normal row expert_offset[e] + j.  recv_expert_count[E]
+ * (int32) = rows written per expert.  Requires T <= num_max_tokens; a row at
+ * slot >= num_max_tokens (possible only when a token names an expert twice)
+ * is dropped and sets EP_DEV_CAPACITY.  Unused slots are not written.
+ */
+EP_API ep_status ep_low_latency_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                  int32_t num_experts, int32_t num_max_tokens, const void* x,
+                                  const int64_t* topk_idx, void* recv_x, float* recv_scales,
+                                  int32_t* recv_expert_count, const ep_ll_handle* handle,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Low-latency combine: the combine reduce above over
+ * expert_out BF16 [E, num_max_tokens, H] addressed by handle->row_of.
+ */
+EP_API ep_status ep_low_latency_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                 int32_t num_experts, int32_t num_max_tokens,
+                                 const void* expert_out, const ep_ll_handle* handle,
+                                 const float* topk_weights, void* y, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
+ * Test hook for the bounded device waits: launches one tiny kernel that waits
+ * on a workspace flag nothing sets and on an mbarrier transaction nothing
+ * completes, each for at most timeout_ns; both give up, set EP_DEV_TIMEOUT and
+ * return, leaving the context usable.
+ */
+EP_API ep_status ep_debug_wait_probe(uint64_t timeout_ns, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_B200_H */

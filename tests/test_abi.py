@@ -1,0 +1,168 @@
+"""The C-ABI library without a GPU: it loads, it exports every entry point the
+header declares, and the host-side argument checks reject bad calls before
+anything touches CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ep_b200.h")
+
+
+@pytest.fixture(scope="module")
+def ep():
+    from combine_get_dispatch_05_b200 import build
+
+    build.build()
+    import combine_get_dispatch_05_b200 as m
+
+    return m
+
+
+def _declared():
+    text = open(HEADER).read()
+    return re.findall(r"^EP_API\s+[\w\s\*]+?\b(ep_\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_the_calls():
+    names = set(_declared())
+    for n in ("ep_get_dispatch_layout", "ep_dispatch", "ep_combine", "ep_low_latency_dispatch",
+              "ep_low_latency_combine"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(ep):
+    lib = ctypes.CDLL(ep.LIB_PATH)
+    declared = _declared()
+    assert declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(ep._lib.EXPORTED)
+
+
+def test_built_for_sm100a_only():
+    from combine_get_dispatch_05_b200 import build
+
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    assert "--use_fast_math" not in build.NVCC_FLAGS and "-prec-div=true" in build.NVCC_FLAGS
+
+
+def test_version_and_strings(ep):
+    assert ep.lib.ep_abi_version() == 1
+    assert ep.status_string(ep.EP_ERR_SHAPE) == "unsupported size"
+    assert ep.status_string(99) == "unknown status"
+
+
+def test_workspace_bytes(ep):
+    b = ep.ep_workspace_bytes(4096, 256, 8)
+    # header + one int per (expert or partition, 256-token chunk), chunk count padded to 4
+    assert b == ((256 + 4 * 16 * (256 + 8)) + 255) // 256 * 256
+    assert ep.ep_workspace_bytes(0, 256, 8) > 0
+    assert ep.ep_workspace_bytes(-1, 256, 8) == 0
+    assert ep.ep_workspace_bytes(10, 0, 1) == 0
+    assert ep.ep_workspace_bytes(32768, 288, 8) >= ep.ep_workspace_bytes(4096, 288, 8)
+
+
+class _Fake:
+    """Aligned non-null addresses: the checks below fail before any dereference."""
+    P = 0x100000
+
+
+def _layout_struct(ep, valid=True):
+    p = _Fake.P if valid else None
+    return ep._lib.ep_layout(p, p, p, p, p, p, p)
+
+
+def _dispatch(ep, T=16, H=256, K=4, E=8, P=2, quant=1, ws_bytes=1 << 20, **over):
+    f = _Fake.P
+    args = dict(T=T, H=H, K=K, E=E, P=P, quant=quant, x=f, idx=f, w=f, rx=f, rs=f, ri=f, rw=f,
+                lay=_layout_struct(ep), ws=f, ws_bytes=ws_bytes)
+    args.update(over)
+    lay = args["lay"]
+    return ep.lib.ep_dispatch(args["T"], args["H"], args["K"], args["E"], args["P"], args["quant"],
+                              args["x"], args["idx"], args["w"], args["rx"], args["rs"],
+                              args["ri"], args["rw"], ctypes.byref(lay) if lay is not None else None,
+                              args["ws"], args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(K=0), 2), (dict(K=33), 2), (dict(E=7, P=2), 2), (dict(P=65, E=65 * 2), 2),
+    (dict(E=4097, P=1), 2), (dict(T=-1), 2), (dict(H=200), 2), (dict(H=0), 2),
+    (dict(H=16512), 2), (dict(quant=1, H=136), 2), (dict(quant=5), 1), (dict(x=None), 1),
+    (dict(rs=None), 1), (dict(x=_Fake.P + 8), 1), (dict(rx=_Fake.P + 4), 1), (dict(rs=_Fake.P + 4), 1),
+    (dict(ws=None), 1), (dict(lay=None), 1), (dict(ws_bytes=64), 3),
+    (dict(T=1 << 28, K=8), 2),
+])
+def test_dispatch_host_checks(ep, over, status):
+    assert _dispatch(ep, **over) == status
+
+
+def test_dispatch_bf16_needs_no_scales_but_checks_hidden(ep):
+    # quant NONE accepts H % 8 == 0 and a NULL recv_scales; it then reaches CUDA,
+    # which on a machine without a GPU reports a runtime error, not a crash
+    import torch
+
+    st = _dispatch(ep, quant=0, H=136, rs=None)
+    if torch.cuda.is_available():
+        pytest.skip("only meaningful without a GPU")
+    assert st == ep.EP_ERR_CUDA
+    assert _dispatch(ep, quant=0, H=132) == ep.EP_ERR_SHAPE
+
+
+def test_layout_host_checks(ep):
+    f = _Fake.P
+    lay = _layout_struct(ep)
+    L = ep.lib
+    assert L.ep_get_dispatch_layout(4, 0, 8, 2, f, ctypes.byref(lay), f, 1 << 20, None) == 2
+    assert L.ep_get_dispatch_layout(4, 2, 8, 3, f, ctypes.byref(lay), f, 1 << 20, None) == 2
+    assert L.ep_get_dispatch_layout(4, 2, 8, 2, None, ctypes.byref(lay), f, 1 << 20, None) == 1
+    bad = ep._lib.ep_layout(f, f, f, f, None, f, f)
+    assert L.ep_get_dispatch_layout(4, 2, 8, 2, f, ctypes.byref(bad), f, 1 << 20, None) == 1
+    assert L.ep_get_dispatch_layout(4, 2, 8, 2, f, ctypes.byref(lay), f, 16, None) == 3
+
+
+def test_combine_host_checks(ep):
+    f = _Fake.P
+    lay = _layout_struct(ep)
+    L = ep.lib
+    assert L.ep_combine(4, 100, 2, f, 8, ctypes.byref(lay), f, f, f, 4096, None) == 2  # H % 8
+    assert L.ep_combine(4, 128, 0, f, 8, ctypes.byref(lay), f, f, f, 4096, None) == 2
+    assert L.ep_combine(4, 128, 2, f, -1, ctypes.byref(lay), f, f, f, 4096, None) == 2
+    assert L.ep_combine(4, 128, 2, f, 8, None, f, f, f, 4096, None) == 1
+    assert L.ep_combine(4, 128, 2, f, 8, ctypes.byref(lay), f, f + 2, f, 4096, None) == 1
+    assert L.ep_combine(4, 128, 2, f, 8, ctypes.byref(lay), None, f, f, 4096, None) == 1
+    assert L.ep_combine(4, 128, 2, f, 8, ctypes.byref(lay), f, f, f, 8, None) == 1
+    # an empty batch is a no-op that succeeds without touching the device
+    assert L.ep_combine(0, 128, 2, None, 0, ctypes.byref(lay), None, None, f, 4096, None) == 0
+
+
+def test_low_latency_host_checks(ep):
+    f = _Fake.P
+    h = ep._lib.ep_ll_handle(f, f)
+    L = ep.lib
+    ok = dict(T=8, H=256, K=4, E=16, cap=8)
+
+    def call(**o):
+        a = dict(ok)
+        a.update(o)
+        return L.ep_low_latency_dispatch(a["T"], a["H"], a["K"], a["E"], a["cap"], f, f, f, f, f,
+                                         ctypes.byref(h), f, 4096, None)
+
+    assert call(T=9) == 2            # more tokens than capacity
+    assert call(cap=0) == 2
+    assert call(H=136) == 2          # FP8 needs H % 128 == 0
+    assert call(K=33) == 2
+    assert call(E=1 << 20, cap=1 << 12) == 2
+    assert L.ep_low_latency_combine(8, 256, 4, 0, 8, f, ctypes.byref(h), f, f, f, 4096, None) == 2
+    assert L.ep_low_latency_combine(8, 256, 4, 16, 8, f, None, f, f, f, 4096, None) == 1
+
+
+def test_read_status_and_probe_argument_checks(ep):
+    L = ep.lib
+    bits = ctypes.c_uint32(0)
+    assert L.ep_read_status(None, 4096, None, ctypes.byref(bits)) == 1
+    assert L.ep_read_status(_Fake.P, 16, None, ctypes.byref(bits)) == 1
+    assert L.ep_debug_wait_probe(1000, None, 4096, None) == 1
+    assert L.ep_workspace_init(None, 4096, None) == 1

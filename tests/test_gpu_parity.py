@@ -1,0 +1,286 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bit-exact comparisons throughout: layout arrays, E4M3 payload bytes, fp32
+scale bits, BF16 copies, and combine outputs (the kernel keeps the oracle's
+fixed k-order fmaf chain).  Sizes span several layout chunks (256 tokens) and
+ragged tails; edge cases cover empty batches, single tokens, all-masked
+tokens, duplicate experts, out-of-range ids, K = 1 / 32, E = 1 and the scale
+paths with H/128 blocks not a multiple of 4.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import oracle  # noqa: E402
+from workloads import make_custom, make_workload, random_bf16  # noqa: E402
+
+from gpu_path import (bf16_to_u16, gpu_combine, gpu_dispatch, gpu_layout,  # noqa: E402
+                      layout_numpy, new_workspace, torch_identity_expert)
+
+
+@pytest.fixture(scope="module")
+def ep():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import combine_get_dispatch_05_b200 as m
+    return m
+
+
+LAYOUT_KEYS = ("num_tokens_per_expert", "num_tokens_per_partition", "is_token_in_partition",
+               "expert_offset", "row_of", "src_of", "num_recv")
+
+
+def _assert_layout(got, want):
+    for k in LAYOUT_KEYS:
+        assert np.array_equal(got[k], want[k]), k
+
+
+def _cases():
+    yield "normal-300", make_workload("normal", seed=1, num_tokens=300, hidden=512)
+    yield "skew-700", make_workload("skew", seed=2, num_tokens=700, hidden=256)
+    yield "ll-128", make_workload("ll", seed=3, hidden=384)
+    yield "bf16-600", make_workload("bf16", seed=4, num_tokens=600, hidden=136)
+    yield "stress-1000", make_workload("stress", seed=5, num_tokens=1000, hidden=128)
+    yield "t1", make_custom(1, 128, 8, 256, 8, seed=6)
+    yield "k1", make_custom(257, 256, 1, 16, 4, seed=7)
+    yield "k32-dups", make_custom(70, 128, 32, 48, 6, seed=8, duplicates=True)
+    yield "e1", make_custom(33, 128, 2, 1, 1, seed=9, duplicates=True)
+    yield "masked", make_custom(513, 640, 6, 64, 16, seed=10, mask_frac=0.3)
+    yield "hot", make_custom(800, 128, 4, 32, 8, seed=11, hot_expert=5)
+    yield "e4096", make_custom(300, 128, 8, 4096, 64, seed=12)
+
+
+CASES = list(_cases())
+
+
+@pytest.mark.parametrize("name,w", CASES, ids=[c[0] for c in CASES])
+def test_layout_parity(ep, name, w):
+    lay, ws = gpu_layout(ep, w.topk_idx, w.num_experts, w.num_partitions)
+    got = layout_numpy(lay, w.num_tokens, w.num_topk)
+    want = oracle.layout(w.topk_idx, w.num_experts, w.num_partitions)
+    _assert_layout(got, want)
+    assert ep.ep_read_status(ws) == 0
+
+
+@pytest.mark.parametrize("name,w", CASES, ids=[c[0] for c in CASES])
+def test_dispatch_parity(ep, name, w):
+    quant = w.quant if w.hidden % 128 == 0 else "none"
+    got, _ = gpu_dispatch(ep, w, quant=quant)
+    want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, w.num_experts, w.num_partitions,
+                           quant=quant)
+    _assert_layout(got, want)
+    assert np.array_equal(got["recv_x"], want["recv_x"])
+    if quant == "fp8":
+        assert np.array_equal(got["recv_scales"].view(np.uint32),
+                              want["recv_scales"].view(np.uint32))
+    assert np.array_equal(got["recv_topk_idx"], want["recv_topk_idx"])
+    assert np.array_equal(got["recv_topk_weights"].view(np.uint32),
+                          want["recv_topk_weights"].view(np.uint32))
+    assert got["canaries_ok"]
+
+
+@pytest.mark.parametrize("name,w", CASES, ids=[c[0] for c in CASES])
+def test_combine_parity_random_expert_out(ep, name, w):
+    rng = np.random.default_rng(100)
+    lay, ws = gpu_layout(ep, w.topk_idx, w.num_experts, w.num_partitions)
+    want_lay = oracle.layout(w.topk_idx, w.num_experts, w.num_partitions)
+    R = int(want_lay["num_recv"][0])
+    H = w.hidden if w.hidden % 8 == 0 else 128
+    eo = random_bf16(rng, (R, H), scale=3.0)
+    y, canary = gpu_combine(ep, eo, lay, w.topk_weights, ws)
+    y_ref, st = oracle.combine(eo, want_lay["row_of"], w.topk_weights)
+    assert st == 0 and canary
+    assert np.array_equal(y, y_ref)
+
+
+@pytest.mark.parametrize("name", ["normal", "skew", "bf16"])
+def test_chain_dispatch_identity_combine(ep, name):
+    w = make_workload(name, seed=21, num_tokens=520, hidden=1024 if name != "bf16" else 264)
+    got, st = gpu_dispatch(ep, w)
+    if w.quant == "fp8":
+        eo = torch_identity_expert(st["recv_x"], st["recv_s"])
+    else:
+        eo = st["recv_x"]
+    y = torch.empty((w.num_tokens, w.hidden), dtype=torch.bfloat16, device="cuda")
+    ep.ep_combine(eo, st["layout"], st["wts"], y, st["ws"])
+    want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, w.num_experts, w.num_partitions,
+                           quant=w.quant)
+    eo_ref = oracle.identity_expert(want["recv_x"], want.get("recv_scales"), quant=w.quant)
+    y_ref, _ = oracle.combine(eo_ref, want["row_of"], w.topk_weights)
+    assert np.array_equal(bf16_to_u16(y), y_ref)
+
+
+def test_dispatch_is_deterministic(ep):
+    w = make_workload("skew", seed=3, num_tokens=1500, hidden=512)
+    a, _ = gpu_dispatch(ep, w)
+    b, _ = gpu_dispatch(ep, w)
+    for k in ("row_of", "src_of", "recv_x", "recv_scales"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_empty_batch(ep):
+    w = make_custom(0, 128, 8, 32, 4)
+    got, st = gpu_dispatch(ep, w)
+    assert got["num_recv"][0] == 0
+    assert np.all(got["expert_offset"] == 0) and np.all(got["num_tokens_per_expert"] == 0)
+    y = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    ep.ep_combine(torch.empty((0, 128), dtype=torch.bfloat16, device="cuda"), st["layout"],
+                  st["wts"], y, st["ws"])
+
+
+def test_workspace_reuse_across_batch_sizes(ep):
+    # one workspace sized for the largest batch serves smaller, ragged ones
+    ws = new_workspace(ep, 2000, 256, 8)
+    for T in (2000, 1999, 257, 3, 1024):
+        w = make_workload("normal", seed=T, num_tokens=T, hidden=128)
+        got, _ = gpu_dispatch(ep, w, workspace=ws)
+        want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, 256, 8)
+        _assert_layout(got, want)
+        assert np.array_equal(got["recv_x"], want["recv_x"])
+
+
+def test_out_of_range_ids_are_skipped_and_reported(ep):
+    w = make_custom(300, 256, 4, 16, 4, seed=13)
+    w.topk_idx[5, 1] = 16
+    w.topk_idx[77, 3] = -9
+    w.topk_idx[299, 0] = 1 << 40
+    got, st = gpu_dispatch(ep, w)
+    want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, 16, 4)
+    assert want["status"] & oracle.INDEX_RANGE
+    _assert_layout(got, want)
+    assert np.array_equal(got["recv_x"], want["recv_x"])
+    assert ep.ep_read_status(st["ws"]) & ep.EP_DEV_INDEX_RANGE
+    assert ep.ep_read_status(st["ws"]) == 0  # read clears
+
+
+def test_combine_row_outside_buffer_is_reported(ep):
+    rng = np.random.default_rng(1)
+    T, K, H = 40, 3, 256
+    eo = random_bf16(rng, (10, H))
+    lay = ep.Layout.empty(T, K, 4, 1, "cuda")
+    row_of = rng.integers(-1, 10, size=(T, K)).astype(np.int32)
+    row_of[7, 2] = 10  # one past the end
+    lay.row_of.copy_(torch.from_numpy(row_of))
+    w = rng.standard_normal((T, K)).astype(np.float32)
+    ws = new_workspace(ep, T, 4, 1)
+    y, ok = gpu_combine(ep, eo, lay, w, ws)
+    y_ref, st = oracle.combine(eo, row_of, w)
+    assert st & oracle.INDEX_RANGE and ok
+    assert np.array_equal(y, y_ref)
+    assert ep.ep_read_status(ws) & ep.EP_DEV_INDEX_RANGE
+
+
+# ---------------------------------------------------------------- low latency --
+
+def _ll_gpu(ep, w, cap):
+    T, H, K, E = w.num_tokens, w.hidden, w.num_topk, w.num_experts
+    x = torch.from_numpy(w.x.view(np.int16)).cuda().view(torch.bfloat16)
+    idx = torch.from_numpy(w.topk_idx).cuda()
+    recv_x = torch.full((E, cap, H), 0xA5, dtype=torch.uint8, device="cuda")
+    recv_s = torch.full((E, cap, H // 128), -1.0, dtype=torch.float32, device="cuda")
+    count = torch.empty(E, dtype=torch.int32, device="cuda")
+    h = ep.LowLatencyHandle.empty(T, K, E, cap, "cuda")
+    h.src_of.fill_(-1)
+    ws = new_workspace(ep, 1, E, 1)
+    ep.ep_low_latency_dispatch(x, idx, cap, E, recv_x, recv_s, count, h, ws)
+    torch.cuda.synchronize()
+    return dict(recv_x=recv_x.cpu().numpy(), recv_scales=recv_s.cpu().numpy(),
+                recv_expert_count=count.cpu().numpy(), ll_row_of=h.row_of.cpu().numpy(),
+                ll_src_of=h.src_of.cpu().numpy()), (h, ws, recv_x, recv_s)
+
+
+LL_CASES = [
+    ("ll", make_workload("ll", seed=0, hidden=512), 128),
+    ("ll-7168", make_workload("ll", seed=1, num_tokens=40), 128),
+    ("ll-h384", make_workload("ll", seed=2, num_tokens=97, hidden=384), 100),
+    ("ll-masked", make_custom(64, 256, 6, 32, 1, seed=3, mask_frac=0.2), 64),
+    ("ll-dups-overflow", make_custom(20, 128, 4, 3, 1, seed=4, duplicates=True), 20),
+    ("ll-t1", make_custom(1, 128, 8, 256, 1, seed=5), 128),
+]
+
+
+@pytest.mark.parametrize("name,w,cap", LL_CASES, ids=[c[0] for c in LL_CASES])
+def test_ll_dispatch_parity(ep, name, w, cap):
+    got, (h, ws, _, _) = _ll_gpu(ep, w, cap)
+    want = oracle.ll_dispatch(w.x, w.topk_idx, w.num_experts, cap, fill=0xA5)
+    assert np.array_equal(got["recv_expert_count"], want["recv_expert_count"])
+    assert np.array_equal(got["ll_row_of"], want["ll_row_of"])
+    # the whole padded tensor: written slots bit-exact, unwritten slots untouched
+    assert np.array_equal(got["recv_x"], want["recv_x"])
+    assert np.array_equal(got["recv_scales"].view(np.uint32), want["recv_scales"].view(np.uint32))
+    assert np.array_equal(got["ll_src_of"], want["ll_src_of"])
+    bits = ep.ep_read_status(ws)
+    assert bool(bits & ep.EP_DEV_CAPACITY) == bool(want["status"] & oracle.CAPACITY)
+
+
+@pytest.mark.parametrize("name,w,cap", LL_CASES, ids=[c[0] for c in LL_CASES])
+def test_ll_combine_parity(ep, name, w, cap):
+    got, (h, ws, _, _) = _ll_gpu(ep, w, cap)
+    rng = np.random.default_rng(9)
+    eo = random_bf16(rng, (w.num_experts, cap, w.hidden))
+    y = torch.empty((w.num_tokens, w.hidden), dtype=torch.bfloat16, device="cuda")
+    eo_d = torch.from_numpy(eo.view(np.int16)).cuda().view(torch.bfloat16)
+    wts = torch.from_numpy(w.topk_weights).cuda()
+    ep.ep_low_latency_combine(eo_d, h, wts, y, ws)
+    want = oracle.ll_dispatch(w.x, w.topk_idx, w.num_experts, cap)
+    y_ref, _ = oracle.ll_combine(eo, want["ll_row_of"], w.topk_weights)
+    assert np.array_equal(bf16_to_u16(y), y_ref)
+
+
+def test_ll_equals_normal(ep):
+    w = make_workload("ll", seed=7, hidden=1024)
+    cap = w.num_max_tokens
+    ll, (h, ws, recv_q, recv_s) = _ll_gpu(ep, w, cap)
+    nd, st = gpu_dispatch(ep, w)
+    off = nd["expert_offset"]
+    for e in range(w.num_experts):
+        n = ll["recv_expert_count"][e]
+        assert np.array_equal(ll["recv_x"][e, :n], nd["recv_x"][off[e]:off[e] + n])
+    # LL combine == normal combine on identity experts, bit for bit
+    y_n = torch.empty((w.num_tokens, w.hidden), dtype=torch.bfloat16, device="cuda")
+    ep.ep_combine(torch_identity_expert(st["recv_x"], st["recv_s"]), st["layout"], st["wts"], y_n,
+                  st["ws"])
+    y_l = torch.empty_like(y_n)
+    ep.ep_low_latency_combine(torch_identity_expert(recv_q, recv_s), h, st["wts"], y_l, ws)
+    assert torch.equal(y_n.view(torch.int16), y_l.view(torch.int16))
+
+
+# ----------------------------------------------------- status / bounded waits --
+
+def test_bounded_wait_gives_up_and_context_survives(ep):
+    ws = new_workspace(ep, 1, 1, 1)
+    ep.ep_debug_wait_probe(2_000_000, ws)  # 2 ms
+    assert ep.ep_read_status(ws) & ep.EP_DEV_TIMEOUT
+    # the context is still usable
+    w = make_custom(50, 128, 2, 8, 2, seed=1)
+    got, _ = gpu_dispatch(ep, w)
+    want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, 8, 2)
+    assert np.array_equal(got["recv_x"], want["recv_x"])
+
+
+# ------------------------------------------------------------------ Buffer API --
+
+def test_buffer_api_matches_pages_call_shapes(ep):
+    w = make_workload("normal", seed=2, num_tokens=333, hidden=256)
+    buf = ep.Buffer(num_experts=256, num_partitions=8, max_tokens=512)
+    x = torch.from_numpy(w.x.view(np.int16)).cuda().view(torch.bfloat16)
+    idx = torch.from_numpy(w.topk_idx).cuda()
+    wts = torch.from_numpy(w.topk_weights).cuda()
+    recv_x, recv_topk_idx, recv_topk_weights, handle, event = buf.dispatch(x, idx, wts, 256)
+    event.synchronize()
+    want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, 256, 8)
+    q, s = recv_x
+    assert q.dtype == torch.float8_e4m3fn and q.shape[0] == int(want["num_recv"][0])
+    assert np.array_equal(q.view(torch.uint8).cpu().numpy(), want["recv_x"])
+    assert np.array_equal(recv_topk_idx.cpu().numpy(), want["recv_topk_idx"])
+    y, ev = buf.combine(torch_identity_expert(q, s), handle, wts)
+    eo_ref = oracle.identity_expert(want["recv_x"], want["recv_scales"])
+    y_ref, _ = oracle.combine(eo_ref, want["row_of"], w.topk_weights)
+    assert np.array_equal(bf16_to_u16(y), y_ref)
+    (rq, rs), cnt, lh, ev, hook = buf.low_latency_dispatch(x[:128], idx[:128], 128, 256)
+    hook()
+    assert np.array_equal(cnt.cpu().numpy(),
+                          oracle.layout(w.topk_idx[:128], 256, 8)["num_tokens_per_expert"])
+    assert buf.read_status() == 0
