@@ -47,7 +47,7 @@ class ep_ll_handle(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m combine_get_dispatch_05_b200.build`")
+            f"{LIB_PATH} is missing: build it with `python combine_get_dispatch_05_b200/build.py`")
     L = ctypes.CDLL(LIB_PATH)
     i64, i32, sz, vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t, ctypes.c_void_p
     st = ctypes.c_int32

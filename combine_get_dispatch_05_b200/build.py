@@ -1,6 +1,8 @@
 """Build ``libep_b200.so`` (the C-ABI CUDA library) in-tree for sm_100a.
 
-    python -m combine_get_dispatch_05_b200.build [--force] [--verbose]
+    python combine_get_dispatch_05_b200/build.py [--force] [--verbose]
+
+(run as a script: importing the package would load the library it builds)
 
 nvcc cross-compiles for sm_100a without a GPU.  Flags: IEEE division and
 square root (no --use_fast_math), -O3, line info for profilers, the CUDA

@@ -13,9 +13,9 @@ HEADER = os.path.join(ROOT, "include", "ep_b200.h")
 
 @pytest.fixture(scope="module")
 def ep():
-    from combine_get_dispatch_05_b200 import build
+    import __graft_entry__
 
-    build.build()
+    __graft_entry__.build()
     import combine_get_dispatch_05_b200 as m
 
     return m
@@ -43,7 +43,9 @@ def test_library_exports_every_declared_symbol(ep):
 
 
 def test_built_for_sm100a_only():
-    from combine_get_dispatch_05_b200 import build
+    import __graft_entry__
+
+    build = __graft_entry__._load_by_path("_ep_build_check", "combine_get_dispatch_05_b200/build.py")
 
     assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
     assert "--use_fast_math" not in build.NVCC_FLAGS and "-prec-div=true" in build.NVCC_FLAGS
