@@ -25,6 +25,7 @@ EXPORTED = (
     "ep_abi_version", "ep_status_string", "ep_workspace_bytes", "ep_workspace_init",
     "ep_read_status", "ep_get_dispatch_layout", "ep_dispatch", "ep_combine",
     "ep_low_latency_dispatch", "ep_low_latency_combine", "ep_debug_wait_probe",
+    "ep_get_dispatch_layout_static",
 )
 
 
@@ -72,6 +73,9 @@ def _load() -> ctypes.CDLL:
                                          ctypes.POINTER(ep_ll_handle), vp, vp, vp, sz, vp]
     L.ep_low_latency_combine.restype = st
     L.ep_debug_wait_probe.argtypes, L.ep_debug_wait_probe.restype = [ctypes.c_uint64, vp, sz, vp], st
+    L.ep_get_dispatch_layout_static.argtypes = [i64, i32, i32, i32, vp,
+                                                ctypes.POINTER(ep_layout), vp]
+    L.ep_get_dispatch_layout_static.restype = st
     return L
 
 

@@ -154,6 +154,36 @@ EP_API ep_status ep_get_dispatch_layout(int64_t num_tokens, int32_t num_topk, in
                                  const ep_layout* layout, void* workspace, size_t workspace_bytes,
                                  void* stream);
 
+/* Size of the scratch array compiled into the library for
+ * ep_get_dispatch_layout_static (per GPU, held until the process exits). */
+#define EP_STATIC_SCRATCH_BYTES (1u << 20)
+
+/*
+ * ep_get_dispatch_layout without a workspace.  The DeepEP pages have no
+ * counterpart: this entry point exists for callers that cannot allocate device
+ * memory where they call the layout -- an engine that gives all of HBM to its
+ * own pool at start-up, a plugin whose enqueue step must not allocate, or a
+ * latency-critical path where cudaMalloc's implicit synchronisation would stall
+ * other streams.  It computes exactly what ep_get_dispatch_layout computes, with
+ * its scratch in a fixed EP_STATIC_SCRATCH_BYTES array inside the library.
+ *   - Allocates nothing (no cudaMalloc / cudaFree / allocating library call).
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Returns EP_ERR_WORKSPACE when the batch needs more scratch than the
+ *     array holds, i.e. ep_workspace_bytes(T, E, P) > EP_STATIC_SCRATCH_BYTES
+ *     (about 250k tokens at E = 256, P = 8).
+ *   - Every call shares the one array and it keeps the last call's contents:
+ *     each call clears the part that must start at zero, and calls that overlap
+ *     on the GPU (other streams or host threads on the same device) race.
+ *   - Ids outside [-1, E) are skipped as masked; this variant has no status word
+ *     the caller can read, so they are not reported.
+ */
+EP_API ep_status ep_get_dispatch_layout_static(int64_t num_tokens, int32_t num_topk,
+                                               int32_t num_experts, int32_t num_partitions,
+                                               const int64_t* topk_idx, const ep_layout* layout,
+                                               void* stream);
+
 /*
  * Dispatch (deepseek.csdn.net/67bd3eb22e30c863900615cc, "使用示例":
  * dispatch(x, topk_idx, topk_weights, num_experts) -> recv_x, recv_topk_idx,
