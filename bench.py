@@ -13,8 +13,11 @@ dispatched rows dequantised, i.e. identity experts).
 Prints ONE JSON line (rank 0).  `value` is algorithmic HBM GB/s of the whole
 step (bytes the method must move / device time, summed over ranks' batches,
 max time over ranks).  Each step is captured as two CUDA graphs (dispatch,
-combine) and timed with CUDA events on the launching stream; L2 (126 MB) is
-flushed by a 256 MiB write before every timed step, outside the events.
+combine) and timed with CUDA events on the launching stream.  Steps run back
+to back: every step reads 529 MB of inputs (x and the expert outputs) and
+writes 294 MB, several times the 126 MB L2, so nothing a step reads is still in
+L2 from the step before.  `--l2-flush write|read` instead flushes L2 with a
+256 MiB buffer before every step (outside the events).
 `--impl reference` times the CPU oracle on a bounded sample instead.
 """
 from __future__ import annotations
@@ -250,18 +253,21 @@ class PathRunner:
         else:
             self.combine()
 
-    def time_steps(self, steps, warmup, flush):
-        """Per-step (dispatch ms, combine ms) with an L2 flush before each step."""
+    def time_steps(self, steps, warmup, flush=None):
+        """Per-step (dispatch ms, combine ms); `flush` (if given) runs before each step,
+        outside the events."""
         import torch
 
         for _ in range(warmup):
-            flush.zero_()
+            if flush is not None:
+                flush()
             self.run_dispatch()
             self.run_combine()
         torch.cuda.synchronize()
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
         for i in range(steps):
-            flush.zero_()
+            if flush is not None:
+                flush()
             evs[i][0].record()
             self.run_dispatch()
             evs[i][1].record()
@@ -393,6 +399,29 @@ def cpu_baseline(w, min_seconds=10.0):
                       f"{t:.1f} s, single-threaded C"}
 
 
+def make_flush(mode, dev):
+    """L2 flush before a step: write (zero) or read (sum) a 256 MiB buffer."""
+    import torch
+
+    if mode == "none":
+        return None
+    buf = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    if mode == "write":
+        return lambda: buf.zero_()
+    return lambda: buf.sum()
+
+
+def reduce_max_over_ranks(values, world, device):
+    """Element-wise max of per-rank float values across the process group."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -412,7 +441,7 @@ def run_ours(args):
     sampler.start()
     w = make_workload("normal", seed=args.seed + rank)
     runner = PathRunner(ep, w, dev, use_graphs=not args.eager)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = make_flush(args.l2_flush, dev)
 
     if world > 1:
         dist.barrier()
@@ -426,11 +455,8 @@ def run_ours(args):
     sampler.mark(t0, t1)
     status = ep.ep_read_status(runner.ws)
 
-    total_ms = sum(d_ms) + sum(c_ms)
-    tot = torch.tensor([total_ms, sum(c_ms), sum(d_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
-    total_ms = float(tot[0])
+    tot = reduce_max_over_ranks([sum(d_ms) + sum(c_ms), sum(c_ms), sum(d_ms)], world, dev)
+    total_ms = tot[0]
     ms_step = total_ms / args.steps
     step_bytes = runner.bytes_dispatch + runner.bytes_combine
     value = world * step_bytes / (ms_step * 1e-3) / 1e9
@@ -450,8 +476,8 @@ def run_ours(args):
         return
 
     peak, peak_kind = measured_peaks()
-    comb_us = float(tot[1]) / args.steps * 1e3
-    disp_us = float(tot[2]) / args.steps * 1e3
+    comb_us = tot[1] / args.steps * 1e3
+    disp_us = tot[2] / args.steps * 1e3
     comb_gbs = runner.bytes_combine / (comb_us * 1e-6) / 1e9
     disp_gbs = runner.bytes_dispatch / (disp_us * 1e-6) / 1e9
     result = {
@@ -474,15 +500,17 @@ def run_ours(args):
             "tokens_per_gpu": w.num_tokens, "hidden": w.hidden, "topk": w.num_topk,
             "experts": w.num_experts, "partitions": w.num_partitions, "recv_rows": runner.R,
             "bytes_per_step": step_bytes, "seed": args.seed,
-            "l2": "flushed before every timed step (256 MiB write, outside the events)",
-            "launch": "CUDA graphs (dispatch: 3 kernels with programmatic dependent launch; "
+            "l2": ("inputs larger than L2: each step reads 529 MB (x + expert outputs) and "
+                   "writes 294 MB, steps back to back, no flush") if args.l2_flush == "none"
+            else f"flushed before every step by a 256 MiB {args.l2_flush} (outside the events)",
+            "launch": "CUDA graphs (dispatch: layout + dispatch kernels, programmatic dependent launch; "
                       "combine: 1 kernel)" if not args.eager else "eager",
             "parallelism": f"replicas x{world} (independent batches, no exchange)",
         },
         "breakdown": {
             "dispatch": {"us": round(disp_us, 2), "bytes": runner.bytes_dispatch,
                          "gbs": round(disp_gbs, 1), "frac": round(disp_gbs / peak, 4),
-                         "kernels": "layout_count + layout_rank + dispatch_fp8"},
+                         "kernels": "layout (cooperative) + dispatch_fp8 (programmatic dependent launch)"},
             "combine": {"us": round(comb_us, 2), "bytes": runner.bytes_combine,
                         "gbs": round(comb_gbs, 1), "frac": round(comb_gbs / peak, 4),
                         "kernels": "combine"},
@@ -494,7 +522,7 @@ def run_ours(args):
             "unit": "GB/s", "frac": round(comb_gbs / peak, 4),
             "traffic": profiled_traffic("combine_kernel_normal_4096x7168.md", COMBINE_SOURCES),
         },
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 3 * args.steps,
         "device_status": status,
         "clocks": clocks,
     }
@@ -601,6 +629,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--extra-steps", type=int, default=50)
     ap.add_argument("--eager", action="store_true", help="launch eagerly instead of CUDA graphs")
+    ap.add_argument("--l2-flush", choices=("none", "write", "read"), default="none")
     ap.add_argument("--no-extra", action="store_true", help="skip the ll/skew/bf16/stress configs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -24,8 +24,8 @@ namespace ep {
 
 namespace {
 
-constexpr int kFp8Stages = 3;     // input ring depth (tokens in flight per CTA)
-constexpr int kFp8OutStages = 2;  // output staging buffers
+constexpr int kFp8InStages = 3;   // input ring: rows in flight from HBM per CTA
+constexpr int kFp8OutStages = 3;  // quantised rows staged for the bulk stores
 constexpr int kBf16Stages = 4;
 
 struct Fp8Smem {
@@ -40,88 +40,154 @@ __host__ __device__ inline Fp8Smem fp8_smem(int64_t H) {
     s.q_bytes = static_cast<uint32_t>(H);
     s.s_bytes = (nb * 4u + 15u) & ~15u;
     s.out_bytes = s.q_bytes + s.s_bytes;
-    s.off_out = kFp8Stages * s.in_bytes;
+    s.off_out = kFp8InStages * s.in_bytes;
     s.off_bars = s.off_out + kFp8OutStages * s.out_bytes;
-    s.off_rows = s.off_bars + 8u * kFp8Stages;
+    s.off_rows = s.off_bars + 8u * 2u * (kFp8InStages + kFp8OutStages);
     s.off_flag = s.off_rows + 4u * 32u * kFp8OutStages;
     s.total = s.off_flag + 16u;
     return s;
 }
 
-__global__ void __launch_bounds__(256) dispatch_fp8_kernel(DispatchParams p) {
+// Wait for a phase, giving up after timeout_ns or as soon as another warp of the
+// CTA has given up (*abort_flag set).  On its own timeout it sets *abort_flag.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
+                                              volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > timeout_ns) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+// Warp-specialised pipeline, one CTA = 1 loader warp + nq quantiser warps + 1 storer
+// warp, coupled only by mbarriers (no CTA-wide barrier after set-up):
+//   loader (warp 0, lane 0): bulk-loads token rows into the input ring
+//       (in_full[s]: transaction bytes; waits in_empty[s] before reusing a stage);
+//   quantisers (warps 1..nq): quantise their share of the row's 128-channel blocks
+//       from input stage s into output stage o, then arrive on in_empty[s] and
+//       out_full[o] (waiting out_empty[o] before reusing an output stage);
+//   storer (last warp): lane k bulk-stores the staged row and its scales to row
+//       row_of[t, k], writes recv_topk_idx / recv_topk_weights, and releases the
+//       output stage (out_empty) once its stores have read it.
+// Only the storer reads what the layout kernel wrote, so only it waits on the
+// programmatic dependency; loads and quantisation overlap the layout.
+__global__ void __launch_bounds__(352) dispatch_fp8_kernel(DispatchParams p) {
     extern __shared__ __align__(128) uint8_t sm[];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nq = (blockDim.x >> 5) - 2;
     const int64_t T = p.T, H = p.H;
     const int K = p.K, nb = static_cast<int>(H >> 7);
     const Fp8Smem L = fp8_smem(H);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.off_bars);
+    uint64_t* in_full = reinterpret_cast<uint64_t*>(sm + L.off_bars);
+    uint64_t* in_empty = in_full + kFp8InStages;
+    uint64_t* out_full = in_empty + kFp8InStages;
+    uint64_t* out_empty = out_full + kFp8OutStages;
     int* rows_sm = reinterpret_cast<int*>(sm + L.off_rows);
     volatile int* abort_flag = reinterpret_cast<int*>(sm + L.off_flag);
     const bool scale_bulk = (static_cast<uint32_t>(nb) * 4u) == L.s_bytes;
-    const uint8_t* x = static_cast<const uint8_t*>(p.x);
-    uint8_t* recv_x = static_cast<uint8_t*>(p.recv_x);
 
     const int64_t G = gridDim.x, first = blockIdx.x;
     const int64_t n_mine = first < T ? (T - 1 - first) / G + 1 : 0;
 
     if (tid == 0) {
-        for (int s = 0; s < kFp8Stages; ++s) mbar_init(&bars[s], 1);
+        for (int s = 0; s < kFp8InStages; ++s) {
+            mbar_init(&in_full[s], 1);
+            mbar_init(&in_empty[s], nq);
+        }
+        for (int o = 0; o < kFp8OutStages; ++o) {
+            mbar_init(&out_full[o], nq);
+            mbar_init(&out_empty[o], 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
-    int64_t issued = 0;  // loads issued (meaningful in thread 0)
-    if (tid == 0) {
-        for (; issued < kFp8Stages && issued < n_mine; ++issued) {
-            const int64_t t = first + issued * G;
-            mbar_arrive_expect_tx(&bars[issued], L.in_bytes);
-            bulk_load(sm + issued * L.in_bytes, x + t * H * 2, L.in_bytes, &bars[issued]);
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- loader
+        if (lane == 0) {
+            const uint8_t* x = static_cast<const uint8_t*>(p.x);
+            int64_t issued = 0;
+            for (; issued < n_mine; ++issued) {
+                const int s = static_cast<int>(issued % kFp8InStages);
+                if (issued >= kFp8InStages &&
+                    !wait_or_abort(&in_empty[s],
+                                   static_cast<uint32_t>((issued / kFp8InStages - 1) & 1),
+                                   p.timeout_ns, abort_flag))
+                    break;
+                const int64_t t = first + issued * G;
+                mbar_arrive_expect_tx(&in_full[s], L.in_bytes);
+                bulk_load(sm + s * L.in_bytes, x + t * H * 2, L.in_bytes, &in_full[s]);
+            }
+            if (*abort_flag) {
+                // let this CTA's loads still in flight land before it exits: the
+                // latest load of each stage is its barrier's current phase
+                for (int64_t j = issued - 1; j >= 0 && j >= issued - kFp8InStages; --j)
+                    mbar_wait_bounded(&in_full[j % kFp8InStages],
+                                      static_cast<uint32_t>((j / kFp8InStages) & 1),
+                                      kDefaultTimeoutNs);
+            }
         }
-    }
-
-    pdl_wait();  // row_of from the layout kernels is complete and visible
-
-    // warp 0, lane k < K: (row, expert, weight) of slot k, prefetched one token ahead
-    int nrow = -1;
-    int64_t nexp = -1;
-    float nwt = 0.0f;
-    const bool slot_lane = (warp == 0) && (lane < K);
-    if (slot_lane && n_mine > 0) {
-        const int64_t g = first * K + lane;
-        nrow = p.row_of[g];
-        nexp = p.topk_idx[g];
-        nwt = p.topk_weights[g];
-    }
-
-    int64_t i = 0;
-    for (; i < n_mine; ++i) {
-        const int64_t t = first + i * G;
-        const int s = static_cast<int>(i % kFp8Stages);
-        const uint32_t par = static_cast<uint32_t>((i / kFp8Stages) & 1);
-        const int o = static_cast<int>(i % kFp8OutStages);
-        uint8_t* out_q = sm + L.off_out + o * L.out_bytes;
-        float* out_s = reinterpret_cast<float*>(out_q + L.q_bytes);
-        const int row = nrow;
-        const int64_t e = nexp;
-        const float wt = nwt;
-        if (slot_lane) {
-            rows_sm[o * 32 + lane] = row;
-            if (i + 1 < n_mine) {
+    } else if (warp <= nq) {
+        // ------------------------------------------------------------ quantisers
+        const int qw = warp - 1;
+        for (int64_t i = 0; i < n_mine; ++i) {
+            const int s = static_cast<int>(i % kFp8InStages);
+            const int o = static_cast<int>(i % kFp8OutStages);
+            if (!wait_or_abort(&in_full[s], static_cast<uint32_t>((i / kFp8InStages) & 1),
+                               p.timeout_ns, abort_flag))
+                break;
+            if (i >= kFp8OutStages &&
+                !wait_or_abort(&out_empty[o], static_cast<uint32_t>((i / kFp8OutStages - 1) & 1),
+                               p.timeout_ns, abort_flag))
+                break;
+            uint8_t* out_q = sm + L.off_out + o * L.out_bytes;
+            quantize_row_fp8(sm + s * L.in_bytes, out_q, reinterpret_cast<float*>(out_q + L.q_bytes),
+                             nb, qw, nq, lane);
+            fence_proxy_async_smem();  // staged row visible to the bulk stores
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&in_empty[s]);
+                mbar_arrive(&out_full[o]);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- storer
+        pdl_wait();  // row_of from the layout kernel is complete and visible
+        uint8_t* recv_x = static_cast<uint8_t*>(p.recv_x);
+        const bool slot_lane = lane < K;
+        int nrow = -1;
+        int64_t nexp = -1;
+        float nwt = 0.0f;
+        if (slot_lane && n_mine > 0) {
+            const int64_t g = first * K + lane;
+            nrow = p.row_of[g];
+            nexp = p.topk_idx[g];
+            nwt = p.topk_weights[g];
+        }
+        for (int64_t i = 0; i < n_mine; ++i) {
+            const int64_t t = first + i * G;
+            const int o = static_cast<int>(i % kFp8OutStages);
+            const int row = nrow;
+            const int64_t e = nexp;
+            const float wt = nwt;
+            if (slot_lane && i + 1 < n_mine) {
                 const int64_t g = (t + G) * K + lane;
                 nrow = p.row_of[g];
                 nexp = p.topk_idx[g];
                 nwt = p.topk_weights[g];
             }
-            bulk_wait_read<kFp8OutStages - 1>();  // out stage o is no longer being read
-        }
-        __syncthreads();
-        if (!mbar_wait_bounded(&bars[s], par, p.timeout_ns)) *abort_flag = 1;
-        quantize_row_fp8(sm + s * L.in_bytes, out_q, out_s, nb, warp, nwarps, lane);
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (*abort_flag) break;
-        if (warp == 0) {
-            if (lane < K) {
+            if (!wait_or_abort(&out_full[o], static_cast<uint32_t>((i / kFp8OutStages) & 1),
+                               p.timeout_ns, abort_flag))
+                break;
+            uint8_t* out_q = sm + L.off_out + o * L.out_bytes;
+            const float* out_s = reinterpret_cast<const float*>(out_q + L.q_bytes);
+            if (slot_lane) {
                 if (row >= 0) {
                     bulk_store(recv_x + static_cast<int64_t>(row) * H, out_q, L.q_bytes);
                     if (scale_bulk)
@@ -132,33 +198,24 @@ __global__ void __launch_bounds__(256) dispatch_fp8_kernel(DispatchParams p) {
                     p.recv_topk_weights[row] = wt;
                 }
                 bulk_commit();
+                rows_sm[o * 32 + lane] = row;
             }
+            if (!scale_bulk) {
+                __syncwarp();
+                for (int idx = lane; idx < K * nb; idx += 32) {
+                    const int k = idx / nb, b = idx - k * nb;
+                    const int r = rows_sm[o * 32 + k];
+                    if (r >= 0) p.recv_scales[static_cast<int64_t>(r) * nb + b] = out_s[b];
+                }
+            }
+            // release the previous output stage once this warp's stores have read it
+            if (slot_lane) bulk_wait_read<1>();
             __syncwarp();
-            // every thread is done reading input stage s: refill it
-            if (lane == 0 && issued < n_mine) {
-                const int64_t t2 = first + issued * G;
-                mbar_arrive_expect_tx(&bars[s], L.in_bytes);
-                bulk_load(sm + s * L.in_bytes, x + t2 * H * 2, L.in_bytes, &bars[s]);
-                ++issued;
-            }
+            if (lane == 0 && i >= 1) mbar_arrive(&out_empty[(i - 1) % kFp8OutStages]);
         }
-        if (!scale_bulk) {
-            for (int idx = tid; idx < K * nb; idx += blockDim.x) {
-                const int k = idx / nb, b = idx - k * nb;
-                const int r = rows_sm[o * 32 + k];
-                if (r >= 0) p.recv_scales[static_cast<int64_t>(r) * nb + b] = out_s[b];
-            }
-        }
+        if (slot_lane) bulk_wait_all<0>();
     }
-    if (i < n_mine && tid == 0) {
-        // a bounded wait gave up: report, then let the loads still in flight land
-        // before this CTA's shared memory goes away
-        raise_status(p.status, kDevTimeout);
-        for (int64_t j = i; j < issued; ++j)
-            mbar_wait_bounded(&bars[j % kFp8Stages],
-                              static_cast<uint32_t>((j / kFp8Stages) & 1), kDefaultTimeoutNs);
-    }
-    if (slot_lane) bulk_wait_all<0>();
+    if (tid == 0 && *abort_flag) raise_status(p.status, kDevTimeout);
 }
 
 __global__ void __launch_bounds__(32) dispatch_bf16_kernel(DispatchParams p) {
@@ -290,11 +347,11 @@ cudaError_t launch_dispatch_fp8(const DispatchParams& p, cudaStream_t stream) {
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(L.total));
     if (err != cudaSuccess) return err;
-    // warps: enough that every warp quantises the same number of block pairs
+    // quantiser warps: enough that each quantises the same number of block pairs
     const int pairs = static_cast<int>((p.H / 128 + 1) / 2);
     const int iters = (pairs + 7) / 8;
-    const int warps = (pairs + iters - 1) / iters;
-    const int threads = 32 * (warps > 0 ? warps : 1);
+    const int nq = (pairs + iters - 1) / iters;
+    const int threads = 32 * (nq + 2);
     const int grid = grid_for(kernel, threads, L.total, p.T, dev.num_sms);
     return launch_pdl(kernel, dim3(grid), dim3(threads), L.total, stream, p);
 }

@@ -91,7 +91,7 @@ const char* ep_status_string(int32_t status) {
 
 size_t ep_workspace_bytes(int64_t num_tokens, int32_t num_experts, int32_t num_partitions) {
     if (num_tokens < 0 || num_experts < 1 || num_partitions < 1) return 0;
-    const size_t body = sizeof(int32_t) * static_cast<size_t>(chunk_stride(num_tokens)) *
+    const size_t body = sizeof(int32_t) * static_cast<size_t>(max_layout_chunks(num_tokens)) *
                         (static_cast<size_t>(num_experts) + static_cast<size_t>(num_partitions));
     return (kWsHeader + body + 255) / 256 * 256;
 }
@@ -123,7 +123,8 @@ ep_status ep_get_dispatch_layout(int64_t num_tokens, int32_t num_topk, int32_t n
     ep_status st = check_routing(num_tokens, num_topk, num_experts, num_partitions);
     if (st != EP_OK) return st;
     if ((st = check_layout_ptrs(layout, num_tokens)) != EP_OK) return st;
-    if (!workspace || (num_tokens > 0 && !topk_idx)) return EP_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace) || (num_tokens > 0 && !topk_idx))
+        return EP_ERR_INVALID_ARG;
     if (workspace_bytes < ep_workspace_bytes(num_tokens, num_experts, num_partitions))
         return EP_ERR_WORKSPACE;
     const Workspace ws = carve_workspace(workspace, num_tokens, num_experts);
@@ -142,7 +143,7 @@ ep_status ep_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk, int3
     if (st != EP_OK) return st;
     if ((st = check_hidden(hidden, fp8)) != EP_OK) return st;
     if ((st = check_layout_ptrs(handle, num_tokens)) != EP_OK) return st;
-    if (!workspace) return EP_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace)) return EP_ERR_INVALID_ARG;
     if (num_tokens > 0) {
         if (!x || !topk_idx || !topk_weights || !recv_x || !recv_topk_idx || !recv_topk_weights)
             return EP_ERR_INVALID_ARG;

@@ -13,16 +13,11 @@ constexpr uint32_t kDevIndexRange = 0x1u;
 constexpr uint32_t kDevTimeout = 0x2u;
 constexpr uint32_t kDevCapacity = 0x4u;
 
-// Workspace header (bytes): status word, layout ticket, probe flag.
+// Workspace header (bytes): status word, probe flag, layout grid-barrier word.
 constexpr size_t kWsStatus = 0;
-constexpr size_t kWsTicket = 4;
-constexpr size_t kWsProbeFlag = 8;
+constexpr size_t kWsProbeFlag = 4;
+constexpr size_t kWsBar = 8;
 constexpr size_t kWsHeader = 256;
-
-// Tokens per layout chunk: one CTA of the count kernel and one CTA of the rank
-// kernel per chunk; each of the rank CTA's 8 warps ranks 32 of its tokens.
-constexpr int kChunkTokens = 256;
-constexpr int kRankWarps = kChunkTokens / 32;
 
 __device__ __forceinline__ void raise_status(uint32_t* status, uint32_t bits) {
     atomicOr(status, bits);
@@ -63,6 +58,10 @@ __device__ __forceinline__ void fence_mbar_init() {
 // Order this thread's generic-proxy shared-memory writes before later async-proxy reads.
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {

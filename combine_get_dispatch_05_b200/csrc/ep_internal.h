@@ -16,22 +16,21 @@ struct DeviceInfo {
 };
 cudaError_t device_info(DeviceInfo* out);
 
-// Number of layout chunks (kChunkTokens tokens each) and their padded stride.
-int64_t num_chunks(int64_t num_tokens);
-int64_t chunk_stride(int64_t num_tokens);
+// Upper bound on the layout kernel's CTAs (chunks) for a batch of num_tokens.
+int64_t max_layout_chunks(int64_t num_tokens);
 
 struct Workspace {
     uint32_t* status;
-    uint32_t* ticket;
     uint32_t* probe_flag;
-    int32_t* chunk_expert;     // [E][chunk_stride]
-    int32_t* chunk_partition;  // [P][chunk_stride]
+    unsigned long long* bar;
+    int32_t* chunk_expert;     // [chunks][E]
+    int32_t* chunk_partition;  // [chunks][P]
 };
 Workspace carve_workspace(void* ws, int64_t num_tokens, int32_t num_experts);
 
-// Launch the layout kernels (count + rank) on `stream`.  The first launch waits
-// for all earlier work in the stream; the rank launch is programmatically
-// dependent on the count launch.
+// Launch the (cooperative) layout kernel on `stream`.  It waits for all earlier
+// work in the stream and lets the next kernel start early (programmatic
+// dependent launch).
 cudaError_t launch_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int64_t* topk_idx,
                           const ep_layout& lay, const Workspace& ws, cudaStream_t stream);
 
@@ -51,7 +50,7 @@ struct DispatchParams {
     uint32_t* status;
     uint64_t timeout_ns;
 };
-// Launched programmatically dependent on the preceding (layout) kernel.
+// Launched programmatically dependent on the preceding layout kernel.
 cudaError_t launch_dispatch_fp8(const DispatchParams& p, cudaStream_t stream);
 cudaError_t launch_dispatch_bf16(const DispatchParams& p, cudaStream_t stream);
 

@@ -7,16 +7,18 @@
 // (deepseek.csdn.net/67bd3eb22e30c863900615cc, section "使用示例": dispatch returns
 // recv_x, recv_topk_idx, recv_topk_weights, handle).
 //
-// Two kernels, one CTA per chunk of kChunkTokens tokens:
-//   count: per-chunk expert histogram (shared-memory atomics: counts do not depend
-//          on order), token -> partition flags; the last CTA to finish (atomic
-//          ticket, no waiting) scans the [expert][chunk] counts into expert offsets
-//          and per-chunk row bases.
-//   rank:  per warp, a match_any / popc rank of each pair among equal expert ids,
-//          per-warp counts scanned across the CTA's warps, plus the chunk base:
-//          row = expert_offset[e] + rows of e in earlier chunks
-//                + rows of e in earlier warps of this chunk + rank in this warp.
-//          Deterministic: the result never depends on the order atomics land in.
+// One cooperative kernel; CTA c owns a contiguous chunk of tokens:
+//   1. stage the chunk's expert ids in shared memory, histogram them (shared-memory
+//      atomics: counts do not depend on order), flag the partitions each token
+//      touches, publish the chunk's counts;
+//   2. grid barrier (bounded wait);
+//   3. every CTA reads all chunks' counts, scans the totals into expert offsets and
+//      adds the counts of earlier chunks: base[e] = first row of e in this chunk;
+//   4. ranks: each warp takes a contiguous run of (t, k) entries, 32 at a time; a
+//      32-step shuffle loop ranks every pair among equal ids in the batch, giving
+//      its rank within the run; the per-warp counts are scanned across the warps, so
+//      row = base[e] + rows of e in earlier warps + rank within the run.
+// Deterministic: nothing depends on the order atomics land in.
 #include "ep_device.cuh"
 #include "ep_internal.h"
 
@@ -24,288 +26,361 @@ namespace ep {
 
 namespace {
 
-constexpr int kCountThreads = 512;
-constexpr int kRankThreads = kRankWarps * 32;
+constexpr int kLayoutThreads = 512;
+constexpr int kLayoutWarps = kLayoutThreads / 32;
+constexpr size_t kRankTableBytes = 32 * 1024;  // per-warp count table budget (shared memory)
 
-struct CountArgs {
+struct LayoutArgs {
     const int64_t* topk_idx;
     int64_t T;
     int32_t K, E, P, epp;
-    int64_t Cs;  // chunk stride of the [E][Cs] / [P][Cs] arrays
-    int32_t* chunk_expert;
-    int32_t* chunk_partition;
+    int32_t chunk_tokens;  // tokens per CTA, a multiple of 32
+    int32_t round_warps;   // warps ranking, each a contiguous run (bounded by the table budget)
+    int32_t flags_vec;     // is_token_in_partition is 8-byte aligned and P % 8 == 0
+    int32_t parts;         // thread groups splitting the chunks in the cross-chunk sums
+    int32_t* chunk_expert;     // [G][E]
+    int32_t* chunk_partition;  // [G][P]
     uint8_t* is_token_in_partition;
     int32_t* num_tokens_per_expert;
     int32_t* num_tokens_per_partition;
     int32_t* expert_offset;
     int32_t* num_recv;
-    uint32_t* ticket;
+    int32_t* row_of;
+    int32_t* src_of;
+    unsigned long long* bar;  // grid-barrier word (8-byte aligned)
     uint32_t* status;
+    uint64_t timeout_ns;
 };
 
-__global__ void __launch_bounds__(kCountThreads) layout_count_kernel(CountArgs a) {
-    pdl_launch_dependents();
-    extern __shared__ __align__(16) int sm_count[];
-    int* hist = sm_count;            // [E]
-    int* phist = hist + a.E;         // [P]
-    int* warp_sums = phist + a.P;    // [32]
-    int* is_last = warp_sums + 32;   // [1]
-    const int tid = threadIdx.x;
+__device__ __forceinline__ unsigned long long atom_add_release_gpu(unsigned long long* p,
+                                                                   unsigned long long v) {
+    unsigned long long old;
+    asm volatile("atom.add.release.gpu.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+    return old;
+}
 
-    for (int e = tid; e < a.E; e += blockDim.x) hist[e] = 0;
-    for (int p = tid; p < a.P; p += blockDim.x) phist[p] = 0;
+__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// All CTAs of the (co-resident, cooperatively launched) grid meet here.  One 64-bit
+// word holds (generation << 32 | arrivals): each CTA adds 1 with release semantics
+// (its writes before the barrier become visible); the last arrival adds
+// 2^32 - G, which bumps the generation and resets the count in one step; the
+// others poll with acquire loads until the generation changes, for at most
+// timeout_ns.  Returns false on timeout.
+__device__ bool grid_barrier(unsigned long long* word, uint64_t timeout_ns, int* flag_sm) {
     __syncthreads();
+    if (threadIdx.x == 0) {
+        bool ok = true;
+        const unsigned long long old = atom_add_release_gpu(word, 1ull);
+        const unsigned long long gen = old >> 32;
+        if ((old & 0xFFFFFFFFull) == gridDim.x - 1) {
+            atom_add_release_gpu(word, (1ull << 32) - gridDim.x);
+        } else {
+            const uint64_t t0 = globaltimer_ns();
+            while ((ld_acquire_gpu(word) >> 32) == gen) {
+                if (globaltimer_ns() - t0 > timeout_ns) {
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        *flag_sm = ok ? 1 : 0;
+    }
+    __syncthreads();
+    return *flag_sm != 0;
+}
+
+// The low 8 bits of m as eight 0/1 bytes (bit i -> byte i).
+__device__ __forceinline__ uint2 flag_bytes(uint64_t m) {
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        lo |= static_cast<uint32_t>((m >> i) & 1u) << (8 * i);
+        hi |= static_cast<uint32_t>((m >> (i + 4)) & 1u) << (8 * i);
+    }
+    return make_uint2(lo, hi);
+}
+
+__global__ void __launch_bounds__(kLayoutThreads, 1) layout_kernel(LayoutArgs a) {
+    pdl_launch_dependents();  // the dispatch kernel may start loading x
+    extern __shared__ __align__(16) int sm[];
+    const int K = a.K, E = a.E, P = a.P, W = a.round_warps;
+    const int Es = E + 1;  // padded row stride of the per-warp table (no bank conflicts)
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int* ent = sm;                                // [chunk_tokens * K] ids, -1 = skip
+    int* base = ent + a.chunk_tokens * K;         // [E] counts, then next row per expert
+    int* wcnt = base + E;                         // [W][E + 1] per-warp counts / first rows
+    int* part = wcnt + W * Es;                    // [2][parts][E] partial sums over chunks
+    int* phist = part + 2 * a.parts * E;          // [P]
+    int* part_of = phist + P + 32 + 4;            // [E] partition of each expert
+    int* rir = part_of + E;                       // [chunk_tokens * K] rank within the run
+    int* warp_sums = phist + P;                   // [32]
+    int* flag = warp_sums + 32;                   // [1]
 
     const int64_t c = blockIdx.x;
-    const int64_t t0 = c * kChunkTokens;
-    const int64_t t1 = min(a.T, t0 + kChunkTokens);
-    bool bad = false;
-    for (int64_t j = t0 * a.K + tid; j < t1 * a.K; j += blockDim.x) {
-        const int64_t e = a.topk_idx[j];
-        if (e == -1) continue;
-        if (e < 0 || e >= a.E) {
-            bad = true;
-            continue;
-        }
-        atomicAdd(&hist[e], 1);
+    const int64_t t0 = c * a.chunk_tokens;
+    const int64_t t1 = min(a.T, t0 + a.chunk_tokens);
+    const int n = t1 > t0 ? static_cast<int>((t1 - t0) * K) : 0;
+
+    for (int e = tid; e < E; e += blockDim.x) {
+        base[e] = 0;
+        part_of[e] = e / a.epp;
     }
-    for (int64_t t = t0 + tid; t < t1; t += blockDim.x) {
-        uint64_t mask = 0;
-        for (int k = 0; k < a.K; ++k) {
-            const int64_t e = a.topk_idx[t * a.K + k];
-            if (e >= 0 && e < a.E) mask |= 1ull << (e / a.epp);
-        }
-        uint8_t* flags = a.is_token_in_partition + t * a.P;
-        for (int p = 0; p < a.P; ++p) flags[p] = static_cast<uint8_t>((mask >> p) & 1u);
-        while (mask) {
-            const int p = __ffsll(static_cast<long long>(mask)) - 1;
-            atomicAdd(&phist[p], 1);
-            mask &= mask - 1;
-        }
+    for (int p = tid; p < P; p += blockDim.x) phist[p] = 0;
+    bool bad = false;
+    for (int j = tid; j < n; j += blockDim.x) {
+        const int64_t e = a.topk_idx[t0 * K + j];
+        const bool ok = e >= 0 && e < E;
+        bad |= (e != -1) && !ok;
+        ent[j] = ok ? static_cast<int>(e) : -1;
     }
     if (bad) raise_status(a.status, kDevIndexRange);
     __syncthreads();
 
-    for (int e = tid; e < a.E; e += blockDim.x) a.chunk_expert[e * a.Cs + c] = hist[e];
-    for (int p = tid; p < a.P; p += blockDim.x) a.chunk_partition[p * a.Cs + c] = phist[p];
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) *is_last = (atomicAdd(a.ticket, 1u) == gridDim.x - 1) ? 1 : 0;
-    __syncthreads();
-    if (!*is_last) return;
-
-    // ---- last CTA: every other chunk's counts are published (fence before ticket) ----
-    __threadfence();
-    const int64_t C = gridDim.x;
-    int carry = 0;
-    for (int e0 = 0; e0 < a.E; e0 += blockDim.x) {
-        const int e = e0 + tid;
-        int tot = 0;
-        if (e < a.E) {
-            const int32_t* col = a.chunk_expert + e * a.Cs;
-            int64_t cc = 0;
-            for (; cc + 4 <= C; cc += 4) {
-                const int4 v = __ldcg(reinterpret_cast<const int4*>(col + cc));
-                tot += v.x + v.y + v.z + v.w;
+    // 1. histogram and partition flags
+    for (int j = tid; j < n; j += blockDim.x)
+        if (ent[j] >= 0) atomicAdd(&base[ent[j]], 1);
+    // token -> partition flags: every thread takes one token's K slots (K <= 32
+    // consecutive ids in shared memory), ORs its partition bits, writes the P
+    // flags; per-partition token counts by ballot
+    for (int tb = warp * 32; tb < t1 - t0; tb += blockDim.x) {  // warp-uniform trip count
+        const int tl = tb + lane;
+        uint64_t mask = 0;
+        if (tl < t1 - t0) {
+#pragma unroll 4
+            for (int k = 0; k < K; ++k) {
+                const int e = ent[tl * K + ((k + lane) % K)];  // rotated: fewer bank conflicts
+                if (e >= 0) mask |= 1ull << part_of[e];
             }
-            for (; cc < C; ++cc) tot += __ldcg(col + cc);
+            uint8_t* flags = a.is_token_in_partition + (t0 + tl) * P;
+            if (a.flags_vec) {
+                for (int p = 0; p < P; p += 8)
+                    *reinterpret_cast<uint2*>(flags + p) = flag_bytes(mask >> p);
+            } else {
+                for (int p = 0; p < P; ++p) flags[p] = static_cast<uint8_t>((mask >> p) & 1u);
+            }
+        }
+        for (int p = 0; p < P; ++p) {
+            const unsigned b = __ballot_sync(0xffffffffu, (mask >> p) & 1u);
+            if (lane == 0 && b) atomicAdd(&phist[p], __popc(b));
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) a.chunk_expert[c * E + e] = base[e];
+    for (int p = tid; p < P; p += blockDim.x) a.chunk_partition[c * P + p] = phist[p];
+
+    // 2. every chunk's counts are published
+    if (!grid_barrier(a.bar, a.timeout_ns, flag)) {
+        if (tid == 0) raise_status(a.status, kDevTimeout);
+        return;
+    }
+
+    // 3. per expert: rows in all chunks and in earlier chunks.  `parts` groups of
+    //    threads split the chunks; each thread issues its loads 16 at a time into
+    //    registers so a whole batch is in flight (a loop over a runtime stride would
+    //    wait for every load in turn).
+    const int64_t G = gridDim.x;
+    {
+        for (int i = tid; i < a.parts * E; i += blockDim.x) {
+            const int e = i % E, q = i / E;
+            int tot = 0, before = 0;
+            for (int64_t c0 = q; c0 < G; c0 += 16 * static_cast<int64_t>(a.parts)) {
+                int v[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int64_t cc = c0 + static_cast<int64_t>(u) * a.parts;
+                    v[u] = cc < G ? __ldcg(a.chunk_expert + cc * E + e) : 0;
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int64_t cc = c0 + static_cast<int64_t>(u) * a.parts;
+                    tot += v[u];
+                    before += cc < c ? v[u] : 0;
+                }
+            }
+            part[q * E + e] = tot;
+            part[(a.parts + q) * E + e] = before;
+        }
+        __syncthreads();
+    }
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+        const int e = e0 + tid;
+        int tot = 0, before = 0;
+        if (e < E) {
+            for (int q = 0; q < a.parts; ++q) {
+                tot += part[q * E + e];
+                before += part[(a.parts + q) * E + e];
+            }
         }
         int tile_total;
         const int excl = block_exclusive_scan(tot, warp_sums, &tile_total);
-        if (e < a.E) {
-            a.num_tokens_per_expert[e] = tot;
-            a.expert_offset[e] = carry + excl;
-            hist[e] = carry + excl;
+        if (e < E) {
+            base[e] = carry + excl + before;
+            if (c == 0) {
+                a.num_tokens_per_expert[e] = tot;
+                a.expert_offset[e] = carry + excl;
+            }
         }
         carry += tile_total;
     }
-    if (tid == 0) {
-        a.expert_offset[a.E] = carry;
-        *a.num_recv = carry;
+    if (c == 0) {
+        if (tid == 0) {
+            a.expert_offset[E] = carry;
+            *a.num_recv = carry;
+        }
+        for (int p = warp; p < P; p += blockDim.x >> 5) {
+            int tot = 0;
+            for (int64_t cc = lane; cc < G; cc += 32) tot += __ldcg(a.chunk_partition + cc * P + p);
+            tot = __reduce_add_sync(0xffffffffu, tot);
+            if (lane == 0) a.num_tokens_per_partition[p] = tot;
+        }
+    }
+
+    // 4. stable ranks.  The chunk's n entries are split into W contiguous runs, one
+    //    per warp, taken 32 at a time; a shuffle loop ranks equal ids inside a batch,
+    //    and a running per-warp count per expert turns that into the entry's rank
+    //    within the run (kept in shared memory).  The per-warp counts are scanned
+    //    across the W warps (one thread per expert) into each warp's first row per
+    //    expert, and every entry's row is that first row + its rank in the run.
+    const int run = (n + W * 32 - 1) / (W * 32) * 32;  // entries per warp, multiple of 32
+    for (int i = tid; i < W * Es; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
+    if (warp < W) {
+        int* my = wcnt + warp * Es;
+        const int j0 = warp * run, j1 = min(n, j0 + run);
+        for (int j = j0 + lane; j - lane < j1; j += 32) {
+            const bool in = j < j1;
+            const int e = in ? ent[j] : -1;
+            int rank = 0, same = 0;  // equal ids in lower lanes / in the whole batch
+#pragma unroll
+            for (int l = 0; l < 32; ++l) {
+                const int el = __shfl_sync(0xffffffffu, e, l);
+                same += el == e ? 1 : 0;
+                rank += (l < lane && el == e) ? 1 : 0;
+            }
+            if (e >= 0) rir[j] = my[e] + rank;
+            __syncwarp();
+            if (e >= 0 && rank == 0) my[e] += same;  // first lane of its id
+            __syncwarp();
+        }
     }
     __syncthreads();
-    // chunk base of expert e = expert_offset[e] + rows of e in earlier chunks (in place)
-    for (int e = tid; e < a.E; e += blockDim.x) {
-        int32_t* col = a.chunk_expert + e * a.Cs;
-        int run = hist[e];
-        int64_t cc = 0;
-        for (; cc + 4 <= C; cc += 4) {
-            int4 v = __ldcg(reinterpret_cast<const int4*>(col + cc));
-            int4 b;
-            b.x = run; run += v.x;
-            b.y = run; run += v.y;
-            b.z = run; run += v.z;
-            b.w = run; run += v.w;
-            *reinterpret_cast<int4*>(col + cc) = b;
-        }
-        for (; cc < C; ++cc) {
-            const int v = __ldcg(col + cc);
-            col[cc] = run;
-            run += v;
+    for (int e = tid; e < E; e += blockDim.x) {
+        int r = base[e];
+        for (int w = 0; w < W; ++w) {
+            const int v = wcnt[w * Es + e];
+            wcnt[w * Es + e] = r;
+            r += v;
         }
     }
-    for (int p = tid; p < a.P; p += blockDim.x) {
-        const int32_t* col = a.chunk_partition + p * a.Cs;
-        int tot = 0;
-        for (int64_t cc = 0; cc < C; ++cc) tot += __ldcg(col + cc);
-        a.num_tokens_per_partition[p] = tot;
+    __syncthreads();
+    for (int j = tid; j < n; j += blockDim.x) {
+        const int e = ent[j];
+        const int row = e >= 0 ? wcnt[(j / run) * Es + e] + rir[j] : -1;
+        const int64_t g = t0 * K + j;
+        a.row_of[g] = row;
+        if (row >= 0) a.src_of[row] = static_cast<int32_t>(g);
     }
-    if (tid == 0) *a.ticket = 0u;  // ready for the next launch on this workspace
 }
 
-struct RankArgs {
-    const int64_t* topk_idx;
-    int64_t T;
-    int32_t K, E;
-    int64_t Cs;
-    const int32_t* chunk_base;  // [E][Cs], written by the count kernel's last CTA
-    int32_t* row_of;
-    int32_t* src_of;
-};
+// Tokens per CTA: about kTargetChunk, but never more CTAs than SMs (the grid must
+// be co-resident for its barrier).
+constexpr int64_t kTargetChunk = 128;
 
-__global__ void __launch_bounds__(kRankThreads) layout_rank_kernel(RankArgs a) {
-    pdl_launch_dependents();
-    extern __shared__ __align__(16) int sm_rank[];
-    const int K = a.K, E = a.E;
-    int* ent = sm_rank;                     // [kChunkTokens * K] expert ids, -1 = skip
-    int* wcnt = ent + kChunkTokens * K;     // [kRankWarps][E]
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t c = blockIdx.x;
-    const int64_t t0 = c * kChunkTokens;
-    const int64_t t1 = min(a.T, t0 + kChunkTokens);
-    const int n = static_cast<int>((t1 - t0) * K);
-
-    // topk_idx is an input of the whole call, so it may be read before the count
-    // kernel has finished.
-    for (int j = tid; j < n; j += blockDim.x) {
-        const int64_t e = a.topk_idx[t0 * K + j];
-        ent[j] = (e >= 0 && e < E) ? static_cast<int>(e) : -1;
-    }
-    for (int i = tid; i < kRankWarps * E; i += blockDim.x) wcnt[i] = 0;
-    __syncthreads();
-
-    // this warp's 32 tokens: entries [jw0, jw1)
-    const int jw0 = min(n, warp * 32 * K);
-    const int jw1 = min(n, jw0 + 32 * K);
-    int* my = wcnt + warp * E;
-    for (int j = jw0 + lane; j - lane < jw1; j += 32) {
-        const int e = j < jw1 ? ent[j] : -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        if (e >= 0 && (__ffs(peers) - 1) == lane) my[e] += __popc(peers);
-        __syncwarp();
-    }
-    __syncthreads();
-
-    pdl_wait();  // chunk bases are final
-    for (int e = tid; e < E; e += blockDim.x) {
-        int run = a.chunk_base[e * a.Cs + c];
-        for (int w = 0; w < kRankWarps; ++w) {
-            const int v = wcnt[w * E + e];
-            wcnt[w * E + e] = run;
-            run += v;
-        }
-    }
-    __syncthreads();
-
-    const unsigned lt = (1u << lane) - 1u;
-    for (int j = jw0 + lane; j - lane < jw1; j += 32) {
-        const bool in = j < jw1;
-        const int e = in ? ent[j] : -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        int row = -1;
-        if (e >= 0) row = my[e] + __popc(peers & lt);
-        __syncwarp();
-        if (e >= 0 && (__ffs(peers) - 1) == lane) my[e] += __popc(peers);
-        __syncwarp();
-        if (in) {
-            const int64_t g = t0 * K + j;
-            a.row_of[g] = row;
-            if (row >= 0) a.src_of[row] = static_cast<int32_t>(g);
-        }
-    }
+int64_t layout_grid(int64_t T, int num_sms) {
+    int64_t g = (T + kTargetChunk - 1) / kTargetChunk;
+    if (g > num_sms) g = num_sms;
+    return g < 1 ? 1 : g;
 }
 
 }  // namespace
 
-int64_t num_chunks(int64_t num_tokens) { return (num_tokens + kChunkTokens - 1) / kChunkTokens; }
-
-int64_t chunk_stride(int64_t num_tokens) {
-    const int64_t c = num_chunks(num_tokens);
-    return ((c > 0 ? c : 1) + 3) / 4 * 4;
+int64_t max_layout_chunks(int64_t num_tokens) {
+    const int64_t g = (num_tokens + kTargetChunk - 1) / kTargetChunk;
+    return g < 1 ? 1 : g;
 }
 
 Workspace carve_workspace(void* ws, int64_t num_tokens, int32_t num_experts) {
-    uint8_t* base = static_cast<uint8_t*>(ws);
+    uint8_t* b = static_cast<uint8_t*>(ws);
     Workspace w;
-    w.status = reinterpret_cast<uint32_t*>(base + kWsStatus);
-    w.ticket = reinterpret_cast<uint32_t*>(base + kWsTicket);
-    w.probe_flag = reinterpret_cast<uint32_t*>(base + kWsProbeFlag);
-    w.chunk_expert = reinterpret_cast<int32_t*>(base + kWsHeader);
-    w.chunk_partition = w.chunk_expert + static_cast<int64_t>(num_experts) * chunk_stride(num_tokens);
+    w.status = reinterpret_cast<uint32_t*>(b + kWsStatus);
+    w.bar = reinterpret_cast<unsigned long long*>(b + kWsBar);
+    w.probe_flag = reinterpret_cast<uint32_t*>(b + kWsProbeFlag);
+    w.chunk_expert = reinterpret_cast<int32_t*>(b + kWsHeader);
+    w.chunk_partition =
+        w.chunk_expert + static_cast<int64_t>(num_experts) * max_layout_chunks(num_tokens);
     return w;
 }
 
 cudaError_t launch_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int64_t* topk_idx,
                           const ep_layout& lay, const Workspace& ws, cudaStream_t stream) {
-    const int64_t C = num_chunks(T);
-    const int64_t Cs = chunk_stride(T);
+    DeviceInfo dev;
+    cudaError_t err = device_info(&dev);
+    if (err != cudaSuccess) return err;
+    const int64_t G = layout_grid(T, dev.num_sms);
+    int64_t chunk = (T + G - 1) / G;
+    chunk = (chunk + 31) / 32 * 32;
+    if (chunk < 32) chunk = 32;
+    int W = static_cast<int>(kRankTableBytes / (sizeof(int) * (static_cast<size_t>(E) + 1)));
+    if (W > kLayoutWarps) W = kLayoutWarps;
+    if (W < 1) W = 1;
+    // thread groups splitting the chunks: enough that every thread has an
+    // (expert, group) pair, at least one, at most one per chunk
+    int parts = (kLayoutThreads + E - 1) / E;
+    if (parts > G) parts = static_cast<int>(G);
+    if (parts < 1) parts = 1;
 
-    CountArgs ca;
-    ca.topk_idx = topk_idx;
-    ca.T = T;
-    ca.K = K;
-    ca.E = E;
-    ca.P = P;
-    ca.epp = E / P;
-    ca.Cs = Cs;
-    ca.chunk_expert = ws.chunk_expert;
-    ca.chunk_partition = ws.chunk_partition;
-    ca.is_token_in_partition = lay.is_token_in_partition;
-    ca.num_tokens_per_expert = lay.num_tokens_per_expert;
-    ca.num_tokens_per_partition = lay.num_tokens_per_partition;
-    ca.expert_offset = lay.expert_offset;
-    ca.num_recv = lay.num_recv;
-    ca.ticket = ws.ticket;
-    ca.status = ws.status;
-    const size_t count_smem = sizeof(int) * (static_cast<size_t>(E) + P + 32 + 4);
-    if (count_smem > 48 * 1024) {
-        cudaError_t err = cudaFuncSetAttribute(
-            layout_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)count_smem);
-        if (err != cudaSuccess) return err;
-    }
-    // First kernel of the call: ordinary launch, so it waits for all earlier work.
-    layout_count_kernel<<<dim3(static_cast<unsigned>(C > 0 ? C : 1)), kCountThreads, count_smem,
-                          stream>>>(ca);
-    cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess || C == 0) return err;
+    LayoutArgs a;
+    a.topk_idx = topk_idx;
+    a.T = T;
+    a.K = K;
+    a.E = E;
+    a.P = P;
+    a.epp = E / P;
+    a.chunk_tokens = static_cast<int32_t>(chunk);
+    a.round_warps = W;
+    a.flags_vec = (P % 8 == 0) && ((reinterpret_cast<uintptr_t>(lay.is_token_in_partition) & 7u) == 0);
+    a.parts = parts;
+    a.chunk_expert = ws.chunk_expert;
+    a.chunk_partition = ws.chunk_partition;
+    a.is_token_in_partition = lay.is_token_in_partition;
+    a.num_tokens_per_expert = lay.num_tokens_per_expert;
+    a.num_tokens_per_partition = lay.num_tokens_per_partition;
+    a.expert_offset = lay.expert_offset;
+    a.num_recv = lay.num_recv;
+    a.row_of = lay.row_of;
+    a.src_of = lay.src_of;
+    a.bar = ws.bar;
+    a.status = ws.status;
+    a.timeout_ns = kDefaultTimeoutNs;
 
-    RankArgs ra;
-    ra.topk_idx = topk_idx;
-    ra.T = T;
-    ra.K = K;
-    ra.E = E;
-    ra.Cs = Cs;
-    ra.chunk_base = ws.chunk_expert;
-    ra.row_of = lay.row_of;
-    ra.src_of = lay.src_of;
-    const size_t rank_smem =
-        sizeof(int) * (static_cast<size_t>(kChunkTokens) * K + static_cast<size_t>(kRankWarps) * E);
-    if (rank_smem > 48 * 1024) {
-        err = cudaFuncSetAttribute(layout_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)rank_smem);
-        if (err != cudaSuccess) return err;
-    }
+    const size_t smem =
+        sizeof(int) * (static_cast<size_t>(chunk) * K + static_cast<size_t>(E) +
+                       static_cast<size_t>(W) * (E + 1) + 2 * static_cast<size_t>(parts) * E + P +
+                       32 + 4 + static_cast<size_t>(E) + static_cast<size_t>(chunk) * K);
+    if (smem > dev.max_smem_optin) return cudaErrorInvalidValue;
+    err = cudaFuncSetAttribute(layout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    // First kernel of the call: an ordinary (not programmatic) launch, so it waits for
+    // all earlier work in the stream.  Cooperative: the grid barrier needs every CTA
+    // resident at once.
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(C));
-    cfg.blockDim = dim3(kRankThreads);
-    cfg.dynamicSmemBytes = rank_smem;
+    cfg.gridDim = dim3(static_cast<unsigned>(G));
+    cfg.blockDim = dim3(kLayoutThreads);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, layout_rank_kernel, ra);
+    return cudaLaunchKernelEx(&cfg, layout_kernel, a);
 }
 
 }  // namespace ep

@@ -6,7 +6,7 @@
 // whose enqueue step must not allocate, or a latency-critical path where the
 // implicit device synchronisation of cudaMalloc would stall other streams.  This
 // entry point gives them the same layout as ep_get_dispatch_layout, with its
-// scratch (status word, layout ticket, per-chunk expert and partition counts) in
+// scratch (status word, grid-barrier words, per-chunk expert and partition counts) in
 // a fixed array compiled into the library instead of a workspace.
 //
 // The array below is EP_STATIC_SCRATCH_BYTES (1 MiB) per GPU; every GPU that
@@ -87,7 +87,7 @@ extern "C" ep_status ep_get_dispatch_layout_static(int64_t num_tokens, int32_t n
     void* scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return EP_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // status word and layout ticket must start at zero; the per-chunk counts are
+    // status word and grid-barrier counter must start at zero; the per-chunk counts are
     // fully written before they are read
     if (cudaMemsetAsync(scratch, 0, kWsHeader, s) != cudaSuccess) return EP_ERR_CUDA;
     const Workspace ws = carve_workspace(scratch, num_tokens, num_experts);

@@ -53,8 +53,9 @@
  *   - Sizes: T = num_tokens >= 0, K = num_topk in [1, 32], E = num_experts in
  *     [1, 4096], P = num_partitions in [1, 64] dividing E, H = hidden > 0 with
  *     H % 8 == 0 (BF16) or H % 128 == 0 (FP8), H <= 16384; T * K < 2^31.
- *     Base pointers of x, recv_x, recv_scales, expert_out, y must be 16-byte
- *     aligned (the rows move by 16-byte vectors and bulk copies).
+ *     Base pointers of x, recv_x, recv_scales, expert_out, y and the workspace
+ *     must be 16-byte aligned (rows move by 16-byte vectors and bulk copies;
+ *     the workspace holds 64-bit atomics).
  */
 #ifndef EP_B200_H
 #define EP_B200_H
@@ -136,7 +137,9 @@ EP_API const char* ep_status_string(int32_t status);
  * serves every entry point for batches up to that size. */
 EP_API size_t ep_workspace_bytes(int64_t num_tokens, int32_t num_experts, int32_t num_partitions);
 
-/* Zero a workspace (once, after allocating it) on `stream`. */
+/* Zero a workspace (once, after allocating it) on `stream`.  Zero it again
+ * after a call reported EP_DEV_TIMEOUT: a layout that gave up at its grid
+ * barrier leaves the barrier word mid-count. */
 EP_API ep_status ep_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronise `stream`, return the sticky device status bits in *bits_out and
@@ -172,7 +175,7 @@ EP_API ep_status ep_get_dispatch_layout(int64_t num_tokens, int32_t num_topk, in
  *     stream capture.
  *   - Returns EP_ERR_WORKSPACE when the batch needs more scratch than the
  *     array holds, i.e. ep_workspace_bytes(T, E, P) > EP_STATIC_SCRATCH_BYTES
- *     (about 250k tokens at E = 256, P = 8).
+ *     (about 125k tokens at E = 256, P = 8).
  *   - Every call shares the one array and it keeps the last call's contents:
  *     each call clears the part that must start at zero, and calls that overlap
  *     on the GPU (other streams or host threads on the same device) race.

@@ -59,8 +59,8 @@ def test_version_and_strings(ep):
 
 def test_workspace_bytes(ep):
     b = ep.ep_workspace_bytes(4096, 256, 8)
-    # header + one int per (expert or partition, 256-token chunk), chunk count padded to 4
-    assert b == ((256 + 4 * 16 * (256 + 8)) + 255) // 256 * 256
+    # header + one int per (expert or partition, layout chunk of up to 128 tokens)
+    assert b == ((256 + 4 * 32 * (256 + 8)) + 255) // 256 * 256
     assert ep.ep_workspace_bytes(0, 256, 8) > 0
     assert ep.ep_workspace_bytes(-1, 256, 8) == 0
     assert ep.ep_workspace_bytes(10, 0, 1) == 0
@@ -94,7 +94,7 @@ def _dispatch(ep, T=16, H=256, K=4, E=8, P=2, quant=1, ws_bytes=1 << 20, **over)
     (dict(E=4097, P=1), 2), (dict(T=-1), 2), (dict(H=200), 2), (dict(H=0), 2),
     (dict(H=16512), 2), (dict(quant=1, H=136), 2), (dict(quant=5), 1), (dict(x=None), 1),
     (dict(rs=None), 1), (dict(x=_Fake.P + 8), 1), (dict(rx=_Fake.P + 4), 1), (dict(rs=_Fake.P + 4), 1),
-    (dict(ws=None), 1), (dict(lay=None), 1), (dict(ws_bytes=64), 3),
+    (dict(ws=None), 1), (dict(ws=_Fake.P + 8), 1), (dict(lay=None), 1), (dict(ws_bytes=64), 3),
     (dict(T=1 << 28, K=8), 2),
 ])
 def test_dispatch_host_checks(ep, over, status):
