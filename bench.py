@@ -277,9 +277,13 @@ class PathRunner:
         return ([e[0].elapsed_time(e[1]) for e in evs], [e[1].elapsed_time(e[2]) for e in evs])
 
 
-def time_low_latency(ep, w, dev, reps=200):
-    """LL dispatch / combine: CUDA-graph replay median (kernel-only, back to back, L2
-    warm as in decode) and eager call + synchronize wall time (launch-inclusive)."""
+def time_low_latency(ep, w, dev, reps=200, per_graph=20):
+    """LL dispatch / combine latency (L2 warm, as in decode):
+    graph_replay_us -- one call per CUDA-graph replay, replays back to back
+                       (launch-inclusive: includes the graph launch cost);
+    gpu_us          -- per_graph calls captured in one graph (device time per call);
+    eager_call_us   -- one eager call through the Python binding + synchronize
+                       (host wall time)."""
     import numpy as np
     import torch
 
@@ -308,8 +312,7 @@ def time_low_latency(ep, w, dev, reps=200):
     def comb():
         ep.ep_low_latency_combine(eo, h, wts, y, ws)
 
-    out = {}
-    for name, fn in (("dispatch", disp), ("combine", comb)):
+    def capture(fn, n):
         s = torch.cuda.Stream(device=dev)
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
@@ -319,24 +322,38 @@ def time_low_latency(ep, w, dev, reps=200):
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            fn()
-        for _ in range(20):
+            for _ in range(n):
+                fn()
+        for _ in range(5):
             g.replay()
         torch.cuda.synchronize()
+        return g
+
+    out = {}
+    for name, fn in (("dispatch", disp), ("combine", comb)):
+        g1 = capture(fn, 1)
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
         evs[0].record()
         for i in range(reps):
-            g.replay()
+            g1.replay()
             evs[i + 1].record()
         torch.cuda.synchronize()
-        graph_us = statistics.median(evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(reps))
+        replay_us = statistics.median(evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(reps))
+        gn = capture(fn, per_graph)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(10):
+            gn.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        gpu_us = e0.elapsed_time(e1) * 1e3 / (10 * per_graph)
         walls = []
         for _ in range(50):
             t0 = time.perf_counter()
             fn()
             torch.cuda.synchronize()
             walls.append((time.perf_counter() - t0) * 1e6)
-        out[name] = {"graph_replay_us": round(graph_us, 2),
+        out[name] = {"gpu_us": round(gpu_us, 2), "graph_replay_us": round(replay_us, 2),
                      "eager_call_us": round(statistics.median(walls), 2)}
     if ep.ep_read_status(ws) != 0:
         raise RuntimeError("device status set in the low-latency run")

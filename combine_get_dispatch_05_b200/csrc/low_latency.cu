@@ -7,14 +7,15 @@
 // expert.  "DeepSeek 开源周第二弹：DeepEP", section "DeepEP 的常规内核和低延迟内核":
 // 128-token decode batches, FP8 dispatch.
 //
-// One CTA per token does everything the normal path does in three kernels:
-//   - its row's bulk load is issued first, so HBM latency overlaps the rest;
+// One kernel does everything the normal path does in its layout and dispatch
+// kernels; each token's row is split into slices, one CTA per (token, slice):
+//   - the slice's bulk load is issued first, so its latency overlaps the rest;
 //   - slot of (t, k) in expert e = number of earlier (t', k') routed to e, counted
 //     directly over the topk_idx prefix (the batch is small, the prefix is L2-hot);
 //     the order is the normal layout's, so slot j of e holds normal row
 //     expert_offset[e] + j;
 //   - CTA 0 also histograms all T*K ids into recv_expert_count;
-//   - quantise (same arithmetic as the normal FP8 path) and bulk-store the row
+//   - quantise the slice (same arithmetic as the normal FP8 path) and bulk-store it
 //     into slot e * num_max_tokens + j of each destination expert.
 #include "ep_device.cuh"
 #include "ep_internal.h"
@@ -24,19 +25,21 @@ namespace ep {
 
 namespace {
 
-constexpr int kLLThreads = 256;
+constexpr int kLLMaxThreads = 256;
 
+// Shared memory of one (token, slice) CTA: the slice's BF16 input, its E4M3 codes
+// and scales, an mbarrier, the token's K rows / slot counters / ids, and (CTA 0
+// only) the expert histogram.
 struct LLSmem {
     uint32_t in_bytes, q_bytes, s_bytes;
     uint32_t off_q, off_s, off_bar, off_rows, off_cnt, off_eid, off_hist, total;
 };
 
-__host__ __device__ inline LLSmem ll_smem(int64_t H, int32_t E) {
+__host__ __device__ inline LLSmem ll_smem(int nbs, int32_t E) {
     LLSmem s;
-    const uint32_t nb = static_cast<uint32_t>(H / 128);
-    s.in_bytes = static_cast<uint32_t>(H) * 2u;
-    s.q_bytes = static_cast<uint32_t>(H);
-    s.s_bytes = (nb * 4u + 15u) & ~15u;
+    s.in_bytes = static_cast<uint32_t>(nbs) * 256u;
+    s.q_bytes = static_cast<uint32_t>(nbs) * 128u;
+    s.s_bytes = (static_cast<uint32_t>(nbs) * 4u + 15u) & ~15u;
     s.off_q = s.in_bytes;
     s.off_s = s.off_q + s.q_bytes;
     s.off_bar = s.off_s + s.s_bytes;
@@ -48,12 +51,17 @@ __host__ __device__ inline LLSmem ll_smem(int64_t H, int32_t E) {
     return s;
 }
 
-__global__ void __launch_bounds__(kLLThreads) ll_dispatch_kernel(LowLatencyDispatchParams p) {
+// grid = (T, S): CTA (t, y) handles token t's 128-channel blocks
+// [y * nbs, min(nb, (y + 1) * nbs)).  Every slice computes the token's slots (the
+// prefix is short and L2-hot); slice 0 also writes the handle; CTA (0, 0) writes
+// recv_expert_count.
+__global__ void __launch_bounds__(kLLMaxThreads) ll_dispatch_kernel(LowLatencyDispatchParams p,
+                                                                    int nbs) {
     extern __shared__ __align__(128) uint8_t sm[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     const int64_t H = p.H;
     const int K = p.K, E = p.E, cap = p.cap, nb = static_cast<int>(H >> 7);
-    const LLSmem L = ll_smem(H, E);
+    const LLSmem L = ll_smem(nbs, E);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.off_bar);
     int* rows_sm = reinterpret_cast<int*>(sm + L.off_rows);
     int* cnt_sm = reinterpret_cast<int*>(sm + L.off_cnt);
@@ -61,8 +69,14 @@ __global__ void __launch_bounds__(kLLThreads) ll_dispatch_kernel(LowLatencyDispa
     int* hist = reinterpret_cast<int*>(sm + L.off_hist);
     uint8_t* out_q = sm + L.off_q;
     float* out_s = reinterpret_cast<float*>(sm + L.off_s);
-    const bool scale_bulk = (static_cast<uint32_t>(nb) * 4u) == L.s_bytes;
     const int64_t t = blockIdx.x;
+    const int y = blockIdx.y;
+    const int b0 = y * nbs;
+    const int nbl = min(nb, b0 + nbs) - b0;  // blocks in this slice (>= 1)
+    const bool head = (y == 0);
+    const bool all = (t == 0 && y == 0);
+    // scales go out by bulk copy when every row's slice of them is 16-byte aligned
+    const bool scale_bulk = (nb % 4 == 0) && (nbs % 4 == 0) && (nbl % 4 == 0);
 
     if (tid == 0) {
         mbar_init(bar, 1);
@@ -70,14 +84,15 @@ __global__ void __launch_bounds__(kLLThreads) ll_dispatch_kernel(LowLatencyDispa
     }
     __syncthreads();
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar, L.in_bytes);
-        bulk_load(sm, static_cast<const uint8_t*>(p.x) + t * H * 2, L.in_bytes, bar);
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbl) * 256u);
+        bulk_load(sm, static_cast<const uint8_t*>(p.x) + t * H * 2 + static_cast<int64_t>(b0) * 256,
+                  static_cast<uint32_t>(nbl) * 256u, bar);
     }
     if (tid < K) {
         eid_sm[tid] = p.topk_idx[t * K + tid];
         cnt_sm[tid] = 0;
     }
-    if (blockIdx.x == 0)
+    if (all)
         for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
 
@@ -88,7 +103,7 @@ __global__ void __launch_bounds__(kLLThreads) ll_dispatch_kernel(LowLatencyDispa
         for (int k = 0; k < K; ++k)
             if (j < base + k && ej == eid_sm[k]) atomicAdd(&cnt_sm[k], 1);
     }
-    if (blockIdx.x == 0) {
+    if (all) {
         for (int64_t j = tid; j < p.T * K; j += blockDim.x) {
             const int64_t ej = p.topk_idx[j];
             if (ej >= 0 && ej < E) atomicAdd(&hist[ej], 1);
@@ -99,19 +114,21 @@ __global__ void __launch_bounds__(kLLThreads) ll_dispatch_kernel(LowLatencyDispa
         const int64_t e = eid_sm[tid];
         int row = -1;
         if (e != -1 && (e < 0 || e >= E)) {
-            raise_status(p.status, kDevIndexRange);
+            if (head) raise_status(p.status, kDevIndexRange);
         } else if (e >= 0) {
             const int j = cnt_sm[tid];
             if (j < cap)
                 row = static_cast<int>(e * cap + j);
-            else
+            else if (head)
                 raise_status(p.status, kDevCapacity);
         }
         rows_sm[tid] = row;
-        p.row_of[base + tid] = row;
-        if (row >= 0) p.src_of[row] = static_cast<int32_t>(base + tid);
+        if (head) {
+            p.row_of[base + tid] = row;
+            if (row >= 0) p.src_of[row] = static_cast<int32_t>(base + tid);
+        }
     }
-    if (blockIdx.x == 0)
+    if (all)
         for (int e = tid; e < E; e += blockDim.x) p.recv_expert_count[e] = min(hist[e], cap);
 
     const bool ok = mbar_wait_bounded(bar, 0, p.timeout_ns);
@@ -122,25 +139,26 @@ __global__ void __launch_bounds__(kLLThreads) ll_dispatch_kernel(LowLatencyDispa
         }
         return;
     }
-    quantize_row_fp8(sm, out_q, out_s, nb, warp, nwarps, lane);
+    quantize_row_fp8(sm, out_q, out_s, nbl, warp, nwarps, lane);
     fence_proxy_async_smem();
     __syncthreads();
     uint8_t* recv_x = static_cast<uint8_t*>(p.recv_x);
     if (warp == 0 && lane < K) {
         const int row = rows_sm[lane];
         if (row >= 0) {
-            bulk_store(recv_x + static_cast<int64_t>(row) * H, out_q, L.q_bytes);
+            bulk_store(recv_x + static_cast<int64_t>(row) * H + static_cast<int64_t>(b0) * 128,
+                       out_q, static_cast<uint32_t>(nbl) * 128u);
             if (scale_bulk)
-                bulk_store(p.recv_scales + static_cast<int64_t>(row) * nb, out_s,
-                           static_cast<uint32_t>(nb) * 4u);
+                bulk_store(p.recv_scales + static_cast<int64_t>(row) * nb + b0, out_s,
+                           static_cast<uint32_t>(nbl) * 4u);
         }
         bulk_commit();
     }
     if (!scale_bulk) {
-        for (int idx = tid; idx < K * nb; idx += blockDim.x) {
-            const int k = idx / nb, b = idx - k * nb;
+        for (int idx = tid; idx < K * nbl; idx += blockDim.x) {
+            const int k = idx / nbl, b = idx - k * nbl;
             const int r = rows_sm[k];
-            if (r >= 0) p.recv_scales[static_cast<int64_t>(r) * nb + b] = out_s[b];
+            if (r >= 0) p.recv_scales[static_cast<int64_t>(r) * nb + b0 + b] = out_s[b];
         }
     }
     if (warp == 0 && lane < K) bulk_wait_all<0>();
@@ -173,12 +191,26 @@ cudaError_t launch_ll_dispatch(const LowLatencyDispatchParams& p, cudaStream_t s
     DeviceInfo dev;
     cudaError_t err = device_info(&dev);
     if (err != cudaSuccess) return err;
-    const LLSmem L = ll_smem(p.H, p.E);
+    // slices per token: enough (token, slice) CTAs to cover every SM about four
+    // times, a multiple of 4 blocks per slice where possible (bulk scale stores)
+    const int nb = static_cast<int>(p.H / 128);
+    int64_t S = (4LL * dev.num_sms + p.T - 1) / p.T;
+    if (S > nb) S = nb;
+    if (S < 1) S = 1;
+    int nbs = static_cast<int>((nb + S - 1) / S);
+    if (nbs % 4 != 0 && nbs > 4 && nb % 4 == 0) nbs = (nbs + 3) / 4 * 4;
+    S = (nb + nbs - 1) / nbs;
+    if (S > 65535) return cudaErrorInvalidValue;
+    const LLSmem L = ll_smem(nbs, p.E);
     if (L.total > dev.max_smem_optin) return cudaErrorInvalidValue;
     err = cudaFuncSetAttribute(ll_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(L.total));
     if (err != cudaSuccess) return err;
-    ll_dispatch_kernel<<<dim3(static_cast<unsigned>(p.T)), kLLThreads, L.total, stream>>>(p);
+    const int pairs = (nbs + 1) / 2;
+    int threads = 32 * (pairs < 2 ? 2 : pairs);
+    if (threads > kLLMaxThreads) threads = kLLMaxThreads;
+    ll_dispatch_kernel<<<dim3(static_cast<unsigned>(p.T), static_cast<unsigned>(S)), threads, L.total,
+                         stream>>>(p, nbs);
     return cudaGetLastError();
 }
 
