@@ -37,6 +37,17 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "dispatch/combine HBM GB/s (% of B200 peak) at 4096x7168 top-8; LL latency µs"
+WORKLOAD_TEXT = {
+    "normal": "normal: 4096 tokens x hidden 7168 BF16, top-8 of 256 experts in 8 logical "
+              "partitions, top-4-of-8-group routing, FP8 (E4M3, 1x128 scales) dispatch + BF16 "
+              "combine",
+    "skew": "skew: 4096 tokens x hidden 7168, top-8 of 256 experts (Zipf 1.2 popularity, 5% "
+            "of slots masked), FP8 dispatch + BF16 combine",
+    "bf16": "bf16: 8192 tokens x hidden 4096, top-6 of 64 experts in 16 partitions, 1% "
+            "outlier rows, BF16 dispatch (no quantisation) + BF16 combine",
+    "stress": "stress: 32768 tokens x hidden 7168, top-8 over 288 expert slots (256 + 32 "
+              "replicas) in 8 partitions, FP8 dispatch + BF16 combine",
+}
 FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 256 << 20
 
@@ -400,19 +411,19 @@ def cpu_baseline(w, min_seconds=10.0):
     import oracle
 
     T, H, K, E, P = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
-    d = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, E, P)
-    eo = oracle.identity_expert(d["recv_x"], d["recv_scales"])
-    bd, bc = algorithmic_bytes(T, H, K, E, P, int(d["num_recv"][0]), True)
+    d = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, E, P, quant=w.quant)
+    eo = oracle.identity_expert(d["recv_x"], d["recv_scales"], quant=w.quant)
+    bd, bc = algorithmic_bytes(T, H, K, E, P, int(d["num_recv"][0]), w.quant == "fp8")
     passes, t = 0, 0.0
     while t < min_seconds and passes < 50:
         t0 = time.perf_counter()
-        dd = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, E, P)
+        dd = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, E, P, quant=w.quant)
         oracle.combine(eo, dd["row_of"], w.topk_weights)
         t += time.perf_counter() - t0
         passes += 1
     return {"value": round((bd + bc) * passes / t / 1e9, 3), "unit": "GB/s", "cores": 1,
             "kind": "oracle",
-            "sample": f"the full {T}-token batch (layout + FP8 dispatch + combine), {passes} passes, "
+            "sample": f"the full {T}-token batch (layout + dispatch + combine), {passes} passes, "
                       f"{t:.1f} s, single-threaded C"}
 
 
@@ -456,7 +467,7 @@ def run_ours(args):
 
     sampler = ClockSampler(local)
     sampler.start()
-    w = make_workload("normal", seed=args.seed + rank)
+    w = make_workload(args.workload, seed=args.seed + rank)
     runner = PathRunner(ep, w, dev, use_graphs=not args.eager)
     flush = make_flush(args.l2_flush, dev)
 
@@ -511,9 +522,7 @@ def run_ours(args):
         "dtype": "f32 arithmetic; fp8-e4m3 dispatch payload, bf16 combine",
         "data": "synthetic",
         "config": {
-            "workload": "normal: 4096 tokens x hidden 7168 BF16, top-8 of 256 experts in 8 "
-                        "logical partitions, top-4-of-8-group routing, FP8 (E4M3, 1x128 scales) "
-                        "dispatch + BF16 combine",
+            "workload": WORKLOAD_TEXT[args.workload],
             "tokens_per_gpu": w.num_tokens, "hidden": w.hidden, "topk": w.num_topk,
             "experts": w.num_experts, "partitions": w.num_partitions, "recv_rows": runner.R,
             "bytes_per_step": step_bytes, "seed": args.seed,
@@ -527,7 +536,8 @@ def run_ours(args):
         "breakdown": {
             "dispatch": {"us": round(disp_us, 2), "bytes": runner.bytes_dispatch,
                          "gbs": round(disp_gbs, 1), "frac": round(disp_gbs / peak, 4),
-                         "kernels": "layout (cooperative) + dispatch_fp8 (programmatic dependent launch)"},
+                         "kernels": "layout (cooperative) + dispatch_%s (programmatic dependent "
+                                    "launch)" % ("fp8" if runner.fp8 else "bf16")},
             "combine": {"us": round(comb_us, 2), "bytes": runner.bytes_combine,
                         "gbs": round(comb_gbs, 1), "frac": round(comb_gbs / peak, 4),
                         "kernels": "combine"},
@@ -647,6 +657,8 @@ def main():
     ap.add_argument("--extra-steps", type=int, default=50)
     ap.add_argument("--eager", action="store_true", help="launch eagerly instead of CUDA graphs")
     ap.add_argument("--l2-flush", choices=("none", "write", "read"), default="none")
+    ap.add_argument("--workload", choices=("normal", "skew", "bf16", "stress"), default="normal",
+                    help="workload of the timed step (the headline metric is quoted on normal)")
     ap.add_argument("--no-extra", action="store_true", help="skip the ll/skew/bf16/stress configs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -26,7 +26,7 @@ namespace {
 
 constexpr int kFp8InStages = 3;   // input ring: rows in flight from HBM per CTA
 constexpr int kFp8OutStages = 3;  // quantised rows staged for the bulk stores
-constexpr int kBf16Stages = 4;
+constexpr int kBf16Stages = 4;    // BF16 rows in flight per CTA
 
 struct Fp8Smem {
     uint32_t in_bytes, q_bytes, s_bytes, out_bytes;
@@ -218,94 +218,105 @@ __global__ void __launch_bounds__(352) dispatch_fp8_kernel(DispatchParams p) {
     if (tid == 0 && *abort_flag) raise_status(p.status, kDevTimeout);
 }
 
-__global__ void __launch_bounds__(32) dispatch_bf16_kernel(DispatchParams p) {
+// BF16 rows are copied bit for bit, so the row staged by the bulk load is itself
+// the source of the K bulk stores.  One CTA = a loader warp and a storer warp
+// coupled by full/empty mbarriers over a ring of kBf16Stages rows:
+//   loader (warp 0, lane 0): waits empty[s], bulk-loads the next token's row into
+//       stage s (full[s] counts its transaction bytes);
+//   storer (warp 1): waits for the layout, then per token waits full[s], lane k
+//       bulk-stores the row to row_of[t, k] and writes recv_topk_idx / weights;
+//       once this token's stores have read the stage it arrives on empty[s].
+__global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
     extern __shared__ __align__(128) uint8_t sm[];
-    const int lane = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t T = p.T, H = p.H;
     const int K = p.K;
     const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kBf16Stages * row_bytes);
-    const uint8_t* x = static_cast<const uint8_t*>(p.x);
-    uint8_t* recv_x = static_cast<uint8_t*>(p.recv_x);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kBf16Stages * row_bytes);
+    uint64_t* empty = full + kBf16Stages;
+    volatile int* abort_flag = reinterpret_cast<int*>(empty + kBf16Stages);
 
     const int64_t G = gridDim.x, first = blockIdx.x;
     const int64_t n_mine = first < T ? (T - 1 - first) / G + 1 : 0;
 
-    if (lane == 0) {
-        for (int s = 0; s < kBf16Stages; ++s) mbar_init(&bars[s], 1);
+    if (tid == 0) {
+        for (int s = 0; s < kBf16Stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        *abort_flag = 0;
         fence_mbar_init();
     }
-    __syncwarp();
-    int64_t issued = 0;
-    if (lane == 0) {
-        for (; issued < kBf16Stages && issued < n_mine; ++issued) {
-            const int64_t t = first + issued * G;
-            mbar_arrive_expect_tx(&bars[issued], row_bytes);
-            bulk_load(sm + issued * row_bytes, x + t * row_bytes, row_bytes, &bars[issued]);
+    __syncthreads();
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- loader
+        if (lane == 0) {
+            const uint8_t* x = static_cast<const uint8_t*>(p.x);
+            int64_t issued = 0;
+            for (; issued < n_mine; ++issued) {
+                const int s = static_cast<int>(issued % kBf16Stages);
+                if (issued >= kBf16Stages &&
+                    !wait_or_abort(&empty[s], static_cast<uint32_t>((issued / kBf16Stages - 1) & 1),
+                                   p.timeout_ns, abort_flag))
+                    break;
+                const int64_t t = first + issued * G;
+                mbar_arrive_expect_tx(&full[s], row_bytes);
+                bulk_load(sm + s * row_bytes, x + t * row_bytes, row_bytes, &full[s]);
+            }
+            if (*abort_flag) {
+                for (int64_t j = issued - 1; j >= 0 && j >= issued - kBf16Stages; --j)
+                    mbar_wait_bounded(&full[j % kBf16Stages],
+                                      static_cast<uint32_t>((j / kBf16Stages) & 1),
+                                      kDefaultTimeoutNs);
+            }
         }
-    }
-
-    pdl_wait();
-
-    const bool slot_lane = lane < K;
-    int nrow = -1;
-    int64_t nexp = -1;
-    float nwt = 0.0f;
-    if (slot_lane && n_mine > 0) {
-        const int64_t g = first * K + lane;
-        nrow = p.row_of[g];
-        nexp = p.topk_idx[g];
-        nwt = p.topk_weights[g];
-    }
-
-    int64_t i = 0;
-    bool aborted = false;
-    for (; i < n_mine; ++i) {
-        const int64_t t = first + i * G;
-        const int s = static_cast<int>(i % kBf16Stages);
-        const uint32_t par = static_cast<uint32_t>((i / kBf16Stages) & 1);
-        const int row = nrow;
-        const int64_t e = nexp;
-        const float wt = nwt;
-        if (slot_lane && i + 1 < n_mine) {
-            const int64_t g = (t + G) * K + lane;
+    } else {
+        // ---------------------------------------------------------------- storer
+        pdl_wait();  // row_of from the layout kernel is complete and visible
+        uint8_t* recv_x = static_cast<uint8_t*>(p.recv_x);
+        const bool slot_lane = lane < K;
+        int nrow = -1;
+        int64_t nexp = -1;
+        float nwt = 0.0f;
+        if (slot_lane && n_mine > 0) {
+            const int64_t g = first * K + lane;
             nrow = p.row_of[g];
             nexp = p.topk_idx[g];
             nwt = p.topk_weights[g];
         }
-        const bool ok = mbar_wait_bounded(&bars[s], par, p.timeout_ns);
-        if (!__all_sync(0xffffffffu, ok)) {
-            aborted = true;
-            break;
-        }
-        if (slot_lane) {
-            if (row >= 0) {
-                bulk_store(recv_x + static_cast<int64_t>(row) * row_bytes, sm + s * row_bytes,
-                           row_bytes);
-                const int64_t epp = p.experts_per_partition;
-                p.recv_topk_idx[row] = static_cast<int32_t>(e - (e / epp) * epp);
-                p.recv_topk_weights[row] = wt;
+        for (int64_t i = 0; i < n_mine; ++i) {
+            const int64_t t = first + i * G;
+            const int s = static_cast<int>(i % kBf16Stages);
+            const int row = nrow;
+            const int64_t e = nexp;
+            const float wt = nwt;
+            if (slot_lane && i + 1 < n_mine) {
+                const int64_t g = (t + G) * K + lane;
+                nrow = p.row_of[g];
+                nexp = p.topk_idx[g];
+                nwt = p.topk_weights[g];
             }
-            bulk_commit();
-            bulk_wait_read<1>();  // this lane's stores of token i-1 have read their stage
+            if (!wait_or_abort(&full[s], static_cast<uint32_t>((i / kBf16Stages) & 1), p.timeout_ns,
+                               abort_flag))
+                break;
+            if (slot_lane) {
+                if (row >= 0) {
+                    bulk_store(recv_x + static_cast<int64_t>(row) * row_bytes, sm + s * row_bytes,
+                               row_bytes);
+                    const int64_t epp = p.experts_per_partition;
+                    p.recv_topk_idx[row] = static_cast<int32_t>(e - (e / epp) * epp);
+                    p.recv_topk_weights[row] = wt;
+                }
+                bulk_commit();
+                bulk_wait_read<1>();  // the previous token's stores have read their stage
+            }
+            __syncwarp();
+            if (lane == 0 && i >= 1) mbar_arrive(&empty[(i - 1) % kBf16Stages]);
         }
-        __syncwarp();
-        // stage of token i-1 is free: refill it with the next token of this CTA
-        if (lane == 0 && i >= 1 && issued < n_mine) {
-            const int ps = static_cast<int>((i - 1) % kBf16Stages);
-            const int64_t t2 = first + issued * G;
-            mbar_arrive_expect_tx(&bars[ps], row_bytes);
-            bulk_load(sm + ps * row_bytes, x + t2 * row_bytes, row_bytes, &bars[ps]);
-            ++issued;
-        }
+        if (slot_lane) bulk_wait_all<0>();
     }
-    if (aborted && lane == 0) {
-        raise_status(p.status, kDevTimeout);
-        for (int64_t j = i; j < issued; ++j)
-            mbar_wait_bounded(&bars[j % kBf16Stages], static_cast<uint32_t>((j / kBf16Stages) & 1),
-                              kDefaultTimeoutNs);
-    }
-    if (slot_lane) bulk_wait_all<0>();
+    if (tid == 0 && *abort_flag) raise_status(p.status, kDevTimeout);
 }
 
 int grid_for(const void* kernel, int threads, size_t smem, int64_t work, int num_sms) {
@@ -361,14 +372,14 @@ cudaError_t launch_dispatch_bf16(const DispatchParams& p, cudaStream_t stream) {
     DeviceInfo dev;
     cudaError_t err = device_info(&dev);
     if (err != cudaSuccess) return err;
-    const size_t smem = static_cast<size_t>(kBf16Stages) * p.H * 2 + 8 * kBf16Stages;
+    const size_t smem = static_cast<size_t>(kBf16Stages) * p.H * 2 + 16 * kBf16Stages + 16;
     if (smem > dev.max_smem_optin) return cudaErrorInvalidValue;
     const void* kernel = reinterpret_cast<const void*>(dispatch_bf16_kernel);
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    const int grid = grid_for(kernel, 32, smem, p.T, dev.num_sms);
-    return launch_pdl(kernel, dim3(grid), dim3(32), smem, stream, p);
+    const int grid = grid_for(kernel, 64, smem, p.T, dev.num_sms);
+    return launch_pdl(kernel, dim3(grid), dim3(64), smem, stream, p);
 }
 
 }  // namespace ep

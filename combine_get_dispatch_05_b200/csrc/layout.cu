@@ -11,13 +11,15 @@
 //   1. stage the chunk's expert ids in shared memory, histogram them (shared-memory
 //      atomics: counts do not depend on order), flag the partitions each token
 //      touches, publish the chunk's counts;
-//   2. grid barrier (bounded wait);
-//   3. every CTA reads all chunks' counts, scans the totals into expert offsets and
+//   2. arrive at a grid barrier, and while the other chunks arrive
+//   3. rank inside the chunk: each warp takes a contiguous run of (t, k) entries, 32
+//      at a time; a 32-step shuffle loop ranks every pair among equal ids in the
+//      batch, giving its rank within the run; the per-warp counts are scanned
+//      across the warps;
+//   4. wait at the barrier (bounded);
+//   5. every CTA reads all chunks' counts, scans the totals into expert offsets and
 //      adds the counts of earlier chunks: base[e] = first row of e in this chunk;
-//   4. ranks: each warp takes a contiguous run of (t, k) entries, 32 at a time; a
-//      32-step shuffle loop ranks every pair among equal ids in the batch, giving
-//      its rank within the run; the per-warp counts are scanned across the warps, so
-//      row = base[e] + rows of e in earlier warps + rank within the run.
+//   6. row = base[e] + rows of e in earlier warps of the chunk + rank within the run.
 // Deterministic: nothing depends on the order atomics land in.
 #include "ep_device.cuh"
 #include "ep_internal.h"
@@ -65,33 +67,28 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long
     return v;
 }
 
-// All CTAs of the (co-resident, cooperatively launched) grid meet here.  One 64-bit
+// Grid barrier of the (co-resident, cooperatively launched) grid, split into an
+// arrive and a wait so that a CTA can do independent work in between.  One 64-bit
 // word holds (generation << 32 | arrivals): each CTA adds 1 with release semantics
-// (its writes before the barrier become visible); the last arrival adds
-// 2^32 - G, which bumps the generation and resets the count in one step; the
-// others poll with acquire loads until the generation changes, for at most
-// timeout_ns.  Returns false on timeout.
-__device__ bool grid_barrier(unsigned long long* word, uint64_t timeout_ns, int* flag_sm) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        bool ok = true;
-        const unsigned long long old = atom_add_release_gpu(word, 1ull);
-        const unsigned long long gen = old >> 32;
-        if ((old & 0xFFFFFFFFull) == gridDim.x - 1) {
-            atom_add_release_gpu(word, (1ull << 32) - gridDim.x);
-        } else {
-            const uint64_t t0 = globaltimer_ns();
-            while ((ld_acquire_gpu(word) >> 32) == gen) {
-                if (globaltimer_ns() - t0 > timeout_ns) {
-                    ok = false;
-                    break;
-                }
-            }
-        }
-        *flag_sm = ok ? 1 : 0;
+// (its writes before the arrive become visible); the last arrival adds 2^32 - G,
+// which bumps the generation and resets the count in one step; the others poll
+// with acquire loads until the generation changes, for at most timeout_ns.
+// Thread 0 of each CTA calls both; the returned token is the generation to leave.
+__device__ __forceinline__ unsigned long long grid_arrive(unsigned long long* word) {
+    const unsigned long long old = atom_add_release_gpu(word, 1ull);
+    if ((old & 0xFFFFFFFFull) == gridDim.x - 1)
+        atom_add_release_gpu(word, (1ull << 32) - gridDim.x);
+    return old >> 32;
+}
+
+__device__ __forceinline__ bool grid_wait(const unsigned long long* word, unsigned long long gen,
+                                          uint64_t timeout_ns) {
+    if ((ld_acquire_gpu(word) >> 32) != gen) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while ((ld_acquire_gpu(word) >> 32) == gen) {
+        if (globaltimer_ns() - t0 > timeout_ns) return false;
     }
-    __syncthreads();
-    return *flag_sm != 0;
+    return true;
 }
 
 // The low 8 bits of m as eight 0/1 bytes (bit i -> byte i).
@@ -173,80 +170,17 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_kernel(LayoutArgs a)
     for (int e = tid; e < E; e += blockDim.x) a.chunk_expert[c * E + e] = base[e];
     for (int p = tid; p < P; p += blockDim.x) a.chunk_partition[c * P + p] = phist[p];
 
-    // 2. every chunk's counts are published
-    if (!grid_barrier(a.bar, a.timeout_ns, flag)) {
-        if (tid == 0) raise_status(a.status, kDevTimeout);
-        return;
-    }
+    // 2. publish: arrive at the grid barrier (release), but do not wait yet
+    __syncthreads();
+    unsigned long long gen = 0;
+    if (tid == 0) gen = grid_arrive(a.bar);
 
-    // 3. per expert: rows in all chunks and in earlier chunks.  `parts` groups of
-    //    threads split the chunks; each thread issues its loads 16 at a time into
-    //    registers so a whole batch is in flight (a loop over a runtime stride would
-    //    wait for every load in turn).
-    const int64_t G = gridDim.x;
-    {
-        for (int i = tid; i < a.parts * E; i += blockDim.x) {
-            const int e = i % E, q = i / E;
-            int tot = 0, before = 0;
-            for (int64_t c0 = q; c0 < G; c0 += 16 * static_cast<int64_t>(a.parts)) {
-                int v[16];
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int64_t cc = c0 + static_cast<int64_t>(u) * a.parts;
-                    v[u] = cc < G ? __ldcg(a.chunk_expert + cc * E + e) : 0;
-                }
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int64_t cc = c0 + static_cast<int64_t>(u) * a.parts;
-                    tot += v[u];
-                    before += cc < c ? v[u] : 0;
-                }
-            }
-            part[q * E + e] = tot;
-            part[(a.parts + q) * E + e] = before;
-        }
-        __syncthreads();
-    }
-    int carry = 0;
-    for (int e0 = 0; e0 < E; e0 += blockDim.x) {
-        const int e = e0 + tid;
-        int tot = 0, before = 0;
-        if (e < E) {
-            for (int q = 0; q < a.parts; ++q) {
-                tot += part[q * E + e];
-                before += part[(a.parts + q) * E + e];
-            }
-        }
-        int tile_total;
-        const int excl = block_exclusive_scan(tot, warp_sums, &tile_total);
-        if (e < E) {
-            base[e] = carry + excl + before;
-            if (c == 0) {
-                a.num_tokens_per_expert[e] = tot;
-                a.expert_offset[e] = carry + excl;
-            }
-        }
-        carry += tile_total;
-    }
-    if (c == 0) {
-        if (tid == 0) {
-            a.expert_offset[E] = carry;
-            *a.num_recv = carry;
-        }
-        for (int p = warp; p < P; p += blockDim.x >> 5) {
-            int tot = 0;
-            for (int64_t cc = lane; cc < G; cc += 32) tot += __ldcg(a.chunk_partition + cc * P + p);
-            tot = __reduce_add_sync(0xffffffffu, tot);
-            if (lane == 0) a.num_tokens_per_partition[p] = tot;
-        }
-    }
-
-    // 4. stable ranks.  The chunk's n entries are split into W contiguous runs, one
-    //    per warp, taken 32 at a time; a shuffle loop ranks equal ids inside a batch,
-    //    and a running per-warp count per expert turns that into the entry's rank
-    //    within the run (kept in shared memory).  The per-warp counts are scanned
-    //    across the W warps (one thread per expert) into each warp's first row per
-    //    expert, and every entry's row is that first row + its rank in the run.
+    // 3. chunk-local ranks, which need no other chunk.  The n entries are split into
+    //    W contiguous runs, one per warp, taken 32 at a time; a shuffle loop ranks
+    //    equal ids inside a batch and a running per-warp count per expert turns that
+    //    into the entry's rank within the run (kept in shared memory).  The per-warp
+    //    counts are then scanned across the W warps: wcnt[w][e] = rows of e in this
+    //    chunk before warp w's run.
     const int run = (n + W * 32 - 1) / (W * 32) * 32;  // entries per warp, multiple of 32
     for (int i = tid; i < W * Es; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
@@ -271,17 +205,96 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_kernel(LayoutArgs a)
     }
     __syncthreads();
     for (int e = tid; e < E; e += blockDim.x) {
-        int r = base[e];
+        int r = 0;
         for (int w = 0; w < W; ++w) {
             const int v = wcnt[w * Es + e];
             wcnt[w * Es + e] = r;
             r += v;
         }
     }
+
+    // 4. wait for every chunk's counts
+    if (tid == 0) *flag = grid_wait(a.bar, gen, a.timeout_ns) ? 1 : 0;
     __syncthreads();
+    if (!*flag) {
+        if (tid == 0) raise_status(a.status, kDevTimeout);
+        return;
+    }
+
+    // 5. per expert: rows in all chunks and in earlier chunks.  `parts` groups of
+    //    threads split the chunks; each thread issues its loads 16 at a time into
+    //    registers so a whole batch is in flight (a loop over a runtime stride would
+    //    wait for every load in turn).  CTA p < P also sums partition p's tokens.
+    const int64_t G = gridDim.x;
+    int ptot = 0;
+    if (c < P && warp == (blockDim.x >> 5) - 1) {
+        for (int64_t cc = lane; cc < G; cc += 32) ptot += __ldcg(a.chunk_partition + cc * P + c);
+    }
+    for (int i = tid; i < a.parts * E; i += blockDim.x) {
+        const int e = i % E, q = i / E;
+        int tot = 0, before = 0;
+        for (int64_t c0 = q; c0 < G; c0 += 16 * static_cast<int64_t>(a.parts)) {
+            int v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int64_t cc = c0 + static_cast<int64_t>(u) * a.parts;
+                v[u] = cc < G ? __ldcg(a.chunk_expert + cc * E + e) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int64_t cc = c0 + static_cast<int64_t>(u) * a.parts;
+                tot += v[u];
+                before += cc < c ? v[u] : 0;
+            }
+        }
+        part[q * E + e] = tot;
+        part[(a.parts + q) * E + e] = before;
+    }
+    if (c < P && warp == (blockDim.x >> 5) - 1) {
+        ptot = __reduce_add_sync(0xffffffffu, ptot);
+        if (lane == 0) a.num_tokens_per_partition[c] = ptot;
+    }
+    __syncthreads();
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+        const int e = e0 + tid;
+        int tot = 0, before = 0;
+        if (e < E) {
+            for (int q = 0; q < a.parts; ++q) {
+                tot += part[q * E + e];
+                before += part[(a.parts + q) * E + e];
+            }
+        }
+        int tile_total;
+        const int excl = block_exclusive_scan(tot, warp_sums, &tile_total);
+        if (e < E) {
+            base[e] = carry + excl + before;
+            if (c == 0) {
+                a.num_tokens_per_expert[e] = tot;
+                a.expert_offset[e] = carry + excl;
+            }
+        }
+        carry += tile_total;
+    }
+    if (c == 0 && tid == 0) {
+        a.expert_offset[E] = carry;
+        *a.num_recv = carry;
+    }
+    // partitions beyond the grid (P > G) hold the remaining sums
+    for (int p = static_cast<int>(G) + static_cast<int>(c); p < P; p += static_cast<int>(G)) {
+        if (warp == 0) {
+            int t2 = 0;
+            for (int64_t cc = lane; cc < G; cc += 32) t2 += __ldcg(a.chunk_partition + cc * P + p);
+            t2 = __reduce_add_sync(0xffffffffu, t2);
+            if (lane == 0) a.num_tokens_per_partition[p] = t2;
+        }
+    }
+    __syncthreads();
+
+    // 6. rows: first row of e in this chunk + rows before this warp's run + rank in run
     for (int j = tid; j < n; j += blockDim.x) {
         const int e = ent[j];
-        const int row = e >= 0 ? wcnt[(j / run) * Es + e] + rir[j] : -1;
+        const int row = e >= 0 ? base[e] + wcnt[(j / run) * Es + e] + rir[j] : -1;
         const int64_t g = t0 * K + j;
         a.row_of[g] = row;
         if (row >= 0) a.src_of[row] = static_cast<int32_t>(g);
