@@ -61,6 +61,10 @@ def lib() -> ctypes.CDLL:
         L.oracle_combine.restype = ctypes.c_uint32
         L.oracle_ll_dispatch.argtypes = [_i64, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p, _p]
         L.oracle_ll_dispatch.restype = ctypes.c_uint32
+        L.oracle_dispatch_backward.argtypes = [_i64, _i64, _i32, _p, _i64, _p, _p, _p, _p]
+        L.oracle_dispatch_backward.restype = ctypes.c_uint32
+        L.oracle_combine_backward.argtypes = [_i64, _i64, _i32, _p, _p, _i64, _p, _p, _p, _p]
+        L.oracle_combine_backward.restype = ctypes.c_uint32
         _lib = L
     return _lib
 
@@ -244,3 +248,40 @@ def ll_combine(expert_out: np.ndarray, ll_row_of: np.ndarray, topk_weights: np.n
     """Low-latency combine: the same k-way reduce over a padded [E, cap, H] output."""
     E, cap, H = expert_out.shape
     return combine(expert_out.reshape(E * cap, H), ll_row_of, topk_weights)
+
+
+# ---------------------------------------------------------------- backward --
+
+def dispatch_backward(grad_recv_x: np.ndarray, row_of: np.ndarray,
+                      grad_recv_topk_weights=None):
+    """grad_x (BF16 bits [T, H]) and grad_topk_weights (fp32 [T, K] or None)."""
+    g = _c(grad_recv_x, np.uint16)
+    rows, H = g.shape
+    ro = _c(row_of, np.int32)
+    T, K = ro.shape
+    gx = np.empty((T, H), np.uint16)
+    gw = np.zeros((T, K), np.float32) if grad_recv_topk_weights is not None else None
+    grw = _c(grad_recv_topk_weights, np.float32) if grad_recv_topk_weights is not None else None
+    g_p = g if rows else np.zeros((1, H), np.uint16)
+    st = lib().oracle_dispatch_backward(T, H, K, _ptr(g_p), rows, _ptr(ro),
+                                        _ptr(grw) if grw is not None else None, _ptr(gx),
+                                        _ptr(gw) if gw is not None else None)
+    return gx, gw, int(st)
+
+
+def combine_backward(grad_y: np.ndarray, expert_out: np.ndarray, row_of: np.ndarray,
+                     topk_weights: np.ndarray, fill: int = 0xA5A5):
+    """grad_expert_out (BF16 bits [rows, H]; rows no slot points at keep `fill`) and
+    grad_topk_weights (fp32 [T, K])."""
+    gy = _c(grad_y, np.uint16)
+    eo = _c(expert_out, np.uint16)
+    rows, H = eo.shape
+    ro = _c(row_of, np.int32)
+    w = _c(topk_weights, np.float32)
+    T, K = ro.shape
+    geo = np.full((max(rows, 1), H), fill, np.uint16)
+    gw = np.empty((T, K), np.float32)
+    eo_p = eo if rows else np.zeros((1, H), np.uint16)
+    st = lib().oracle_combine_backward(T, H, K, _ptr(gy), _ptr(eo_p), rows, _ptr(ro), _ptr(w),
+                                       _ptr(geo), _ptr(gw))
+    return geo[:rows], gw, int(st)

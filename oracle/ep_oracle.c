@@ -337,3 +337,79 @@ uint32_t oracle_ll_dispatch(int64_t T, int64_t H, int32_t K, int32_t E, int32_t 
     free(s);
     return status;
 }
+
+/* ------------------------------------------------------------ backward -- */
+
+/* Backward of dispatch ("deepseek-ai/DeepEP" (agentlenshq.com), section
+ * "典型工作流程": combine "or the backward helpers" reduce results back).  Every
+ * receive row is a copy of its token, so the gradient of x sums the gradients of
+ * the token's rows:
+ *   grad_x[t][i] = bf16_rne( +0.0f + grad_recv_x[row_of[t][0]][i] + ... ), rows in
+ *   k order, masked slots skipped;
+ * and recv_topk_weights[row] = topk_weights[t][k] gives
+ *   grad_topk_weights[t][k] = grad_recv_topk_weights[row_of[t][k]] (0 if masked).
+ * grad_recv_topk_weights / grad_topk_weights may be NULL. */
+uint32_t oracle_dispatch_backward(int64_t T, int64_t H, int32_t K, const uint16_t* grad_recv_x,
+                                  int64_t rows, const int32_t* row_of,
+                                  const float* grad_recv_topk_weights, uint16_t* grad_x,
+                                  float* grad_topk_weights) {
+    uint32_t status = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t i = 0; i < H; ++i) {
+            float acc = 0.0f;
+            for (int32_t k = 0; k < K; ++k) {
+                int32_t row = row_of[t * K + k];
+                if (row < 0) continue;
+                if ((int64_t)row >= rows) {
+                    status |= ORACLE_INDEX_RANGE;
+                    continue;
+                }
+                acc = acc + oracle_bf16_to_f32(grad_recv_x[(int64_t)row * H + i]);
+            }
+            grad_x[t * H + i] = oracle_bf16_from_f32(acc);
+        }
+        if (grad_recv_topk_weights && grad_topk_weights) {
+            for (int32_t k = 0; k < K; ++k) {
+                int32_t row = row_of[t * K + k];
+                grad_topk_weights[t * K + k] =
+                    (row >= 0 && (int64_t)row < rows) ? grad_recv_topk_weights[row] : 0.0f;
+            }
+        }
+    }
+    return status;
+}
+
+/* Backward of combine y[t] = sum_k w[t][k] * expert_out[row_of[t][k]]:
+ *   grad_expert_out[row_of[t][k]][i] = bf16_rne( w[t][k] * float(grad_y[t][i]) )
+ *     (one binary32 multiply; rows no slot points at are not written);
+ *   grad_topk_weights[t][k] = float( sum over i = 0..H-1 of
+ *     (double)grad_y[t][i] * (double)expert_out[row][i] ), 0 for masked slots.
+ * Each product of two BF16 values is exact in binary32 (8 + 8 significant bits)
+ * and the sum runs in binary64, so while the products' magnitudes span fewer
+ * than 37 binades the sum is exact and its rounding to binary32 does not depend
+ * on the order of the terms. */
+uint32_t oracle_combine_backward(int64_t T, int64_t H, int32_t K, const uint16_t* grad_y,
+                                 const uint16_t* expert_out, int64_t rows, const int32_t* row_of,
+                                 const float* topk_weights, uint16_t* grad_expert_out,
+                                 float* grad_topk_weights) {
+    uint32_t status = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t k = 0; k < K; ++k) {
+            int32_t row = row_of[t * K + k];
+            double dot = 0.0;
+            int valid = row >= 0 && (int64_t)row < rows;
+            if (row >= 0 && !valid) status |= ORACLE_INDEX_RANGE;
+            if (valid) {
+                float w = topk_weights[t * K + k];
+                for (int64_t i = 0; i < H; ++i) {
+                    float g = oracle_bf16_to_f32(grad_y[t * H + i]);
+                    float e = oracle_bf16_to_f32(expert_out[(int64_t)row * H + i]);
+                    grad_expert_out[(int64_t)row * H + i] = oracle_bf16_from_f32(w * g);
+                    dot += (double)g * (double)e;
+                }
+            }
+            grad_topk_weights[t * K + k] = valid ? (float)dot : 0.0f;
+        }
+    }
+    return status;
+}
