@@ -25,7 +25,7 @@ EXPORTED = (
     "ep_abi_version", "ep_status_string", "ep_workspace_bytes", "ep_workspace_init",
     "ep_read_status", "ep_get_dispatch_layout", "ep_dispatch", "ep_combine",
     "ep_low_latency_dispatch", "ep_low_latency_combine", "ep_debug_wait_probe",
-    "ep_get_dispatch_layout_static",
+    "ep_get_dispatch_layout_static", "ep_dispatch_backward", "ep_combine_backward",
 )
 
 
@@ -76,6 +76,12 @@ def _load() -> ctypes.CDLL:
     L.ep_get_dispatch_layout_static.argtypes = [i64, i32, i32, i32, vp,
                                                 ctypes.POINTER(ep_layout), vp]
     L.ep_get_dispatch_layout_static.restype = st
+    L.ep_dispatch_backward.argtypes = [i64, i64, i32, vp, i64, ctypes.POINTER(ep_layout), vp, vp, vp,
+                                       vp, sz, vp]
+    L.ep_dispatch_backward.restype = st
+    L.ep_combine_backward.argtypes = [i64, i64, i32, vp, vp, i64, ctypes.POINTER(ep_layout), vp, vp,
+                                      vp, vp, sz, vp]
+    L.ep_combine_backward.restype = st
     return L
 
 
@@ -305,3 +311,45 @@ def ep_debug_wait_probe(timeout_ns: int, workspace: torch.Tensor, stream=None) -
     _need(workspace, "workspace", torch.uint8)
     _check("ep_debug_wait_probe", lib.ep_debug_wait_probe(
         int(timeout_ns), workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_dispatch_backward(grad_recv_x: torch.Tensor, handle: Layout, grad_x: torch.Tensor,
+                         workspace: torch.Tensor, grad_recv_topk_weights=None,
+                         grad_topk_weights=None, stream=None) -> None:
+    _need(grad_recv_x, "grad_recv_x", torch.bfloat16)
+    H = grad_recv_x.shape[-1]
+    rows = grad_recv_x.numel() // H if H else 0
+    T, K = handle.row_of.shape
+    _need(handle.row_of, "handle.row_of", torch.int32)
+    _need(grad_x, "grad_x", torch.bfloat16, shape=(T, H))
+    _need(workspace, "workspace", torch.uint8)
+    if grad_recv_topk_weights is not None:
+        _need(grad_recv_topk_weights, "grad_recv_topk_weights", torch.float32,
+              numel_at_least=rows)
+        _need(grad_topk_weights, "grad_topk_weights", torch.float32, shape=(T, K))
+    c = ep_layout(row_of=handle.row_of.data_ptr())
+    _check("ep_dispatch_backward", lib.ep_dispatch_backward(
+        T, H, K, grad_recv_x.data_ptr(), rows, ctypes.byref(c), _ptr(grad_recv_topk_weights),
+        grad_x.data_ptr(), _ptr(grad_topk_weights), workspace.data_ptr(), workspace.numel(),
+        _stream(stream)))
+
+
+def ep_combine_backward(grad_y: torch.Tensor, expert_out: torch.Tensor, handle: Layout,
+                        topk_weights: torch.Tensor, grad_expert_out: torch.Tensor,
+                        grad_topk_weights: torch.Tensor, workspace: torch.Tensor,
+                        stream=None) -> None:
+    _need(grad_y, "grad_y", torch.bfloat16)
+    T, H = grad_y.shape
+    _need(expert_out, "expert_out", torch.bfloat16)
+    rows = expert_out.numel() // H if H else 0
+    K = handle.row_of.shape[1]
+    _need(handle.row_of, "handle.row_of", torch.int32, shape=(T, K))
+    _need(topk_weights, "topk_weights", torch.float32, shape=(T, K))
+    _need(grad_expert_out, "grad_expert_out", torch.bfloat16, numel_at_least=rows * H)
+    _need(grad_topk_weights, "grad_topk_weights", torch.float32, shape=(T, K))
+    _need(workspace, "workspace", torch.uint8)
+    c = ep_layout(row_of=handle.row_of.data_ptr())
+    _check("ep_combine_backward", lib.ep_combine_backward(
+        T, H, K, grad_y.data_ptr(), expert_out.data_ptr(), rows, ctypes.byref(c),
+        topk_weights.data_ptr(), grad_expert_out.data_ptr(), grad_topk_weights.data_ptr(),
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))

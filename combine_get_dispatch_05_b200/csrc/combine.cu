@@ -39,10 +39,10 @@ __global__ void __launch_bounds__(kCombineMaxThreads) combine_kernel(CombinePara
     uint4* y = static_cast<uint4*>(p.y);
 
     int nrow = -1;
-    float nw = 0.0f;
+    float nw = 1.0f;
     if (tid < K && static_cast<int64_t>(blockIdx.x) < T) {
         nrow = p.row_of[static_cast<int64_t>(blockIdx.x) * K + tid];
-        nw = p.topk_weights[static_cast<int64_t>(blockIdx.x) * K + tid];
+        if (p.topk_weights) nw = p.topk_weights[static_cast<int64_t>(blockIdx.x) * K + tid];
     }
     int buf = 0;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x, buf ^= 1) {
@@ -54,10 +54,12 @@ __global__ void __launch_bounds__(kCombineMaxThreads) combine_kernel(CombinePara
             }
             rows_sm[buf][tid] = r;
             w_sm[buf][tid] = nw;
+            if (p.grad_w && blockIdx.y == 0)
+                p.grad_w[t * K + tid] = r >= 0 ? p.grad_recv_w[r] : 0.0f;
             const int64_t tn = t + gridDim.x;
             if (tn < T) {
                 nrow = p.row_of[tn * K + tid];
-                nw = p.topk_weights[tn * K + tid];
+                if (p.topk_weights) nw = p.topk_weights[tn * K + tid];
             }
         }
         __syncthreads();
@@ -103,6 +105,95 @@ __global__ void __launch_bounds__(kCombineMaxThreads) combine_kernel(CombinePara
     }
 }
 
+// Backward of combine y[t] = sum_k w[t, k] * expert_out[row_of[t, k]]:
+//   grad_expert_out[row, i] = bf16_rne(w[t, k] * grad_y[t, i])   (one fp32 multiply)
+//   grad_topk_weights[t, k] = float(sum_i double(grad_y[t, i] * expert_out[row, i]))
+// A product of two BF16 values is exact in fp32 (8 + 8 significant bits); the sum
+// runs in fp64, which is exact -- and so independent of the summation order -- while
+// the products span fewer than 37 binades.  One CTA per token row (grid-stride);
+// each thread owns 8-channel vectors and issues the loads of up to 8 slots before
+// using them; the per-slot dot products are reduced across the CTA in a fixed
+// order (warp shuffles, then warps in index order).
+constexpr int kBwdThreads = 448;
+
+__global__ void __launch_bounds__(kBwdThreads) combine_backward_kernel(CombineBackwardParams p) {
+    __shared__ int rows_sm[32];
+    __shared__ float w_sm[32];
+    __shared__ double red[kBwdThreads / 32][kLoadBatch];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    const int K = p.K;
+    const int64_t T = p.T, V = p.H / 8;
+    const uint4* gy = static_cast<const uint4*>(p.grad_y);
+    const uint4* eo = static_cast<const uint4*>(p.expert_out);
+    uint4* geo = static_cast<uint4*>(p.grad_expert_out);
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        if (tid < K) {
+            int r = p.row_of[t * K + tid];
+            if (r >= 0 && static_cast<int64_t>(r) >= p.expert_out_rows) {
+                raise_status(p.status, kDevIndexRange);
+                r = -1;
+            }
+            rows_sm[tid] = r;
+            w_sm[tid] = p.topk_weights[t * K + tid];
+        }
+        __syncthreads();
+        for (int k0 = 0; k0 < K; k0 += kLoadBatch) {
+            double dot[kLoadBatch];
+#pragma unroll
+            for (int u = 0; u < kLoadBatch; ++u) dot[u] = 0.0;
+            for (int64_t v = tid; v < V; v += blockDim.x) {
+                const uint4 g = ld_stream_v4(gy + t * V + v);
+                float gf[8];
+                gf[0] = bf16_lo(g.x); gf[1] = bf16_hi(g.x); gf[2] = bf16_lo(g.y); gf[3] = bf16_hi(g.y);
+                gf[4] = bf16_lo(g.z); gf[5] = bf16_hi(g.z); gf[6] = bf16_lo(g.w); gf[7] = bf16_hi(g.w);
+                uint4 d[kLoadBatch];
+#pragma unroll
+                for (int u = 0; u < kLoadBatch; ++u) {
+                    const int k = k0 + u;
+                    const int r = k < K ? rows_sm[k] : -1;
+                    d[u] = r >= 0 ? ld_stream_v4(eo + static_cast<int64_t>(r) * V + v)
+                                  : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int u = 0; u < kLoadBatch; ++u) {
+                    const int k = k0 + u;
+                    const int r = k < K ? rows_sm[k] : -1;
+                    if (r < 0) continue;
+                    float ef[8];
+                    ef[0] = bf16_lo(d[u].x); ef[1] = bf16_hi(d[u].x);
+                    ef[2] = bf16_lo(d[u].y); ef[3] = bf16_hi(d[u].y);
+                    ef[4] = bf16_lo(d[u].z); ef[5] = bf16_hi(d[u].z);
+                    ef[6] = bf16_lo(d[u].w); ef[7] = bf16_hi(d[u].w);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) dot[u] += static_cast<double>(__fmul_rn(gf[j], ef[j]));
+                    const float w = w_sm[k];
+                    uint4 o;
+                    o.x = bf16x2_rn(__fmul_rn(w, gf[0]), __fmul_rn(w, gf[1]));
+                    o.y = bf16x2_rn(__fmul_rn(w, gf[2]), __fmul_rn(w, gf[3]));
+                    o.z = bf16x2_rn(__fmul_rn(w, gf[4]), __fmul_rn(w, gf[5]));
+                    o.w = bf16x2_rn(__fmul_rn(w, gf[6]), __fmul_rn(w, gf[7]));
+                    geo[static_cast<int64_t>(r) * V + v] = o;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kLoadBatch; ++u) {
+                double s = dot[u];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                if (lane == 0) red[warp][u] = s;
+            }
+            __syncthreads();
+            if (tid < kLoadBatch && k0 + tid < K) {
+                double s = 0.0;
+                for (int w2 = 0; w2 < nwarps; ++w2) s += red[w2][tid];
+                const int k = k0 + tid;
+                p.grad_topk_weights[t * K + k] = rows_sm[k] >= 0 ? __double2float_rn(s) : 0.0f;
+            }
+            __syncthreads();
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
@@ -133,6 +224,29 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
     if (gx > 2147483647LL) gx = 2147483647LL;
     combine_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(slices)), threads, 0,
                      stream>>>(p, per_slice);
+    return cudaGetLastError();
+}
+
+}  // namespace ep
+
+namespace ep {
+
+cudaError_t launch_combine_backward(const CombineBackwardParams& p, cudaStream_t stream) {
+    if (p.T == 0) return cudaSuccess;
+    DeviceInfo dev;
+    cudaError_t err = device_info(&dev);
+    if (err != cudaSuccess) return err;
+    const int64_t V = p.H / 8;
+    int threads = static_cast<int>((V + 31) / 32 * 32);
+    if (threads > kBwdThreads) threads = kBwdThreads;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_backward_kernel, threads,
+                                                      0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    int64_t grid = static_cast<int64_t>(per_sm) * dev.num_sms;
+    if (grid > p.T) grid = p.T;
+    combine_backward_kernel<<<static_cast<unsigned>(grid), threads, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

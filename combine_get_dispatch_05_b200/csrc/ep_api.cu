@@ -197,8 +197,73 @@ ep_status ep_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk, const
     p.row_of = handle->row_of;
     p.topk_weights = topk_weights;
     p.y = y;
+    p.grad_recv_w = nullptr;
+    p.grad_w = nullptr;
     p.status = carve_workspace(workspace, 0, 1).status;
     return cuda_status(launch_combine(p, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_dispatch_backward(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                               const void* grad_recv_x, int64_t grad_recv_rows,
+                               const ep_layout* handle, const float* grad_recv_topk_weights,
+                               void* grad_x, float* grad_topk_weights, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    if (num_tokens < 0 || num_topk < 1 || num_topk > 32 || grad_recv_rows < 0) return EP_ERR_SHAPE;
+    if (num_tokens * static_cast<int64_t>(num_topk) >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    ep_status st = check_hidden(hidden, false);
+    if (st != EP_OK) return st;
+    if (!handle || !workspace || !aligned16(workspace) || workspace_bytes < kWsHeader)
+        return EP_ERR_INVALID_ARG;
+    if ((grad_recv_topk_weights == nullptr) != (grad_topk_weights == nullptr))
+        return EP_ERR_INVALID_ARG;
+    if (num_tokens == 0) return EP_OK;
+    if (!handle->row_of || !grad_x || (!grad_recv_x && grad_recv_rows > 0)) return EP_ERR_INVALID_ARG;
+    if (!aligned16(grad_x) || !aligned16(grad_recv_x)) return EP_ERR_INVALID_ARG;
+    CombineParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = num_topk;
+    p.expert_out = grad_recv_x;
+    p.expert_out_rows = grad_recv_rows;
+    p.row_of = handle->row_of;
+    p.topk_weights = nullptr;  // every weight 1: the plain sum of the token's rows
+    p.y = grad_x;
+    p.grad_recv_w = grad_recv_topk_weights;
+    p.grad_w = grad_topk_weights;
+    p.status = carve_workspace(workspace, 0, 1).status;
+    return cuda_status(launch_combine(p, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_combine_backward(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                              const void* grad_y, const void* expert_out, int64_t expert_out_rows,
+                              const ep_layout* handle, const float* topk_weights,
+                              void* grad_expert_out, float* grad_topk_weights, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    if (num_tokens < 0 || num_topk < 1 || num_topk > 32 || expert_out_rows < 0) return EP_ERR_SHAPE;
+    if (num_tokens * static_cast<int64_t>(num_topk) >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    ep_status st = check_hidden(hidden, false);
+    if (st != EP_OK) return st;
+    if (!handle || !workspace || !aligned16(workspace) || workspace_bytes < kWsHeader)
+        return EP_ERR_INVALID_ARG;
+    if (num_tokens == 0) return EP_OK;
+    if (!handle->row_of || !grad_y || !topk_weights || !grad_topk_weights ||
+        (expert_out_rows > 0 && (!expert_out || !grad_expert_out)))
+        return EP_ERR_INVALID_ARG;
+    if (!aligned16(grad_y) || !aligned16(expert_out) || !aligned16(grad_expert_out))
+        return EP_ERR_INVALID_ARG;
+    CombineBackwardParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = num_topk;
+    p.grad_y = grad_y;
+    p.expert_out = expert_out;
+    p.expert_out_rows = expert_out_rows;
+    p.row_of = handle->row_of;
+    p.topk_weights = topk_weights;
+    p.grad_expert_out = grad_expert_out;
+    p.grad_topk_weights = grad_topk_weights;
+    p.status = carve_workspace(workspace, 0, 1).status;
+    return cuda_status(launch_combine_backward(p, static_cast<cudaStream_t>(stream)));
 }
 
 ep_status ep_low_latency_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk,

@@ -61,11 +61,28 @@ struct CombineParams {
     const void* expert_out;
     int64_t expert_out_rows;
     const int32_t* row_of;
-    const float* topk_weights;
+    const float* topk_weights;  // NULL: every weight is 1 (the backward of dispatch)
     void* y;
+    const float* grad_recv_w;   // optional gather: grad_w[t, k] = grad_recv_w[row_of[t, k]]
+    float* grad_w;
     uint32_t* status;
 };
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+
+struct CombineBackwardParams {
+    int64_t T;
+    int64_t H;
+    int32_t K;
+    const void* grad_y;
+    const void* expert_out;
+    int64_t expert_out_rows;
+    const int32_t* row_of;
+    const float* topk_weights;
+    void* grad_expert_out;
+    float* grad_topk_weights;
+    uint32_t* status;
+};
+cudaError_t launch_combine_backward(const CombineBackwardParams& p, cudaStream_t stream);
 
 struct LowLatencyDispatchParams {
     int64_t T;

@@ -224,6 +224,41 @@ EP_API ep_status ep_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk
                      void* y, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward of dispatch ("deepseek-ai/DeepEP" (agentlenshq.com), section
+ * "典型工作流程": combine or the backward helpers reduce results back).  Each
+ * receive row is a copy of its token, so the gradient of x is the plain sum of
+ * the gradients of the token's rows:
+ *   grad_x[t, i] = bf16_rne( ((+0.0f + g[row_of[t,0], i]) + g[row_of[t,1], i]) + ... )
+ * over valid slots in k order (fp32 adds), g = grad_recv_x BF16 [grad_recv_rows, H];
+ * and, if both pointers are given (else both NULL),
+ *   grad_topk_weights[t, k] = grad_recv_topk_weights[row_of[t, k]] (0 for masked slots).
+ * grad_x: BF16 [T, H].  Only handle->row_of is read.
+ */
+EP_API ep_status ep_dispatch_backward(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                      const void* grad_recv_x, int64_t grad_recv_rows,
+                                      const ep_layout* handle, const float* grad_recv_topk_weights,
+                                      void* grad_x, float* grad_topk_weights, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
+/*
+ * Backward of combine (y[t] = sum_k w[t,k] * expert_out[row_of[t,k]]):
+ *   grad_expert_out[row_of[t,k], i] = bf16_rne( w[t,k] * float(grad_y[t, i]) )  (fp32 multiply)
+ *   grad_topk_weights[t, k] = float( sum_i (double)grad_y[t,i] * (double)expert_out[row,i] ),
+ *                             0 for masked slots.
+ * BF16 products are exact in fp32 and the sum runs in fp64, which is exact (so
+ * order-independent) while the products span fewer than 37 binades.  Rows that
+ * no slot points at are not written; each row must be named by at most one slot
+ * (true of every layout this library produces).  grad_y, expert_out,
+ * grad_expert_out: BF16; grad_topk_weights: fp32 [T, K].
+ */
+EP_API ep_status ep_combine_backward(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                     const void* grad_y, const void* expert_out,
+                                     int64_t expert_out_rows, const ep_layout* handle,
+                                     const float* topk_weights, void* grad_expert_out,
+                                     float* grad_topk_weights, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
  * Low-latency dispatch (deepseek.csdn.net/67bd3eb22e30c863900615cc,
  * "推理解码阶段的应用").  One fused kernel: layout, FP8 quantisation and
  * scatter into the padded tensors

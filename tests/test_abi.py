@@ -168,3 +168,24 @@ def test_read_status_and_probe_argument_checks(ep):
     assert L.ep_read_status(_Fake.P, 16, None, ctypes.byref(bits)) == 1
     assert L.ep_debug_wait_probe(1000, None, 4096, None) == 1
     assert L.ep_workspace_init(None, 4096, None) == 1
+
+
+def test_backward_host_checks(ep):
+    f = _Fake.P
+    lay = _layout_struct(ep)
+    L = ep.lib
+    # dispatch backward: both weight-gradient pointers or neither
+    assert L.ep_dispatch_backward(4, 128, 2, f, 8, ctypes.byref(lay), f, f, None, f, 4096, None) == 1
+    assert L.ep_dispatch_backward(4, 124, 2, f, 8, ctypes.byref(lay), None, f, None, f, 4096, None) == 2
+    assert L.ep_dispatch_backward(4, 128, 33, f, 8, ctypes.byref(lay), None, f, None, f, 4096, None) == 2
+    assert L.ep_dispatch_backward(4, 128, 2, f, 8, ctypes.byref(lay), None, f + 8, None, f, 4096,
+                                  None) == 1
+    assert L.ep_dispatch_backward(0, 128, 2, None, 0, ctypes.byref(lay), None, None, None, f, 4096,
+                                  None) == 0
+    # combine backward
+    assert L.ep_combine_backward(4, 128, 2, f, f, 8, ctypes.byref(lay), None, f, f, f, 4096, None) == 1
+    assert L.ep_combine_backward(4, 128, 2, f, f, -1, ctypes.byref(lay), f, f, f, f, 4096, None) == 2
+    assert L.ep_combine_backward(4, 128, 2, f, f + 4, 8, ctypes.byref(lay), f, f, f, f, 4096,
+                                 None) == 1
+    assert L.ep_combine_backward(0, 128, 2, None, None, 0, ctypes.byref(lay), None, None, None, f,
+                                 4096, None) == 0
