@@ -372,6 +372,59 @@ def time_low_latency(ep, w, dev, reps=200, per_graph=20):
     return out
 
 
+def time_backward(ep, runner, steps):
+    """Backward pair on the runner's workload: ep_dispatch_backward (row gradients ->
+    grad_x, weight-gradient gather) and ep_combine_backward (grad_y -> expert-row
+    gradients and weight gradients), each captured as a CUDA graph, back to back."""
+    import torch
+
+    T, H, K, R = runner.T, runner.H, runner.K, runner.R
+    dev = runner.x.device
+    g_rows = runner.eo  # any BF16 [rows, H] buffer serves as the row gradients
+    grw = torch.randn(max(R, 1), device=dev)
+    gx = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    gw1 = torch.empty((T, K), dtype=torch.float32, device=dev)
+    gy = torch.randn((T, H), device=dev).to(torch.bfloat16)
+    geo = torch.empty_like(runner.eo)
+    gw2 = torch.empty((T, K), dtype=torch.float32, device=dev)
+
+    def dbwd():
+        ep.ep_dispatch_backward(g_rows, runner.lay, gx, runner.ws, grw, gw1)
+
+    def cbwd():
+        ep.ep_combine_backward(gy, runner.eo, runner.lay, runner.wts, geo, gw2, runner.ws)
+
+    out = {}
+    bytes_d = R * H * 2 + T * H * 2 + T * K * 4 + R * 4 + T * K * 4
+    bytes_c = T * H * 2 + R * H * 2 * 2 + T * K * 8 + T * K * 4
+    for name, fn, nbytes in (("dispatch_backward", dbwd, bytes_d),
+                             ("combine_backward", cbwd, bytes_c)):
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            fn()
+            fn()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        evs[0].record()
+        for i in range(steps):
+            g.replay()
+            evs[i + 1].record()
+        torch.cuda.synchronize()
+        us = statistics.mean(evs[i].elapsed_time(evs[i + 1]) for i in range(steps)) * 1e3
+        out[name] = {"us": round(us, 2), "bytes": nbytes, "gbs": round(nbytes / (us * 1e-6) / 1e9, 1)}
+    if ep.ep_read_status(runner.ws) != 0:
+        raise RuntimeError("device status set in the backward run")
+    return out
+
+
 def time_e2e(ep, runner, steps):
     """The same step through the public API with host buffers, pipelined the way a
     serving loop would run it: every step copies its inputs (x, topk_idx,
@@ -592,6 +645,11 @@ def run_ours(args):
         result["cpu_baseline"] = cpu_baseline(w)
     if not args.no_extra:
         extra = {}
+        try:
+            extra["backward"] = time_backward(ep, runner, args.extra_steps)
+            extra["backward"]["workload"] = args.workload
+        except Exception as exc:  # report, do not hide
+            extra["backward"] = {"error": repr(exc)}
         try:
             extra["ll"] = time_low_latency(ep, make_workload("ll", seed=args.seed), dev)
         except Exception as exc:  # report, do not hide

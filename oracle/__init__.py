@@ -65,6 +65,13 @@ def lib() -> ctypes.CDLL:
         L.oracle_dispatch_backward.restype = ctypes.c_uint32
         L.oracle_combine_backward.argtypes = [_i64, _i64, _i32, _p, _p, _i64, _p, _p, _p, _p]
         L.oracle_combine_backward.restype = ctypes.c_uint32
+        L.oracle_dispatch_dedup.argtypes = [_i64, _i64, _i32, _i32, _i32, _i32, _p, _p, _p, _p,
+                                            _p, _p, _p, _p, _p, _p, _p, _p]
+        L.oracle_dispatch_dedup.restype = ctypes.c_uint32
+        L.oracle_partition_identity.argtypes = [_i64, _i64, _i32, _i32, _p, _p, _p, _p, _p]
+        L.oracle_partition_identity.restype = None
+        L.oracle_combine_dedup.argtypes = [_i64, _i64, _i32, _p, _i64, _p, _p]
+        L.oracle_combine_dedup.restype = ctypes.c_uint32
         _lib = L
     return _lib
 
@@ -285,3 +292,65 @@ def combine_backward(grad_y: np.ndarray, expert_out: np.ndarray, row_of: np.ndar
     st = lib().oracle_combine_backward(T, H, K, _ptr(gy), _ptr(eo_p), rows, _ptr(ro), _ptr(w),
                                        _ptr(geo), _ptr(gw))
     return geo[:rows], gw, int(st)
+
+
+# ---------------------------------------------------- deduplicated dispatch --
+
+def dispatch_dedup(x: np.ndarray, topk_idx: np.ndarray, topk_weights: np.ndarray,
+                   num_experts: int, num_partitions: int, quant: str = "fp8"):
+    """One row per (token, partition).  Returns prow_of [T, P], part_count [P],
+    part_offset [P+1], src_tok [rows], num_rows, recv_x, recv_scales,
+    recv_topk_idx [rows, K], recv_topk_weights [rows, K], status."""
+    x = _c(x, np.uint16)
+    idx = _c(topk_idx, np.int64)
+    w = _c(topk_weights, np.float32)
+    T, H = x.shape
+    K = idx.shape[1]
+    P = num_partitions
+    qm = 1 if quant == "fp8" else 0
+    cap = max(T * min(P, K), 1)
+    out = dict(prow_of=np.empty((T, P), np.int32), part_count=np.empty(P, np.int32),
+               part_offset=np.empty(P + 1, np.int32), src_tok=np.full(cap, -1, np.int32),
+               num_rows=np.zeros(1, np.int32),
+               recv_x=np.zeros((cap, H), np.uint8 if qm else np.uint16),
+               recv_scales=np.zeros((cap, max(H // 128, 1)), np.float32),
+               recv_topk_idx=np.zeros((cap, K), np.int32),
+               recv_topk_weights=np.zeros((cap, K), np.float32))
+    st = lib().oracle_dispatch_dedup(
+        T, H, K, num_experts, P, qm, _ptr(x), _ptr(idx), _ptr(w), _ptr(out["prow_of"]),
+        _ptr(out["part_count"]), _ptr(out["part_offset"]), _ptr(out["src_tok"]),
+        _ptr(out["num_rows"]), _ptr(out["recv_x"]), _ptr(out["recv_scales"]),
+        _ptr(out["recv_topk_idx"]), _ptr(out["recv_topk_weights"]))
+    R = int(out["num_rows"][0])
+    for k in ("src_tok", "recv_x", "recv_topk_idx", "recv_topk_weights"):
+        out[k] = out[k][:R]
+    out["recv_scales"] = out["recv_scales"][:R, : H // 128]
+    out["status"] = int(st)
+    return out
+
+
+def partition_identity(recv_x, recv_scales, recv_topk_idx, recv_topk_weights, quant="fp8"):
+    """Partition-local stand-in expert output for the deduplicated path."""
+    R, H = recv_x.shape
+    K = recv_topk_idx.shape[1]
+    qm = 1 if quant == "fp8" else 0
+    rx = _c(recv_x, np.uint8 if qm else np.uint16)
+    rs = _c(recv_scales if recv_scales is not None else np.zeros((R, 1), np.float32), np.float32)
+    ri = _c(recv_topk_idx, np.int32)
+    rw = _c(recv_topk_weights, np.float32)
+    out = np.empty((R, H), np.uint16)
+    if R:
+        lib().oracle_partition_identity(R, H, K, qm, _ptr(rx), _ptr(rs), _ptr(ri), _ptr(rw),
+                                        _ptr(out))
+    return out
+
+
+def combine_dedup(part_out: np.ndarray, prow_of: np.ndarray):
+    po = _c(part_out, np.uint16)
+    rows, H = po.shape
+    pr = _c(prow_of, np.int32)
+    T, P = pr.shape
+    y = np.empty((T, H), np.uint16)
+    po_p = po if rows else np.zeros((1, H), np.uint16)
+    st = lib().oracle_combine_dedup(T, H, P, _ptr(po_p), rows, _ptr(pr), _ptr(y))
+    return y, int(st)

@@ -413,3 +413,135 @@ uint32_t oracle_combine_backward(int64_t T, int64_t H, int32_t K, const uint16_t
     }
     return status;
 }
+
+/* ------------------------------------------------- deduplicated dispatch -- */
+
+/* Dispatch with one receive row per (token, partition) instead of one per
+ * (token, expert): DeepEP's normal kernels send a token once to each rank that
+ * holds any of its experts, with the list of that rank's experts and weights
+ * (deepseek.csdn.net/67bd3eb22e30c863900615cc, section "使用示例": dispatch
+ * returns recv_x, recv_topk_idx, recv_topk_weights; "DeepSeek 开源周第二弹：DeepEP",
+ * section "DeepEP 的常规内核和低延迟内核": top-4 groups of top-8 experts).
+ * Partitions stand for the ranks: partition p owns experts [p*E/P, (p+1)*E/P).
+ *   prow_of[t][p]  row of (t, p): partition-major, token ascending; -1 if token t
+ *                  names no expert of partition p
+ *   part_count[p], part_offset[P+1], src_tok[row] = t, *num_rows
+ *   recv_x[row]    the token's row (E4M3 + 1x128 scales, or BF16 bits)
+ *   recv_topk_idx[row][k]     e - p*E/P if topk_idx[t][k] = e lies in p, else -1
+ *   recv_topk_weights[row][k] topk_weights[t][k] for those k, else 0
+ * Ids outside [-1, E) are skipped and reported. */
+uint32_t oracle_dispatch_dedup(int64_t T, int64_t H, int32_t K, int32_t E, int32_t P,
+                               int32_t quant, const uint16_t* x, const int64_t* topk_idx,
+                               const float* topk_weights, int32_t* prow_of, int32_t* part_count,
+                               int32_t* part_offset, int32_t* src_tok, int32_t* num_rows,
+                               uint8_t* recv_x, float* recv_scales, int32_t* recv_topk_idx,
+                               float* recv_topk_weights) {
+    uint32_t status = 0;
+    int32_t epp = E / P;
+    int64_t nb = H / 128;
+    uint8_t* in_part = (uint8_t*)calloc((size_t)(T * P > 0 ? T * P : 1), 1);
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t k = 0; k < K; ++k) {
+            int64_t e = topk_idx[t * K + k];
+            if (e == -1) continue;
+            if (e < 0 || e >= E) {
+                status |= ORACLE_INDEX_RANGE;
+                continue;
+            }
+            in_part[t * P + e / epp] = 1;
+        }
+    }
+    for (int32_t p = 0; p < P; ++p) {
+        part_count[p] = 0;
+        for (int64_t t = 0; t < T; ++t) part_count[p] += in_part[t * P + p];
+    }
+    part_offset[0] = 0;
+    for (int32_t p = 0; p < P; ++p) part_offset[p + 1] = part_offset[p] + part_count[p];
+    *num_rows = part_offset[P];
+    uint8_t* q = (uint8_t*)malloc((size_t)H);
+    float* s = (float*)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    for (int32_t p = 0; p < P; ++p) {
+        int32_t row = part_offset[p];
+        for (int64_t t = 0; t < T; ++t) {
+            if (!in_part[t * P + p]) {
+                prow_of[t * P + p] = -1;
+                continue;
+            }
+            prow_of[t * P + p] = row;
+            src_tok[row] = (int32_t)t;
+            if (quant == 1) {
+                oracle_quantize_row(H, x + t * H, q, s);
+                memcpy(recv_x + (int64_t)row * H, q, (size_t)H);
+                memcpy(recv_scales + (int64_t)row * nb, s, sizeof(float) * (size_t)nb);
+            } else {
+                memcpy(recv_x + (int64_t)row * H * 2, x + t * H, (size_t)H * 2);
+            }
+            for (int32_t k = 0; k < K; ++k) {
+                int64_t e = topk_idx[t * K + k];
+                int in = e >= 0 && e < E && e / epp == p;
+                recv_topk_idx[(int64_t)row * K + k] = in ? (int32_t)(e - (int64_t)p * epp) : -1;
+                recv_topk_weights[(int64_t)row * K + k] = in ? topk_weights[t * K + k] : 0.0f;
+            }
+            row += 1;
+        }
+    }
+    free(in_part);
+    free(q);
+    free(s);
+    return status;
+}
+
+/* Stand-in for a partition's experts in tests and benchmarks of the
+ * deduplicated path: every expert returns its input, and the partition reduces
+ * its experts' outputs with their weights before sending the row back, so
+ *   out[row][i] = bf16_rne( fmaf chain over k with recv_topk_idx[row][k] >= 0 of
+ *                 recv_topk_weights[row][k] * v[i] ),  v = the dequantised row
+ *   (q * scale in one binary32 multiply, or the BF16 row). */
+void oracle_partition_identity(int64_t rows, int64_t H, int32_t K, int32_t quant,
+                               const uint8_t* recv_x, const float* recv_scales,
+                               const int32_t* recv_topk_idx, const float* recv_topk_weights,
+                               uint16_t* out) {
+    int64_t nb = H / 128;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t i = 0; i < H; ++i) {
+            float v;
+            if (quant == 1) {
+                v = oracle_e4m3_to_f32(recv_x[r * H + i]) * recv_scales[r * nb + i / 128];
+            } else {
+                uint16_t b;
+                memcpy(&b, recv_x + (r * H + i) * 2, 2);
+                v = oracle_bf16_to_f32(b);
+            }
+            float acc = 0.0f;
+            for (int32_t k = 0; k < K; ++k) {
+                if (recv_topk_idx[r * K + k] < 0) continue;
+                acc = fmaf(recv_topk_weights[r * K + k], v, acc);
+            }
+            out[r * H + i] = oracle_bf16_from_f32(acc);
+        }
+    }
+}
+
+/* Combine of the deduplicated path: each partition returns one already-weighted
+ * row per token, so y[t][i] = bf16_rne( +0.0f + out[prow_of[t][0]][i] + ... ) over
+ * the partitions the token touched, in partition order (binary32 adds). */
+uint32_t oracle_combine_dedup(int64_t T, int64_t H, int32_t P, const uint16_t* part_out,
+                              int64_t rows, const int32_t* prow_of, uint16_t* y) {
+    uint32_t status = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t i = 0; i < H; ++i) {
+            float acc = 0.0f;
+            for (int32_t p = 0; p < P; ++p) {
+                int32_t row = prow_of[t * P + p];
+                if (row < 0) continue;
+                if ((int64_t)row >= rows) {
+                    status |= ORACLE_INDEX_RANGE;
+                    continue;
+                }
+                acc = acc + oracle_bf16_to_f32(part_out[(int64_t)row * H + i]);
+            }
+            y[t * H + i] = oracle_bf16_from_f32(acc);
+        }
+    }
+    return status;
+}
