@@ -26,6 +26,7 @@ EXPORTED = (
     "ep_read_status", "ep_get_dispatch_layout", "ep_dispatch", "ep_combine",
     "ep_low_latency_dispatch", "ep_low_latency_combine", "ep_debug_wait_probe",
     "ep_get_dispatch_layout_static", "ep_dispatch_backward", "ep_combine_backward",
+    "ep_dispatch_dedup", "ep_combine_dedup",
 )
 
 
@@ -82,6 +83,12 @@ def _load() -> ctypes.CDLL:
     L.ep_combine_backward.argtypes = [i64, i64, i32, vp, vp, i64, ctypes.POINTER(ep_layout), vp, vp,
                                       vp, vp, sz, vp]
     L.ep_combine_backward.restype = st
+    L.ep_dispatch_dedup.argtypes = [i64, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp,
+                                    ctypes.POINTER(ep_layout), vp, sz, vp]
+    L.ep_dispatch_dedup.restype = st
+    L.ep_combine_dedup.argtypes = [i64, i64, i32, vp, i64, ctypes.POINTER(ep_layout), vp, vp, sz,
+                                   vp]
+    L.ep_combine_dedup.restype = st
     return L
 
 
@@ -352,4 +359,54 @@ def ep_combine_backward(grad_y: torch.Tensor, expert_out: torch.Tensor, handle: 
     _check("ep_combine_backward", lib.ep_combine_backward(
         T, H, K, grad_y.data_ptr(), expert_out.data_ptr(), rows, ctypes.byref(c),
         topk_weights.data_ptr(), grad_expert_out.data_ptr(), grad_topk_weights.data_ptr(),
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_dispatch_dedup(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
+                      num_experts: int, num_partitions: int, quant: int, recv_x: torch.Tensor,
+                      recv_scales: Optional[torch.Tensor], recv_topk_idx: torch.Tensor,
+                      recv_topk_weights: torch.Tensor, handle: Layout, workspace: torch.Tensor,
+                      stream=None) -> None:
+    """Deduplicated dispatch; handle = Layout.empty(T, P, P, P) (partition-sized)."""
+    _need(x, "x", torch.bfloat16)
+    T, H = x.shape
+    K = topk_idx.shape[1]
+    P = num_partitions
+    rows = max(T * min(P, K), 1)
+    _need(topk_idx, "topk_idx", torch.int64, shape=(T, K))
+    _need(topk_weights, "topk_weights", torch.float32, shape=(T, K))
+    if quant == EP_QUANT_FP8_E4M3_1X128:
+        _need(recv_x, "recv_x", (torch.uint8, torch.float8_e4m3fn), numel_at_least=rows * H)
+        _need(recv_scales, "recv_scales", torch.float32, numel_at_least=rows * (H // 128))
+    else:
+        _need(recv_x, "recv_x", torch.bfloat16, numel_at_least=rows * H)
+    _need(recv_topk_idx, "recv_topk_idx", torch.int32, numel_at_least=rows * K)
+    _need(recv_topk_weights, "recv_topk_weights", torch.float32, numel_at_least=rows * K)
+    _need(handle.row_of, "handle.row_of", torch.int32, shape=(T, P))
+    _need(handle.src_of, "handle.src_of", torch.int32, numel_at_least=rows)
+    _need(handle.num_tokens_per_expert, "handle.num_tokens_per_expert", torch.int32, shape=(P,))
+    _need(handle.expert_offset, "handle.expert_offset", torch.int32, shape=(P + 1,))
+    _need(handle.is_token_in_partition, "handle.is_token_in_partition", torch.uint8,
+          shape=(T, P))
+    _need(workspace, "workspace", torch.uint8)
+    c = handle.c()
+    _check("ep_dispatch_dedup", lib.ep_dispatch_dedup(
+        T, H, K, num_experts, P, quant, x.data_ptr(), topk_idx.data_ptr(),
+        topk_weights.data_ptr(), recv_x.data_ptr(), _ptr(recv_scales), recv_topk_idx.data_ptr(),
+        recv_topk_weights.data_ptr(), ctypes.byref(c), workspace.data_ptr(), workspace.numel(),
+        _stream(stream)))
+
+
+def ep_combine_dedup(partition_out: torch.Tensor, handle: Layout, y: torch.Tensor,
+                     workspace: torch.Tensor, stream=None) -> None:
+    _need(partition_out, "partition_out", torch.bfloat16)
+    H = partition_out.shape[-1]
+    rows = partition_out.numel() // H if H else 0
+    T, P = handle.row_of.shape
+    _need(handle.row_of, "handle.row_of", torch.int32)
+    _need(y, "y", torch.bfloat16, shape=(T, H))
+    _need(workspace, "workspace", torch.uint8)
+    c = ep_layout(row_of=handle.row_of.data_ptr())
+    _check("ep_combine_dedup", lib.ep_combine_dedup(
+        T, H, P, partition_out.data_ptr(), rows, ctypes.byref(c), y.data_ptr(),
         workspace.data_ptr(), workspace.numel(), _stream(stream)))

@@ -64,6 +64,33 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, ui
     return true;
 }
 
+// Metadata of one token's receive rows, written by the storer warp.  Per-expert
+// rows: lane k owns slot k and writes the local id and weight of its row.
+// Deduplicated rows (one per partition): lane p owns partition p's row and writes
+// its K-entry lists, reading every slot's id and weight from the id lanes by
+// shuffle (all lanes take part in the shuffles).
+__device__ __forceinline__ void write_row_metadata(const DispatchParams& p, int lane, int row,
+                                                   int64_t e, float wt) {
+    const int64_t epp = p.experts_per_partition;
+    if (!p.dedup) {
+        if (lane < p.slots && row >= 0) {
+            p.recv_topk_idx[row] = static_cast<int32_t>(e - (e / epp) * epp);
+            p.recv_topk_weights[row] = wt;
+        }
+        return;
+    }
+    for (int k = 0; k < p.K; ++k) {
+        const int64_t ek = __shfl_sync(0xffffffffu, e, k);
+        const float wk = __shfl_sync(0xffffffffu, wt, k);
+        if (lane < p.slots && row >= 0) {
+            const bool in = ek >= 0 && ek < p.num_experts && ek / epp == lane;
+            p.recv_topk_idx[static_cast<int64_t>(row) * p.K + k] =
+                in ? static_cast<int32_t>(ek - lane * epp) : -1;
+            p.recv_topk_weights[static_cast<int64_t>(row) * p.K + k] = in ? wk : 0.0f;
+        }
+    }
+}
+
 // Warp-specialised pipeline, one CTA = 1 loader warp + nq quantiser warps + 1 storer
 // warp, coupled only by mbarriers (no CTA-wide barrier after set-up):
 //   loader (warp 0, lane 0): bulk-loads token rows into the input ring
@@ -160,15 +187,18 @@ __global__ void __launch_bounds__(352) dispatch_fp8_kernel(DispatchParams p) {
         // ---------------------------------------------------------------- storer
         pdl_wait();  // row_of from the layout kernel is complete and visible
         uint8_t* recv_x = static_cast<uint8_t*>(p.recv_x);
-        const bool slot_lane = lane < K;
+        const int S = p.slots;
+        const bool slot_lane = lane < S;  // lane s stores slot s's row
+        const bool id_lane = lane < K;    // lane k holds routing entry k
         int nrow = -1;
         int64_t nexp = -1;
         float nwt = 0.0f;
-        if (slot_lane && n_mine > 0) {
-            const int64_t g = first * K + lane;
-            nrow = p.row_of[g];
-            nexp = p.topk_idx[g];
-            nwt = p.topk_weights[g];
+        if (n_mine > 0) {
+            if (slot_lane) nrow = p.row_of[first * S + lane];
+            if (id_lane) {
+                nexp = p.topk_idx[first * K + lane];
+                nwt = p.topk_weights[first * K + lane];
+            }
         }
         for (int64_t i = 0; i < n_mine; ++i) {
             const int64_t t = first + i * G;
@@ -176,11 +206,12 @@ __global__ void __launch_bounds__(352) dispatch_fp8_kernel(DispatchParams p) {
             const int row = nrow;
             const int64_t e = nexp;
             const float wt = nwt;
-            if (slot_lane && i + 1 < n_mine) {
-                const int64_t g = (t + G) * K + lane;
-                nrow = p.row_of[g];
-                nexp = p.topk_idx[g];
-                nwt = p.topk_weights[g];
+            if (i + 1 < n_mine) {
+                if (slot_lane) nrow = p.row_of[(t + G) * S + lane];
+                if (id_lane) {
+                    nexp = p.topk_idx[(t + G) * K + lane];
+                    nwt = p.topk_weights[(t + G) * K + lane];
+                }
             }
             if (!wait_or_abort(&out_full[o], static_cast<uint32_t>((i / kFp8OutStages) & 1),
                                p.timeout_ns, abort_flag))
@@ -193,16 +224,14 @@ __global__ void __launch_bounds__(352) dispatch_fp8_kernel(DispatchParams p) {
                     if (scale_bulk)
                         bulk_store(p.recv_scales + static_cast<int64_t>(row) * nb, out_s,
                                    static_cast<uint32_t>(nb) * 4u);
-                    const int64_t epp = p.experts_per_partition;
-                    p.recv_topk_idx[row] = static_cast<int32_t>(e - (e / epp) * epp);
-                    p.recv_topk_weights[row] = wt;
                 }
                 bulk_commit();
                 rows_sm[o * 32 + lane] = row;
             }
+            write_row_metadata(p, lane, row, e, wt);
             if (!scale_bulk) {
                 __syncwarp();
-                for (int idx = lane; idx < K * nb; idx += 32) {
+                for (int idx = lane; idx < S * nb; idx += 32) {
                     const int k = idx / nb, b = idx - k * nb;
                     const int r = rows_sm[o * 32 + k];
                     if (r >= 0) p.recv_scales[static_cast<int64_t>(r) * nb + b] = out_s[b];
@@ -275,15 +304,18 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
         // ---------------------------------------------------------------- storer
         pdl_wait();  // row_of from the layout kernel is complete and visible
         uint8_t* recv_x = static_cast<uint8_t*>(p.recv_x);
-        const bool slot_lane = lane < K;
+        const int S = p.slots;
+        const bool slot_lane = lane < S;  // lane s stores slot s's row
+        const bool id_lane = lane < K;    // lane k holds routing entry k
         int nrow = -1;
         int64_t nexp = -1;
         float nwt = 0.0f;
-        if (slot_lane && n_mine > 0) {
-            const int64_t g = first * K + lane;
-            nrow = p.row_of[g];
-            nexp = p.topk_idx[g];
-            nwt = p.topk_weights[g];
+        if (n_mine > 0) {
+            if (slot_lane) nrow = p.row_of[first * S + lane];
+            if (id_lane) {
+                nexp = p.topk_idx[first * K + lane];
+                nwt = p.topk_weights[first * K + lane];
+            }
         }
         for (int64_t i = 0; i < n_mine; ++i) {
             const int64_t t = first + i * G;
@@ -291,26 +323,24 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
             const int row = nrow;
             const int64_t e = nexp;
             const float wt = nwt;
-            if (slot_lane && i + 1 < n_mine) {
-                const int64_t g = (t + G) * K + lane;
-                nrow = p.row_of[g];
-                nexp = p.topk_idx[g];
-                nwt = p.topk_weights[g];
+            if (i + 1 < n_mine) {
+                if (slot_lane) nrow = p.row_of[(t + G) * S + lane];
+                if (id_lane) {
+                    nexp = p.topk_idx[(t + G) * K + lane];
+                    nwt = p.topk_weights[(t + G) * K + lane];
+                }
             }
             if (!wait_or_abort(&full[s], static_cast<uint32_t>((i / kBf16Stages) & 1), p.timeout_ns,
                                abort_flag))
                 break;
             if (slot_lane) {
-                if (row >= 0) {
+                if (row >= 0)
                     bulk_store(recv_x + static_cast<int64_t>(row) * row_bytes, sm + s * row_bytes,
                                row_bytes);
-                    const int64_t epp = p.experts_per_partition;
-                    p.recv_topk_idx[row] = static_cast<int32_t>(e - (e / epp) * epp);
-                    p.recv_topk_weights[row] = wt;
-                }
                 bulk_commit();
-                bulk_wait_read<1>();  // the previous token's stores have read their stage
             }
+            write_row_metadata(p, lane, row, e, wt);
+            if (slot_lane) bulk_wait_read<1>();  // the previous token's stores have read their stage
             __syncwarp();
             if (lane == 0 && i >= 1) mbar_arrive(&empty[(i - 1) % kBf16Stages]);
         }

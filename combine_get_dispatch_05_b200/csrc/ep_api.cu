@@ -162,6 +162,9 @@ ep_status ep_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk, int3
     p.T = num_tokens;
     p.H = hidden;
     p.K = num_topk;
+    p.slots = num_topk;
+    p.dedup = 0;
+    p.num_experts = num_experts;
     p.experts_per_partition = num_experts / num_partitions;
     p.x = x;
     p.topk_idx = topk_idx;
@@ -196,6 +199,86 @@ ep_status ep_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk, const
     p.expert_out_rows = expert_out_rows;
     p.row_of = handle->row_of;
     p.topk_weights = topk_weights;
+    p.y = y;
+    p.grad_recv_w = nullptr;
+    p.grad_w = nullptr;
+    p.status = carve_workspace(workspace, 0, 1).status;
+    return cuda_status(launch_combine(p, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_dispatch_dedup(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                            int32_t num_experts, int32_t num_partitions, int32_t quant,
+                            const void* x, const int64_t* topk_idx, const float* topk_weights,
+                            void* recv_x, float* recv_scales, int32_t* recv_topk_idx,
+                            float* recv_topk_weights, const ep_layout* handle, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    if (quant != EP_QUANT_NONE && quant != EP_QUANT_FP8_E4M3_1X128) return EP_ERR_INVALID_ARG;
+    const bool fp8 = quant == EP_QUANT_FP8_E4M3_1X128;
+    ep_status st = check_routing(num_tokens, num_topk, num_experts, num_partitions);
+    if (st != EP_OK) return st;
+    if (num_partitions > 32) return EP_ERR_SHAPE;  // one storer lane per partition
+    if (num_tokens * static_cast<int64_t>(num_partitions) >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    if ((st = check_hidden(hidden, fp8)) != EP_OK) return st;
+    if ((st = check_layout_ptrs(handle, num_tokens)) != EP_OK) return st;
+    if (!workspace || !aligned16(workspace)) return EP_ERR_INVALID_ARG;
+    if (num_tokens > 0) {
+        if (!x || !topk_idx || !topk_weights || !recv_x || !recv_topk_idx || !recv_topk_weights)
+            return EP_ERR_INVALID_ARG;
+        if (fp8 && !recv_scales) return EP_ERR_INVALID_ARG;
+        if (!aligned16(x) || !aligned16(recv_x) || (fp8 && !aligned16(recv_scales)))
+            return EP_ERR_INVALID_ARG;
+    }
+    if (workspace_bytes < ep_workspace_bytes(num_tokens, num_experts, num_partitions))
+        return EP_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Workspace ws = carve_workspace(workspace, num_tokens, num_partitions);
+    cudaError_t err = launch_layout(num_tokens, num_topk, num_experts, num_partitions, topk_idx,
+                                    *handle, ws, s, /*by_partition=*/true);
+    if (err != cudaSuccess) return EP_ERR_CUDA;
+    DispatchParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = num_topk;
+    p.slots = num_partitions;
+    p.dedup = 1;
+    p.num_experts = num_experts;
+    p.experts_per_partition = num_experts / num_partitions;
+    p.x = x;
+    p.topk_idx = topk_idx;
+    p.topk_weights = topk_weights;
+    p.row_of = handle->row_of;
+    p.recv_x = recv_x;
+    p.recv_scales = recv_scales;
+    p.recv_topk_idx = recv_topk_idx;
+    p.recv_topk_weights = recv_topk_weights;
+    p.status = ws.status;
+    p.timeout_ns = kDefaultTimeoutNs;
+    return cuda_status(fp8 ? launch_dispatch_fp8(p, s) : launch_dispatch_bf16(p, s));
+}
+
+ep_status ep_combine_dedup(int64_t num_tokens, int64_t hidden, int32_t num_partitions,
+                           const void* partition_out, int64_t partition_out_rows,
+                           const ep_layout* handle, void* y, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    if (num_tokens < 0 || num_partitions < 1 || num_partitions > 32 || partition_out_rows < 0)
+        return EP_ERR_SHAPE;
+    if (num_tokens * static_cast<int64_t>(num_partitions) >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    ep_status st = check_hidden(hidden, false);
+    if (st != EP_OK) return st;
+    if (!handle || !workspace || !aligned16(workspace) || workspace_bytes < kWsHeader)
+        return EP_ERR_INVALID_ARG;
+    if (num_tokens == 0) return EP_OK;
+    if (!handle->row_of || !y || (!partition_out && partition_out_rows > 0))
+        return EP_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(partition_out)) return EP_ERR_INVALID_ARG;
+    CombineParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = num_partitions;  // slots are partitions
+    p.expert_out = partition_out;
+    p.expert_out_rows = partition_out_rows;
+    p.row_of = handle->row_of;
+    p.topk_weights = nullptr;  // partitions return weighted rows: a plain sum
     p.y = y;
     p.grad_recv_w = nullptr;
     p.grad_w = nullptr;

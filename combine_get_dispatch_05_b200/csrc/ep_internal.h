@@ -31,13 +31,19 @@ Workspace carve_workspace(void* ws, int64_t num_tokens, int32_t num_experts);
 // Launch the (cooperative) layout kernel on `stream`.  It waits for all earlier
 // work in the stream and lets the next kernel start early (programmatic
 // dependent launch).
+// by_partition: the deduplicated layout (one slot per partition, rows
+// partition-major); the layout arrays are then P-sized and row_of is [T, P].
 cudaError_t launch_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int64_t* topk_idx,
-                          const ep_layout& lay, const Workspace& ws, cudaStream_t stream);
+                          const ep_layout& lay, const Workspace& ws, cudaStream_t stream,
+                          bool by_partition = false);
 
 struct DispatchParams {
     int64_t T;
     int64_t H;
-    int32_t K;
+    int32_t K;       // routing ids per token (topk_idx / topk_weights row length)
+    int32_t slots;   // receive rows per token in row_of: K, or P when dedup
+    int32_t dedup;   // 1: a row per (token, partition) with [rows, K] expert lists
+    int32_t num_experts;
     int32_t experts_per_partition;
     const void* x;
     const int64_t* topk_idx;

@@ -39,6 +39,11 @@ struct LayoutArgs {
     int32_t chunk_tokens;  // tokens per CTA, a multiple of 32
     int32_t round_warps;   // warps ranking, each a contiguous run (bounded by the table budget)
     int32_t flags_vec;     // is_token_in_partition is 8-byte aligned and P % 8 == 0
+    // partition mode (deduplicated dispatch): the slots of a token are the P
+    // partitions and the "ids" are partitions (K = E = P, epp = 1 below); the
+    // routing is read as K_src ids per token among E_src experts, epp_src per partition
+    int32_t by_partition;
+    int32_t K_src, E_src, epp_src;
     int32_t parts;         // thread groups splitting the chunks in the cross-chunk sums
     int32_t* chunk_expert;     // [G][E]
     int32_t* chunk_partition;  // [G][P]
@@ -129,11 +134,25 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_kernel(LayoutArgs a)
     }
     for (int p = tid; p < P; p += blockDim.x) phist[p] = 0;
     bool bad = false;
-    for (int j = tid; j < n; j += blockDim.x) {
-        const int64_t e = a.topk_idx[t0 * K + j];
-        const bool ok = e >= 0 && e < E;
-        bad |= (e != -1) && !ok;
-        ent[j] = ok ? static_cast<int>(e) : -1;
+    if (!a.by_partition) {
+        for (int j = tid; j < n; j += blockDim.x) {
+            const int64_t e = a.topk_idx[t0 * K + j];
+            const bool ok = e >= 0 && e < E;
+            bad |= (e != -1) && !ok;
+            ent[j] = ok ? static_cast<int>(e) : -1;
+        }
+    } else {
+        // slot p of token t holds p if the token names any expert of partition p
+        for (int tl = tid; tl < t1 - t0; tl += blockDim.x) {
+            uint64_t mask = 0;
+            for (int k = 0; k < a.K_src; ++k) {
+                const int64_t e = a.topk_idx[(t0 + tl) * a.K_src + k];
+                const bool ok = e >= 0 && e < a.E_src;
+                bad |= (e != -1) && !ok;
+                if (ok) mask |= 1ull << (e / a.epp_src);
+            }
+            for (int p = 0; p < K; ++p) ent[tl * K + p] = ((mask >> p) & 1u) ? p : -1;
+        }
     }
     if (bad) raise_status(a.status, kDevIndexRange);
     __syncthreads();
@@ -331,7 +350,13 @@ Workspace carve_workspace(void* ws, int64_t num_tokens, int32_t num_experts) {
 }
 
 cudaError_t launch_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int64_t* topk_idx,
-                          const ep_layout& lay, const Workspace& ws, cudaStream_t stream) {
+                          const ep_layout& lay, const Workspace& ws, cudaStream_t stream,
+                          bool by_partition) {
+    const int32_t K_src = K, E_src = E, epp_src = E / P;
+    if (by_partition) {  // slots and ids are partitions
+        K = P;
+        E = P;
+    }
     DeviceInfo dev;
     cudaError_t err = device_info(&dev);
     if (err != cudaSuccess) return err;
@@ -354,7 +379,11 @@ cudaError_t launch_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int6
     a.K = K;
     a.E = E;
     a.P = P;
-    a.epp = E / P;
+    a.epp = by_partition ? 1 : E / P;
+    a.by_partition = by_partition ? 1 : 0;
+    a.K_src = K_src;
+    a.E_src = E_src;
+    a.epp_src = epp_src;
     a.chunk_tokens = static_cast<int32_t>(chunk);
     a.round_warps = W;
     a.flags_vec = (P % 8 == 0) && ((reinterpret_cast<uintptr_t>(lay.is_token_in_partition) & 7u) == 0);

@@ -224,6 +224,43 @@ EP_API ep_status ep_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk
                      void* y, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Deduplicated dispatch: one receive row per (token, partition) instead of one per
+ * (token, expert), as DeepEP's normal kernels send a token once to each rank that
+ * holds any of its experts (deepseek.csdn.net/67bd3eb22e30c863900615cc, "使用示例":
+ * recv_topk_idx / recv_topk_weights list each received token's local experts;
+ * "DeepSeek 开源周第二弹：DeepEP", "DeepEP 的常规内核和低延迟内核": top-4 groups of
+ * top-8 experts).  Under top-4-group routing a token reaches at most 4 of 8
+ * partitions, so this writes at most half the rows of ep_dispatch.
+ * The handle's arrays are partition-sized: num_tokens_per_expert[P] = rows per
+ * partition, expert_offset[P+1], row_of[T, P] (-1 where the token names no
+ * expert of the partition), src_of[rows] = t*P + p, num_recv; plus the usual
+ * is_token_in_partition / num_tokens_per_partition.  Rows are partition-major,
+ * token ascending.  Payload as ep_dispatch.  recv_topk_idx / recv_topk_weights
+ * are [rows, K]: entry k of token t's row in partition p holds e - p*E/P and
+ * topk_weights[t, k] if e = topk_idx[t, k] lies in p, else -1 and 0.
+ * Receive buffers: worst case T * min(P, K) rows.  Requires P <= 32.
+ */
+EP_API ep_status ep_dispatch_dedup(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                   int32_t num_experts, int32_t num_partitions, int32_t quant,
+                                   const void* x, const int64_t* topk_idx,
+                                   const float* topk_weights, void* recv_x, float* recv_scales,
+                                   int32_t* recv_topk_idx, float* recv_topk_weights,
+                                   const ep_layout* handle, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/*
+ * Combine of the deduplicated path: each partition returns one row per received
+ * token, already reduced over its own experts with their weights, so
+ *   y[t, i] = bf16_rne( (+0.0f + out[row_of[t,0], i]) + out[row_of[t,1], i] + ... )
+ * over the token's partitions in partition order (fp32 adds).
+ * partition_out: BF16 [partition_out_rows, H]; row_of from ep_dispatch_dedup's handle.
+ */
+EP_API ep_status ep_combine_dedup(int64_t num_tokens, int64_t hidden, int32_t num_partitions,
+                                  const void* partition_out, int64_t partition_out_rows,
+                                  const ep_layout* handle, void* y, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/*
  * Backward of dispatch ("deepseek-ai/DeepEP" (agentlenshq.com), section
  * "典型工作流程": combine or the backward helpers reduce results back).  Each
  * receive row is a copy of its token, so the gradient of x is the plain sum of

@@ -189,3 +189,21 @@ def test_backward_host_checks(ep):
                                  None) == 1
     assert L.ep_combine_backward(0, 128, 2, None, None, 0, ctypes.byref(lay), None, None, None, f,
                                  4096, None) == 0
+
+
+def test_dedup_host_checks(ep):
+    f = _Fake.P
+    lay = _layout_struct(ep)
+    L = ep.lib
+
+    def call(T=16, H=256, K=4, E=64, P=8, quant=1, ws=f):
+        return L.ep_dispatch_dedup(T, H, K, E, P, quant, f, f, f, f, f, f, f, ctypes.byref(lay),
+                                   ws, 1 << 20, None)
+
+    assert call(P=64, E=128) == 2   # one storer lane per partition: P <= 32
+    assert call(E=60) == 2           # E % P
+    assert call(quant=3) == 1
+    assert call(ws=f + 8) == 1
+    assert L.ep_combine_dedup(4, 128, 33, f, 8, ctypes.byref(lay), f, f, 4096, None) == 2
+    assert L.ep_combine_dedup(4, 128, 8, f, 8, None, f, f, 4096, None) == 1
+    assert L.ep_combine_dedup(0, 128, 8, None, 0, ctypes.byref(lay), None, f, 4096, None) == 0

@@ -1,0 +1,132 @@
+"""GPU parity for the deduplicated path (one row per token and partition) against
+the oracle, bit for bit: partition layout, payload and scales, the [rows, K]
+expert lists and weights, and the combine of partition partials."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import oracle  # noqa: E402
+from workloads import make_custom, make_workload, random_bf16  # noqa: E402
+
+from gpu_path import Guarded, bf16_to_u16, dev_u16_as_bf16, new_workspace  # noqa: E402
+
+
+@pytest.fixture(scope="module")
+def ep():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import combine_get_dispatch_05_b200 as m
+    return m
+
+
+def run_dedup(ep, w, quant):
+    T, H, K, E, P = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
+    fp8 = quant == "fp8"
+    rows = max(T * min(P, K), 1)
+    x = dev_u16_as_bf16(w.x)
+    idx = torch.from_numpy(np.ascontiguousarray(w.topk_idx)).cuda()
+    wts = torch.from_numpy(np.ascontiguousarray(w.topk_weights)).cuda()
+    rx = Guarded((rows, H), torch.uint8 if fp8 else torch.bfloat16)
+    rs = Guarded((rows, max(H // 128, 1)), torch.float32) if fp8 else None
+    ri = Guarded((rows, K), torch.int32)
+    rw = Guarded((rows, K), torch.float32)
+    lay = ep.Layout.empty(T, P, P, P, "cuda")
+    ws = new_workspace(ep, T, E, P)
+    ep.ep_dispatch_dedup(x, idx, wts, E, P,
+                         ep.EP_QUANT_FP8_E4M3_1X128 if fp8 else ep.EP_QUANT_NONE,
+                         rx.t, rs.t if fp8 else None, ri.t, rw.t, lay, ws)
+    torch.cuda.synchronize()
+    R = int(lay.num_recv.item())
+    out = dict(R=R, lay=lay, ws=ws,
+               row_of=lay.row_of.cpu().numpy(), count=lay.num_tokens_per_expert.cpu().numpy(),
+               offset=lay.expert_offset.cpu().numpy(), src_of=lay.src_of[:R].cpu().numpy(),
+               itp=lay.is_token_in_partition.cpu().numpy(),
+               ntp=lay.num_tokens_per_partition.cpu().numpy(),
+               recv_topk_idx=ri.t[:R].cpu().numpy(), recv_topk_weights=rw.t[:R].cpu().numpy())
+    if fp8:
+        out["recv_x"] = rx.t[:R].cpu().numpy()
+        out["recv_scales"] = rs.t[:R, : H // 128].cpu().numpy()
+    else:
+        out["recv_x"] = bf16_to_u16(rx.t[:R])
+    out["canaries_ok"] = all(g.canary_ok() for g in [rx, ri, rw] + ([rs] if fp8 else []))
+    return out
+
+
+CASES = [
+    ("normal-300", lambda: make_workload("normal", seed=1, num_tokens=300, hidden=512)),
+    ("skew-700", lambda: make_workload("skew", seed=2, num_tokens=700, hidden=256)),
+    ("bf16-600", lambda: make_workload("bf16", seed=4, num_tokens=600, hidden=136)),
+    ("stress-1000", lambda: make_workload("stress", seed=5, num_tokens=1000, hidden=128)),
+    ("k32-dups", lambda: make_custom(70, 128, 32, 48, 6, seed=8, duplicates=True)),
+    ("masked", lambda: make_custom(513, 640, 6, 64, 16, seed=10, mask_frac=0.3)),
+    ("p1", lambda: make_custom(90, 128, 4, 8, 1, seed=11)),
+    ("e-eq-p", lambda: make_custom(257, 256, 3, 16, 16, seed=12)),
+    ("t1", lambda: make_custom(1, 128, 8, 256, 8, seed=6)),
+]
+
+
+@pytest.mark.parametrize("name,mk", CASES, ids=[c[0] for c in CASES])
+def test_dispatch_dedup_parity(ep, name, mk):
+    w = mk()
+    quant = w.quant if w.hidden % 128 == 0 else "none"
+    got = run_dedup(ep, w, quant)
+    want = oracle.dispatch_dedup(w.x, w.topk_idx, w.topk_weights, w.num_experts,
+                                 w.num_partitions, quant=quant)
+    lay = oracle.layout(w.topk_idx, w.num_experts, w.num_partitions)
+    P = w.num_partitions
+    assert got["R"] == want["num_rows"][0]
+    assert np.array_equal(got["row_of"], want["prow_of"])
+    assert np.array_equal(got["count"], want["part_count"])
+    assert np.array_equal(got["offset"], want["part_offset"])
+    assert np.array_equal(got["src_of"] // P, want["src_tok"])
+    assert np.array_equal(got["itp"], lay["is_token_in_partition"])
+    assert np.array_equal(got["ntp"], lay["num_tokens_per_partition"])
+    assert np.array_equal(got["recv_x"], want["recv_x"])
+    if quant == "fp8":
+        assert np.array_equal(got["recv_scales"].view(np.uint32), want["recv_scales"].view(np.uint32))
+    assert np.array_equal(got["recv_topk_idx"], want["recv_topk_idx"])
+    assert np.array_equal(got["recv_topk_weights"].view(np.uint32),
+                          want["recv_topk_weights"].view(np.uint32))
+    assert got["canaries_ok"]
+    assert ep.ep_read_status(got["ws"]) == 0
+
+
+@pytest.mark.parametrize("name,mk", CASES, ids=[c[0] for c in CASES])
+def test_combine_dedup_parity(ep, name, mk):
+    w = mk()
+    got = run_dedup(ep, w, "none" if w.hidden % 128 else w.quant)
+    want = oracle.dispatch_dedup(w.x, w.topk_idx, w.topk_weights, w.num_experts,
+                                 w.num_partitions, quant="none")
+    R = got["R"]
+    part = random_bf16(np.random.default_rng(3), (R, w.hidden), scale=2.0)
+    y = torch.empty((w.num_tokens, w.hidden), dtype=torch.bfloat16, device="cuda")
+    pd = dev_u16_as_bf16(part) if R else torch.empty((0, w.hidden), dtype=torch.bfloat16,
+                                                     device="cuda")
+    ep.ep_combine_dedup(pd, got["lay"], y, got["ws"])
+    torch.cuda.synchronize()
+    y_ref, st = oracle.combine_dedup(part, want["prow_of"])
+    assert st == 0
+    assert np.array_equal(bf16_to_u16(y), y_ref)
+
+
+def test_dedup_full_size_sampled(ep):
+    w = make_workload("normal", seed=4)
+    got = run_dedup(ep, w, "fp8")
+    lay = oracle.layout(w.topk_idx, 256, 8)
+    assert got["R"] == int(lay["num_tokens_per_partition"].sum())
+    assert got["R"] * 2 <= int(lay["num_recv"][0])
+    rng = np.random.default_rng(2)
+    for t in rng.choice(w.num_tokens, 32, replace=False):
+        q, s = oracle.quantize_row(w.x[t])
+        for p in range(8):
+            r = got["row_of"][t, p]
+            touches = bool(((w.topk_idx[t] // 32) == p).any())
+            assert (r >= 0) == touches
+            if r >= 0:
+                assert np.array_equal(got["recv_x"][r], q)
+                assert np.array_equal(got["recv_scales"][r], s)
+                inside = (w.topk_idx[t] // 32) == p
+                assert np.array_equal(got["recv_topk_idx"][r],
+                                      np.where(inside, w.topk_idx[t] - 32 * p, -1))
