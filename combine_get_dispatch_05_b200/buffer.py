@@ -10,7 +10,12 @@ Shapes of the calls follow the DeepEP pages:
   buffer.low_latency_dispatch(hidden_states, topk_idx, num_max_tokens, num_experts)``
   with a buffer of ``num_max_tokens * hidden * num_experts`` elements;
 * "deepseek-ai/DeepEP" (agentlenshq.com), section "典型工作流程": dispatch, expert
-  GEMM, ``buffer.combine(...)`` reduces the expert outputs back.
+  GEMM, ``buffer.combine(...)`` (or the backward helpers) reduces the expert
+  outputs back.
+
+Besides the per-expert dispatch (one receive row per token and expert), the
+buffer offers the deduplicated dispatch (one row per token and partition, with
+the partition's expert list per row) and the backward pair.
 
 Everything runs on one GPU: the ``num_partitions`` logical partitions stand for
 the EP ranks, so there is no process group.  torch provides device memory and
@@ -163,3 +168,70 @@ class Buffer:
         y = torch.empty((T, H), dtype=torch.bfloat16, device=self.device)
         _lib.ep_low_latency_combine(expert_out, handle, topk_weights, y, self.workspace)
         return y, self._event(), _noop_hook
+
+    # ------------------------------------------------------- deduplicated --
+    def dispatch_dedup(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
+                       use_fp8: bool = True, exact: bool = True):
+        """One receive row per (token, partition).  Returns ``(recv_x, recv_topk_idx
+        [R, K], recv_topk_weights [R, K], handle, event)``; handle.row_of is [T, P]."""
+        T, H = x.shape
+        K = topk_idx.shape[1]
+        P = self.num_partitions
+        self._check_tokens(T)
+        if P > 32:
+            raise ValueError("the deduplicated dispatch supports at most 32 partitions")
+        rows = max(T * min(P, K), 1)
+        dev = self.device
+        handle = Layout.empty(T, P, P, P, dev)
+        ri = torch.empty((rows, K), dtype=torch.int32, device=dev)
+        rw = torch.empty((rows, K), dtype=torch.float32, device=dev)
+        if use_fp8:
+            rq = torch.empty((rows, H), dtype=torch.float8_e4m3fn, device=dev)
+            rs = torch.empty((rows, H // 128), dtype=torch.float32, device=dev)
+            quant = EP_QUANT_FP8_E4M3_1X128
+        else:
+            rq = torch.empty((rows, H), dtype=torch.bfloat16, device=dev)
+            rs = None
+            quant = EP_QUANT_NONE
+        _lib.ep_dispatch_dedup(x, topk_idx, topk_weights, self.num_experts, P, quant, rq, rs, ri,
+                               rw, handle, self.workspace)
+        event = self._event()
+        if exact:
+            R = int(handle.num_recv.item())
+            rq, ri, rw = rq[:R], ri[:R], rw[:R]
+            if rs is not None:
+                rs = rs[:R]
+        return ((rq, rs) if use_fp8 else rq), ri, rw, handle, event
+
+    def combine_dedup(self, partition_out: torch.Tensor, handle: Layout):
+        """Returns ``(y, event)``: y[t] = sum over the token's partitions of their rows."""
+        T = handle.row_of.shape[0]
+        H = partition_out.shape[-1]
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=self.device)
+        _lib.ep_combine_dedup(partition_out, handle, y, self.workspace)
+        return y, self._event()
+
+    # ----------------------------------------------------------- backward --
+    def dispatch_backward(self, grad_recv_x: torch.Tensor, handle: Layout,
+                          grad_recv_topk_weights: Optional[torch.Tensor] = None):
+        """Returns ``(grad_x, grad_topk_weights or None, event)``."""
+        T, K = handle.row_of.shape
+        H = grad_recv_x.shape[-1]
+        gx = torch.empty((T, H), dtype=torch.bfloat16, device=self.device)
+        gw = None
+        if grad_recv_topk_weights is not None:
+            gw = torch.empty((T, K), dtype=torch.float32, device=self.device)
+        _lib.ep_dispatch_backward(grad_recv_x, handle, gx, self.workspace, grad_recv_topk_weights,
+                                  gw)
+        return gx, gw, self._event()
+
+    def combine_backward(self, grad_y: torch.Tensor, expert_out: torch.Tensor, handle: Layout,
+                         topk_weights: torch.Tensor):
+        """Returns ``(grad_expert_out, grad_topk_weights, event)``; rows no slot names
+        are left as zeros."""
+        T, K = handle.row_of.shape
+        geo = torch.zeros_like(expert_out)
+        gw = torch.empty((T, K), dtype=torch.float32, device=self.device)
+        _lib.ep_combine_backward(grad_y, expert_out, handle, topk_weights, geo, gw,
+                                 self.workspace)
+        return geo, gw, self._event()

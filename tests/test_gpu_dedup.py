@@ -130,3 +130,34 @@ def test_dedup_full_size_sampled(ep):
                 inside = (w.topk_idx[t] // 32) == p
                 assert np.array_equal(got["recv_topk_idx"][r],
                                       np.where(inside, w.topk_idx[t] - 32 * p, -1))
+
+
+def test_buffer_dedup_and_backward_methods(ep):
+    w = make_workload("normal", seed=8, num_tokens=200, hidden=256)
+    buf = ep.Buffer(num_experts=256, num_partitions=8, max_tokens=256)
+    x = dev_u16_as_bf16(w.x)
+    idx = torch.from_numpy(w.topk_idx).cuda()
+    wts = torch.from_numpy(w.topk_weights).cuda()
+    (q, s), ri, rw, h, ev = buf.dispatch_dedup(x, idx, wts)
+    want = oracle.dispatch_dedup(w.x, w.topk_idx, w.topk_weights, 256, 8)
+    assert q.shape[0] == want["num_rows"][0]
+    assert np.array_equal(q.view(torch.uint8).cpu().numpy(), want["recv_x"])
+    assert np.array_equal(ri.cpu().numpy(), want["recv_topk_idx"])
+    part = random_bf16(np.random.default_rng(1), (q.shape[0], 256))
+    y, _ = buf.combine_dedup(dev_u16_as_bf16(part), h)
+    assert np.array_equal(bf16_to_u16(y), oracle.combine_dedup(part, want["prow_of"])[0])
+    # backward pair through the buffer on the per-expert layout
+    _, _, _, hk, _ = buf.dispatch(x, idx, wts)
+    R = int(hk.num_recv.item())
+    g = random_bf16(np.random.default_rng(2), (R, 256))
+    gx, gw, _ = buf.dispatch_backward(dev_u16_as_bf16(g), hk)
+    lay = oracle.layout(w.topk_idx, 256, 8)
+    assert gw is None
+    assert np.array_equal(bf16_to_u16(gx), oracle.dispatch_backward(g, lay["row_of"])[0])
+    eo = random_bf16(np.random.default_rng(3), (R, 256))
+    gy = random_bf16(np.random.default_rng(4), (200, 256))
+    geo, gwt, _ = buf.combine_backward(dev_u16_as_bf16(gy), dev_u16_as_bf16(eo), hk, wts)
+    geo_ref, gw_ref, _ = oracle.combine_backward(gy, eo, lay["row_of"], w.topk_weights)
+    assert np.array_equal(bf16_to_u16(geo), geo_ref)
+    assert np.array_equal(gwt.cpu().numpy().view(np.uint32), gw_ref.view(np.uint32))
+    assert buf.read_status() == 0
