@@ -48,6 +48,10 @@ def lib() -> ctypes.CDLL:
         L.oracle_bf16_from_f32_n.restype = None
         L.oracle_block_scale.argtypes = [ctypes.c_float]
         L.oracle_block_scale.restype = ctypes.c_float
+        L.oracle_block_scale_pow2.argtypes = [ctypes.c_float]
+        L.oracle_block_scale_pow2.restype = ctypes.c_float
+        L.oracle_quantize_row_mode.argtypes = [_i64, _p, _p, _p, _i32]
+        L.oracle_quantize_row_mode.restype = None
         L.oracle_quantize_row.argtypes = [_i64, _p, _p, _p]
         L.oracle_quantize_row.restype = None
         L.oracle_layout.argtypes = [_i64, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p, _p, _p]
@@ -107,6 +111,13 @@ def block_scale(amax: float) -> float:
     return float(lib().oracle_block_scale(float(amax)))
 
 
+def block_scale_pow2(amax: float) -> float:
+    return float(lib().oracle_block_scale_pow2(float(amax)))
+
+
+QUANT_MODES = {"none": 0, "fp8": 1, "fp8_pow2": 2}
+
+
 # ----------------------------------------------------- vectorised wrappers --
 # The array codecs loop in C over the elements; the Python side only moves
 # buffers.
@@ -129,13 +140,13 @@ def bf16_from_f32_array(v: np.ndarray) -> np.ndarray:
     return out
 
 
-def quantize_row(x_row: np.ndarray):
+def quantize_row(x_row: np.ndarray, pow2: bool = False):
     """E4M3 codes and 1x128 fp32 scales of one BF16 row (uint16 bit patterns)."""
     x_row = _c(x_row, np.uint16).reshape(-1)
     H = x_row.size
     q = np.empty(H, dtype=np.uint8)
     s = np.empty(H // 128, dtype=np.float32)
-    lib().oracle_quantize_row(H, _ptr(x_row), _ptr(q), _ptr(s))
+    lib().oracle_quantize_row_mode(H, _ptr(x_row), _ptr(q), _ptr(s), 1 if pow2 else 0)
     return q, s
 
 
@@ -187,7 +198,7 @@ def dispatch(x: np.ndarray, topk_idx: np.ndarray, topk_weights: np.ndarray, num_
     K = idx.shape[1]
     lay = layout(idx, num_experts, num_partitions)
     R = int(lay["num_recv"][0])
-    qm = 1 if quant == "fp8" else 0
+    qm = QUANT_MODES[quant]
     rows = max(R, 1)
     recv_x = np.zeros((rows, H), np.uint8) if qm else np.zeros((rows, H), np.uint16)
     recv_scales = np.zeros((rows, max(H // 128, 1)), np.float32)
@@ -205,7 +216,7 @@ def dispatch(x: np.ndarray, topk_idx: np.ndarray, topk_weights: np.ndarray, num_
 def identity_expert(recv_x: np.ndarray, recv_scales, quant: str = "fp8") -> np.ndarray:
     """BF16 expert output of the identity expert (dequantised receive rows)."""
     R, H = recv_x.shape
-    qm = 1 if quant == "fp8" else 0
+    qm = QUANT_MODES[quant]
     rx = _c(recv_x, np.uint8 if qm else np.uint16)
     rs = _c(recv_scales if recv_scales is not None else np.zeros((R, 1), np.float32), np.float32)
     out = np.empty((R, H), np.uint16)
@@ -307,7 +318,7 @@ def dispatch_dedup(x: np.ndarray, topk_idx: np.ndarray, topk_weights: np.ndarray
     T, H = x.shape
     K = idx.shape[1]
     P = num_partitions
-    qm = 1 if quant == "fp8" else 0
+    qm = QUANT_MODES[quant]
     cap = max(T * min(P, K), 1)
     out = dict(prow_of=np.empty((T, P), np.int32), part_count=np.empty(P, np.int32),
                part_offset=np.empty(P + 1, np.int32), src_tok=np.full(cap, -1, np.int32),

@@ -133,20 +133,36 @@ float oracle_block_scale(float amax) {
     return a / 448.0f;
 }
 
+/* Power-of-two scale of one block, for consumers that take scales as an 8-bit
+ * exponent (UE8M0): the smallest power of two not below max(amax, 1e-4) / 448.
+ * The quotient x / s is then an exact exponent shift and |x / s| <= 448.  The
+ * pages fix no scale format; this is the library's optional second one. */
+float oracle_block_scale_pow2(float amax) {
+    float s = oracle_block_scale(amax);
+    int e;
+    double m = frexp((double)s, &e); /* s = m * 2^e, m in [0.5, 1) */
+    if (m == 0.5) return s;          /* already a power of two */
+    return (float)ldexp(1.0, e);
+}
+
 /* Quantise one BF16 row of H channels (H a multiple of 128) into E4M3 codes
- * and H/128 fp32 scales. */
-void oracle_quantize_row(int64_t H, const uint16_t* x, uint8_t* q, float* scales) {
+ * and H/128 fp32 scales; pow2 selects the power-of-two scales. */
+void oracle_quantize_row_mode(int64_t H, const uint16_t* x, uint8_t* q, float* scales, int pow2) {
     int64_t nb = H / 128;
     for (int64_t b = 0; b < nb; ++b) {
         float amax = 0.0f;
         for (int i = 0; i < 128; ++i) amax = fmaxf(amax, fabsf(oracle_bf16_to_f32(x[b * 128 + i])));
-        float s = oracle_block_scale(amax);
+        float s = pow2 ? oracle_block_scale_pow2(amax) : oracle_block_scale(amax);
         for (int i = 0; i < 128; ++i) {
             float xv = oracle_bf16_to_f32(x[b * 128 + i]);
             q[b * 128 + i] = oracle_e4m3_from_f32(xv / s);
         }
         scales[b] = s;
     }
+}
+
+void oracle_quantize_row(int64_t H, const uint16_t* x, uint8_t* q, float* scales) {
+    oracle_quantize_row_mode(H, x, q, scales, 0);
 }
 
 /* -------------------------------------------------------------- layout -- */
@@ -210,6 +226,7 @@ uint32_t oracle_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int64_t
 
 /* Copy every token to the rows the layout gave it.
  *   quant = 1: recv_x is E4M3 [rows][H], recv_scales fp32 [rows][H/128]
+ *   quant = 2: the same with power-of-two scales (oracle_block_scale_pow2)
  *   quant = 0: recv_x is the BF16 row, bit for bit [rows][H]; recv_scales unused
  *   recv_topk_idx[row]     = local expert id e - p*E/P of the row's expert
  *   recv_topk_weights[row] = topk_weights[t][k]                              */
@@ -222,12 +239,12 @@ uint32_t oracle_dispatch(int64_t T, int64_t H, int32_t K, int32_t E, int32_t P, 
     uint8_t* q = (uint8_t*)malloc((size_t)H);
     float* s = (float*)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
     for (int64_t t = 0; t < T; ++t) {
-        if (quant == 1) oracle_quantize_row(H, x + t * H, q, s);
+        if (quant >= 1) oracle_quantize_row_mode(H, x + t * H, q, s, quant == 2);
         for (int32_t k = 0; k < K; ++k) {
             int32_t row = row_of[t * K + k];
             if (row < 0) continue;
             int64_t e = topk_idx[t * K + k];
-            if (quant == 1) {
+            if (quant >= 1) {
                 memcpy(recv_x + (int64_t)row * H, q, (size_t)H);
                 memcpy(recv_scales + (int64_t)row * nb, s, sizeof(float) * (size_t)nb);
             } else {
@@ -250,7 +267,7 @@ void oracle_identity_expert(int64_t R, int64_t H, int32_t quant, const uint8_t* 
     int64_t nb = H / 128;
     for (int64_t r = 0; r < R; ++r) {
         for (int64_t i = 0; i < H; ++i) {
-            if (quant == 1) {
+            if (quant >= 1) {
                 float v = oracle_e4m3_to_f32(recv_x[r * H + i]) * recv_scales[r * nb + i / 128];
                 expert_out[r * H + i] = oracle_bf16_from_f32(v);
             } else {
@@ -469,8 +486,8 @@ uint32_t oracle_dispatch_dedup(int64_t T, int64_t H, int32_t K, int32_t E, int32
             }
             prow_of[t * P + p] = row;
             src_tok[row] = (int32_t)t;
-            if (quant == 1) {
-                oracle_quantize_row(H, x + t * H, q, s);
+            if (quant >= 1) {
+                oracle_quantize_row_mode(H, x + t * H, q, s, quant == 2);
                 memcpy(recv_x + (int64_t)row * H, q, (size_t)H);
                 memcpy(recv_scales + (int64_t)row * nb, s, sizeof(float) * (size_t)nb);
             } else {
@@ -505,7 +522,7 @@ void oracle_partition_identity(int64_t rows, int64_t H, int32_t K, int32_t quant
     for (int64_t r = 0; r < rows; ++r) {
         for (int64_t i = 0; i < H; ++i) {
             float v;
-            if (quant == 1) {
+            if (quant >= 1) {
                 v = oracle_e4m3_to_f32(recv_x[r * H + i]) * recv_scales[r * nb + i / 128];
             } else {
                 uint16_t b;

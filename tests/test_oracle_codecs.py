@@ -14,6 +14,8 @@ independent implementations fix:
   2M random values inside [-448, 448] (outside it torch returns NaN instead
   of saturating, so the two are not compared there).
 * BF16 rounding: torch's float32 -> bfloat16 cast on random bit patterns.
+* Power-of-two (UE8M0) scales: the scale is a power of two and the smallest
+  one not below the plain scale; codes are torch's cast of the exact quotient.
 """
 import numpy as np
 import pytest
@@ -222,3 +224,46 @@ def test_quantize_roundtrip_error_bound_and_block_independence():
     other[256:384] = False
     assert np.array_equal(q[other], q2[other])
     assert np.array_equal(np.delete(s, 2), np.delete(s2, 2))
+
+
+# ------------------------------------------------------- power-of-two scales --
+
+def test_pow2_scale_closed_forms_and_bracket():
+    assert oracle.block_scale_pow2(448.0) == 1.0
+    assert oracle.block_scale_pow2(449.0) == 2.0
+    assert oracle.block_scale_pow2(224.0) == 0.5
+    assert oracle.block_scale_pow2(0.0) == 2.0 ** -22  # 1e-4 / 448 = 2.23e-7 -> 2^-22
+    rng = np.random.default_rng(12)
+    for a in np.exp2(rng.uniform(-20, 20, 2000)).astype(np.float32):
+        s = oracle.block_scale_pow2(float(a))
+        r = oracle.block_scale(float(a))
+        m, _ = np.frexp(s)
+        assert m == 0.5                  # a power of two
+        assert s >= r and s / 2 < r      # the smallest one not below the plain scale
+
+
+def test_pow2_quantise_matches_torch_cast_of_exact_quotient():
+    rng = np.random.default_rng(13)
+    f = (rng.standard_normal(1024) * np.exp2(rng.uniform(-6, 6, 1024))).astype(np.float32)
+    x = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    q, s = oracle.quantize_row(x, pow2=True)
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    quot = (xf / np.repeat(s, 128)).astype(np.float32)  # division by a power of two: exact
+    assert np.all(np.abs(quot) <= 448.0)
+    ref = torch.from_numpy(quot).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(q, ref)
+
+
+def test_pow2_dispatch_rows_are_pow2_quantised_token_rows():
+    from workloads import make_workload
+    w = make_workload("normal", seed=3, num_tokens=40, hidden=256)
+    d = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, 256, 8, quant="fp8_pow2")
+    d1 = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, 256, 8, quant="fp8")
+    R = int(d["num_recv"][0])
+    assert R == int(d1["num_recv"][0]) and np.array_equal(d["src_of"], d1["src_of"])
+    for r in range(R):
+        t = int(d["src_of"][r]) // w.num_topk
+        q, s = oracle.quantize_row(w.x[t], pow2=True)
+        assert np.array_equal(d["recv_x"][r], q) and np.array_equal(d["recv_scales"][r], s)
+    # the power-of-two scales never fall below the plain ones
+    assert np.all(d["recv_scales"][:R] >= d1["recv_scales"][:R])
