@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libep_b200.
 
 EP_OK, EP_ERR_INVALID_ARG, EP_ERR_SHAPE, EP_ERR_WORKSPACE, EP_ERR_CUDA = 0, 1, 2, 3, 4
 EP_DEV_INDEX_RANGE, EP_DEV_TIMEOUT, EP_DEV_CAPACITY = 0x1, 0x2, 0x4
-EP_QUANT_NONE, EP_QUANT_FP8_E4M3_1X128 = 0, 1
+EP_QUANT_NONE, EP_QUANT_FP8_E4M3_1X128, EP_QUANT_FP8_E4M3_1X128_POW2 = 0, 1, 2
 
 EXPORTED = (
     "ep_abi_version", "ep_status_string", "ep_workspace_bytes", "ep_workspace_init",
@@ -236,7 +236,7 @@ def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Ten
     K = topk_idx.shape[1]
     _need(topk_idx, "topk_idx", torch.int64, shape=(T, K))
     _need(topk_weights, "topk_weights", torch.float32, shape=(T, K))
-    if quant == EP_QUANT_FP8_E4M3_1X128:
+    if quant in (EP_QUANT_FP8_E4M3_1X128, EP_QUANT_FP8_E4M3_1X128_POW2):
         _need(recv_x, "recv_x", (torch.uint8, torch.float8_e4m3fn), numel_at_least=T * K * H)
         _need(recv_scales, "recv_scales", torch.float32, numel_at_least=T * K * (H // 128))
     else:
@@ -375,7 +375,7 @@ def ep_dispatch_dedup(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: tor
     rows = max(T * min(P, K), 1)
     _need(topk_idx, "topk_idx", torch.int64, shape=(T, K))
     _need(topk_weights, "topk_weights", torch.float32, shape=(T, K))
-    if quant == EP_QUANT_FP8_E4M3_1X128:
+    if quant in (EP_QUANT_FP8_E4M3_1X128, EP_QUANT_FP8_E4M3_1X128_POW2):
         _need(recv_x, "recv_x", (torch.uint8, torch.float8_e4m3fn), numel_at_least=rows * H)
         _need(recv_scales, "recv_scales", torch.float32, numel_at_least=rows * (H // 128))
     else:

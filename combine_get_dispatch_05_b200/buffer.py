@@ -30,7 +30,8 @@ from typing import Optional, Tuple, Union
 import torch
 
 from . import _lib
-from ._lib import EP_QUANT_FP8_E4M3_1X128, EP_QUANT_NONE, Layout, LowLatencyHandle
+from ._lib import (EP_QUANT_FP8_E4M3_1X128, EP_QUANT_FP8_E4M3_1X128_POW2, EP_QUANT_NONE,
+                   Layout, LowLatencyHandle)
 
 __all__ = ["Buffer"]
 
@@ -88,11 +89,13 @@ class Buffer:
 
     # ----------------------------------------------------------- dispatch --
     def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
-                 num_experts: Optional[int] = None, use_fp8: bool = True, exact: bool = True):
+                 num_experts: Optional[int] = None, use_fp8: bool = True, exact: bool = True,
+                 pow2_scales: bool = False):
         """Returns ``(recv_x, recv_topk_idx, recv_topk_weights, handle, event)``.
 
         With ``use_fp8`` recv_x is ``(payload float8_e4m3fn [R, H], scales float32
-        [R, H/128])``; otherwise a BF16 ``[R, H]`` tensor.  ``exact`` trims the
+        [R, H/128])``; otherwise a BF16 ``[R, H]`` tensor.  ``pow2_scales`` rounds
+        every scale up to a power of two.  ``exact`` trims the
         worst-case (T*K-row) buffers to the R received rows, which reads R back to
         the host once; ``exact=False`` returns the untrimmed buffers and never
         synchronises (R is then ``handle.num_recv`` on the device).
@@ -111,7 +114,8 @@ class Buffer:
             recv_q = torch.empty((rows, H), dtype=torch.float8_e4m3fn, device=dev)
             recv_s = torch.empty((rows, H // 128), dtype=torch.float32, device=dev)
             _lib.ep_dispatch(x, topk_idx, topk_weights, self.num_experts, self.num_partitions,
-                             EP_QUANT_FP8_E4M3_1X128, recv_q, recv_s, recv_topk_idx,
+                             EP_QUANT_FP8_E4M3_1X128_POW2 if pow2_scales
+                             else EP_QUANT_FP8_E4M3_1X128, recv_q, recv_s, recv_topk_idx,
                              recv_topk_weights, handle, self.workspace)
         else:
             recv_q = torch.empty((rows, H), dtype=torch.bfloat16, device=dev)
@@ -171,7 +175,7 @@ class Buffer:
 
     # ------------------------------------------------------- deduplicated --
     def dispatch_dedup(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
-                       use_fp8: bool = True, exact: bool = True):
+                       use_fp8: bool = True, exact: bool = True, pow2_scales: bool = False):
         """One receive row per (token, partition).  Returns ``(recv_x, recv_topk_idx
         [R, K], recv_topk_weights [R, K], handle, event)``; handle.row_of is [T, P]."""
         T, H = x.shape
@@ -188,7 +192,7 @@ class Buffer:
         if use_fp8:
             rq = torch.empty((rows, H), dtype=torch.float8_e4m3fn, device=dev)
             rs = torch.empty((rows, H // 128), dtype=torch.float32, device=dev)
-            quant = EP_QUANT_FP8_E4M3_1X128
+            quant = EP_QUANT_FP8_E4M3_1X128_POW2 if pow2_scales else EP_QUANT_FP8_E4M3_1X128
         else:
             rq = torch.empty((rows, H), dtype=torch.bfloat16, device=dev)
             rs = None

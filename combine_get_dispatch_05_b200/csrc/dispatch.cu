@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(352) dispatch_fp8_kernel(DispatchParams p) {
                 break;
             uint8_t* out_q = sm + L.off_out + o * L.out_bytes;
             quantize_row_fp8(sm + s * L.in_bytes, out_q, reinterpret_cast<float*>(out_q + L.q_bytes),
-                             nb, qw, nq, lane);
+                             nb, qw, nq, lane, p.pow2_scales != 0);
             fence_proxy_async_smem();  // staged row visible to the bulk stores
             __syncwarp();
             if (lane == 0) {

@@ -43,6 +43,7 @@ struct DispatchParams {
     int32_t K;       // routing ids per token (topk_idx / topk_weights row length)
     int32_t slots;   // receive rows per token in row_of: K, or P when dedup
     int32_t dedup;   // 1: a row per (token, partition) with [rows, K] expert lists
+    int32_t pow2_scales;  // FP8: power-of-two block scales
     int32_t num_experts;
     int32_t experts_per_partition;
     const void* x;

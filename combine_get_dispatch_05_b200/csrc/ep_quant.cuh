@@ -14,10 +14,13 @@ namespace ep {
 // Quantise one BF16 row held in shared memory.  A warp takes two 128-channel
 // blocks at a time: lanes 0-15 the even block, lanes 16-31 the odd one, 8
 // channels (16 bytes) per lane; the block amax is a 16-lane xor-shuffle max.
+//
+// pow2: round each scale up to the next power of two (for consumers that take
+// scales as an 8-bit exponent); x / s is then an exact exponent shift.
 __device__ __forceinline__ void quantize_row_fp8(const uint8_t* __restrict__ in,
                                              uint8_t* __restrict__ out_q,
                                              float* __restrict__ out_s, int nb, int warp,
-                                             int nwarps, int lane) {
+                                             int nwarps, int lane, bool pow2 = false) {
     const int half = lane >> 4, l16 = lane & 15;
     for (int bp = warp; 2 * bp < nb; bp += nwarps) {
         const int b = 2 * bp + half;
@@ -36,7 +39,11 @@ __device__ __forceinline__ void quantize_row_fp8(const uint8_t* __restrict__ in,
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        const float s = fmaxf(amax, 1e-4f) / 448.0f;  // IEEE division (no fast-math)
+        float s = fmaxf(amax, 1e-4f) / 448.0f;  // IEEE division (no fast-math)
+        if (pow2) {
+            const uint32_t b = __float_as_uint(s);  // s is normal and positive
+            if (b & 0x007FFFFFu) s = __uint_as_float((b & 0x7F800000u) + 0x00800000u);
+        }
         uint2 q;
         q.x = e4m3x2(f[0] / s, f[1] / s) | (e4m3x2(f[2] / s, f[3] / s) << 16);
         q.y = e4m3x2(f[4] / s, f[5] / s) | (e4m3x2(f[6] / s, f[7] / s) << 16);

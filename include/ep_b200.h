@@ -89,8 +89,11 @@ typedef enum ep_status {
 
 /* Dispatch payload format. */
 typedef enum ep_quant {
-    EP_QUANT_NONE = 0,           /* BF16 rows copied bit for bit */
-    EP_QUANT_FP8_E4M3_1X128 = 1  /* E4M3 codes + one fp32 scale per 128 channels */
+    EP_QUANT_NONE = 0,                /* BF16 rows copied bit for bit */
+    EP_QUANT_FP8_E4M3_1X128 = 1,      /* E4M3 codes + one fp32 scale per 128 channels */
+    EP_QUANT_FP8_E4M3_1X128_POW2 = 2  /* the same with each scale rounded up to a power of
+                                         two (an 8-bit exponent, UE8M0, for FP8 GEMMs that
+                                         take exponent-only scales); x / s is exact */
 } ep_quant;
 
 /*

@@ -68,11 +68,16 @@ def layout_numpy(lay, T, K):
     )
 
 
+def quant_code(ep, quant: str) -> int:
+    return {"none": ep.EP_QUANT_NONE, "fp8": ep.EP_QUANT_FP8_E4M3_1X128,
+            "fp8_pow2": ep.EP_QUANT_FP8_E4M3_1X128_POW2}[quant]
+
+
 def gpu_dispatch(ep, w, workspace=None, quant=None):
     """Layout + dispatch of workload `w` on the GPU; returns (numpy dict, device state)."""
     quant = w.quant if quant is None else quant
     T, H, K, E, P = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
-    fp8 = quant == "fp8"
+    fp8 = quant in ("fp8", "fp8_pow2")
     x = dev_u16_as_bf16(w.x)
     idx = torch.from_numpy(np.ascontiguousarray(w.topk_idx)).cuda()
     wts = torch.from_numpy(np.ascontiguousarray(w.topk_weights)).cuda()
@@ -83,8 +88,7 @@ def gpu_dispatch(ep, w, workspace=None, quant=None):
     recv_w = Guarded((rows,), torch.float32)
     lay = ep.Layout.empty(T, K, E, P, "cuda")
     ws = workspace if workspace is not None else new_workspace(ep, T, E, P)
-    ep.ep_dispatch(x, idx, wts, E, P,
-                   ep.EP_QUANT_FP8_E4M3_1X128 if fp8 else ep.EP_QUANT_NONE,
+    ep.ep_dispatch(x, idx, wts, E, P, quant_code(ep, quant),
                    recv_x.t, recv_s.t if fp8 else None, recv_i.t, recv_w.t, lay, ws)
     torch.cuda.synchronize()
     out = layout_numpy(lay, T, K)

@@ -10,7 +10,8 @@ pytestmark = pytest.mark.gpu
 import oracle  # noqa: E402
 from workloads import make_custom, make_workload, random_bf16  # noqa: E402
 
-from gpu_path import Guarded, bf16_to_u16, dev_u16_as_bf16, new_workspace  # noqa: E402
+from gpu_path import (Guarded, bf16_to_u16, dev_u16_as_bf16, new_workspace,  # noqa: E402
+                      quant_code)
 
 
 @pytest.fixture(scope="module")
@@ -23,7 +24,7 @@ def ep():
 
 def run_dedup(ep, w, quant):
     T, H, K, E, P = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
-    fp8 = quant == "fp8"
+    fp8 = quant in ("fp8", "fp8_pow2")
     rows = max(T * min(P, K), 1)
     x = dev_u16_as_bf16(w.x)
     idx = torch.from_numpy(np.ascontiguousarray(w.topk_idx)).cuda()
@@ -34,8 +35,7 @@ def run_dedup(ep, w, quant):
     rw = Guarded((rows, K), torch.float32)
     lay = ep.Layout.empty(T, P, P, P, "cuda")
     ws = new_workspace(ep, T, E, P)
-    ep.ep_dispatch_dedup(x, idx, wts, E, P,
-                         ep.EP_QUANT_FP8_E4M3_1X128 if fp8 else ep.EP_QUANT_NONE,
+    ep.ep_dispatch_dedup(x, idx, wts, E, P, quant_code(ep, quant),
                          rx.t, rs.t if fp8 else None, ri.t, rw.t, lay, ws)
     torch.cuda.synchronize()
     R = int(lay.num_recv.item())
@@ -84,7 +84,7 @@ def test_dispatch_dedup_parity(ep, name, mk):
     assert np.array_equal(got["itp"], lay["is_token_in_partition"])
     assert np.array_equal(got["ntp"], lay["num_tokens_per_partition"])
     assert np.array_equal(got["recv_x"], want["recv_x"])
-    if quant == "fp8":
+    if quant != "none":
         assert np.array_equal(got["recv_scales"].view(np.uint32), want["recv_scales"].view(np.uint32))
     assert np.array_equal(got["recv_topk_idx"], want["recv_topk_idx"])
     assert np.array_equal(got["recv_topk_weights"].view(np.uint32),
@@ -161,3 +161,14 @@ def test_buffer_dedup_and_backward_methods(ep):
     assert np.array_equal(bf16_to_u16(geo), geo_ref)
     assert np.array_equal(gwt.cpu().numpy().view(np.uint32), gw_ref.view(np.uint32))
     assert buf.read_status() == 0
+
+
+def test_dispatch_dedup_pow2_scales_parity(ep):
+    w = make_workload("normal", seed=41, num_tokens=333, hidden=768)
+    got = run_dedup(ep, w, "fp8_pow2")
+    want = oracle.dispatch_dedup(w.x, w.topk_idx, w.topk_weights, w.num_experts,
+                                 w.num_partitions, quant="fp8_pow2")
+    assert got["R"] == want["num_rows"][0]
+    assert np.array_equal(got["recv_x"], want["recv_x"])
+    assert np.array_equal(got["recv_scales"].view(np.uint32), want["recv_scales"].view(np.uint32))
+    assert got["canaries_ok"]

@@ -284,3 +284,38 @@ def test_buffer_api_matches_pages_call_shapes(ep):
     assert np.array_equal(cnt.cpu().numpy(),
                           oracle.layout(w.topk_idx[:128], 256, 8)["num_tokens_per_expert"])
     assert buf.read_status() == 0
+
+
+POW2_CASES = [c for c in CASES if c[0] in ("normal-300", "masked", "k32-dups", "e4096", "t1")]
+
+
+@pytest.mark.parametrize("name,w", POW2_CASES, ids=[c[0] for c in POW2_CASES])
+def test_dispatch_pow2_scales_parity(ep, name, w):
+    got, _ = gpu_dispatch(ep, w, quant="fp8_pow2")
+    want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, w.num_experts, w.num_partitions,
+                           quant="fp8_pow2")
+    _assert_layout(got, want)
+    assert np.array_equal(got["recv_x"], want["recv_x"])
+    assert np.array_equal(got["recv_scales"].view(np.uint32), want["recv_scales"].view(np.uint32))
+    assert np.all((got["recv_scales"].view(np.uint32) & 0x007FFFFF) == 0)  # exponent only
+    assert got["canaries_ok"]
+
+
+def test_pow2_scales_on_extreme_blocks(ep):
+    # blocks whose amax sits exactly on, just above and just below 448 * 2^n, and
+    # all-zero / subnormal-only blocks (the 1e-4 floor)
+    f = np.zeros((4, 1024), np.float32)
+    f[0, :128] = 448.0
+    f[0, 128:256] = np.float32(448.0 * 2 ** -3)
+    f[0, 256:384] = 449.0
+    f[0, 384:512] = 447.0
+    f[1, :128] = 1e-40
+    f[2] = np.linspace(-3000, 3000, 1024, dtype=np.float32)
+    f[3, ::7] = -2.0 ** 100
+    x = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    w = make_custom(4, 1024, 2, 8, 2, seed=30)
+    w.x[:] = x
+    got, _ = gpu_dispatch(ep, w, quant="fp8_pow2")
+    want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, 8, 2, quant="fp8_pow2")
+    assert np.array_equal(got["recv_x"], want["recv_x"])
+    assert np.array_equal(got["recv_scales"].view(np.uint32), want["recv_scales"].view(np.uint32))
