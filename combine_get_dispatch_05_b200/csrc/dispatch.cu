@@ -7,8 +7,12 @@
 //
 // BF16 path: the row is copied bit for bit.
 //
-// Both kernels are persistent pipelines over the CTA's tokens (t = blockIdx.x,
-// blockIdx.x + gridDim.x, ...).  Input rows arrive by 1-D bulk async copies
+// Both kernels are persistent pipelines; a CTA takes its next token from a ticket
+// counter in the workspace (one atomic per token), so CTAs that started late (on
+// the SMs the layout kernel held) or that see less bandwidth take fewer tokens
+// and all finish together.  The last CTA to finish re-zeroes the counter for the
+// next call.  Which CTA writes a token does not change what is written: the
+// output is deterministic.  Input rows arrive by 1-D bulk async copies
 // (cp.async.bulk, mbarrier completion) into a ring of shared-memory stages, so
 // several 14 KB rows per SM are in flight from HBM at once; output rows leave by
 // bulk stores from shared memory, one per destination row, issued by one lane
@@ -24,28 +28,67 @@ namespace ep {
 
 namespace {
 
-constexpr int kFp8InStages = 3;   // input ring: rows in flight from HBM per CTA
-constexpr int kFp8OutStages = 3;  // quantised rows staged for the bulk stores
-constexpr int kBf16Stages = 4;    // BF16 rows in flight per CTA
+constexpr int kFp8InStages = 3;      // input ring: rows in flight from HBM per CTA
+constexpr int kFp8MaxOutStages = 40;  // quantised rows staged per CTA, at most
+constexpr int kFp8CtasPerSm = 2;      // the output ring fills this share of an SM
+constexpr int kBf16Stages = 4;        // BF16 rows in flight per CTA
+// Token log: the token of pipeline step i sits in tok[i % kTokLog] from the
+// loader's ticket until the storer has read it.  The loader runs at most
+// (input stages + output stages) steps ahead of the storer.
+constexpr int kTokLog = 64;
+static_assert(kTokLog > kFp8InStages + kFp8MaxOutStages + 1, "token log too short");
+static_assert(kTokLog > kBf16Stages + 1, "token log too short");
+static_assert((kTokLog & (kTokLog - 1)) == 0, "token log size is a power of two");
 
+// FP8 kernel shared memory: input ring | output ring (E4M3 row + scales per stage) |
+// mbarriers | staged rows per output stage | token log | abort flag.
 struct Fp8Smem {
     uint32_t in_bytes, q_bytes, s_bytes, out_bytes;
-    uint32_t off_out, off_bars, off_rows, off_flag, total;
+    uint32_t off_out, off_bars, off_rows, off_tok, off_flag, total;
 };
 
-__host__ __device__ inline Fp8Smem fp8_smem(int64_t H) {
+__host__ __device__ inline Fp8Smem fp8_smem(int64_t H, int in_stages, int out_stages) {
     Fp8Smem s;
     const uint32_t nb = static_cast<uint32_t>(H / 128);
     s.in_bytes = static_cast<uint32_t>(H) * 2u;
     s.q_bytes = static_cast<uint32_t>(H);
     s.s_bytes = (nb * 4u + 15u) & ~15u;
     s.out_bytes = s.q_bytes + s.s_bytes;
-    s.off_out = kFp8InStages * s.in_bytes;
-    s.off_bars = s.off_out + kFp8OutStages * s.out_bytes;
-    s.off_rows = s.off_bars + 8u * 2u * (kFp8InStages + kFp8OutStages);
-    s.off_flag = s.off_rows + 4u * 32u * kFp8OutStages;
+    s.off_out = in_stages * s.in_bytes;
+    s.off_bars = s.off_out + out_stages * s.out_bytes;
+    s.off_rows = s.off_bars + 8u * 2u * (in_stages + out_stages);
+    s.off_tok = s.off_rows + 4u * 32u * out_stages;
+    s.off_flag = s.off_tok + 4u * kTokLog;
     s.total = s.off_flag + 16u;
     return s;
+}
+
+// A ring position: stage index and the parity of that stage's current use.
+struct Ring {
+    int stage = 0;
+    uint32_t parity = 0;
+    __device__ __forceinline__ void next(int n) {
+        if (++stage == n) {
+            stage = 0;
+            parity ^= 1u;
+        }
+    }
+};
+
+// Next token for this CTA, or -1 when the batch is exhausted.
+__device__ __forceinline__ int take_ticket(const DispatchParams& p) {
+    const int t = atomicAdd(p.ticket, 1);
+    return t < p.T ? t : -1;
+}
+
+// Called by thread 0 after the whole CTA is done (every ticket it will take is
+// taken): count the finished CTAs; the last one re-zeroes the ticket counter.
+__device__ __forceinline__ void finish_tickets(const DispatchParams& p) {
+    __threadfence();
+    if (atomicAdd(p.done, 1u) == gridDim.x - 1) {
+        atomicExch(p.ticket, 0);
+        atomicExch(p.done, 0u);
+    }
 }
 
 // Wait for a phase, giving up after timeout_ns or as soon as another warp of the
@@ -92,41 +135,43 @@ __device__ __forceinline__ void write_row_metadata(const DispatchParams& p, int 
 }
 
 // Warp-specialised pipeline, one CTA = 1 loader warp + nq quantiser warps + 1 storer
-// warp, coupled only by mbarriers (no CTA-wide barrier after set-up):
-//   loader (warp 0, lane 0): bulk-loads token rows into the input ring
-//       (in_full[s]: transaction bytes; waits in_empty[s] before reusing a stage);
+// warp, coupled only by mbarriers (no CTA-wide barrier between set-up and the end):
+//   loader (warp 0, lane 0): takes a ticket, records the token in the token log and
+//       bulk-loads its row into the input ring (in_full[s]: transaction bytes;
+//       waits in_empty[s] before reusing a stage); when the tickets run out it
+//       records -1 and arrives on in_full[s] without a load;
 //   quantisers (warps 1..nq): quantise their share of the row's 128-channel blocks
 //       from input stage s into output stage o, then arrive on in_empty[s] and
-//       out_full[o] (waiting out_empty[o] before reusing an output stage);
+//       out_full[o] (waiting out_empty[o] before reusing an output stage); a -1
+//       token is passed on without work and ends the warp;
 //   storer (last warp): lane k bulk-stores the staged row and its scales to row
 //       row_of[t, k], writes recv_topk_idx / recv_topk_weights, and releases the
-//       output stage (out_empty) once its stores have read it.
+//       output stage (out_empty) once its stores have read it; a -1 token ends it.
 // Only the storer reads what the layout kernel wrote, so only it waits on the
 // programmatic dependency; loads and quantisation overlap the layout.
 __global__ void __launch_bounds__(352) dispatch_fp8_kernel(DispatchParams p) {
     extern __shared__ __align__(128) uint8_t sm[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nq = (blockDim.x >> 5) - 2;
-    const int64_t T = p.T, H = p.H;
+    const int64_t H = p.H;
     const int K = p.K, nb = static_cast<int>(H >> 7);
-    const Fp8Smem L = fp8_smem(H);
+    const int NI = p.in_stages, NO = p.out_stages;
+    const Fp8Smem L = fp8_smem(H, NI, NO);
     uint64_t* in_full = reinterpret_cast<uint64_t*>(sm + L.off_bars);
-    uint64_t* in_empty = in_full + kFp8InStages;
-    uint64_t* out_full = in_empty + kFp8InStages;
-    uint64_t* out_empty = out_full + kFp8OutStages;
+    uint64_t* in_empty = in_full + NI;
+    uint64_t* out_full = in_empty + NI;
+    uint64_t* out_empty = out_full + NO;
     int* rows_sm = reinterpret_cast<int*>(sm + L.off_rows);
+    volatile int* tok = reinterpret_cast<volatile int*>(sm + L.off_tok);
     volatile int* abort_flag = reinterpret_cast<int*>(sm + L.off_flag);
     const bool scale_bulk = (static_cast<uint32_t>(nb) * 4u) == L.s_bytes;
 
-    const int64_t G = gridDim.x, first = blockIdx.x;
-    const int64_t n_mine = first < T ? (T - 1 - first) / G + 1 : 0;
-
     if (tid == 0) {
-        for (int s = 0; s < kFp8InStages; ++s) {
+        for (int s = 0; s < NI; ++s) {
             mbar_init(&in_full[s], 1);
             mbar_init(&in_empty[s], nq);
         }
-        for (int o = 0; o < kFp8OutStages; ++o) {
+        for (int o = 0; o < NO; ++o) {
             mbar_init(&out_full[o], nq);
             mbar_init(&out_empty[o], 1);
         }
@@ -139,49 +184,54 @@ __global__ void __launch_bounds__(352) dispatch_fp8_kernel(DispatchParams p) {
         // ---------------------------------------------------------------- loader
         if (lane == 0) {
             const uint8_t* x = static_cast<const uint8_t*>(p.x);
-            int64_t issued = 0;
-            for (; issued < n_mine; ++issued) {
-                const int s = static_cast<int>(issued % kFp8InStages);
-                if (issued >= kFp8InStages &&
-                    !wait_or_abort(&in_empty[s],
-                                   static_cast<uint32_t>((issued / kFp8InStages - 1) & 1),
-                                   p.timeout_ns, abort_flag))
+            int issued = 0;  // bulk loads issued (steps 0 .. issued-1)
+            Ring in;
+            for (int i = 0;; ++i, in.next(NI)) {
+                if (i >= NI && !wait_or_abort(&in_empty[in.stage], in.parity ^ 1u, p.timeout_ns,
+                                              abort_flag))
                     break;
-                const int64_t t = first + issued * G;
-                mbar_arrive_expect_tx(&in_full[s], L.in_bytes);
-                bulk_load(sm + s * L.in_bytes, x + t * H * 2, L.in_bytes, &in_full[s]);
+                const int t = take_ticket(p);
+                tok[i & (kTokLog - 1)] = t;
+                if (t < 0) {
+                    mbar_arrive(&in_full[in.stage]);  // the end marker: no load
+                    break;
+                }
+                mbar_arrive_expect_tx(&in_full[in.stage], L.in_bytes);
+                bulk_load(sm + in.stage * L.in_bytes, x + static_cast<int64_t>(t) * H * 2, L.in_bytes,
+                          &in_full[in.stage]);
+                ++issued;
             }
             if (*abort_flag) {
                 // let this CTA's loads still in flight land before it exits: the
                 // latest load of each stage is its barrier's current phase
-                for (int64_t j = issued - 1; j >= 0 && j >= issued - kFp8InStages; --j)
-                    mbar_wait_bounded(&in_full[j % kFp8InStages],
-                                      static_cast<uint32_t>((j / kFp8InStages) & 1),
+                for (int j = issued - 1; j >= 0 && j >= issued - NI; --j)
+                    mbar_wait_bounded(&in_full[j % NI], static_cast<uint32_t>((j / NI) & 1),
                                       kDefaultTimeoutNs);
             }
         }
     } else if (warp <= nq) {
         // ------------------------------------------------------------ quantisers
         const int qw = warp - 1;
-        for (int64_t i = 0; i < n_mine; ++i) {
-            const int s = static_cast<int>(i % kFp8InStages);
-            const int o = static_cast<int>(i % kFp8OutStages);
-            if (!wait_or_abort(&in_full[s], static_cast<uint32_t>((i / kFp8InStages) & 1),
-                               p.timeout_ns, abort_flag))
+        Ring in, out;
+        for (int i = 0;; ++i, in.next(NI), out.next(NO)) {
+            if (!wait_or_abort(&in_full[in.stage], in.parity, p.timeout_ns, abort_flag)) break;
+            if (i >= NO &&
+                !wait_or_abort(&out_empty[out.stage], out.parity ^ 1u, p.timeout_ns, abort_flag))
                 break;
-            if (i >= kFp8OutStages &&
-                !wait_or_abort(&out_empty[o], static_cast<uint32_t>((i / kFp8OutStages - 1) & 1),
-                               p.timeout_ns, abort_flag))
-                break;
-            uint8_t* out_q = sm + L.off_out + o * L.out_bytes;
-            quantize_row_fp8(sm + s * L.in_bytes, out_q, reinterpret_cast<float*>(out_q + L.q_bytes),
-                             nb, qw, nq, lane, p.pow2_scales != 0);
-            fence_proxy_async_smem();  // staged row visible to the bulk stores
+            const int t = tok[i & (kTokLog - 1)];
+            if (t >= 0) {
+                uint8_t* out_q = sm + L.off_out + out.stage * L.out_bytes;
+                quantize_row_fp8(sm + in.stage * L.in_bytes, out_q,
+                                 reinterpret_cast<float*>(out_q + L.q_bytes), nb, qw, nq, lane,
+                                 p.pow2_scales != 0);
+                fence_proxy_async_smem();  // staged row visible to the bulk stores
+            }
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&in_empty[s]);
-                mbar_arrive(&out_full[o]);
+                mbar_arrive(&in_empty[in.stage]);
+                mbar_arrive(&out_full[out.stage]);
             }
+            if (t < 0) break;
         }
     } else {
         // ---------------------------------------------------------------- storer
@@ -190,32 +240,16 @@ __global__ void __launch_bounds__(352) dispatch_fp8_kernel(DispatchParams p) {
         const int S = p.slots;
         const bool slot_lane = lane < S;  // lane s stores slot s's row
         const bool id_lane = lane < K;    // lane k holds routing entry k
-        int nrow = -1;
-        int64_t nexp = -1;
-        float nwt = 0.0f;
-        if (n_mine > 0) {
-            if (slot_lane) nrow = p.row_of[first * S + lane];
-            if (id_lane) {
-                nexp = p.topk_idx[first * K + lane];
-                nwt = p.topk_weights[first * K + lane];
-            }
-        }
-        for (int64_t i = 0; i < n_mine; ++i) {
-            const int64_t t = first + i * G;
-            const int o = static_cast<int>(i % kFp8OutStages);
-            const int row = nrow;
-            const int64_t e = nexp;
-            const float wt = nwt;
-            if (i + 1 < n_mine) {
-                if (slot_lane) nrow = p.row_of[(t + G) * S + lane];
-                if (id_lane) {
-                    nexp = p.topk_idx[(t + G) * K + lane];
-                    nwt = p.topk_weights[(t + G) * K + lane];
-                }
-            }
-            if (!wait_or_abort(&out_full[o], static_cast<uint32_t>((i / kFp8OutStages) & 1),
-                               p.timeout_ns, abort_flag))
-                break;
+        Ring out;
+        int prev = -1;  // output stage of the previous step
+        for (int i = 0;; ++i, out.next(NO)) {
+            if (!wait_or_abort(&out_full[out.stage], out.parity, p.timeout_ns, abort_flag)) break;
+            const int t = tok[i & (kTokLog - 1)];
+            if (t < 0) break;
+            const int o = out.stage;
+            const int row = slot_lane ? p.row_of[static_cast<int64_t>(t) * S + lane] : -1;
+            const int64_t e = id_lane ? p.topk_idx[static_cast<int64_t>(t) * K + lane] : -1;
+            const float wt = id_lane ? p.topk_weights[static_cast<int64_t>(t) * K + lane] : 0.0f;
             uint8_t* out_q = sm + L.off_out + o * L.out_bytes;
             const float* out_s = reinterpret_cast<const float*>(out_q + L.q_bytes);
             if (slot_lane) {
@@ -240,33 +274,38 @@ __global__ void __launch_bounds__(352) dispatch_fp8_kernel(DispatchParams p) {
             // release the previous output stage once this warp's stores have read it
             if (slot_lane) bulk_wait_read<1>();
             __syncwarp();
-            if (lane == 0 && i >= 1) mbar_arrive(&out_empty[(i - 1) % kFp8OutStages]);
+            if (lane == 0 && prev >= 0) mbar_arrive(&out_empty[prev]);
+            prev = o;
         }
         if (slot_lane) bulk_wait_all<0>();
     }
-    if (tid == 0 && *abort_flag) raise_status(p.status, kDevTimeout);
+    __syncthreads();
+    if (tid == 0) {
+        if (*abort_flag) raise_status(p.status, kDevTimeout);
+        finish_tickets(p);
+    }
 }
 
 // BF16 rows are copied bit for bit, so the row staged by the bulk load is itself
 // the source of the K bulk stores.  One CTA = a loader warp and a storer warp
 // coupled by full/empty mbarriers over a ring of kBf16Stages rows:
-//   loader (warp 0, lane 0): waits empty[s], bulk-loads the next token's row into
-//       stage s (full[s] counts its transaction bytes);
-//   storer (warp 1): waits for the layout, then per token waits full[s], lane k
+//   loader (warp 0, lane 0): waits empty[s], takes a ticket, records the token in
+//       the token log and bulk-loads its row into stage s (full[s] counts its
+//       transaction bytes); when the tickets run out it records -1 and arrives on
+//       full[s] without a load;
+//   storer (warp 1): waits for the layout, then per step waits full[s], lane k
 //       bulk-stores the row to row_of[t, k] and writes recv_topk_idx / weights;
 //       once this token's stores have read the stage it arrives on empty[s].
 __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
     extern __shared__ __align__(128) uint8_t sm[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t T = p.T, H = p.H;
+    const int64_t H = p.H;
     const int K = p.K;
     const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + kBf16Stages * row_bytes);
     uint64_t* empty = full + kBf16Stages;
-    volatile int* abort_flag = reinterpret_cast<int*>(empty + kBf16Stages);
-
-    const int64_t G = gridDim.x, first = blockIdx.x;
-    const int64_t n_mine = first < T ? (T - 1 - first) / G + 1 : 0;
+    volatile int* tok = reinterpret_cast<volatile int*>(empty + kBf16Stages);
+    volatile int* abort_flag = tok + kTokLog;
 
     if (tid == 0) {
         for (int s = 0; s < kBf16Stages; ++s) {
@@ -283,15 +322,22 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
         if (lane == 0) {
             const uint8_t* x = static_cast<const uint8_t*>(p.x);
             int64_t issued = 0;
-            for (; issued < n_mine; ++issued) {
-                const int s = static_cast<int>(issued % kBf16Stages);
-                if (issued >= kBf16Stages &&
-                    !wait_or_abort(&empty[s], static_cast<uint32_t>((issued / kBf16Stages - 1) & 1),
+            for (int64_t i = 0;; ++i) {
+                const int s = static_cast<int>(i % kBf16Stages);
+                if (i >= kBf16Stages &&
+                    !wait_or_abort(&empty[s], static_cast<uint32_t>((i / kBf16Stages - 1) & 1),
                                    p.timeout_ns, abort_flag))
                     break;
-                const int64_t t = first + issued * G;
+                const int t = take_ticket(p);
+                tok[i % kTokLog] = t;
+                if (t < 0) {
+                    mbar_arrive(&full[s]);  // the end marker: no load
+                    break;
+                }
                 mbar_arrive_expect_tx(&full[s], row_bytes);
-                bulk_load(sm + s * row_bytes, x + t * row_bytes, row_bytes, &full[s]);
+                bulk_load(sm + s * row_bytes, x + static_cast<int64_t>(t) * row_bytes, row_bytes,
+                          &full[s]);
+                ++issued;
             }
             if (*abort_flag) {
                 for (int64_t j = issued - 1; j >= 0 && j >= issued - kBf16Stages; --j)
@@ -307,32 +353,16 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
         const int S = p.slots;
         const bool slot_lane = lane < S;  // lane s stores slot s's row
         const bool id_lane = lane < K;    // lane k holds routing entry k
-        int nrow = -1;
-        int64_t nexp = -1;
-        float nwt = 0.0f;
-        if (n_mine > 0) {
-            if (slot_lane) nrow = p.row_of[first * S + lane];
-            if (id_lane) {
-                nexp = p.topk_idx[first * K + lane];
-                nwt = p.topk_weights[first * K + lane];
-            }
-        }
-        for (int64_t i = 0; i < n_mine; ++i) {
-            const int64_t t = first + i * G;
+        for (int64_t i = 0;; ++i) {
             const int s = static_cast<int>(i % kBf16Stages);
-            const int row = nrow;
-            const int64_t e = nexp;
-            const float wt = nwt;
-            if (i + 1 < n_mine) {
-                if (slot_lane) nrow = p.row_of[(t + G) * S + lane];
-                if (id_lane) {
-                    nexp = p.topk_idx[(t + G) * K + lane];
-                    nwt = p.topk_weights[(t + G) * K + lane];
-                }
-            }
             if (!wait_or_abort(&full[s], static_cast<uint32_t>((i / kBf16Stages) & 1), p.timeout_ns,
                                abort_flag))
                 break;
+            const int t = tok[i % kTokLog];
+            if (t < 0) break;
+            const int row = slot_lane ? p.row_of[static_cast<int64_t>(t) * S + lane] : -1;
+            const int64_t e = id_lane ? p.topk_idx[static_cast<int64_t>(t) * K + lane] : -1;
+            const float wt = id_lane ? p.topk_weights[static_cast<int64_t>(t) * K + lane] : 0.0f;
             if (slot_lane) {
                 if (row >= 0)
                     bulk_store(recv_x + static_cast<int64_t>(row) * row_bytes, sm + s * row_bytes,
@@ -346,7 +376,11 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
         }
         if (slot_lane) bulk_wait_all<0>();
     }
-    if (tid == 0 && *abort_flag) raise_status(p.status, kDevTimeout);
+    __syncthreads();
+    if (tid == 0) {
+        if (*abort_flag) raise_status(p.status, kDevTimeout);
+        finish_tickets(p);
+    }
 }
 
 int grid_for(const void* kernel, int threads, size_t smem, int64_t work, int num_sms) {
@@ -377,12 +411,27 @@ cudaError_t launch_pdl(const void* kernel, dim3 grid, dim3 block, size_t smem, c
 
 }  // namespace
 
-cudaError_t launch_dispatch_fp8(const DispatchParams& p, cudaStream_t stream) {
-    if (p.T == 0) return cudaSuccess;
+cudaError_t launch_dispatch_fp8(const DispatchParams& params, cudaStream_t stream) {
+    if (params.T == 0) return cudaSuccess;
     DeviceInfo dev;
     cudaError_t err = device_info(&dev);
     if (err != cudaSuccess) return err;
-    const Fp8Smem L = fp8_smem(p.H);
+    // Output ring: as many staged rows as fit in 1/kFp8CtasPerSm of the SM's shared
+    // memory, so that while the layout kernel runs each SM reads and quantises as
+    // many of its tokens as it can hold.
+    DispatchParams p = params;
+    p.in_stages = kFp8InStages;
+    const Fp8Smem one = fp8_smem(p.H, kFp8InStages, 1);
+    const Fp8Smem two = fp8_smem(p.H, kFp8InStages, 2);
+    const size_t per_out = two.total - one.total;
+    size_t budget = dev.smem_per_sm / kFp8CtasPerSm;
+    budget = budget > dev.smem_reserved ? budget - dev.smem_reserved : 0;
+    if (budget > dev.max_smem_optin) budget = dev.max_smem_optin;
+    int no = budget >= one.total ? 1 + static_cast<int>((budget - one.total) / per_out) : 1;
+    if (no > kFp8MaxOutStages) no = kFp8MaxOutStages;
+    if (no < 2) no = 2;
+    p.out_stages = no;
+    const Fp8Smem L = fp8_smem(p.H, p.in_stages, p.out_stages);
     if (L.total > dev.max_smem_optin) return cudaErrorInvalidValue;
     const void* kernel = reinterpret_cast<const void*>(dispatch_fp8_kernel);
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -402,7 +451,8 @@ cudaError_t launch_dispatch_bf16(const DispatchParams& p, cudaStream_t stream) {
     DeviceInfo dev;
     cudaError_t err = device_info(&dev);
     if (err != cudaSuccess) return err;
-    const size_t smem = static_cast<size_t>(kBf16Stages) * p.H * 2 + 16 * kBf16Stages + 16;
+    const size_t smem = static_cast<size_t>(kBf16Stages) * p.H * 2 + 16 * kBf16Stages +
+                        4 * kTokLog + 16;
     if (smem > dev.max_smem_optin) return cudaErrorInvalidValue;
     const void* kernel = reinterpret_cast<const void*>(dispatch_bf16_kernel);
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -62,6 +62,13 @@ cudaError_t device_info(DeviceInfo* out) {
     err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (err != cudaSuccess) return err;
     d.max_smem_optin = static_cast<size_t>(optin);
+    int per_sm = 0, reserved = 0;
+    err = cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    if (err != cudaSuccess) return err;
+    err = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    if (err != cudaSuccess) return err;
+    d.smem_per_sm = static_cast<size_t>(per_sm);
+    d.smem_reserved = static_cast<size_t>(reserved);
     if (dev >= 0 && dev < kMaxDevices) {
         g_info[dev] = d;
         g_have_info[dev].store(1, std::memory_order_release);
@@ -178,6 +185,8 @@ ep_status ep_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk, int3
     p.recv_topk_idx = recv_topk_idx;
     p.recv_topk_weights = recv_topk_weights;
     p.status = ws.status;
+    p.ticket = ws.ticket;
+    p.done = ws.done;
     p.timeout_ns = kDefaultTimeoutNs;
     return cuda_status(fp8 ? launch_dispatch_fp8(p, s) : launch_dispatch_bf16(p, s));
 }
@@ -258,6 +267,8 @@ ep_status ep_dispatch_dedup(int64_t num_tokens, int64_t hidden, int32_t num_topk
     p.recv_topk_idx = recv_topk_idx;
     p.recv_topk_weights = recv_topk_weights;
     p.status = ws.status;
+    p.ticket = ws.ticket;
+    p.done = ws.done;
     p.timeout_ns = kDefaultTimeoutNs;
     return cuda_status(fp8 ? launch_dispatch_fp8(p, s) : launch_dispatch_bf16(p, s));
 }

@@ -13,10 +13,13 @@ constexpr uint32_t kDevIndexRange = 0x1u;
 constexpr uint32_t kDevTimeout = 0x2u;
 constexpr uint32_t kDevCapacity = 0x4u;
 
-// Workspace header (bytes): status word, probe flag, layout grid-barrier word.
+// Workspace header (bytes): status word, probe flag, layout grid-barrier word,
+// dispatch token ticket and finished-CTA count (both zero between calls).
 constexpr size_t kWsStatus = 0;
 constexpr size_t kWsProbeFlag = 4;
 constexpr size_t kWsBar = 8;
+constexpr size_t kWsTicket = 16;
+constexpr size_t kWsDone = 20;
 constexpr size_t kWsHeader = 256;
 
 __device__ __forceinline__ void raise_status(uint32_t* status, uint32_t bits) {

@@ -12,7 +12,9 @@ namespace ep {
 struct DeviceInfo {
     int device;
     int num_sms;
-    size_t max_smem_optin;
+    size_t max_smem_optin;   // per CTA
+    size_t smem_per_sm;      // per SM
+    size_t smem_reserved;    // reserved by the runtime per resident CTA
 };
 cudaError_t device_info(DeviceInfo* out);
 
@@ -23,6 +25,8 @@ struct Workspace {
     uint32_t* status;
     uint32_t* probe_flag;
     unsigned long long* bar;
+    int32_t* ticket;           // next token a dispatch CTA takes
+    uint32_t* done;            // dispatch CTAs finished
     int32_t* chunk_expert;     // [chunks][E]
     int32_t* chunk_partition;  // [chunks][P]
 };
@@ -44,6 +48,8 @@ struct DispatchParams {
     int32_t slots;   // receive rows per token in row_of: K, or P when dedup
     int32_t dedup;   // 1: a row per (token, partition) with [rows, K] expert lists
     int32_t pow2_scales;  // FP8: power-of-two block scales
+    int32_t in_stages;    // FP8: input ring depth (rows in flight from HBM per CTA)
+    int32_t out_stages;   // FP8: quantised rows staged per CTA
     int32_t num_experts;
     int32_t experts_per_partition;
     const void* x;
@@ -55,6 +61,8 @@ struct DispatchParams {
     int32_t* recv_topk_idx;
     float* recv_topk_weights;
     uint32_t* status;
+    int32_t* ticket;  // token counter (zero on entry; the last CTA to finish re-zeroes it)
+    uint32_t* done;
     uint64_t timeout_ns;
 };
 // Launched programmatically dependent on the preceding layout kernel.

@@ -136,13 +136,16 @@ EP_API int32_t ep_abi_version(void);
 EP_API const char* ep_status_string(int32_t status);
 
 /* Bytes of device workspace the calls need for a batch of num_tokens tokens
- * (status word, scan counters, per-chunk expert counts).  The same workspace
- * serves every entry point for batches up to that size. */
+ * (status word, grid-barrier word, the dispatch kernels' token ticket counter,
+ * per-chunk expert counts).  The same workspace serves every entry point for
+ * batches up to that size. */
 EP_API size_t ep_workspace_bytes(int64_t num_tokens, int32_t num_experts, int32_t num_partitions);
 
-/* Zero a workspace (once, after allocating it) on `stream`.  Zero it again
- * after a call reported EP_DEV_TIMEOUT: a layout that gave up at its grid
- * barrier leaves the barrier word mid-count. */
+/* Zero a workspace (once, after allocating it) on `stream`.  Every call leaves
+ * the barrier word and the ticket counter as it found them (the last dispatch
+ * CTA to finish re-zeroes the counter).  Zero it again after a call reported
+ * EP_DEV_TIMEOUT: a layout that gave up at its grid barrier leaves the barrier
+ * word mid-count. */
 EP_API ep_status ep_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronise `stream`, return the sticky device status bits in *bits_out and

@@ -319,3 +319,61 @@ def test_pow2_scales_on_extreme_blocks(ep):
     want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, 8, 2, quant="fp8_pow2")
     assert np.array_equal(got["recv_x"], want["recv_x"])
     assert np.array_equal(got["recv_scales"].view(np.uint32), want["recv_scales"].view(np.uint32))
+
+
+@pytest.mark.parametrize("T,K,E,P", [(40000, 8, 256, 8), (65536, 8, 256, 8), (16384, 32, 64, 8)])
+def test_layout_parity_large_batches(ep, T, K, E, P):
+    # batches whose ids no longer fit one cluster's shared memory take the
+    # cooperative-grid layout; those just below take the cluster with large chunks
+    w = make_custom(T, 128, K, E, P, seed=T + K, mask_frac=0.05)
+    lay, ws = gpu_layout(ep, w.topk_idx, E, P)
+    got = layout_numpy(lay, T, K)
+    _assert_layout(got, oracle.layout(w.topk_idx, E, P))
+    assert ep.ep_read_status(ws) == 0
+
+
+def test_dispatch_ticket_words_return_to_zero(ep):
+    # the dispatch kernels hand tokens out from a counter in the workspace header
+    # (bytes 16..23); the last CTA to finish re-zeroes it for the next call
+    ws = new_workspace(ep, 700, 256, 8)
+    for name, T, H in (("normal", 700, 256), ("bf16", 333, 136), ("normal", 5, 128)):
+        w = make_workload(name, seed=T, num_tokens=T, hidden=H)
+        quant = w.quant if H % 128 == 0 else "none"
+        got, _ = gpu_dispatch(ep, w, workspace=ws, quant=quant)
+        want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, w.num_experts, w.num_partitions,
+                               quant=quant)
+        assert np.array_equal(got["recv_x"], want["recv_x"])
+        assert np.array_equal(got["src_of"], want["src_of"])
+        assert ws[16:24].cpu().numpy().tolist() == [0] * 8
+
+
+def test_quantiser_quotients_on_exact_midpoints(ep):
+    # Blocks whose scale s = c * 2^k has few significant bits (c in 1, 3, 5) and whose
+    # elements are E4M3 values and midpoints times s, all exact in BF16: x / s is then
+    # exactly an E4M3 value or a tie, so a quotient off by one ulp would change the
+    # code.  The kernel's quotient (Markstein correction step) must give the oracle's
+    # IEEE division result everywhere.
+    rng = np.random.default_rng(77)
+    codes = np.arange(0x7F)
+    E_, m_ = codes >> 3, codes & 7
+    vals = np.where(E_ == 0, m_ * 2.0 ** -9, (1 + m_ / 8.0) * 2.0 ** (E_ - 7))
+    grid = np.unique(np.concatenate([vals, (vals[:-1] + vals[1:]) / 2]))
+    T, H = 96, 1024
+    f = np.zeros((T, H), np.float64)
+    for t in range(T):
+        for b in range(H // 128):
+            c = rng.choice([1.0, 3.0, 5.0])
+            s = c * 2.0 ** int(rng.integers(-20, 13))
+            blk = rng.choice(grid, 128) * s * np.where(rng.random(128) < 0.5, -1.0, 1.0)
+            blk[rng.integers(0, 128)] = 448.0 * s * (1 if rng.random() < 0.5 else -1)
+            f[t, b * 128:(b + 1) * 128] = blk
+    x32 = f.astype(np.float32)
+    x = torch.from_numpy(x32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal((x.astype(np.uint32) << 16).view(np.float32), x32)  # exact in BF16
+    w = make_custom(T, H, 2, 8, 2, seed=78)
+    w.x[:] = x
+    for quant in ("fp8", "fp8_pow2"):
+        got, _ = gpu_dispatch(ep, w, quant=quant)
+        want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, 8, 2, quant=quant)
+        assert np.array_equal(got["recv_x"], want["recv_x"]), quant
+        assert np.array_equal(got["recv_scales"].view(np.uint32), want["recv_scales"].view(np.uint32))
