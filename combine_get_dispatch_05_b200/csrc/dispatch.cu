@@ -28,9 +28,11 @@ namespace ep {
 
 namespace {
 
-constexpr int kFp8InStages = 3;      // input ring: rows in flight from HBM per CTA
+constexpr int kFp8InStages = 4;      // input ring: rows in flight from HBM per CTA
 constexpr int kFp8MaxOutStages = 40;  // quantised rows staged per CTA, at most
 constexpr int kFp8CtasPerSm = 2;      // the output ring fills this share of an SM
+constexpr int kFp8MaxQuantWarps = 14; // quantiser warps per CTA, at most
+constexpr int kFp8MaxThreads = 32 * (kFp8MaxQuantWarps + 2);
 constexpr int kBf16Stages = 4;        // BF16 rows in flight per CTA
 // Token log: the token of pipeline step i sits in tok[i % kTokLog] from the
 // loader's ticket until the storer has read it.  The loader runs at most
@@ -149,7 +151,7 @@ __device__ __forceinline__ void write_row_metadata(const DispatchParams& p, int 
 //       output stage (out_empty) once its stores have read it; a -1 token ends it.
 // Only the storer reads what the layout kernel wrote, so only it waits on the
 // programmatic dependency; loads and quantisation overlap the layout.
-__global__ void __launch_bounds__(352) dispatch_fp8_kernel(DispatchParams p) {
+__global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchParams p) {
     extern __shared__ __align__(128) uint8_t sm[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nq = (blockDim.x >> 5) - 2;
@@ -187,10 +189,11 @@ __global__ void __launch_bounds__(352) dispatch_fp8_kernel(DispatchParams p) {
             int issued = 0;  // bulk loads issued (steps 0 .. issued-1)
             Ring in;
             for (int i = 0;; ++i, in.next(NI)) {
+                // the ticket's round trip overlaps the wait for a free stage
+                const int t = take_ticket(p);
                 if (i >= NI && !wait_or_abort(&in_empty[in.stage], in.parity ^ 1u, p.timeout_ns,
                                               abort_flag))
                     break;
-                const int t = take_ticket(p);
                 tok[i & (kTokLog - 1)] = t;
                 if (t < 0) {
                     mbar_arrive(&in_full[in.stage]);  // the end marker: no load
@@ -324,11 +327,11 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
             int64_t issued = 0;
             for (int64_t i = 0;; ++i) {
                 const int s = static_cast<int>(i % kBf16Stages);
+                const int t = take_ticket(p);  // overlaps the wait for a free stage
                 if (i >= kBf16Stages &&
                     !wait_or_abort(&empty[s], static_cast<uint32_t>((i / kBf16Stages - 1) & 1),
                                    p.timeout_ns, abort_flag))
                     break;
-                const int t = take_ticket(p);
                 tok[i % kTokLog] = t;
                 if (t < 0) {
                     mbar_arrive(&full[s]);  // the end marker: no load
@@ -437,9 +440,11 @@ cudaError_t launch_dispatch_fp8(const DispatchParams& params, cudaStream_t strea
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(L.total));
     if (err != cudaSuccess) return err;
-    // quantiser warps: enough that each quantises the same number of block pairs
+    // quantiser warps: at most kFp8MaxQuantWarps, each quantising the same number
+    // of block pairs (a row's quantisation is a latency chain per pair, so more
+    // warps per row shorten the time a row occupies its stages)
     const int pairs = static_cast<int>((p.H / 128 + 1) / 2);
-    const int iters = (pairs + 7) / 8;
+    const int iters = (pairs + kFp8MaxQuantWarps - 1) / kFp8MaxQuantWarps;
     const int nq = (pairs + iters - 1) / iters;
     const int threads = 32 * (nq + 2);
     const int grid = grid_for(kernel, threads, L.total, p.T, dev.num_sms);
