@@ -35,8 +35,11 @@ constexpr int kFp8MaxQuantWarps = 14; // quantiser warps per CTA, at most
 constexpr int kFp8MaxThreads = 32 * (kFp8MaxQuantWarps + 2);
 constexpr int kBf16Stages = 4;        // BF16 rows in flight per CTA
 // Token log: the token of pipeline step i sits in tok[i % kTokLog] from the
-// loader's ticket until the storer has read it.  The loader runs at most
-// (input stages + output stages) steps ahead of the storer.
+// loader's ticket until the storer has read it; the storer then marks the entry
+// consumed (kTokFree).  The loader runs at most (input stages + output stages)
+// steps ahead of the storer.  The storer peeks at the next entry to prefetch that
+// token's routing: a value >= 0 there can only be the next step's token.
+constexpr int kTokFree = -2;
 constexpr int kTokLog = 64;
 static_assert(kTokLog > kFp8InStages + kFp8MaxOutStages + 1, "token log too short");
 static_assert(kTokLog > kBf16Stages + 1, "token log too short");
@@ -77,6 +80,32 @@ struct Ring {
     }
 };
 
+// One token's routing as the storer lanes hold it: lane s the row of slot s,
+// lane k routing entry k (id and weight).
+struct Routing {
+    int token = -1;
+    int row = -1;
+    int64_t e = -1;
+    float wt = 0.0f;
+};
+
+__device__ __forceinline__ Routing load_routing(const DispatchParams& p, int t, int lane) {
+    Routing r;
+    r.token = t;
+    if (lane < p.slots) r.row = p.row_of[static_cast<int64_t>(t) * p.slots + lane];
+    if (lane < p.K) {
+        r.e = p.topk_idx[static_cast<int64_t>(t) * p.K + lane];
+        r.wt = p.topk_weights[static_cast<int64_t>(t) * p.K + lane];
+    }
+    return r;
+}
+
+// Prefetch for a token log entry read without waiting: only a real token (>= 0)
+// is loaded; a free entry or the end marker gives an empty Routing.
+__device__ __forceinline__ Routing peek_routing(const DispatchParams& p, int t, int lane) {
+    return t >= 0 ? load_routing(p, t, lane) : Routing();
+}
+
 // Next token for this CTA, or -1 when the batch is exhausted.
 __device__ __forceinline__ int take_ticket(const DispatchParams& p) {
     const int t = atomicAdd(p.ticket, 1);
@@ -116,21 +145,27 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, ui
 // shuffle (all lanes take part in the shuffles).
 __device__ __forceinline__ void write_row_metadata(const DispatchParams& p, int lane, int row,
                                                    int64_t e, float wt) {
-    const int64_t epp = p.experts_per_partition;
+    // lane k < K: partition and partition-local id of routing entry k, one 32-bit
+    // division per lane (-1: not a valid expert id)
+    const int epp = p.experts_per_partition;
+    const bool valid = e >= 0 && e < p.num_experts;
+    const int ei = valid ? static_cast<int>(e) : 0;
+    const int part = valid ? ei / epp : -1;
+    const int local = ei - (valid ? part : 0) * epp;
     if (!p.dedup) {
-        if (lane < p.slots && row >= 0) {
-            p.recv_topk_idx[row] = static_cast<int32_t>(e - (e / epp) * epp);
+        if (lane < p.slots && row >= 0) {  // a row exists only for a valid id
+            p.recv_topk_idx[row] = local;
             p.recv_topk_weights[row] = wt;
         }
         return;
     }
     for (int k = 0; k < p.K; ++k) {
-        const int64_t ek = __shfl_sync(0xffffffffu, e, k);
+        const int pk = __shfl_sync(0xffffffffu, part, k);
+        const int lk = __shfl_sync(0xffffffffu, local, k);
         const float wk = __shfl_sync(0xffffffffu, wt, k);
         if (lane < p.slots && row >= 0) {
-            const bool in = ek >= 0 && ek < p.num_experts && ek / epp == lane;
-            p.recv_topk_idx[static_cast<int64_t>(row) * p.K + k] =
-                in ? static_cast<int32_t>(ek - lane * epp) : -1;
+            const bool in = pk == lane;
+            p.recv_topk_idx[static_cast<int64_t>(row) * p.K + k] = in ? lk : -1;
             p.recv_topk_weights[static_cast<int64_t>(row) * p.K + k] = in ? wk : 0.0f;
         }
     }
@@ -156,7 +191,7 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nq = (blockDim.x >> 5) - 2;
     const int64_t H = p.H;
-    const int K = p.K, nb = static_cast<int>(H >> 7);
+    const int nb = static_cast<int>(H >> 7);
     const int NI = p.in_stages, NO = p.out_stages;
     const Fp8Smem L = fp8_smem(H, NI, NO);
     uint64_t* in_full = reinterpret_cast<uint64_t*>(sm + L.off_bars);
@@ -177,6 +212,7 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
             mbar_init(&out_full[o], nq);
             mbar_init(&out_empty[o], 1);
         }
+        for (int j = 0; j < kTokLog; ++j) tok[j] = kTokFree;
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -242,17 +278,21 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
         uint8_t* recv_x = static_cast<uint8_t*>(p.recv_x);
         const int S = p.slots;
         const bool slot_lane = lane < S;  // lane s stores slot s's row
-        const bool id_lane = lane < K;    // lane k holds routing entry k
         Ring out;
         int prev = -1;  // output stage of the previous step
+        Routing next;   // prefetched routing of the next step's token
         for (int i = 0;; ++i, out.next(NO)) {
             if (!wait_or_abort(&out_full[out.stage], out.parity, p.timeout_ns, abort_flag)) break;
             const int t = tok[i & (kTokLog - 1)];
             if (t < 0) break;
             const int o = out.stage;
-            const int row = slot_lane ? p.row_of[static_cast<int64_t>(t) * S + lane] : -1;
-            const int64_t e = id_lane ? p.topk_idx[static_cast<int64_t>(t) * K + lane] : -1;
-            const float wt = id_lane ? p.topk_weights[static_cast<int64_t>(t) * K + lane] : 0.0f;
+            const Routing cur = next.token == t ? next : load_routing(p, t, lane);
+            __syncwarp();
+            if (lane == 0) tok[i & (kTokLog - 1)] = kTokFree;
+            next = peek_routing(p, tok[(i + 1) & (kTokLog - 1)], lane);
+            const int row = cur.row;
+            const int64_t e = cur.e;
+            const float wt = cur.wt;
             uint8_t* out_q = sm + L.off_out + o * L.out_bytes;
             const float* out_s = reinterpret_cast<const float*>(out_q + L.q_bytes);
             if (slot_lane) {
@@ -303,7 +343,6 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
     extern __shared__ __align__(128) uint8_t sm[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t H = p.H;
-    const int K = p.K;
     const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + kBf16Stages * row_bytes);
     uint64_t* empty = full + kBf16Stages;
@@ -315,6 +354,7 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
+        for (int j = 0; j < kTokLog; ++j) tok[j] = kTokFree;
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -355,7 +395,7 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
         uint8_t* recv_x = static_cast<uint8_t*>(p.recv_x);
         const int S = p.slots;
         const bool slot_lane = lane < S;  // lane s stores slot s's row
-        const bool id_lane = lane < K;    // lane k holds routing entry k
+        Routing next;  // prefetched routing of the next step's token
         for (int64_t i = 0;; ++i) {
             const int s = static_cast<int>(i % kBf16Stages);
             if (!wait_or_abort(&full[s], static_cast<uint32_t>((i / kBf16Stages) & 1), p.timeout_ns,
@@ -363,9 +403,13 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
                 break;
             const int t = tok[i % kTokLog];
             if (t < 0) break;
-            const int row = slot_lane ? p.row_of[static_cast<int64_t>(t) * S + lane] : -1;
-            const int64_t e = id_lane ? p.topk_idx[static_cast<int64_t>(t) * K + lane] : -1;
-            const float wt = id_lane ? p.topk_weights[static_cast<int64_t>(t) * K + lane] : 0.0f;
+            const Routing cur = next.token == t ? next : load_routing(p, t, lane);
+            __syncwarp();
+            if (lane == 0) tok[i % kTokLog] = kTokFree;
+            next = peek_routing(p, tok[(i + 1) % kTokLog], lane);
+            const int row = cur.row;
+            const int64_t e = cur.e;
+            const float wt = cur.wt;
             if (slot_lane) {
                 if (row >= 0)
                     bulk_store(recv_x + static_cast<int64_t>(row) * row_bytes, sm + s * row_bytes,
