@@ -260,7 +260,7 @@ __device__ __forceinline__ void count_chunk(const LayoutArgs& a, const Smem& s, 
                 const int64_t e = a.topk_idx[(t0 + tl) * a.K_src + k];
                 const bool ok = e >= 0 && e < a.E_src;
                 bad |= (e != -1) && !ok;
-                if (ok) mask |= 1ull << (e / a.epp_src);
+                if (ok) mask |= 1ull << (static_cast<int>(e) / a.epp_src);  // 32-bit division
             }
             s.tmask[tl] = mask;
             for (int p = 0; p < K; ++p) {

@@ -75,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.oracle_partition_identity.argtypes = [_i64, _i64, _i32, _i32, _p, _p, _p, _p, _p]
         L.oracle_partition_identity.restype = None
         L.oracle_combine_dedup.argtypes = [_i64, _i64, _i32, _p, _i64, _p, _p]
+        L.oracle_lb_prefetch_weights.argtypes = [_i32, _i64, _p, _p]
+        L.oracle_lb_prefetch_weights.restype = ctypes.c_uint32
+        L.oracle_lb_reduce_grads.argtypes = [_i32, _i64, _p, _p]
+        L.oracle_lb_reduce_grads.restype = ctypes.c_uint32
         L.oracle_combine_dedup.restype = ctypes.c_uint32
         _lib = L
     return _lib
@@ -365,3 +369,21 @@ def combine_dedup(part_out: np.ndarray, prow_of: np.ndarray):
     po_p = po if rows else np.zeros((1, H), np.uint16)
     st = lib().oracle_combine_dedup(T, H, P, _ptr(po_p), rows, _ptr(pr), _ptr(y))
     return y, int(st)
+
+
+def lb_prefetch_weights(weights: np.ndarray, primary_of: np.ndarray):
+    """weights: uint8 [S, nbytes] (a copy is returned); primary_of: int32 [S]."""
+    w = np.array(weights, dtype=np.uint8, order="C", copy=True)
+    S, nbytes = w.shape
+    po = _c(primary_of, np.int32)
+    st = lib().oracle_lb_prefetch_weights(S, nbytes, _ptr(po), _ptr(w))
+    return w, int(st)
+
+
+def lb_reduce_grads(grads: np.ndarray, primary_of: np.ndarray):
+    """grads: float32 [S, n] (a copy is returned); primary_of: int32 [S]."""
+    g = np.array(grads, dtype=np.float32, order="C", copy=True)
+    S, n = g.shape
+    po = _c(primary_of, np.int32)
+    st = lib().oracle_lb_reduce_grads(S, n, _ptr(po), _ptr(g))
+    return g, int(st)

@@ -562,3 +562,65 @@ uint32_t oracle_combine_dedup(int64_t T, int64_t H, int32_t P, const uint16_t* p
     }
     return status;
 }
+
+/* ---------------------------------------------------- redundant experts -- */
+/*
+ * Expert replication for load balancing.  Pages: "deepseek-ai/DeepEP"
+ * (agentlenshq.com), section "主要特性" (redundant-expert support through
+ * lb_prefetch_weights / lb_reduce_grads) and section "典型工作流程", step 5
+ * (optionally replicate heavily loaded experts across NVLink-connected GPUs);
+ * the page's opening paragraph adds that the kernels prefetch expert weights
+ * and reduce redundant gradients.  The pages name the calls and their purpose
+ * only.  This library's reading, with one GPU's expert slots standing for the
+ * ranks' slots:
+ *  - primary_of[s] is the slot holding the authoritative copy of slot s's
+ *    expert; a primary names itself, a replica names its primary.
+ *  - prefetch_weights: every replica slot receives a byte copy of its
+ *    primary's weight blob; primaries are left as they are.
+ *  - reduce_grads: the fp32 gradients of a primary and its replicas are summed
+ *    in ascending slot order (the first slot's value, then one binary32 add per
+ *    further slot), and the sum is written to every slot of the group, so all
+ *    copies apply the same update.  A slot whose primary_of entry is out of
+ *    range, or names a slot that is not a primary, is skipped (status bit 1).
+ */
+static int oracle_lb_valid(int32_t S, const int32_t* primary_of, int32_t s) {
+    int32_t q = primary_of[s];
+    return q >= 0 && q < S && primary_of[q] == q;
+}
+
+uint32_t oracle_lb_prefetch_weights(int32_t S, int64_t nbytes, const int32_t* primary_of,
+                                    uint8_t* weights) {
+    uint32_t status = 0;
+    for (int32_t s = 0; s < S; ++s) {
+        if (!oracle_lb_valid(S, primary_of, s)) {
+            status |= ORACLE_INDEX_RANGE;
+            continue;
+        }
+        int32_t q = primary_of[s];
+        if (q != s) memcpy(weights + (int64_t)s * nbytes, weights + (int64_t)q * nbytes, (size_t)nbytes);
+    }
+    return status;
+}
+
+uint32_t oracle_lb_reduce_grads(int32_t S, int64_t n, const int32_t* primary_of, float* grads) {
+    uint32_t status = 0;
+    float* acc = (float*)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+    for (int32_t s = 0; s < S; ++s)
+        if (!oracle_lb_valid(S, primary_of, s)) status |= ORACLE_INDEX_RANGE;
+    for (int32_t q = 0; q < S; ++q) {
+        if (primary_of[q] != q) continue; /* q is not a primary */
+        int first = 1;
+        for (int32_t s = 0; s < S; ++s) { /* ascending slot order */
+            if (!oracle_lb_valid(S, primary_of, s) || primary_of[s] != q) continue;
+            const float* g = grads + (int64_t)s * n;
+            for (int64_t i = 0; i < n; ++i) acc[i] = first ? g[i] : acc[i] + g[i];
+            first = 0;
+        }
+        for (int32_t s = 0; s < S; ++s) {
+            if (!oracle_lb_valid(S, primary_of, s) || primary_of[s] != q) continue;
+            memcpy(grads + (int64_t)s * n, acc, sizeof(float) * (size_t)n);
+        }
+    }
+    free(acc);
+    return status;
+}

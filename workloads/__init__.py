@@ -220,8 +220,12 @@ def _stress(seed: int, T: Optional[int], H: Optional[int]) -> Workload:
     idx = slot[logical]
     use_replica = (replica[logical] >= 0) & ((np.arange(T) % 2)[:, None] == 1)
     idx = np.where(use_replica, replica[logical], idx).astype(np.int64)
+    # slot -> the slot holding its expert's primary copy (primaries name themselves)
+    primary_of = np.empty(288, dtype=np.int32)
+    primary_of[slot] = slot
+    primary_of[replica[hottest]] = slot[hottest]
     return _build("stress", seed, T, H, K, 288, P, "fp8", x, idx, w, hottest=hottest,
-                  logical_idx=logical)
+                  logical_idx=logical, primary_of=primary_of)
 
 
 WORKLOADS = {
