@@ -425,6 +425,55 @@ def time_backward(ep, runner, steps):
     return out
 
 
+def time_lb(ep, dev, steps, seed):
+    """Redundant experts on the stress workload's 288-slot map (32 replicas of the
+    hottest experts): weight prefetch with one FP8 expert per slot (gate, up and
+    down projections, 3 x 7168 x 2048 bytes) and the fp32 gradient reduce over
+    one 7168 x 2048 matrix per slot, each captured as a CUDA graph."""
+    import numpy as np
+    import torch
+    from workloads import make_workload
+
+    po = make_workload("stress", seed=seed, num_tokens=64, hidden=128).meta["primary_of"]
+    S = po.size
+    groups = np.bincount(po, minlength=S)
+    replicas = int((po != np.arange(S)).sum())
+    in_groups = int(groups[po][groups[po] > 1].size)  # slots whose group has > 1 member
+    nbytes = 3 * 7168 * 2048
+    n = 7168 * 2048
+    dpo = torch.from_numpy(po).to(dev)
+    weights = torch.empty((S, nbytes), dtype=torch.uint8, device=dev)
+    grads = torch.zeros((S, n), dtype=torch.float32, device=dev)
+    ws = torch.empty(ep.ep_workspace_bytes(1, 1, 1), dtype=torch.uint8, device=dev)
+    ep.ep_workspace_init(ws)
+    out = {"slots": S, "replicas": replicas, "bytes_per_slot": nbytes, "grad_floats_per_slot": n}
+    cases = (("prefetch_weights", lambda: ep.ep_lb_prefetch_weights(dpo, weights, ws),
+              2 * replicas * nbytes),
+             ("reduce_grads", lambda: ep.ep_lb_reduce_grads(dpo, grads, ws), 2 * in_groups * n * 4))
+    for name, fn, nb in cases:
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        evs[0].record()
+        for i in range(steps):
+            g.replay()
+            evs[i + 1].record()
+        torch.cuda.synchronize()
+        us = statistics.mean(evs[i].elapsed_time(evs[i + 1]) for i in range(steps)) * 1e3
+        out[name] = {"us": round(us, 2), "bytes": nb, "gbs": round(nb / (us * 1e-6) / 1e9, 1)}
+    if ep.ep_read_status(ws) != 0:
+        raise RuntimeError("device status set in the redundant-expert run")
+    del weights, grads
+    torch.cuda.empty_cache()
+    return out
+
+
 def time_dedup(ep, w, dev, steps):
     """Deduplicated dispatch (one row per token and partition) and its combine on
     workload w, each captured as a CUDA graph; the partition outputs come from a
@@ -725,6 +774,10 @@ def run_ours(args):
             extra["dedup"]["workload"] = args.workload
         except Exception as exc:
             extra["dedup"] = {"error": repr(exc)}
+        try:
+            extra["lb"] = time_lb(ep, dev, 20, args.seed)
+        except Exception as exc:  # report, do not hide
+            extra["lb"] = {"error": repr(exc)}
         try:
             extra["ll"] = time_low_latency(ep, make_workload("ll", seed=args.seed), dev)
         except Exception as exc:  # report, do not hide

@@ -15,8 +15,9 @@ from ._lib import (  # noqa: F401
     EP_QUANT_NONE, EpError,
     Layout, LowLatencyHandle, LIB_PATH, ep_combine, ep_combine_backward, ep_debug_wait_probe,
     ep_combine_dedup, ep_dispatch, ep_dispatch_backward, ep_dispatch_dedup,
-    ep_get_dispatch_layout, ep_low_latency_combine, ep_low_latency_dispatch, ep_read_status,
-    ep_workspace_bytes, ep_workspace_init, lib, status_string,
+    ep_get_dispatch_layout, ep_lb_prefetch_weights, ep_lb_reduce_grads, ep_low_latency_combine,
+    ep_low_latency_dispatch, ep_read_status, ep_workspace_bytes, ep_workspace_init, lib,
+    status_string,
 )
 from .buffer import Buffer  # noqa: F401
 

@@ -26,7 +26,7 @@ EXPORTED = (
     "ep_read_status", "ep_get_dispatch_layout", "ep_dispatch", "ep_combine",
     "ep_low_latency_dispatch", "ep_low_latency_combine", "ep_debug_wait_probe",
     "ep_get_dispatch_layout_static", "ep_dispatch_backward", "ep_combine_backward",
-    "ep_dispatch_dedup", "ep_combine_dedup",
+    "ep_dispatch_dedup", "ep_combine_dedup", "ep_lb_prefetch_weights", "ep_lb_reduce_grads",
 )
 
 
@@ -74,6 +74,10 @@ def _load() -> ctypes.CDLL:
                                          ctypes.POINTER(ep_ll_handle), vp, vp, vp, sz, vp]
     L.ep_low_latency_combine.restype = st
     L.ep_debug_wait_probe.argtypes, L.ep_debug_wait_probe.restype = [ctypes.c_uint64, vp, sz, vp], st
+    L.ep_lb_prefetch_weights.argtypes = [i32, i64, vp, vp, vp, sz, vp]
+    L.ep_lb_prefetch_weights.restype = st
+    L.ep_lb_reduce_grads.argtypes = [i32, i64, vp, vp, vp, sz, vp]
+    L.ep_lb_reduce_grads.restype = st
     L.ep_get_dispatch_layout_static.argtypes = [i64, i32, i32, i32, vp,
                                                 ctypes.POINTER(ep_layout), vp]
     L.ep_get_dispatch_layout_static.restype = st
@@ -312,6 +316,36 @@ def ep_low_latency_combine(expert_out: torch.Tensor, handle: LowLatencyHandle,
     _check("ep_low_latency_combine", lib.ep_low_latency_combine(
         T, H, K, E, cap, expert_out.data_ptr(), ctypes.byref(c), topk_weights.data_ptr(),
         y.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_lb_prefetch_weights(primary_of: torch.Tensor, weights: torch.Tensor,
+                           workspace: torch.Tensor, stream=None) -> None:
+    """weights: [num_slots, ...] (any dtype, viewed as bytes per slot), updated in place."""
+    _need(primary_of, "primary_of", torch.int32)
+    S = primary_of.numel()
+    _need(weights, "weights", None)
+    if weights.shape[0] != S:
+        raise ValueError("weights must have one row (blob) per slot")
+    nbytes = weights.numel() * weights.element_size() // max(S, 1)
+    _need(workspace, "workspace", torch.uint8)
+    _check("ep_lb_prefetch_weights", lib.ep_lb_prefetch_weights(
+        S, nbytes, primary_of.data_ptr(), weights.data_ptr(), workspace.data_ptr(),
+        workspace.numel(), _stream(stream)))
+
+
+def ep_lb_reduce_grads(primary_of: torch.Tensor, grads: torch.Tensor, workspace: torch.Tensor,
+                       stream=None) -> None:
+    """grads: float32 [num_slots, n], updated in place."""
+    _need(primary_of, "primary_of", torch.int32)
+    S = primary_of.numel()
+    _need(grads, "grads", torch.float32)
+    if grads.shape[0] != S:
+        raise ValueError("grads must have one row per slot")
+    n = grads.numel() // max(S, 1)
+    _need(workspace, "workspace", torch.uint8)
+    _check("ep_lb_reduce_grads", lib.ep_lb_reduce_grads(
+        S, n, primary_of.data_ptr(), grads.data_ptr(), workspace.data_ptr(), workspace.numel(),
+        _stream(stream)))
 
 
 def ep_debug_wait_probe(timeout_ns: int, workspace: torch.Tensor, stream=None) -> None:

@@ -215,6 +215,19 @@ class Buffer:
         _lib.ep_combine_dedup(partition_out, handle, y, self.workspace)
         return y, self._event()
 
+    # -------------------------------------------------- redundant experts --
+    def lb_prefetch_weights(self, primary_of: torch.Tensor, weights: torch.Tensor):
+        """Copy each primary slot's weights into its replica slots (in place);
+        returns ``event``.  ``primary_of[s]`` names slot s's primary."""
+        _lib.ep_lb_prefetch_weights(primary_of, weights, self.workspace)
+        return self._event()
+
+    def lb_reduce_grads(self, primary_of: torch.Tensor, grads: torch.Tensor):
+        """Sum each primary's and its replicas' fp32 gradients (ascending slot
+        order) into every member of the group (in place); returns ``event``."""
+        _lib.ep_lb_reduce_grads(primary_of, grads, self.workspace)
+        return self._event()
+
     # ----------------------------------------------------------- backward --
     def dispatch_backward(self, grad_recv_x: torch.Tensor, handle: Layout,
                           grad_recv_topk_weights: Optional[torch.Tensor] = None):

@@ -416,6 +416,30 @@ ep_status ep_low_latency_combine(int64_t num_tokens, int64_t hidden, int32_t num
                       workspace, workspace_bytes, stream);
 }
 
+ep_status ep_lb_prefetch_weights(int32_t num_slots, int64_t bytes_per_slot,
+                                 const int32_t* primary_of, void* weights, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    if (num_slots < 1 || num_slots > 4096 || bytes_per_slot <= 0 || bytes_per_slot % 16 != 0)
+        return EP_ERR_SHAPE;
+    if (!primary_of || !weights || !aligned16(weights) || !workspace ||
+        workspace_bytes < kWsHeader)
+        return EP_ERR_INVALID_ARG;
+    const Workspace ws = carve_workspace(workspace, 0, 1);
+    return cuda_status(launch_lb_prefetch(num_slots, bytes_per_slot, primary_of, weights, ws.status,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_lb_reduce_grads(int32_t num_slots, int64_t n, const int32_t* primary_of, float* grads,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    if (num_slots < 1 || num_slots > 4096 || n < 0 || n % 4 != 0) return EP_ERR_SHAPE;
+    if (!primary_of || !workspace || workspace_bytes < kWsHeader) return EP_ERR_INVALID_ARG;
+    if (n > 0 && (!grads || !aligned16(grads))) return EP_ERR_INVALID_ARG;
+    if (n == 0) return EP_OK;
+    const Workspace ws = carve_workspace(workspace, 0, 1);
+    return cuda_status(launch_lb_reduce(num_slots, n, primary_of, grads, ws.status,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 ep_status ep_debug_wait_probe(uint64_t timeout_ns, void* workspace, size_t workspace_bytes,
                               void* stream) {
     if (!workspace || workspace_bytes < kWsHeader) return EP_ERR_INVALID_ARG;

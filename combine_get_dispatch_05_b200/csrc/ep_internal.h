@@ -117,6 +117,11 @@ struct LowLatencyDispatchParams {
 };
 cudaError_t launch_ll_dispatch(const LowLatencyDispatchParams& p, cudaStream_t stream);
 
+cudaError_t launch_lb_prefetch(int32_t S, int64_t nbytes, const int32_t* primary_of, void* weights,
+                               uint32_t* status, cudaStream_t stream);
+cudaError_t launch_lb_reduce(int32_t S, int64_t n, const int32_t* primary_of, float* grads,
+                             uint32_t* status, cudaStream_t stream);
+
 cudaError_t launch_wait_probe(uint32_t* status, uint32_t* flag, uint64_t timeout_ns,
                               cudaStream_t stream);
 

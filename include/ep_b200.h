@@ -339,6 +339,38 @@ EP_API ep_status ep_low_latency_combine(int64_t num_tokens, int64_t hidden, int3
 EP_API ep_status ep_debug_wait_probe(uint64_t timeout_ns, void* workspace, size_t workspace_bytes,
                               void* stream);
 
+/* ---- redundant experts ----------------------------------------------------
+ * "deepseek-ai/DeepEP" (agentlenshq.com), section "主要特性" (redundant-expert
+ * support: lb_prefetch_weights / lb_reduce_grads) and section "典型工作流程",
+ * step 5 (optionally replicate heavily loaded experts across NVLink-connected
+ * GPUs).  The pages name the calls and their purpose; this library's reading on
+ * one GPU, whose expert slots stand for the ranks' slots:
+ *   primary_of  device int32 [num_slots]: the slot holding slot s's
+ *               authoritative copy (a primary names itself, a replica its
+ *               primary).  An entry out of [0, num_slots) or naming a slot that
+ *               is not a primary is skipped and sets EP_DEV_INDEX_RANGE.
+ * Asynchronous on `stream`; the workspace carries the status word only
+ * (workspace_bytes >= 256 suffices).  Errors: EP_ERR_INVALID_ARG for NULL or
+ * misaligned pointers, EP_ERR_SHAPE for sizes out of range. */
+
+/* Copy every primary's weight blob into its replica slots.
+ *   weights  device, 16-byte aligned, [num_slots, bytes_per_slot] bytes;
+ *            primaries are read, replicas written.
+ *   bytes_per_slot > 0, a multiple of 16; 1 <= num_slots <= 4096. */
+EP_API ep_status ep_lb_prefetch_weights(int32_t num_slots, int64_t bytes_per_slot,
+                                        const int32_t* primary_of, void* weights, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/* Sum the fp32 gradients of each primary and its replicas in ascending slot order
+ * (the first member's value, then one IEEE binary32 add per further member) and
+ * write the sum to every member, so all copies apply the same update.  Groups of
+ * one are left untouched.
+ *   grads  device, 16-byte aligned, float32 [num_slots, n], updated in place.
+ *   n >= 0, a multiple of 4; 1 <= num_slots <= 4096. */
+EP_API ep_status ep_lb_reduce_grads(int32_t num_slots, int64_t n, const int32_t* primary_of,
+                                    float* grads, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
 #ifdef __cplusplus
 }
 #endif

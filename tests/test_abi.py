@@ -208,3 +208,19 @@ def test_dedup_host_checks(ep):
     assert L.ep_combine_dedup(4, 128, 33, f, 8, ctypes.byref(lay), f, f, 4096, None) == 2
     assert L.ep_combine_dedup(4, 128, 8, f, 8, None, f, f, 4096, None) == 1
     assert L.ep_combine_dedup(0, 128, 8, None, 0, ctypes.byref(lay), None, f, 4096, None) == 0
+
+
+def test_lb_host_checks(ep):
+    f = _Fake.P
+    L = ep.lib
+    pre, red = L.ep_lb_prefetch_weights, L.ep_lb_reduce_grads
+    assert pre(0, 16, f, f, f, 4096, None) == 2          # no slots
+    assert pre(4097, 16, f, f, f, 4096, None) == 2       # too many slots
+    assert pre(4, 24, f, f, f, 4096, None) == 2          # blob not a multiple of 16 bytes
+    assert pre(4, 16, None, f, f, 4096, None) == 1
+    assert pre(4, 16, f, f + 8, f, 4096, None) == 1      # weights not 16-byte aligned
+    assert pre(4, 16, f, f, f, 64, None) == 1            # workspace too small
+    assert red(4, 6, f, f, f, 4096, None) == 2           # n not a multiple of 4
+    assert red(4, -4, f, f, f, 4096, None) == 2
+    assert red(4, 8, f, f + 4, f, 4096, None) == 1       # grads not 16-byte aligned
+    assert red(4, 0, f, None, f, 4096, None) == 0        # nothing to reduce
