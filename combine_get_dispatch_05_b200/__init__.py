@@ -12,7 +12,7 @@ fails (there is no fallback implementation).
 from ._lib import (  # noqa: F401
     EP_DEV_CAPACITY, EP_DEV_INDEX_RANGE, EP_DEV_TIMEOUT, EP_ERR_CUDA, EP_ERR_INVALID_ARG,
     EP_ERR_SHAPE, EP_ERR_WORKSPACE, EP_OK, EP_QUANT_FP8_E4M3_1X128, EP_QUANT_FP8_E4M3_1X128_POW2,
-    EP_QUANT_NONE, EpError,
+    EP_QUANT_NONE, EP_QUANT_SCALES_MN_MAJOR, EpError, scales_ld,
     Layout, LowLatencyHandle, LIB_PATH, ep_combine, ep_combine_backward, ep_debug_wait_probe,
     ep_combine_dedup, ep_dispatch, ep_dispatch_backward, ep_dispatch_dedup,
     ep_get_dispatch_layout, ep_lb_prefetch_weights, ep_lb_reduce_grads, ep_low_latency_combine,

@@ -20,6 +20,16 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libep_b200.
 EP_OK, EP_ERR_INVALID_ARG, EP_ERR_SHAPE, EP_ERR_WORKSPACE, EP_ERR_CUDA = 0, 1, 2, 3, 4
 EP_DEV_INDEX_RANGE, EP_DEV_TIMEOUT, EP_DEV_CAPACITY = 0x1, 0x2, 0x4
 EP_QUANT_NONE, EP_QUANT_FP8_E4M3_1X128, EP_QUANT_FP8_E4M3_1X128_POW2 = 0, 1, 2
+EP_QUANT_SCALES_MN_MAJOR = 0x100  # OR-ed into an FP8 quant: recv_scales [H/128, ld]
+
+
+def scales_ld(rows: int) -> int:
+    """Leading dimension of block-major (MN-major) scales for `rows` worst-case rows."""
+    return (rows + 3) // 4 * 4
+
+
+def _scale_numel(quant: int, rows: int, H: int) -> int:
+    return (H // 128) * (scales_ld(rows) if quant & EP_QUANT_SCALES_MN_MAJOR else rows)
 
 EXPORTED = (
     "ep_abi_version", "ep_status_string", "ep_workspace_bytes", "ep_workspace_init",
@@ -240,9 +250,10 @@ def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Ten
     K = topk_idx.shape[1]
     _need(topk_idx, "topk_idx", torch.int64, shape=(T, K))
     _need(topk_weights, "topk_weights", torch.float32, shape=(T, K))
-    if quant in (EP_QUANT_FP8_E4M3_1X128, EP_QUANT_FP8_E4M3_1X128_POW2):
+    if quant & ~EP_QUANT_SCALES_MN_MAJOR in (EP_QUANT_FP8_E4M3_1X128, EP_QUANT_FP8_E4M3_1X128_POW2):
         _need(recv_x, "recv_x", (torch.uint8, torch.float8_e4m3fn), numel_at_least=T * K * H)
-        _need(recv_scales, "recv_scales", torch.float32, numel_at_least=T * K * (H // 128))
+        _need(recv_scales, "recv_scales", torch.float32,
+              numel_at_least=_scale_numel(quant, T * K, H))
     else:
         _need(recv_x, "recv_x", torch.bfloat16, numel_at_least=T * K * H)
     _need(recv_topk_idx, "recv_topk_idx", torch.int32, numel_at_least=T * K)
@@ -409,9 +420,10 @@ def ep_dispatch_dedup(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: tor
     rows = max(T * min(P, K), 1)
     _need(topk_idx, "topk_idx", torch.int64, shape=(T, K))
     _need(topk_weights, "topk_weights", torch.float32, shape=(T, K))
-    if quant in (EP_QUANT_FP8_E4M3_1X128, EP_QUANT_FP8_E4M3_1X128_POW2):
+    if quant & ~EP_QUANT_SCALES_MN_MAJOR in (EP_QUANT_FP8_E4M3_1X128, EP_QUANT_FP8_E4M3_1X128_POW2):
         _need(recv_x, "recv_x", (torch.uint8, torch.float8_e4m3fn), numel_at_least=rows * H)
-        _need(recv_scales, "recv_scales", torch.float32, numel_at_least=rows * (H // 128))
+        _need(recv_scales, "recv_scales", torch.float32,
+              numel_at_least=_scale_numel(quant, T * min(P, K), H))
     else:
         _need(recv_x, "recv_x", torch.bfloat16, numel_at_least=rows * H)
     _need(recv_topk_idx, "recv_topk_idx", torch.int32, numel_at_least=rows * K)

@@ -31,7 +31,7 @@ import torch
 
 from . import _lib
 from ._lib import (EP_QUANT_FP8_E4M3_1X128, EP_QUANT_FP8_E4M3_1X128_POW2, EP_QUANT_NONE,
-                   Layout, LowLatencyHandle)
+                   EP_QUANT_SCALES_MN_MAJOR, Layout, LowLatencyHandle, scales_ld)
 
 __all__ = ["Buffer"]
 
@@ -90,12 +90,14 @@ class Buffer:
     # ----------------------------------------------------------- dispatch --
     def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
                  num_experts: Optional[int] = None, use_fp8: bool = True, exact: bool = True,
-                 pow2_scales: bool = False):
+                 pow2_scales: bool = False, scales_mn_major: bool = False):
         """Returns ``(recv_x, recv_topk_idx, recv_topk_weights, handle, event)``.
 
         With ``use_fp8`` recv_x is ``(payload float8_e4m3fn [R, H], scales float32
         [R, H/128])``; otherwise a BF16 ``[R, H]`` tensor.  ``pow2_scales`` rounds
-        every scale up to a power of two.  ``exact`` trims the
+        every scale up to a power of two; ``scales_mn_major`` stores the scales
+        block-major (the [R, H/128] tensor is then a strided view of an
+        [H/128, ld] buffer, the layout FP8 grouped GEMMs read).  ``exact`` trims the
         worst-case (T*K-row) buffers to the R received rows, which reads R back to
         the host once; ``exact=False`` returns the untrimmed buffers and never
         synchronises (R is then ``handle.num_recv`` on the device).
@@ -112,11 +114,16 @@ class Buffer:
         recv_topk_weights = torch.empty(rows, dtype=torch.float32, device=dev)
         if use_fp8:
             recv_q = torch.empty((rows, H), dtype=torch.float8_e4m3fn, device=dev)
-            recv_s = torch.empty((rows, H // 128), dtype=torch.float32, device=dev)
+            quant = EP_QUANT_FP8_E4M3_1X128_POW2 if pow2_scales else EP_QUANT_FP8_E4M3_1X128
+            if scales_mn_major:
+                quant |= EP_QUANT_SCALES_MN_MAJOR
+                flat = torch.empty((H // 128, scales_ld(rows)), dtype=torch.float32, device=dev)
+                recv_s = flat.t()[:rows]
+            else:
+                flat = recv_s = torch.empty((rows, H // 128), dtype=torch.float32, device=dev)
             _lib.ep_dispatch(x, topk_idx, topk_weights, self.num_experts, self.num_partitions,
-                             EP_QUANT_FP8_E4M3_1X128_POW2 if pow2_scales
-                             else EP_QUANT_FP8_E4M3_1X128, recv_q, recv_s, recv_topk_idx,
-                             recv_topk_weights, handle, self.workspace)
+                             quant, recv_q, flat, recv_topk_idx, recv_topk_weights, handle,
+                             self.workspace)
         else:
             recv_q = torch.empty((rows, H), dtype=torch.bfloat16, device=dev)
             recv_s = None

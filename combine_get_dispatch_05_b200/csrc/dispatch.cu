@@ -201,7 +201,9 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
     int* rows_sm = reinterpret_cast<int*>(sm + L.off_rows);
     volatile int* tok = reinterpret_cast<volatile int*>(sm + L.off_tok);
     volatile int* abort_flag = reinterpret_cast<int*>(sm + L.off_flag);
-    const bool scale_bulk = (static_cast<uint32_t>(nb) * 4u) == L.s_bytes;
+    // row-major scales whose row is a whole number of 16-byte units go out with the
+    // row's bulk store; otherwise (and block-major) the storer writes them one by one
+    const bool scale_bulk = !p.scales_mn && (static_cast<uint32_t>(nb) * 4u) == L.s_bytes;
 
     if (tid == 0) {
         for (int s = 0; s < NI; ++s) {
@@ -311,7 +313,11 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
                 for (int idx = lane; idx < S * nb; idx += 32) {
                     const int k = idx / nb, b = idx - k * nb;
                     const int r = rows_sm[o * 32 + k];
-                    if (r >= 0) p.recv_scales[static_cast<int64_t>(r) * nb + b] = out_s[b];
+                    if (r >= 0) {
+                        const int64_t at = p.scales_mn ? b * p.scales_ld + r
+                                                       : static_cast<int64_t>(r) * nb + b;
+                        p.recv_scales[at] = out_s[b];
+                    }
                 }
             }
             // release the previous output stage once this warp's stores have read it

@@ -144,10 +144,13 @@ ep_status ep_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk, int3
                       const float* topk_weights, void* recv_x, float* recv_scales,
                       int32_t* recv_topk_idx, float* recv_topk_weights, const ep_layout* handle,
                       void* workspace, size_t workspace_bytes, void* stream) {
+    const bool scales_mn = (quant & EP_QUANT_SCALES_MN_MAJOR) != 0;
+    quant &= ~EP_QUANT_SCALES_MN_MAJOR;
     if (quant != EP_QUANT_NONE && quant != EP_QUANT_FP8_E4M3_1X128 &&
         quant != EP_QUANT_FP8_E4M3_1X128_POW2)
         return EP_ERR_INVALID_ARG;
     const bool fp8 = quant != EP_QUANT_NONE;
+    if (scales_mn && !fp8) return EP_ERR_INVALID_ARG;  // BF16 rows carry no scales
     ep_status st = check_routing(num_tokens, num_topk, num_experts, num_partitions);
     if (st != EP_OK) return st;
     if ((st = check_hidden(hidden, fp8)) != EP_OK) return st;
@@ -174,6 +177,8 @@ ep_status ep_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk, int3
     p.slots = num_topk;
     p.dedup = 0;
     p.pow2_scales = quant == EP_QUANT_FP8_E4M3_1X128_POW2 ? 1 : 0;
+    p.scales_mn = scales_mn ? 1 : 0;
+    p.scales_ld = (num_tokens * num_topk + 3) / 4 * 4;
     p.num_experts = num_experts;
     p.experts_per_partition = num_experts / num_partitions;
     p.x = x;
@@ -224,10 +229,13 @@ ep_status ep_dispatch_dedup(int64_t num_tokens, int64_t hidden, int32_t num_topk
                             void* recv_x, float* recv_scales, int32_t* recv_topk_idx,
                             float* recv_topk_weights, const ep_layout* handle, void* workspace,
                             size_t workspace_bytes, void* stream) {
+    const bool scales_mn = (quant & EP_QUANT_SCALES_MN_MAJOR) != 0;
+    quant &= ~EP_QUANT_SCALES_MN_MAJOR;
     if (quant != EP_QUANT_NONE && quant != EP_QUANT_FP8_E4M3_1X128 &&
         quant != EP_QUANT_FP8_E4M3_1X128_POW2)
         return EP_ERR_INVALID_ARG;
     const bool fp8 = quant != EP_QUANT_NONE;
+    if (scales_mn && !fp8) return EP_ERR_INVALID_ARG;  // BF16 rows carry no scales
     ep_status st = check_routing(num_tokens, num_topk, num_experts, num_partitions);
     if (st != EP_OK) return st;
     if (num_partitions > 32) return EP_ERR_SHAPE;  // one storer lane per partition
@@ -256,6 +264,8 @@ ep_status ep_dispatch_dedup(int64_t num_tokens, int64_t hidden, int32_t num_topk
     p.slots = num_partitions;
     p.dedup = 1;
     p.pow2_scales = quant == EP_QUANT_FP8_E4M3_1X128_POW2 ? 1 : 0;
+    p.scales_mn = scales_mn ? 1 : 0;
+    p.scales_ld = (num_tokens * (num_partitions < num_topk ? num_partitions : num_topk) + 3) / 4 * 4;
     p.num_experts = num_experts;
     p.experts_per_partition = num_experts / num_partitions;
     p.x = x;

@@ -48,6 +48,8 @@ struct DispatchParams {
     int32_t slots;   // receive rows per token in row_of: K, or P when dedup
     int32_t dedup;   // 1: a row per (token, partition) with [rows, K] expert lists
     int32_t pow2_scales;  // FP8: power-of-two block scales
+    int32_t scales_mn;    // FP8: recv_scales block-major, [H/128][scales_ld]
+    int64_t scales_ld;
     int32_t in_stages;    // FP8: input ring depth (rows in flight from HBM per CTA)
     int32_t out_stages;   // FP8: quantised rows staged per CTA
     int32_t num_experts;

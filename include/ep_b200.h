@@ -96,6 +96,16 @@ typedef enum ep_quant {
                                          take exponent-only scales); x / s is exact */
 } ep_quant;
 
+/* OR-ed into an FP8 `quant` of ep_dispatch / ep_dispatch_dedup: write recv_scales
+ * MN-major (block-major), the layout FP8 grouped GEMMs read with TMA: the scale
+ * of row r, block b at recv_scales[b * ld + r], ld = the worst-case row count
+ * (T*K, resp. T*min(P, K)) rounded up to a multiple of 4, so every block's column
+ * starts on a 16-byte boundary; recv_scales then holds (H/128) * ld floats.  The
+ * values are those of the row-major layout.  The pages fix no scale layout; this
+ * is a reading for the downstream expert GEMM ("deepseek-ai/DeepEP", section
+ * "典型工作流程": dispatch, then the expert GEMM). */
+#define EP_QUANT_SCALES_MN_MAJOR 0x100
+
 /*
  * The layout of one batch, and the `handle` that dispatch returns and combine
  * consumes (deepseek.csdn.net/67bd3eb22e30c863900615cc, "使用示例": dispatch

@@ -94,6 +94,8 @@ def _dispatch(ep, T=16, H=256, K=4, E=8, P=2, quant=1, ws_bytes=1 << 20, **over)
     (dict(E=4097, P=1), 2), (dict(T=-1), 2), (dict(H=200), 2), (dict(H=0), 2),
     (dict(H=16512), 2), (dict(quant=1, H=136), 2), (dict(quant=5), 1), (dict(x=None), 1),
     (dict(quant=2, H=136), 2), (dict(quant=2, rs=None), 1), (dict(quant=3), 1),
+    (dict(quant=0x100), 1), (dict(quant=0x200 | 1), 1), (dict(quant=0x101, rs=None), 1),
+    (dict(quant=0x102, H=136), 2),
     (dict(rs=None), 1), (dict(x=_Fake.P + 8), 1), (dict(rx=_Fake.P + 4), 1), (dict(rs=_Fake.P + 4), 1),
     (dict(ws=None), 1), (dict(ws=_Fake.P + 8), 1), (dict(lay=None), 1), (dict(ws_bytes=64), 3),
     (dict(T=1 << 28, K=8), 2),

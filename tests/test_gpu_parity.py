@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
 import oracle  # noqa: E402
 from workloads import make_custom, make_workload, random_bf16  # noqa: E402
 
-from gpu_path import (bf16_to_u16, gpu_combine, gpu_dispatch, gpu_layout,  # noqa: E402
+from gpu_path import (bf16_to_u16, dev_u16_as_bf16, gpu_combine, gpu_dispatch, gpu_layout,  # noqa: E402
                       layout_numpy, new_workspace, torch_identity_expert)
 
 
@@ -377,3 +377,47 @@ def test_quantiser_quotients_on_exact_midpoints(ep):
         want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, 8, 2, quant=quant)
         assert np.array_equal(got["recv_x"], want["recv_x"]), quant
         assert np.array_equal(got["recv_scales"].view(np.uint32), want["recv_scales"].view(np.uint32))
+
+
+@pytest.mark.parametrize("quant,name,mk", [
+    ("fp8", "normal-300", lambda: make_workload("normal", seed=1, num_tokens=300, hidden=512)),
+    ("fp8_pow2", "masked", lambda: make_custom(513, 640, 6, 64, 16, seed=10, mask_frac=0.3)),
+    ("fp8", "t1", lambda: make_custom(1, 128, 8, 256, 8, seed=6)),
+])
+def test_dispatch_block_major_scales(ep, quant, name, mk):
+    # EP_QUANT_SCALES_MN_MAJOR: the scale of row r, block b at [b * ld + r],
+    # ld = T*K rounded up to 4; entries past the received rows are not written
+    w = mk()
+    T, H, K, E, P = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
+    nb, ld = H // 128, ep.scales_ld(T * K)
+    x = dev_u16_as_bf16(w.x)
+    idx = torch.from_numpy(np.ascontiguousarray(w.topk_idx)).cuda()
+    wts = torch.from_numpy(np.ascontiguousarray(w.topk_weights)).cuda()
+    rq = torch.empty((T * K, H), dtype=torch.uint8, device="cuda")
+    rs = torch.full((nb * ld + 4,), float("nan"), dtype=torch.float32, device="cuda")
+    ri = torch.empty(T * K, dtype=torch.int32, device="cuda")
+    rw = torch.empty(T * K, dtype=torch.float32, device="cuda")
+    lay = ep.Layout.empty(T, K, E, P, "cuda")
+    ws = new_workspace(ep, T, E, P)
+    base = {"fp8": ep.EP_QUANT_FP8_E4M3_1X128, "fp8_pow2": ep.EP_QUANT_FP8_E4M3_1X128_POW2}[quant]
+    ep.ep_dispatch(x, idx, wts, E, P, base | ep.EP_QUANT_SCALES_MN_MAJOR, rq, rs, ri, rw, lay, ws)
+    torch.cuda.synchronize()
+    want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, E, P, quant=quant)
+    R = int(want["num_recv"][0])
+    got = rs[:nb * ld].view(nb, ld).cpu().numpy()
+    assert np.array_equal(got[:, :R].T.view(np.uint32), want["recv_scales"].view(np.uint32))
+    assert np.all(np.isnan(got[:, R:])) and bool(torch.isnan(rs[nb * ld:]).all())
+    assert np.array_equal(rq[:R].cpu().numpy(), want["recv_x"])
+    assert ep.ep_read_status(ws) == 0
+
+
+def test_buffer_block_major_scales_view(ep):
+    w = make_workload("normal", seed=3, num_tokens=200, hidden=256)
+    buf = ep.Buffer(num_experts=256, num_partitions=8, max_tokens=256)
+    x = dev_u16_as_bf16(w.x)
+    idx = torch.from_numpy(w.topk_idx).cuda()
+    wts = torch.from_numpy(w.topk_weights).cuda()
+    (q1, s1), *_ = buf.dispatch(x, idx, wts, scales_mn_major=True)
+    (q0, s0), *_ = buf.dispatch(x, idx, wts)
+    assert s1.shape == s0.shape and s1.stride(0) == 1  # an [R, H/128] view, block-major
+    assert torch.equal(s1, s0) and torch.equal(q1.view(torch.uint8), q0.view(torch.uint8))
