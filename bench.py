@@ -425,7 +425,7 @@ def time_backward(ep, runner, steps):
     return out
 
 
-def time_lb(ep, dev, steps, seed):
+def time_lb(ep, dev, steps, seed, scale=1):
     """Redundant experts on the stress workload's 288-slot map (32 replicas of the
     hottest experts): weight prefetch with one FP8 expert per slot (gate, up and
     down projections, 3 x 7168 x 2048 bytes) and the fp32 gradient reduce over
@@ -439,8 +439,8 @@ def time_lb(ep, dev, steps, seed):
     groups = np.bincount(po, minlength=S)
     replicas = int((po != np.arange(S)).sum())
     in_groups = int(groups[po][groups[po] > 1].size)  # slots whose group has > 1 member
-    nbytes = 3 * 7168 * 2048
-    n = 7168 * 2048
+    nbytes = 3 * 7168 * 2048 // scale // 16 * 16
+    n = 7168 * 2048 // scale // 4 * 4
     dpo = torch.from_numpy(po).to(dev)
     weights = torch.empty((S, nbytes), dtype=torch.uint8, device=dev)
     grads = torch.zeros((S, n), dtype=torch.float32, device=dev)
@@ -775,7 +775,7 @@ def run_ours(args):
         except Exception as exc:
             extra["dedup"] = {"error": repr(exc)}
         try:
-            extra["lb"] = time_lb(ep, dev, 20, args.seed)
+            extra["lb"] = time_lb(ep, dev, min(args.extra_steps, 20), args.seed, args.lb_scale)
         except Exception as exc:  # report, do not hide
             extra["lb"] = {"error": repr(exc)}
         try:
@@ -881,6 +881,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the ll/skew/bf16/stress configs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lb-scale", type=int, default=1,
+                    help="divide the redundant-expert per-slot sizes by this (small profiling case)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
