@@ -37,6 +37,9 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "dispatch/combine HBM GB/s (% of B200 peak) at 4096x7168 top-8; LL latency µs"
+DTYPE_TEXT = {True: "f32 arithmetic; fp8-e4m3 dispatch payload, bf16 combine",
+              False: "f32 arithmetic; bf16 dispatch payload, bf16 combine"}
+
 WORKLOAD_TEXT = {
     "normal": "normal: 4096 tokens x hidden 7168 BF16, top-8 of 256 experts in 8 logical "
               "partitions, top-4-of-8-group routing, FP8 (E4M3, 1x128 scales) dispatch + BF16 "
@@ -724,7 +727,7 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32 arithmetic; fp8-e4m3 dispatch payload, bf16 combine",
+        "dtype": DTYPE_TEXT[runner.fp8],
         "data": "synthetic",
         "config": {
             "workload": WORKLOAD_TEXT[args.workload],
@@ -815,16 +818,17 @@ def run_reference(args):
     import oracle
     from workloads import make_workload
 
-    w = make_workload("normal", seed=args.seed)
+    w = make_workload(args.workload, seed=args.seed)
     T, H, K, E, P = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
+    fp8 = w.quant == "fp8"
 
     def make_step(n):
         xs, idxs, wts = w.x[:n], w.topk_idx[:n], w.topk_weights[:n]
-        ds = oracle.dispatch(xs, idxs, wts, E, P)
-        eos = oracle.identity_expert(ds["recv_x"], ds["recv_scales"])
+        ds = oracle.dispatch(xs, idxs, wts, E, P, quant=w.quant)
+        eos = oracle.identity_expert(ds["recv_x"], ds.get("recv_scales"), quant=w.quant)
 
         def step():
-            dx = oracle.dispatch(xs, idxs, wts, E, P)
+            dx = oracle.dispatch(xs, idxs, wts, E, P, quant=w.quant)
             oracle.combine(eos, dx["row_of"], wts)
         return step, int(ds["num_recv"][0])
 
@@ -838,7 +842,7 @@ def run_reference(args):
     budget = 120.0 / max(1, args.steps + args.warmup)
     S = int(max(1, min(T, budget / per_tok)))
     step, R = make_step(S)
-    bd, bc = algorithmic_bytes(S, H, K, E, P, R, True)
+    bd, bc = algorithmic_bytes(S, H, K, E, P, R, fp8)
 
     for _ in range(args.warmup):
         step()
@@ -849,16 +853,17 @@ def run_reference(args):
         times.append(time.perf_counter() - t)
     ms = statistics.mean(times) * 1e3
     value = (bd + bc) / (ms * 1e-3) / 1e9
-    sample = (f"first {S} of {T} tokens of the normal workload per step (layout + FP8 dispatch + "
-              f"combine), single-threaded C oracle")
+    sample = (f"first {S} of {T} tokens of the {args.workload} workload per step (layout + "
+              f"{'FP8' if fp8 else 'BF16'} dispatch + combine), single-threaded C oracle")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32 arithmetic; fp8-e4m3 dispatch payload, bf16 combine",
+        "vs_baseline": None, "dtype": DTYPE_TEXT[fp8],
         "data": "synthetic",
-        "config": {"workload": "normal: 4096 tokens x hidden 7168, top-8 of 256 experts, 8 "
-                               "partitions, FP8 dispatch + BF16 combine", "sample_tokens": S},
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "tokens_per_gpu": T, "hidden": H,
+                   "topk": K, "experts": E, "partitions": P, "seed": args.seed,
+                   "sample_tokens": S},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
