@@ -26,10 +26,16 @@ namespace {
 constexpr int kCombineMaxThreads = 512;
 constexpr int kLoadBatch = 8;  // vector loads issued before the first FMA
 
-__global__ void __launch_bounds__(kCombineMaxThreads) combine_kernel(CombineParams p,
-                                                                    int64_t vec_per_slice) {
+// kBatch: row loads issued per thread before the first FMA.  The token's valid
+// rows are compacted (k order kept) so a batch holds only rows that exist; sparse
+// routings (one slot per partition, about half of them empty) use a batch of 4 and
+// fewer registers, so more threads and more loads are in flight per SM.
+template <int kBatch>
+__global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
+    combine_kernel(CombineParams p, int64_t vec_per_slice) {
     __shared__ int rows_sm[2][32];
     __shared__ float w_sm[2][32];
+    __shared__ int cnt_sm[2];
     const int tid = threadIdx.x;
     const int K = p.K;
     const int64_t T = p.T, V = p.H / 8;
@@ -46,42 +52,49 @@ __global__ void __launch_bounds__(kCombineMaxThreads) combine_kernel(CombinePara
     }
     int buf = 0;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x, buf ^= 1) {
-        if (tid < K) {
-            int r = nrow;
+        if (tid < 32) {  // warp 0: lane k < K holds slot k
+            int r = tid < K ? nrow : -1;
             if (r >= 0 && static_cast<int64_t>(r) >= p.expert_out_rows) {
                 raise_status(p.status, kDevIndexRange);
                 r = -1;
             }
-            rows_sm[buf][tid] = r;
-            w_sm[buf][tid] = nw;
-            if (p.grad_w && blockIdx.y == 0)
-                p.grad_w[t * K + tid] = r >= 0 ? p.grad_recv_w[r] : 0.0f;
-            const int64_t tn = t + gridDim.x;
-            if (tn < T) {
-                nrow = p.row_of[tn * K + tid];
-                if (p.topk_weights) nw = p.topk_weights[tn * K + tid];
+            const unsigned valid = __ballot_sync(0xffffffffu, r >= 0);
+            if (r >= 0) {
+                const int at = __popc(valid & ((1u << tid) - 1u));
+                rows_sm[buf][at] = r;
+                w_sm[buf][at] = nw;
+            }
+            if (tid == 0) cnt_sm[buf] = __popc(valid);
+            if (tid < K) {
+                if (p.grad_w && blockIdx.y == 0)
+                    p.grad_w[t * K + tid] = r >= 0 ? p.grad_recv_w[r] : 0.0f;
+                const int64_t tn = t + gridDim.x;
+                if (tn < T) {
+                    nrow = p.row_of[tn * K + tid];
+                    if (p.topk_weights) nw = p.topk_weights[tn * K + tid];
+                }
             }
         }
         __syncthreads();
         const int* rows = rows_sm[buf];
         const float* ws = w_sm[buf];
+        const int m = cnt_sm[buf];
         for (int64_t v = v0 + tid; v < v1; v += blockDim.x) {
             float acc[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-            for (int k0 = 0; k0 < K; k0 += kLoadBatch) {
-                uint4 d[kLoadBatch];
+            for (int k0 = 0; k0 < m; k0 += kBatch) {
+                uint4 d[kBatch];
 #pragma unroll
-                for (int u = 0; u < kLoadBatch; ++u) {
+                for (int u = 0; u < kBatch; ++u) {
                     const int k = k0 + u;
-                    const int r = k < K ? rows[k] : -1;
-                    d[u] = r >= 0 ? ld_stream_v4(eo + static_cast<int64_t>(r) * V + v)
-                                  : make_uint4(0u, 0u, 0u, 0u);
+                    d[u] = k < m ? ld_stream_v4(eo + static_cast<int64_t>(rows[k]) * V + v)
+                                 : make_uint4(0u, 0u, 0u, 0u);
                 }
 #pragma unroll
-                for (int u = 0; u < kLoadBatch; ++u) {
+                for (int u = 0; u < kBatch; ++u) {
                     const int k = k0 + u;
-                    if (k < K && rows[k] >= 0) {
+                    if (k < m) {
                         const float w = ws[k];
                         acc[0] = __fmaf_rn(w, bf16_lo(d[u].x), acc[0]);
                         acc[1] = __fmaf_rn(w, bf16_hi(d[u].x), acc[1]);
@@ -213,17 +226,21 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
     slices = (V + per_slice - 1) / per_slice;
     int threads = static_cast<int>((per_slice + 31) / 32 * 32);
     if (threads > kCombineMaxThreads) threads = kCombineMaxThreads;
+    const void* kernel = p.sparse ? reinterpret_cast<const void*>(combine_kernel<4>)
+                                  : reinterpret_cast<const void*>(combine_kernel<8>);
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_kernel, threads, 0) !=
-            cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
     int64_t gx = (static_cast<int64_t>(per_sm) * dev.num_sms + slices - 1) / slices;
     if (gx > p.T) gx = p.T;
     if (gx < 1) gx = 1;
     if (gx > 2147483647LL) gx = 2147483647LL;
-    combine_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(slices)), threads, 0,
-                     stream>>>(p, per_slice);
+    const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(slices));
+    if (p.sparse)
+        combine_kernel<4><<<grid, threads, 0, stream>>>(p, per_slice);
+    else
+        combine_kernel<8><<<grid, threads, 0, stream>>>(p, per_slice);
     return cudaGetLastError();
 }
 

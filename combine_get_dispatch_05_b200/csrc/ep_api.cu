@@ -310,6 +310,7 @@ ep_status ep_combine_dedup(int64_t num_tokens, int64_t hidden, int32_t num_parti
     p.grad_recv_w = nullptr;
     p.grad_w = nullptr;
     p.status = carve_workspace(workspace, 0, 1).status;
+    p.sparse = 1;  // a token reaches few of the P partitions
     return cuda_status(launch_combine(p, static_cast<cudaStream_t>(stream)));
 }
 

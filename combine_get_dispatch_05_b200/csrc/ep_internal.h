@@ -83,6 +83,7 @@ struct CombineParams {
     const float* grad_recv_w;   // optional gather: grad_w[t, k] = grad_recv_w[row_of[t, k]]
     float* grad_w;
     uint32_t* status;
+    int32_t sparse = 0;         // about half the slots empty (one slot per partition)
 };
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 
