@@ -44,6 +44,13 @@ ep_status check_layout_ptrs(const ep_layout* lay, int64_t T) {
 
 inline ep_status cuda_status(cudaError_t e) { return e == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
 
+// EP_ERR_SHAPE if the batch is too large for the layout kernels.
+ep_status check_layout_size(int64_t T, int32_t K, int32_t E, int32_t P, bool by_partition) {
+    bool fits = true;
+    if (layout_fits(T, K, E, P, by_partition, &fits) != cudaSuccess) return EP_ERR_CUDA;
+    return fits ? EP_OK : EP_ERR_SHAPE;
+}
+
 }  // namespace
 
 cudaError_t device_info(DeviceInfo* out) {
@@ -134,6 +141,8 @@ ep_status ep_get_dispatch_layout(int64_t num_tokens, int32_t num_topk, int32_t n
         return EP_ERR_INVALID_ARG;
     if (workspace_bytes < ep_workspace_bytes(num_tokens, num_experts, num_partitions))
         return EP_ERR_WORKSPACE;
+    if ((st = check_layout_size(num_tokens, num_topk, num_experts, num_partitions, false)) != EP_OK)
+        return st;
     const Workspace ws = carve_workspace(workspace, num_tokens, num_experts);
     return cuda_status(launch_layout(num_tokens, num_topk, num_experts, num_partitions, topk_idx,
                                      *layout, ws, static_cast<cudaStream_t>(stream)));
@@ -165,6 +174,8 @@ ep_status ep_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk, int3
     }
     if (workspace_bytes < ep_workspace_bytes(num_tokens, num_experts, num_partitions))
         return EP_ERR_WORKSPACE;
+    if ((st = check_layout_size(num_tokens, num_topk, num_experts, num_partitions, false)) != EP_OK)
+        return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const Workspace ws = carve_workspace(workspace, num_tokens, num_experts);
     cudaError_t err =
@@ -252,6 +263,8 @@ ep_status ep_dispatch_dedup(int64_t num_tokens, int64_t hidden, int32_t num_topk
     }
     if (workspace_bytes < ep_workspace_bytes(num_tokens, num_experts, num_partitions))
         return EP_ERR_WORKSPACE;
+    if ((st = check_layout_size(num_tokens, num_topk, num_experts, num_partitions, true)) != EP_OK)
+        return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const Workspace ws = carve_workspace(workspace, num_tokens, num_partitions);
     cudaError_t err = launch_layout(num_tokens, num_topk, num_experts, num_partitions, topk_idx,

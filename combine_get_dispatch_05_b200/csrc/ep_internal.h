@@ -37,6 +37,11 @@ Workspace carve_workspace(void* ws, int64_t num_tokens, int32_t num_experts);
 // dependent launch).
 // by_partition: the deduplicated layout (one slot per partition, rows
 // partition-major); the layout arrays are then P-sized and row_of is [T, P].
+// Whether the layout of a batch of T tokens fits the layout kernels (each SM keeps
+// its chunk of ids in shared memory): *fits = false above about 400k tokens at
+// K = 8, E = 256.  Returns a CUDA error only if the device cannot be queried.
+cudaError_t layout_fits(int64_t T, int32_t K, int32_t E, int32_t P, bool by_partition, bool* fits);
+
 cudaError_t launch_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int64_t* topk_idx,
                           const ep_layout& lay, const Workspace& ws, cudaStream_t stream,
                           bool by_partition = false);

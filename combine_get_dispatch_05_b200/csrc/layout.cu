@@ -564,6 +564,34 @@ Workspace carve_workspace(void* ws, int64_t num_tokens, int32_t num_experts) {
     return w;
 }
 
+cudaError_t layout_fits(int64_t T, int32_t K, int32_t E, int32_t P, bool by_partition,
+                        bool* fits) {
+    if (by_partition) {
+        K = P;
+        E = P;
+    }
+    DeviceInfo dev;
+    cudaError_t err = device_info(&dev);
+    if (err != cudaSuccess) return err;
+    if (T * K <= kSingleMaxEntries) {
+        const int W = rank_warps(kSingleRankTableBytes, E, kSingleThreads / 32);
+        if (sizeof(int) * smem_ints(T > 0 ? T : 1, K, E, P, W, true, 0) <= dev.max_smem_optin) {
+            *fits = true;
+            return cudaSuccess;
+        }
+    }
+    const int64_t G = layout_grid(T, dev.num_sms);
+    int64_t chunk = (T + G - 1) / G;
+    chunk = (chunk + 31) / 32 * 32;
+    if (chunk < 32) chunk = 32;
+    const int W = rank_warps(kRankTableBytes, E, kLayoutThreads / 32);
+    int parts = (kLayoutThreads + E - 1) / E;
+    if (parts > G) parts = static_cast<int>(G);
+    if (parts < 1) parts = 1;
+    *fits = sizeof(int) * smem_ints(chunk, K, E, P, W, false, parts) <= dev.max_smem_optin;
+    return cudaSuccess;
+}
+
 cudaError_t launch_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int64_t* topk_idx,
                           const ep_layout& lay, const Workspace& ws, cudaStream_t stream,
                           bool by_partition) {

@@ -84,6 +84,10 @@ extern "C" ep_status ep_get_dispatch_layout_static(int64_t num_tokens, int32_t n
     if (ep_workspace_bytes(num_tokens, num_experts, num_partitions) > EP_STATIC_SCRATCH_BYTES)
         return EP_ERR_WORKSPACE;
 
+    bool fits = true;
+    if (layout_fits(num_tokens, num_topk, num_experts, num_partitions, false, &fits) != cudaSuccess)
+        return EP_ERR_CUDA;
+    if (!fits) return EP_ERR_SHAPE;
     void* scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return EP_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -77,7 +77,10 @@ extern "C" {
 typedef enum ep_status {
     EP_OK = 0,
     EP_ERR_INVALID_ARG = 1, /* a required pointer is NULL, misaligned, or an enum is unknown */
-    EP_ERR_SHAPE = 2,       /* a size is outside the supported range (see Conventions) */
+    EP_ERR_SHAPE = 2,       /* a size is outside the supported range (see Conventions),
+                               or a batch is too large for the layout kernels, which keep
+                               each SM's chunk of ids in shared memory (about 400k tokens
+                               at K = 8, E = 256) */
     EP_ERR_WORKSPACE = 3,   /* workspace smaller than ep_workspace_bytes() */
     EP_ERR_CUDA = 4         /* the CUDA runtime reported an error (launch / copy) */
 } ep_status;

@@ -421,3 +421,17 @@ def test_buffer_block_major_scales_view(ep):
     (q0, s0), *_ = buf.dispatch(x, idx, wts)
     assert s1.shape == s0.shape and s1.stride(0) == 1  # an [R, H/128] view, block-major
     assert torch.equal(s1, s0) and torch.equal(q1.view(torch.uint8), q0.view(torch.uint8))
+
+
+def test_layout_too_large_batch_is_a_shape_error(ep):
+    # each SM keeps its chunk of ids in shared memory: far beyond that the call
+    # returns EP_ERR_SHAPE before launching anything
+    T, K, E, P = 1 << 21, 8, 256, 8
+    idx = torch.zeros((T, K), dtype=torch.int64, device="cuda")
+    lay = ep.Layout.empty(T, K, E, P, "cuda")
+    ws = new_workspace(ep, 1, E, P)
+    with pytest.raises(ep.EpError) as err:
+        ep.ep_get_dispatch_layout(idx, E, P, lay, torch.empty(ep.ep_workspace_bytes(T, E, P),
+                                                             dtype=torch.uint8, device="cuda"))
+    assert err.value.status == ep.EP_ERR_SHAPE
+    assert ep.ep_read_status(ws) == 0
