@@ -43,28 +43,63 @@ def _noop_hook():
 class Buffer:
     """Dispatch / combine buffer for one GPU.
 
-    ``num_partitions`` logical partitions (the EP ranks of a multi-GPU run)
-    split ``num_experts`` experts into equal contiguous ranges.
-    ``max_tokens`` bounds the batch size the workspace is sized for.
+    Call shapes: ``Buffer(group, num_nvl_bytes, num_rdma_bytes[, low_latency_mode])``
+    as on the pages (deepseek.csdn.net/67bd3eb22e30c863900615cc, sections
+    "使用示例" and "推理解码阶段的应用"), or by keyword ``Buffer(num_experts=,
+    num_partitions=, max_tokens=)``.
+
+    ``num_partitions`` logical partitions (the EP ranks of a multi-GPU run) split
+    the experts into equal contiguous ranges; it defaults to ``group.size()`` when
+    a process group is given, else 1.  ``num_nvl_bytes`` / ``num_rdma_bytes`` size
+    DeepEP's peer buffers; one GPU has none, so they are recorded and unused.
+    ``low_latency_mode`` is recorded; both kinds of calls are always available.
+    ``num_experts`` may be left to the first call that passes it.  The device
+    workspace is sized for the largest batch seen so far (``max_tokens`` to start)
+    and grows, on the current stream, when a larger batch arrives.
     """
 
-    def __init__(self, num_experts: int, num_partitions: int = 1, max_tokens: int = 4096,
+    def __init__(self, group=None, num_nvl_bytes: int = 0, num_rdma_bytes: int = 0,
+                 low_latency_mode: bool = False, *, num_experts: Optional[int] = None,
+                 num_partitions: Optional[int] = None, max_tokens: int = 0,
                  device: Optional[Union[int, str, torch.device]] = None):
-        if num_experts % num_partitions:
+        if num_partitions is None:
+            num_partitions = group.size() if group is not None else 1
+        if num_experts is not None and num_experts % num_partitions:
             raise ValueError("num_experts must be a multiple of num_partitions")
         self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
             else torch.device(device)
+        self.group = group
+        self.num_nvl_bytes = num_nvl_bytes
+        self.num_rdma_bytes = num_rdma_bytes
+        self.low_latency_mode = low_latency_mode
         self.num_experts = num_experts
         self.num_partitions = num_partitions
         self.max_tokens = max_tokens
-        nbytes = _lib.ep_workspace_bytes(max_tokens, num_experts, num_partitions)
-        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
-        _lib.ep_workspace_init(self.workspace)
+        self.workspace: Optional[torch.Tensor] = None
+        self._ensure(max_tokens)
 
     # ------------------------------------------------------------ helpers --
-    def _check_tokens(self, n: int) -> None:
-        if n > self.max_tokens:
-            raise ValueError(f"{n} tokens exceed this buffer's max_tokens={self.max_tokens}")
+    def _ensure(self, num_tokens: int, num_experts: Optional[int] = None) -> None:
+        """Fix num_experts on first use and grow the workspace to fit the batch."""
+        if num_experts is not None:
+            if self.num_experts is None:
+                if num_experts % self.num_partitions:
+                    raise ValueError("num_experts must be a multiple of num_partitions")
+                self.num_experts = num_experts
+                self.workspace = None  # sized for the experts now known
+            elif num_experts != self.num_experts:
+                raise ValueError("num_experts differs from the buffer's")
+        self.max_tokens = max(self.max_tokens, num_tokens)
+        need = _lib.ep_workspace_bytes(max(self.max_tokens, 1), self.num_experts or 1,
+                                       self.num_partitions)
+        if self.workspace is None or self.workspace.numel() < need:
+            self.workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+            _lib.ep_workspace_init(self.workspace)
+
+    def _experts(self) -> int:
+        if self.num_experts is None:
+            raise ValueError("num_experts is not known yet: pass it to this call or to Buffer()")
+        return self.num_experts
 
     def _event(self) -> torch.cuda.Event:
         ev = torch.cuda.Event()
@@ -80,9 +115,10 @@ class Buffer:
         """Returns ``(num_tokens_per_expert, num_tokens_per_partition,
         is_token_in_partition, handle, event)``."""
         T, K = topk_idx.shape
-        self._check_tokens(T)
-        lay = Layout.empty(T, K, self.num_experts, self.num_partitions, self.device)
-        _lib.ep_get_dispatch_layout(topk_idx, self.num_experts, self.num_partitions, lay,
+        self._ensure(T)
+        E = self._experts()
+        lay = Layout.empty(T, K, E, self.num_partitions, self.device)
+        _lib.ep_get_dispatch_layout(topk_idx, E, self.num_partitions, lay,
                                     self.workspace)
         return (lay.num_tokens_per_expert, lay.num_tokens_per_partition,
                 lay.is_token_in_partition, lay, self._event())
@@ -102,11 +138,10 @@ class Buffer:
         the host once; ``exact=False`` returns the untrimmed buffers and never
         synchronises (R is then ``handle.num_recv`` on the device).
         """
-        if num_experts is not None and num_experts != self.num_experts:
-            raise ValueError("num_experts differs from the buffer's")
         T, H = x.shape
         K = topk_idx.shape[1]
-        self._check_tokens(T)
+        self._ensure(T, num_experts)
+        self._experts()
         rows = max(T * K, 1)
         dev = self.device
         handle = Layout.empty(T, K, self.num_experts, self.num_partitions, dev)
@@ -159,6 +194,8 @@ class Buffer:
         recv_expert_count[e] are not written.
         """
         E = self.num_experts if num_experts is None else num_experts
+        if E is None:
+            raise ValueError("num_experts is not known yet: pass it to this call or to Buffer()")
         T, H = hidden_states.shape
         K = topk_idx.shape[1]
         dev = self.device
@@ -188,7 +225,8 @@ class Buffer:
         T, H = x.shape
         K = topk_idx.shape[1]
         P = self.num_partitions
-        self._check_tokens(T)
+        self._ensure(T)
+        self._experts()
         if P > 32:
             raise ValueError("the deduplicated dispatch supports at most 32 partitions")
         rows = max(T * min(P, K), 1)

@@ -435,3 +435,31 @@ def test_layout_too_large_batch_is_a_shape_error(ep):
                                                              dtype=torch.uint8, device="cuda"))
     assert err.value.status == ep.EP_ERR_SHAPE
     assert ep.ep_read_status(ws) == 0
+
+
+class _FakeGroup:
+    """Stands in for a process group of 8 ranks (only size() is read)."""
+
+    def size(self):
+        return 8
+
+
+def test_buffer_pages_constructor_and_growing_workspace(ep):
+    # Buffer(group, num_nvl_bytes, num_rdma_bytes, low_latency_mode) as on the pages;
+    # num_experts comes with the first dispatch; a larger batch grows the workspace
+    buf = ep.Buffer(_FakeGroup(), int(1e9), 0, False)
+    assert buf.num_partitions == 8 and buf.num_experts is None
+    for T in (100, 700):
+        w = make_workload("normal", seed=T, num_tokens=T, hidden=256)
+        x = dev_u16_as_bf16(w.x)
+        idx = torch.from_numpy(w.topk_idx).cuda()
+        wts = torch.from_numpy(w.topk_weights).cuda()
+        (q, s), ri, rw, handle, ev = buf.dispatch(x, idx, wts, 256)
+        ev.synchronize()
+        want = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, 256, 8)
+        assert np.array_equal(q.view(torch.uint8).cpu().numpy(), want["recv_x"])
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), want["recv_scales"].view(np.uint32))
+        assert buf.max_tokens >= T
+    with pytest.raises(ValueError):
+        buf.dispatch(x, idx, wts, 128)  # the buffer's experts are fixed by now
+    assert buf.read_status() == 0
