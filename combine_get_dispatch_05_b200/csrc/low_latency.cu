@@ -10,8 +10,9 @@
 // One kernel does everything the normal path does in its layout and dispatch
 // kernels; each token's row is split into slices, one CTA per (token, slice):
 //   - the slice's bulk load is issued first, so its latency overlaps the rest;
-//   - slot of (t, k) in expert e = number of earlier (t', k') routed to e, counted
-//     directly over the topk_idx prefix (the batch is small, the prefix is L2-hot);
+//   - slot of (t, k) in expert e = number of earlier (t', k') routed to e: a
+//     shared-memory histogram of the earlier tokens' ids (the batch is small, the
+//     prefix is L2-hot) plus equal ids in the token's own earlier slots;
 //     the order is the normal layout's, so slot j of e holds normal row
 //     expert_offset[e] + j;
 //   - CTA 0 also histograms all T*K ids into recv_expert_count;
@@ -26,6 +27,7 @@ namespace ep {
 namespace {
 
 constexpr int kLLMaxThreads = 256;
+constexpr int kPrefixBatch = 4;  // topk_idx loads in flight per thread
 
 // Shared memory of one (token, slice) CTA: the slice's BF16 input, its E4M3 codes
 // and scales, an mbarrier, the token's K rows / slot counters / ids, and (CTA 0
@@ -88,26 +90,35 @@ __global__ void __launch_bounds__(kLLMaxThreads) ll_dispatch_kernel(LowLatencyDi
         bulk_load(sm, static_cast<const uint8_t*>(p.x) + t * H * 2 + static_cast<int64_t>(b0) * 256,
                   static_cast<uint32_t>(nbl) * 256u, bar);
     }
-    if (tid < K) {
-        eid_sm[tid] = p.topk_idx[t * K + tid];
-        cnt_sm[tid] = 0;
-    }
-    if (all)
-        for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
+    if (tid < K) eid_sm[tid] = p.topk_idx[t * K + tid];
+    for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
 
-    // slot of (t, k): pairs (t', k') < (t, k) in (token, k) order with the same expert
+    // slot of (t, k) = pairs (t', k') < (t, k) in (token, k) order with the same
+    // expert: a histogram of the ids of the earlier tokens (shared-memory atomics,
+    // kPrefixBatch loads in flight per thread), plus the equal ids among the
+    // token's own earlier slots.  CTA (0, 0) -- token 0, no earlier tokens --
+    // histograms the whole batch instead, for recv_expert_count.
     const int64_t base = t * K;
-    for (int64_t j = tid; j < base + K; j += blockDim.x) {
-        const int64_t ej = p.topk_idx[j];
-        for (int k = 0; k < K; ++k)
-            if (j < base + k && ej == eid_sm[k]) atomicAdd(&cnt_sm[k], 1);
-    }
-    if (all) {
-        for (int64_t j = tid; j < p.T * K; j += blockDim.x) {
-            const int64_t ej = p.topk_idx[j];
-            if (ej >= 0 && ej < E) atomicAdd(&hist[ej], 1);
+    const int64_t upto = all ? p.T * K : base;
+    const int64_t stride = static_cast<int64_t>(blockDim.x);
+    for (int64_t j0 = tid; j0 < upto; j0 += kPrefixBatch * stride) {
+        int64_t v[kPrefixBatch];
+#pragma unroll
+        for (int u = 0; u < kPrefixBatch; ++u) {
+            const int64_t j = j0 + u * stride;
+            v[u] = j < upto ? p.topk_idx[j] : -1;
         }
+#pragma unroll
+        for (int u = 0; u < kPrefixBatch; ++u)
+            if (v[u] >= 0 && v[u] < E) atomicAdd(&hist[v[u]], 1);
+    }
+    __syncthreads();
+    if (tid < K) {
+        const int64_t e = eid_sm[tid];
+        int same = 0;  // equal ids in this token's earlier slots
+        for (int k = 0; k < tid; ++k) same += eid_sm[k] == e ? 1 : 0;
+        cnt_sm[tid] = (t == 0 || e < 0 || e >= E ? 0 : hist[e]) + same;
     }
     __syncthreads();
     if (tid < K) {
