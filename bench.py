@@ -699,6 +699,7 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         e_ms, h2d, d2h = time_e2e(ep, runner, max(5, min(args.steps, 50)))
+        e_ms = reduce_max_over_ranks([e_ms], world, dev)[0]  # the slowest rank's time
         e2e = {"value": round(world * step_bytes / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                "ms_per_step": round(e_ms, 4), "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
