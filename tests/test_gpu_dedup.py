@@ -172,3 +172,32 @@ def test_dispatch_dedup_pow2_scales_parity(ep):
     assert np.array_equal(got["recv_x"], want["recv_x"])
     assert np.array_equal(got["recv_scales"].view(np.uint32), want["recv_scales"].view(np.uint32))
     assert got["canaries_ok"]
+
+
+def test_dispatch_dedup_block_major_pow2_scales(ep):
+    # deduplicated rows with power-of-two scales stored block-major: scale of row r,
+    # block b at [b * ld + r], ld = T * min(P, K) rounded up to 4
+    w = make_custom(301, 640, 6, 64, 16, seed=13, mask_frac=0.1)
+    T, H, K, E, P = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
+    rows = T * min(P, K)
+    nb, ld = H // 128, ep.scales_ld(rows)
+    x = dev_u16_as_bf16(w.x)
+    idx = torch.from_numpy(np.ascontiguousarray(w.topk_idx)).cuda()
+    wts = torch.from_numpy(np.ascontiguousarray(w.topk_weights)).cuda()
+    rq = torch.empty((rows, H), dtype=torch.uint8, device="cuda")
+    rs = torch.full((nb * ld,), float("nan"), dtype=torch.float32, device="cuda")
+    ri = torch.empty((rows, K), dtype=torch.int32, device="cuda")
+    rw = torch.empty((rows, K), dtype=torch.float32, device="cuda")
+    lay = ep.Layout.empty(T, P, P, P, "cuda")
+    ws = new_workspace(ep, T, E, P)
+    ep.ep_dispatch_dedup(x, idx, wts, E, P,
+                         ep.EP_QUANT_FP8_E4M3_1X128_POW2 | ep.EP_QUANT_SCALES_MN_MAJOR,
+                         rq, rs, ri, rw, lay, ws)
+    torch.cuda.synchronize()
+    want = oracle.dispatch_dedup(w.x, w.topk_idx, w.topk_weights, E, P, quant="fp8_pow2")
+    R = int(want["num_rows"][0])
+    got = rs.view(nb, ld).cpu().numpy()
+    assert np.array_equal(got[:, :R].T.view(np.uint32), want["recv_scales"].view(np.uint32))
+    assert np.all(np.isnan(got[:, R:]))
+    assert np.array_equal(rq[:R].cpu().numpy(), want["recv_x"])
+    assert ep.ep_read_status(ws) == 0

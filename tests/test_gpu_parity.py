@@ -198,6 +198,7 @@ LL_CASES = [
     ("ll-masked", make_custom(64, 256, 6, 32, 1, seed=3, mask_frac=0.2), 64),
     ("ll-dups-overflow", make_custom(20, 128, 4, 3, 1, seed=4, duplicates=True), 20),
     ("ll-t1", make_custom(1, 128, 8, 256, 1, seed=5), 128),
+    ("ll-e2048", make_custom(300, 256, 8, 2048, 1, seed=6), 300),
 ]
 
 
