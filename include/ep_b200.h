@@ -214,12 +214,18 @@ EP_API ep_status ep_get_dispatch_layout_static(int64_t num_tokens, int32_t num_t
  *   quant = EP_QUANT_FP8_E4M3_1X128: recv_x (uint8 [T*K, H]) gets E4M3 codes
  *     q = e4m3_rne_satfinite(x / s) and recv_scales (fp32 [T*K, H/128]) gets
  *     s = max(amax, 1e-4) / 448 of each 128-channel block (fp32 division);
+ *   quant = EP_QUANT_FP8_E4M3_1X128_POW2: the same with every s rounded up to
+ *     a power of two;
+ *   quant | EP_QUANT_SCALES_MN_MAJOR (FP8 only): recv_scales block-major,
+ *     [H/128, ld] with ld = T*K rounded up to 4;
  *   quant = EP_QUANT_NONE: recv_x (BF16 [T*K, H]) gets the row bit for bit;
  *     recv_scales may be NULL.
  *   recv_topk_idx[row] = e - p*E/P (expert id local to its partition, int32),
  *   recv_topk_weights[row] = topk_weights[t, k].
  * Receive buffers are sized for the worst case (T*K rows) so no host sync is
- * needed; the first *handle->num_recv rows are valid.
+ * needed; the first *handle->num_recv rows are valid.  Which CTA writes a token
+ * is decided at run time (a ticket counter in the workspace); what is written
+ * is not, so the output is deterministic.
  * x: BF16 [T, H]; topk_idx: int64 [T, K]; topk_weights: fp32 [T, K] (device).
  */
 EP_API ep_status ep_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk, int32_t num_experts,
