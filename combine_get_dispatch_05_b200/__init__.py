@@ -20,5 +20,6 @@ from ._lib import (  # noqa: F401
     status_string,
 )
 from .buffer import Buffer  # noqa: F401
+from .ep_group import EpContext, EpGroup  # noqa: F401
 
 __version__ = "0.1.0"

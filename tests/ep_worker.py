@@ -1,0 +1,75 @@
+"""One rank of the multi-process EpGroup test (spawned by tests/test_gpu_ep.py).
+
+Every rank draws every rank's tokens from fixed seeds, so it can compute with the
+oracle both what it should receive (each source's partition-r rows of a one-GPU
+dispatch with P = world) and its own combine result."""
+import datetime
+import os
+import sys
+
+import numpy as np
+
+
+def run(rank: int, world: int, port: int, out_dir: str) -> None:
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for p in (root, os.path.join(root, "tests")):
+        if p not in sys.path:
+            sys.path.insert(0, p)
+    import torch
+    import torch.distributed as dist
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    status = "failed"
+    try:
+        import combine_get_dispatch_05_b200 as ep
+        import oracle
+        from gpu_path import bf16_to_u16, dev_u16_as_bf16, torch_identity_expert
+        from workloads import make_custom
+
+        E, H, K = 64, 256, 6
+        tokens = [150 + 71 * r for r in range(world)]
+        loads = [make_custom(tokens[r], H, K, E, world, seed=100 + r, mask_frac=0.1)
+                 for r in range(world)]
+        w = loads[rank]
+        g = ep.EpGroup(E)
+        x = dev_u16_as_bf16(w.x)
+        idx = torch.from_numpy(w.topk_idx).cuda()
+        wts = torch.from_numpy(w.topk_weights).cuda()
+        (rq, rs), ri, rw, per_expert, ctx = g.dispatch(x, idx, wts)
+
+        # received rows: each source's partition-`rank` slice, sources in rank order
+        epp = E // world
+        want_q, want_s, want_i, want_w, want_cnt = [], [], [], [], []
+        for s, ws in enumerate(loads):
+            d = oracle.dispatch(ws.x, ws.topk_idx, ws.topk_weights, E, world)
+            lo, hi = d["expert_offset"][rank * epp], d["expert_offset"][(rank + 1) * epp]
+            want_q.append(d["recv_x"][lo:hi])
+            want_s.append(d["recv_scales"][lo:hi])
+            want_i.append(d["recv_topk_idx"][lo:hi])
+            want_w.append(d["recv_topk_weights"][lo:hi])
+            want_cnt.append(d["num_tokens_per_expert"][rank * epp:(rank + 1) * epp])
+        assert np.array_equal(rq.view(torch.uint8).cpu().numpy(), np.concatenate(want_q))
+        assert np.array_equal(rs.cpu().numpy().view(np.uint32),
+                              np.concatenate(want_s).view(np.uint32))
+        assert np.array_equal(ri.cpu().numpy(), np.concatenate(want_i))
+        assert np.array_equal(rw.cpu().numpy().view(np.uint32),
+                              np.concatenate(want_w).view(np.uint32))
+        assert np.array_equal(per_expert.cpu().numpy(), np.stack(want_cnt))
+
+        # identity experts on the received rows, then combine back at the source
+        y = g.combine(torch_identity_expert(rq.view(torch.uint8), rs), ctx, wts)
+        mine = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, E, world)
+        eo = oracle.identity_expert(mine["recv_x"], mine["recv_scales"])
+        y_ref, st = oracle.combine(eo, mine["row_of"], w.topk_weights)
+        assert st == 0
+        assert np.array_equal(bf16_to_u16(y), y_ref)
+        assert ep.ep_read_status(g.workspace) == 0
+        status = "ok"
+    finally:
+        with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
+            f.write(status)
+        dist.destroy_process_group()
