@@ -33,6 +33,8 @@ constexpr int kLoadBatch = 8;  // vector loads issued before the first FMA
 template <int kBatch>
 __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
     combine_kernel(CombineParams p, int64_t vec_per_slice) {
+    pdl_wait();               // the previous kernel (e.g. the dispatch) is complete
+    pdl_launch_dependents();  // the next kernel may be scheduled
     __shared__ int rows_sm[2][32];
     __shared__ float w_sm[2][32];
     __shared__ int cnt_sm[2];
@@ -236,12 +238,19 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
     if (gx > p.T) gx = p.T;
     if (gx < 1) gx = 1;
     if (gx > 2147483647LL) gx = 2147483647LL;
-    const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(slices));
-    if (p.sparse)
-        combine_kernel<4><<<grid, threads, 0, stream>>>(p, per_slice);
-    else
-        combine_kernel<8><<<grid, threads, 0, stream>>>(p, per_slice);
-    return cudaGetLastError();
+    // Programmatic dependent launch: the CTAs may be scheduled while the previous
+    // kernel finishes; each waits for it (griddepcontrol.wait) before reading anything.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(slices));
+    cfg.blockDim = dim3(threads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (p.sparse) return cudaLaunchKernelEx(&cfg, combine_kernel<4>, p, per_slice);
+    return cudaLaunchKernelEx(&cfg, combine_kernel<8>, p, per_slice);
 }
 
 }  // namespace ep

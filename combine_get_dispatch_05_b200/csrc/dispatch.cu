@@ -187,6 +187,7 @@ __device__ __forceinline__ void write_row_metadata(const DispatchParams& p, int 
 // Only the storer reads what the layout kernel wrote, so only it waits on the
 // programmatic dependency; loads and quantisation overlap the layout.
 __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchParams p) {
+    pdl_launch_dependents();  // the next kernel (e.g. the combine) may be scheduled
     extern __shared__ __align__(128) uint8_t sm[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nq = (blockDim.x >> 5) - 2;
@@ -346,6 +347,7 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
 //       bulk-stores the row to row_of[t, k] and writes recv_topk_idx / weights;
 //       once this token's stores have read the stage it arrives on empty[s].
 __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
+    pdl_launch_dependents();  // the next kernel (e.g. the combine) may be scheduled
     extern __shared__ __align__(128) uint8_t sm[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t H = p.H;

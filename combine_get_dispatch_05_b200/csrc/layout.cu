@@ -416,6 +416,7 @@ __device__ __forceinline__ int run_length(int n, int W) {
 
 // The whole batch in one CTA: the chunk's counts are the totals.
 __global__ void __launch_bounds__(kSingleThreads, 1) layout_single_kernel(LayoutArgs a) {
+    pdl_wait();               // the previous kernel (e.g. the one writing topk_idx) is complete
     pdl_launch_dependents();  // the dispatch kernel may start loading x
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const Smem s = carve_smem(smem_raw, a);
@@ -436,6 +437,7 @@ __global__ void __launch_bounds__(kSingleThreads, 1) layout_single_kernel(Layout
 // ------------------------------------------------------------ grid kernel --
 
 __global__ void __launch_bounds__(kLayoutThreads, 1) layout_kernel(LayoutArgs a) {
+    pdl_wait();               // the previous kernel (e.g. the one writing topk_idx) is complete
     pdl_launch_dependents();  // the dispatch kernel may start loading x
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const Smem s = carve_smem(smem_raw, a);
@@ -630,11 +632,14 @@ cudaError_t launch_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int6
     a.status = ws.status;
     a.timeout_ns = kDefaultTimeoutNs;
 
-    // First kernel of the call: an ordinary (not programmatic) launch, so it waits for
-    // all earlier work in the stream.
+    // First kernel of the call: a programmatic dependent launch, so its CTAs may be
+    // scheduled while the previous kernel in the stream finishes; each waits for it
+    // (griddepcontrol.wait) before reading topk_idx.
     cudaLaunchConfig_t cfg = {};
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
 
@@ -656,7 +661,6 @@ cudaError_t launch_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int6
             cfg.gridDim = dim3(1);
             cfg.blockDim = dim3(kSingleThreads);
             cfg.dynamicSmemBytes = smem;
-            cfg.numAttrs = 0;
             return cudaLaunchKernelEx(&cfg, layout_single_kernel, a);
         }
     }
@@ -685,8 +689,9 @@ cudaError_t launch_layout(int64_t T, int32_t K, int32_t E, int32_t P, const int6
     cfg.gridDim = dim3(static_cast<unsigned>(G));
     cfg.blockDim = dim3(kLayoutThreads);
     cfg.dynamicSmemBytes = smem;
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, layout_kernel, a);
 }
 
