@@ -67,6 +67,19 @@ def run(rank: int, world: int, port: int, out_dir: str) -> None:
         y_ref, st = oracle.combine(eo, mine["row_of"], w.topk_weights)
         assert st == 0
         assert np.array_equal(bf16_to_u16(y), y_ref)
+
+        # BF16 payload: rows copied bit for bit, and back
+        recv_b, ri_b, rw_b, per_b, ctx_b = g.dispatch(x, idx, wts, use_fp8=False)
+        want_b = []
+        for ws in loads:
+            d = oracle.dispatch(ws.x, ws.topk_idx, ws.topk_weights, E, world, quant="none")
+            lo, hi = d["expert_offset"][rank * epp], d["expert_offset"][(rank + 1) * epp]
+            want_b.append(d["recv_x"][lo:hi])
+        assert np.array_equal(bf16_to_u16(recv_b), np.concatenate(want_b))
+        y_b = g.combine(recv_b, ctx_b, wts)
+        mine_b = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, E, world, quant="none")
+        y_ref_b, _ = oracle.combine(mine_b["recv_x"], mine_b["row_of"], w.topk_weights)
+        assert np.array_equal(bf16_to_u16(y_b), y_ref_b)
         assert ep.ep_read_status(g.workspace) == 0
         status = "ok"
     finally:
