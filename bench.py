@@ -154,9 +154,16 @@ class ClockSampler:
 
 
 def source_hash(paths):
+    """Hash of the code in `paths` with comments and blank space removed, so that
+    a comment edit does not invalidate a capture of the same kernel."""
+    import re
+
     h = hashlib.sha256()
     for p in paths:
-        h.update(open(os.path.join(ROOT, p), "rb").read())
+        text = open(os.path.join(ROOT, p), encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)  # block comments
+        text = re.sub(r"//[^\n]*", " ", text)                # line comments
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

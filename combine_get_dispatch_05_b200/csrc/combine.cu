@@ -10,8 +10,9 @@
 //
 // Layout of the work: a CTA owns a slice of a token's row (blockIdx.y) and walks
 // tokens t = blockIdx.x, blockIdx.x + gridDim.x, ...; each thread owns 8 channels
-// (one 16-byte vector) and issues the K vector loads of its channels before it
-// uses any, so K * 16 bytes per thread (128 B at K = 8) are in flight.  The K
+// (one 16-byte vector) and issues the loads of the token's valid rows for its
+// channels (up to kBatch at a time) before it uses any, so up to 128 B per thread
+// are in flight.  The K
 // source rows are contiguous 14 KB rows (hidden 7168), so every warp reads whole
 // 512-byte runs: the reads are coalesced and the traffic is the algorithmic
 // minimum (K rows read once, one row written).  The rows and weights of the
@@ -24,7 +25,7 @@ namespace ep {
 namespace {
 
 constexpr int kCombineMaxThreads = 512;
-constexpr int kLoadBatch = 8;  // vector loads issued before the first FMA
+constexpr int kLoadBatch = 8;  // combine backward: slots handled per batch
 
 // kBatch: row loads issued per thread before the first FMA.  The token's valid
 // rows are compacted (k order kept) so a batch holds only rows that exist; sparse
