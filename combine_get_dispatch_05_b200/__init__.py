@@ -5,6 +5,8 @@ Python binding.
   taking torch tensors for device memory (argument marshalling only).
 * :class:`Buffer`: the DeepEP-style call shapes (dispatch / combine /
   low_latency_dispatch / low_latency_combine) on top of them.
+* :class:`EpGroup`: dispatch / combine across the ranks of a process group (one
+  GPU each), through NCCL all-to-all or straight through peer memory.
 
 Importing this package loads ``libep_b200.so``; if it is missing the import
 fails (there is no fallback implementation).
@@ -17,7 +19,8 @@ from ._lib import (  # noqa: F401
     ep_combine_dedup, ep_dispatch, ep_dispatch_backward, ep_dispatch_dedup,
     ep_get_dispatch_layout, ep_lb_prefetch_weights, ep_lb_reduce_grads, ep_low_latency_combine,
     ep_low_latency_dispatch, ep_read_status, ep_workspace_bytes, ep_workspace_init, lib,
-    status_string,
+    status_string, EP_IPC_HANDLE_BYTES, PeerTables, device_bytes, ep_ipc_alloc, ep_ipc_close,
+    ep_ipc_free, ep_ipc_open, ep_peer_combine, ep_peer_dispatch, ep_peer_plan,
 )
 from .buffer import Buffer  # noqa: F401
 from .ep_group import EpContext, EpGroup  # noqa: F401

@@ -37,7 +37,10 @@ EXPORTED = (
     "ep_low_latency_dispatch", "ep_low_latency_combine", "ep_debug_wait_probe",
     "ep_get_dispatch_layout_static", "ep_dispatch_backward", "ep_combine_backward",
     "ep_dispatch_dedup", "ep_combine_dedup", "ep_lb_prefetch_weights", "ep_lb_reduce_grads",
+    "ep_ipc_alloc", "ep_ipc_free", "ep_ipc_open", "ep_ipc_close", "ep_peer_plan",
+    "ep_peer_dispatch", "ep_peer_combine",
 )
+EP_IPC_HANDLE_BYTES = 64
 
 
 class EpError(RuntimeError):
@@ -54,6 +57,12 @@ class ep_layout(ctypes.Structure):
 
 class ep_ll_handle(ctypes.Structure):
     _fields_ = [("row_of", ctypes.c_void_p), ("src_of", ctypes.c_void_p)]
+
+
+class ep_peer_buffers(ctypes.Structure):
+    _fields_ = [("recv_x", ctypes.c_void_p), ("recv_scales", ctypes.c_void_p),
+                ("recv_topk_idx", ctypes.c_void_p), ("recv_topk_weights", ctypes.c_void_p),
+                ("capacity", ctypes.c_int64)]
 
 
 def _load() -> ctypes.CDLL:
@@ -103,6 +112,20 @@ def _load() -> ctypes.CDLL:
     L.ep_combine_dedup.argtypes = [i64, i64, i32, vp, i64, ctypes.POINTER(ep_layout), vp, vp, sz,
                                    vp]
     L.ep_combine_dedup.restype = st
+    L.ep_ipc_alloc.argtypes = [sz, ctypes.POINTER(vp), vp]
+    L.ep_ipc_alloc.restype = st
+    L.ep_ipc_free.argtypes, L.ep_ipc_free.restype = [vp], st
+    L.ep_ipc_open.argtypes, L.ep_ipc_open.restype = [vp, ctypes.POINTER(vp)], st
+    L.ep_ipc_close.argtypes, L.ep_ipc_close.restype = [vp], st
+    L.ep_peer_plan.argtypes = [i32, i32, i32, vp, vp, i64, vp, vp, vp, vp, sz, vp]
+    L.ep_peer_plan.restype = st
+    L.ep_peer_dispatch.argtypes = [i64, i64, i32, i32, i32, i32, vp, vp, vp,
+                                   ctypes.POINTER(ep_layout), vp, ctypes.POINTER(ep_peer_buffers),
+                                   vp, sz, vp]
+    L.ep_peer_dispatch.restype = st
+    L.ep_peer_combine.argtypes = [i64, i64, i32, i32, i32, vp, i64, ctypes.POINTER(ep_layout), vp,
+                                  vp, vp, vp, vp, sz, vp]
+    L.ep_peer_combine.restype = st
     return L
 
 
@@ -456,3 +479,126 @@ def ep_combine_dedup(partition_out: torch.Tensor, handle: Layout, y: torch.Tenso
     _check("ep_combine_dedup", lib.ep_combine_dedup(
         T, H, P, partition_out.data_ptr(), rows, ctypes.byref(c), y.data_ptr(),
         workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+# ------------------------------------------------ expert parallelism across GPUs --
+
+@dataclass
+class PeerTables:
+    """Every rank's receive buffers as device tables of W addresses (int64 [W],
+    rank order), the ``void* const*`` arguments of ep_peer_dispatch / ep_peer_combine."""
+
+    recv_x: torch.Tensor
+    recv_scales: torch.Tensor
+    recv_topk_idx: torch.Tensor
+    recv_topk_weights: torch.Tensor
+    expert_out: torch.Tensor
+    capacity: int
+
+    @staticmethod
+    def from_addresses(device, capacity: int, recv_x, recv_scales, recv_topk_idx,
+                       recv_topk_weights, expert_out) -> "PeerTables":
+        def table(addrs):
+            return torch.tensor([int(a) for a in addrs], dtype=torch.int64, device=device)
+        return PeerTables(table(recv_x), table(recv_scales), table(recv_topk_idx),
+                          table(recv_topk_weights), table(expert_out), int(capacity))
+
+
+class _DeviceMemory:
+    """Raw device memory exposed through __cuda_array_interface__ (bytes)."""
+
+    def __init__(self, ptr: int, nbytes: int):
+        self.__cuda_array_interface__ = {"shape": (nbytes,), "typestr": "|u1",
+                                         "data": (ptr, False), "version": 3, "strides": None}
+
+
+def device_bytes(ptr: int, nbytes: int, device) -> torch.Tensor:
+    """A uint8 tensor over `nbytes` of device memory at `ptr` (no copy; the memory
+    must outlive the tensor)."""
+    return torch.as_tensor(_DeviceMemory(int(ptr), int(nbytes)), device=device)
+
+
+def ep_ipc_alloc(nbytes: int):
+    """Device memory that other processes can map: returns (address, handle bytes)."""
+    ptr = ctypes.c_void_p()
+    handle = ctypes.create_string_buffer(EP_IPC_HANDLE_BYTES)
+    _check("ep_ipc_alloc", lib.ep_ipc_alloc(int(nbytes), ctypes.byref(ptr), handle))
+    return int(ptr.value), handle.raw
+
+
+def ep_ipc_free(ptr: int) -> None:
+    _check("ep_ipc_free", lib.ep_ipc_free(ptr))
+
+
+def ep_ipc_open(handle: bytes) -> int:
+    if len(handle) != EP_IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle has {EP_IPC_HANDLE_BYTES} bytes")
+    ptr = ctypes.c_void_p()
+    _check("ep_ipc_open", lib.ep_ipc_open(handle, ctypes.byref(ptr)))
+    return int(ptr.value)
+
+
+def ep_ipc_close(ptr: int) -> None:
+    _check("ep_ipc_close", lib.ep_ipc_close(ptr))
+
+
+def ep_peer_plan(counts: torch.Tensor, rank: int, expert_offset: torch.Tensor, capacity: int,
+                 dst_offset: torch.Tensor, recv_count: torch.Tensor, recv_offset: torch.Tensor,
+                 workspace: torch.Tensor, stream=None) -> None:
+    """counts: int32 [W, E], every rank's num_tokens_per_expert."""
+    _need(counts, "counts", torch.int32)
+    W, E = counts.shape
+    _need(expert_offset, "expert_offset", torch.int32, shape=(E + 1,))
+    _need(dst_offset, "dst_offset", torch.int32, shape=(E,))
+    _need(recv_count, "recv_count", torch.int32, shape=(E // W,))
+    _need(recv_offset, "recv_offset", torch.int32, shape=(E // W + 1,))
+    _need(workspace, "workspace", torch.uint8)
+    _check("ep_peer_plan", lib.ep_peer_plan(
+        W, rank, E, counts.data_ptr(), expert_offset.data_ptr(), int(capacity),
+        dst_offset.data_ptr(), recv_count.data_ptr(), recv_offset.data_ptr(),
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_peer_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
+                     num_experts: int, world: int, quant: int, handle: Layout,
+                     dst_offset: torch.Tensor, tables: PeerTables, workspace: torch.Tensor,
+                     stream=None) -> None:
+    _need(x, "x", torch.bfloat16)
+    T, H = x.shape
+    K = topk_idx.shape[1]
+    _need(topk_idx, "topk_idx", torch.int64, shape=(T, K))
+    _need(topk_weights, "topk_weights", torch.float32, shape=(T, K))
+    _need(handle.row_of, "handle.row_of", torch.int32, shape=(T, K))
+    _need(dst_offset, "dst_offset", torch.int32, shape=(num_experts,))
+    for name in ("recv_x", "recv_scales", "recv_topk_idx", "recv_topk_weights"):
+        _need(getattr(tables, name), "tables." + name, torch.int64, shape=(world,))
+    _need(workspace, "workspace", torch.uint8)
+    c = ep_layout(row_of=handle.row_of.data_ptr())
+    fp8 = quant != EP_QUANT_NONE
+    b = ep_peer_buffers(tables.recv_x.data_ptr(),
+                        tables.recv_scales.data_ptr() if fp8 else None,
+                        tables.recv_topk_idx.data_ptr(), tables.recv_topk_weights.data_ptr(),
+                        tables.capacity)
+    _check("ep_peer_dispatch", lib.ep_peer_dispatch(
+        T, H, K, num_experts, world, quant, x.data_ptr(), topk_idx.data_ptr(),
+        topk_weights.data_ptr(), ctypes.byref(c), dst_offset.data_ptr(), ctypes.byref(b),
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_peer_combine(tables: PeerTables, handle: Layout, topk_idx: torch.Tensor,
+                    dst_offset: torch.Tensor, topk_weights: torch.Tensor, y: torch.Tensor,
+                    num_experts: int, world: int, workspace: torch.Tensor, stream=None) -> None:
+    _need(y, "y", torch.bfloat16)
+    T, H = y.shape
+    K = topk_idx.shape[1]
+    _need(topk_idx, "topk_idx", torch.int64, shape=(T, K))
+    _need(topk_weights, "topk_weights", torch.float32, shape=(T, K))
+    _need(handle.row_of, "handle.row_of", torch.int32, shape=(T, K))
+    _need(dst_offset, "dst_offset", torch.int32, shape=(num_experts,))
+    _need(tables.expert_out, "tables.expert_out", torch.int64, shape=(world,))
+    _need(workspace, "workspace", torch.uint8)
+    c = ep_layout(row_of=handle.row_of.data_ptr())
+    _check("ep_peer_combine", lib.ep_peer_combine(
+        T, H, K, num_experts, world, tables.expert_out.data_ptr(), tables.capacity,
+        ctypes.byref(c), topk_idx.data_ptr(), dst_offset.data_ptr(), topk_weights.data_ptr(),
+        y.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)))

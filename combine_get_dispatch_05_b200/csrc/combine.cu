@@ -31,12 +31,16 @@ constexpr int kLoadBatch = 8;  // combine backward: slots handled per batch
 // rows are compacted (k order kept) so a batch holds only rows that exist; sparse
 // routings (one slot per partition, about half of them empty) use a batch of 4 and
 // fewer registers, so more threads and more loads are in flight per SM.
-template <int kBatch>
+// kPeer: partitions are ranks; slot k's row is row_of[t, k] + peer_offset[e] in the
+// expert outputs of the rank that owns e = topk_idx[t, k] (read over NVLink), and
+// the compaction records a pointer to each valid row instead of its index.
+template <int kBatch, bool kPeer>
 __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
     combine_kernel(CombineParams p, int64_t vec_per_slice) {
     pdl_wait();               // the previous kernel (e.g. the dispatch) is complete
     pdl_launch_dependents();  // the next kernel may be scheduled
     __shared__ int rows_sm[2][32];
+    __shared__ const uint4* src_sm[kPeer ? 2 : 1][kPeer ? 32 : 1];
     __shared__ float w_sm[2][32];
     __shared__ int cnt_sm[2];
     const int tid = threadIdx.x;
@@ -49,22 +53,42 @@ __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
 
     int nrow = -1;
     float nw = 1.0f;
+    int64_t ne = -1;
     if (tid < K && static_cast<int64_t>(blockIdx.x) < T) {
         nrow = p.row_of[static_cast<int64_t>(blockIdx.x) * K + tid];
         if (p.topk_weights) nw = p.topk_weights[static_cast<int64_t>(blockIdx.x) * K + tid];
+        if constexpr (kPeer) ne = p.topk_idx[static_cast<int64_t>(blockIdx.x) * K + tid];
     }
     int buf = 0;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x, buf ^= 1) {
         if (tid < 32) {  // warp 0: lane k < K holds slot k
             int r = tid < K ? nrow : -1;
-            if (r >= 0 && static_cast<int64_t>(r) >= p.expert_out_rows) {
+            const uint4* src = nullptr;
+            if constexpr (kPeer) {
+                // rows past the owner's buffer (or with an id the handle does not
+                // match) are skipped
+                if (r >= 0) {
+                    const int ei = ne >= 0 && ne < p.num_experts ? static_cast<int>(ne) : -1;
+                    const int64_t pr = ei >= 0 ? static_cast<int64_t>(r) + p.peer_offset[ei] : -1;
+                    if (pr < 0 || pr >= p.expert_out_rows) {
+                        raise_status(p.status, kDevIndexRange);
+                        r = -1;
+                    } else {
+                        src = static_cast<const uint4*>(p.peer_out[ei / p.experts_per_partition]) +
+                              pr * V;
+                    }
+                }
+            } else if (r >= 0 && static_cast<int64_t>(r) >= p.expert_out_rows) {
                 raise_status(p.status, kDevIndexRange);
                 r = -1;
             }
             const unsigned valid = __ballot_sync(0xffffffffu, r >= 0);
             if (r >= 0) {
                 const int at = __popc(valid & ((1u << tid) - 1u));
-                rows_sm[buf][at] = r;
+                if constexpr (kPeer)
+                    src_sm[buf][at] = src;
+                else
+                    rows_sm[buf][at] = r;
                 w_sm[buf][at] = nw;
             }
             if (tid == 0) cnt_sm[buf] = __popc(valid);
@@ -75,6 +99,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
                 if (tn < T) {
                     nrow = p.row_of[tn * K + tid];
                     if (p.topk_weights) nw = p.topk_weights[tn * K + tid];
+                    if constexpr (kPeer) ne = p.topk_idx[tn * K + tid];
                 }
             }
         }
@@ -91,8 +116,11 @@ __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
 #pragma unroll
                 for (int u = 0; u < kBatch; ++u) {
                     const int k = k0 + u;
-                    d[u] = k < m ? ld_stream_v4(eo + static_cast<int64_t>(rows[k]) * V + v)
-                                 : make_uint4(0u, 0u, 0u, 0u);
+                    if constexpr (kPeer)
+                        d[u] = k < m ? ld_stream_v4(src_sm[buf][k] + v) : make_uint4(0u, 0u, 0u, 0u);
+                    else
+                        d[u] = k < m ? ld_stream_v4(eo + static_cast<int64_t>(rows[k]) * V + v)
+                                     : make_uint4(0u, 0u, 0u, 0u);
                 }
 #pragma unroll
                 for (int u = 0; u < kBatch; ++u) {
@@ -229,8 +257,10 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
     slices = (V + per_slice - 1) / per_slice;
     int threads = static_cast<int>((per_slice + 31) / 32 * 32);
     if (threads > kCombineMaxThreads) threads = kCombineMaxThreads;
-    const void* kernel = p.sparse ? reinterpret_cast<const void*>(combine_kernel<4>)
-                                  : reinterpret_cast<const void*>(combine_kernel<8>);
+    const void* kernel =
+        p.peer_out ? reinterpret_cast<const void*>(combine_kernel<8, true>)
+        : p.sparse ? reinterpret_cast<const void*>(combine_kernel<4, false>)
+                   : reinterpret_cast<const void*>(combine_kernel<8, false>);
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess ||
         per_sm < 1)
@@ -250,8 +280,9 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (p.sparse) return cudaLaunchKernelEx(&cfg, combine_kernel<4>, p, per_slice);
-    return cudaLaunchKernelEx(&cfg, combine_kernel<8>, p, per_slice);
+    if (p.peer_out) return cudaLaunchKernelEx(&cfg, combine_kernel<8, true>, p, per_slice);
+    if (p.sparse) return cudaLaunchKernelEx(&cfg, combine_kernel<4, false>, p, per_slice);
+    return cudaLaunchKernelEx(&cfg, combine_kernel<8, false>, p, per_slice);
 }
 
 }  // namespace ep

@@ -138,13 +138,46 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, ui
     return true;
 }
 
+// Where a storer lane writes its row: payload, scales, local id and weight arrays.
+struct Dest {
+    uint8_t* x;
+    float* s;
+    int32_t* i;
+    float* w;
+};
+
+// Peer mode (partitions are ranks): slot k's row goes to the rank that owns its
+// expert, at row_of[t, k] + peer_offset[e] there.  A row outside the owner's
+// buffers (the owner receives more rows than it has room for) is dropped and
+// reported.  Lane k < K holds both the row and the id of slot k.
+__device__ __forceinline__ int peer_dest(const DispatchParams& p, int row, int64_t e, Dest& d) {
+    if (row < 0) return -1;
+    if (e < 0 || e >= p.num_experts) {  // a handle that does not match topk_idx
+        raise_status(p.status, kDevIndexRange);
+        return -1;
+    }
+    const int ei = static_cast<int>(e);
+    const int part = ei / p.experts_per_partition;
+    const int64_t r = static_cast<int64_t>(row) + p.peer_offset[ei];
+    if (r < 0 || r >= p.peer_rows) {
+        raise_status(p.status, kDevCapacity);
+        return -1;
+    }
+    d.x = static_cast<uint8_t*>(p.peer_recv_x[part]);
+    d.s = p.peer_recv_scales ? p.peer_recv_scales[part] : nullptr;
+    d.i = p.peer_recv_topk_idx[part];
+    d.w = p.peer_recv_topk_weights[part];
+    return static_cast<int>(r);
+}
+
 // Metadata of one token's receive rows, written by the storer warp.  Per-expert
-// rows: lane k owns slot k and writes the local id and weight of its row.
+// rows: lane k owns slot k and writes the local id and weight of its row into
+// ri / rw (its own buffers in peer mode).
 // Deduplicated rows (one per partition): lane p owns partition p's row and writes
 // its K-entry lists, reading every slot's id and weight from the id lanes by
 // shuffle (all lanes take part in the shuffles).
 __device__ __forceinline__ void write_row_metadata(const DispatchParams& p, int lane, int row,
-                                                   int64_t e, float wt) {
+                                                   int64_t e, float wt, int32_t* ri, float* rw) {
     // lane k < K: partition and partition-local id of routing entry k, one 32-bit
     // division per lane (-1: not a valid expert id)
     const int epp = p.experts_per_partition;
@@ -154,8 +187,8 @@ __device__ __forceinline__ void write_row_metadata(const DispatchParams& p, int 
     const int local = ei - (valid ? part : 0) * epp;
     if (!p.dedup) {
         if (lane < p.slots && row >= 0) {  // a row exists only for a valid id
-            p.recv_topk_idx[row] = local;
-            p.recv_topk_weights[row] = wt;
+            ri[row] = local;
+            rw[row] = wt;
         }
         return;
     }
@@ -186,6 +219,8 @@ __device__ __forceinline__ void write_row_metadata(const DispatchParams& p, int 
 //       output stage (out_empty) once its stores have read it; a -1 token ends it.
 // Only the storer reads what the layout kernel wrote, so only it waits on the
 // programmatic dependency; loads and quantisation overlap the layout.
+// kPeer: rows go to the owner ranks' buffers (peer_dest).
+template <bool kPeer>
 __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchParams p) {
     pdl_launch_dependents();  // the next kernel (e.g. the combine) may be scheduled
     extern __shared__ __align__(128) uint8_t sm[];
@@ -293,23 +328,28 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
             __syncwarp();
             if (lane == 0) tok[i & (kTokLog - 1)] = kTokFree;
             next = peek_routing(p, tok[(i + 1) & (kTokLog - 1)], lane);
-            const int row = cur.row;
+            int row = cur.row;
             const int64_t e = cur.e;
             const float wt = cur.wt;
+            Dest d{recv_x, p.recv_scales, p.recv_topk_idx, p.recv_topk_weights};
+            if constexpr (kPeer) row = peer_dest(p, row, e, d);
             uint8_t* out_q = sm + L.off_out + o * L.out_bytes;
             const float* out_s = reinterpret_cast<const float*>(out_q + L.q_bytes);
             if (slot_lane) {
                 if (row >= 0) {
-                    bulk_store(recv_x + static_cast<int64_t>(row) * H, out_q, L.q_bytes);
+                    bulk_store(d.x + static_cast<int64_t>(row) * H, out_q, L.q_bytes);
                     if (scale_bulk)
-                        bulk_store(p.recv_scales + static_cast<int64_t>(row) * nb, out_s,
+                        bulk_store(d.s + static_cast<int64_t>(row) * nb, out_s,
                                    static_cast<uint32_t>(nb) * 4u);
                 }
                 bulk_commit();
                 rows_sm[o * 32 + lane] = row;
             }
-            write_row_metadata(p, lane, row, e, wt);
-            if (!scale_bulk) {
+            write_row_metadata(p, lane, row, e, wt, d.i, d.w);
+            if constexpr (kPeer) {
+                if (!scale_bulk && slot_lane && row >= 0)  // row-major: the lane's own row
+                    for (int b = 0; b < nb; ++b) d.s[static_cast<int64_t>(row) * nb + b] = out_s[b];
+            } else if (!scale_bulk) {
                 __syncwarp();
                 for (int idx = lane; idx < S * nb; idx += 32) {
                     const int k = idx / nb, b = idx - k * nb;
@@ -346,6 +386,8 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
 //   storer (warp 1): waits for the layout, then per step waits full[s], lane k
 //       bulk-stores the row to row_of[t, k] and writes recv_topk_idx / weights;
 //       once this token's stores have read the stage it arrives on empty[s].
+// kPeer: rows go to the owner ranks' buffers (peer_dest).
+template <bool kPeer>
 __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
     pdl_launch_dependents();  // the next kernel (e.g. the combine) may be scheduled
     extern __shared__ __align__(128) uint8_t sm[];
@@ -415,16 +457,18 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
             __syncwarp();
             if (lane == 0) tok[i % kTokLog] = kTokFree;
             next = peek_routing(p, tok[(i + 1) % kTokLog], lane);
-            const int row = cur.row;
+            int row = cur.row;
             const int64_t e = cur.e;
             const float wt = cur.wt;
+            Dest d{recv_x, nullptr, p.recv_topk_idx, p.recv_topk_weights};
+            if constexpr (kPeer) row = peer_dest(p, row, e, d);
             if (slot_lane) {
                 if (row >= 0)
-                    bulk_store(recv_x + static_cast<int64_t>(row) * row_bytes, sm + s * row_bytes,
+                    bulk_store(d.x + static_cast<int64_t>(row) * row_bytes, sm + s * row_bytes,
                                row_bytes);
                 bulk_commit();
             }
-            write_row_metadata(p, lane, row, e, wt);
+            write_row_metadata(p, lane, row, e, wt, d.i, d.w);
             if (slot_lane) bulk_wait_read<1>();  // the previous token's stores have read their stage
             __syncwarp();
             if (lane == 0 && i >= 1) mbar_arrive(&empty[(i - 1) % kBf16Stages]);
@@ -488,7 +532,8 @@ cudaError_t launch_dispatch_fp8(const DispatchParams& params, cudaStream_t strea
     p.out_stages = no;
     const Fp8Smem L = fp8_smem(p.H, p.in_stages, p.out_stages);
     if (L.total > dev.max_smem_optin) return cudaErrorInvalidValue;
-    const void* kernel = reinterpret_cast<const void*>(dispatch_fp8_kernel);
+    const void* kernel = p.peer_offset ? reinterpret_cast<const void*>(dispatch_fp8_kernel<true>)
+                                       : reinterpret_cast<const void*>(dispatch_fp8_kernel<false>);
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(L.total));
     if (err != cudaSuccess) return err;
@@ -511,7 +556,8 @@ cudaError_t launch_dispatch_bf16(const DispatchParams& p, cudaStream_t stream) {
     const size_t smem = static_cast<size_t>(kBf16Stages) * p.H * 2 + 16 * kBf16Stages +
                         4 * kTokLog + 16;
     if (smem > dev.max_smem_optin) return cudaErrorInvalidValue;
-    const void* kernel = reinterpret_cast<const void*>(dispatch_bf16_kernel);
+    const void* kernel = p.peer_offset ? reinterpret_cast<const void*>(dispatch_bf16_kernel<true>)
+                                       : reinterpret_cast<const void*>(dispatch_bf16_kernel<false>);
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;

@@ -1,8 +1,9 @@
 // ep_api.cu -- the exported C ABI (include/ep_b200.h): host-side argument checks,
-// workspace handling and kernel launches.  No allocation, no host synchronisation
-// except in ep_read_status().
+// workspace handling and kernel launches.  No allocation (except ep_ipc_alloc), no
+// host synchronisation except in ep_read_status().
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include <atomic>
 
@@ -90,7 +91,7 @@ using namespace ep;
 
 extern "C" {
 
-int32_t ep_abi_version(void) { return 1; }
+int32_t ep_abi_version(void) { return 2; }
 
 const char* ep_status_string(int32_t status) {
     switch (status) {
@@ -462,6 +463,156 @@ ep_status ep_lb_reduce_grads(int32_t num_slots, int64_t n, const int32_t* primar
     const Workspace ws = carve_workspace(workspace, 0, 1);
     return cuda_status(launch_lb_reduce(num_slots, n, primary_of, grads, ws.status,
                                         static_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_ipc_alloc(size_t bytes, void** ptr, void* handle) {
+    static_assert(sizeof(cudaIpcMemHandle_t) == EP_IPC_HANDLE_BYTES, "IPC handle size");
+    if (!ptr || !handle || bytes == 0) return EP_ERR_INVALID_ARG;
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) return EP_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, p) != cudaSuccess) {
+        cudaFree(p);
+        return EP_ERR_CUDA;
+    }
+    memcpy(handle, &h, sizeof(h));
+    *ptr = p;
+    return EP_OK;
+}
+
+ep_status ep_ipc_free(void* ptr) {
+    if (!ptr) return EP_ERR_INVALID_ARG;
+    return cuda_status(cudaFree(ptr));
+}
+
+ep_status ep_ipc_open(const void* handle, void** ptr) {
+    if (!handle || !ptr) return EP_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t h;
+    memcpy(&h, handle, sizeof(h));
+    void* p = nullptr;
+    if (cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess)
+        return EP_ERR_CUDA;
+    *ptr = p;
+    return EP_OK;
+}
+
+ep_status ep_ipc_close(void* ptr) {
+    if (!ptr) return EP_ERR_INVALID_ARG;
+    return cuda_status(cudaIpcCloseMemHandle(ptr));
+}
+
+ep_status ep_peer_plan(int32_t world, int32_t rank, int32_t num_experts, const int32_t* counts,
+                       const int32_t* expert_offset, int64_t capacity, int32_t* dst_offset,
+                       int32_t* recv_count, int32_t* recv_offset, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    if (world < 1 || world > 64 || num_experts < 1 || num_experts > 4096 ||
+        num_experts % world != 0 || rank < 0 || rank >= world || capacity < 0 ||
+        capacity >= (int64_t(1) << 31))
+        return EP_ERR_SHAPE;
+    if (!counts || !expert_offset || !dst_offset || !recv_count || !recv_offset || !workspace ||
+        workspace_bytes < kWsHeader)
+        return EP_ERR_INVALID_ARG;
+    PeerPlanParams p;
+    p.world = world;
+    p.rank = rank;
+    p.num_experts = num_experts;
+    p.counts = counts;
+    p.expert_offset = expert_offset;
+    p.capacity = capacity;
+    p.dst_offset = dst_offset;
+    p.recv_count = recv_count;
+    p.recv_offset = recv_offset;
+    p.status = carve_workspace(workspace, 0, 1).status;
+    return cuda_status(launch_peer_plan(p, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_peer_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                           int32_t num_experts, int32_t world, int32_t quant, const void* x,
+                           const int64_t* topk_idx, const float* topk_weights,
+                           const ep_layout* handle, const int32_t* dst_offset,
+                           const ep_peer_buffers* peers, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+    if (quant != EP_QUANT_NONE && quant != EP_QUANT_FP8_E4M3_1X128 &&
+        quant != EP_QUANT_FP8_E4M3_1X128_POW2)
+        return EP_ERR_INVALID_ARG;  // block-major scales are not offered here
+    const bool fp8 = quant != EP_QUANT_NONE;
+    ep_status st = check_routing(num_tokens, num_topk, num_experts, world);
+    if (st != EP_OK) return st;
+    if ((st = check_hidden(hidden, fp8)) != EP_OK) return st;
+    if (!peers || peers->capacity < 0 || peers->capacity >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    if (!handle || !workspace || !aligned16(workspace) || workspace_bytes < kWsHeader)
+        return EP_ERR_INVALID_ARG;
+    if (num_tokens == 0) return EP_OK;
+    if (!handle->row_of || !x || !topk_idx || !topk_weights || !dst_offset || !peers->recv_x ||
+        !peers->recv_topk_idx || !peers->recv_topk_weights || (fp8 && !peers->recv_scales) ||
+        !aligned16(x))
+        return EP_ERR_INVALID_ARG;
+    const Workspace ws = carve_workspace(workspace, 0, 1);
+    DispatchParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = num_topk;
+    p.slots = num_topk;
+    p.dedup = 0;
+    p.pow2_scales = quant == EP_QUANT_FP8_E4M3_1X128_POW2 ? 1 : 0;
+    p.scales_mn = 0;
+    p.scales_ld = 0;
+    p.num_experts = num_experts;
+    p.experts_per_partition = num_experts / world;
+    p.x = x;
+    p.topk_idx = topk_idx;
+    p.topk_weights = topk_weights;
+    p.row_of = handle->row_of;
+    p.recv_x = nullptr;
+    p.recv_scales = nullptr;
+    p.recv_topk_idx = nullptr;
+    p.recv_topk_weights = nullptr;
+    p.status = ws.status;
+    p.ticket = ws.ticket;
+    p.done = ws.done;
+    p.timeout_ns = kDefaultTimeoutNs;
+    p.peer_recv_x = peers->recv_x;
+    p.peer_recv_scales = fp8 ? peers->recv_scales : nullptr;
+    p.peer_recv_topk_idx = peers->recv_topk_idx;
+    p.peer_recv_topk_weights = peers->recv_topk_weights;
+    p.peer_offset = dst_offset;
+    p.peer_rows = peers->capacity;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return cuda_status(fp8 ? launch_dispatch_fp8(p, s) : launch_dispatch_bf16(p, s));
+}
+
+ep_status ep_peer_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                          int32_t num_experts, int32_t world, const void* const* expert_out,
+                          int64_t capacity, const ep_layout* handle, const int64_t* topk_idx,
+                          const int32_t* dst_offset, const float* topk_weights, void* y,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+    ep_status st = check_routing(num_tokens, num_topk, num_experts, world);
+    if (st != EP_OK) return st;
+    if ((st = check_hidden(hidden, false)) != EP_OK) return st;
+    if (capacity < 0 || capacity >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    if (!handle || !workspace || workspace_bytes < kWsHeader) return EP_ERR_INVALID_ARG;
+    if (num_tokens == 0) return EP_OK;
+    if (!handle->row_of || !expert_out || !topk_idx || !dst_offset || !topk_weights || !y ||
+        !aligned16(y))
+        return EP_ERR_INVALID_ARG;
+    CombineParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = num_topk;
+    p.expert_out = nullptr;
+    p.expert_out_rows = capacity;
+    p.row_of = handle->row_of;
+    p.topk_weights = topk_weights;
+    p.y = y;
+    p.grad_recv_w = nullptr;
+    p.grad_w = nullptr;
+    p.status = carve_workspace(workspace, 0, 1).status;
+    p.peer_out = expert_out;
+    p.topk_idx = topk_idx;
+    p.peer_offset = dst_offset;
+    p.experts_per_partition = num_experts / world;
+    p.num_experts = num_experts;
+    return cuda_status(launch_combine(p, static_cast<cudaStream_t>(stream)));
 }
 
 ep_status ep_debug_wait_probe(uint64_t timeout_ns, void* workspace, size_t workspace_bytes,

@@ -71,6 +71,15 @@ struct DispatchParams {
     int32_t* ticket;  // token counter (zero on entry; the last CTA to finish re-zeroes it)
     uint32_t* done;
     uint64_t timeout_ns;
+    // Peer mode (partitions are ranks; per-expert rows only): the row of (t, k) is
+    // row_of[t, k] + peer_offset[e] in the buffers of rank e / experts_per_partition,
+    // whose base pointers the tables hold; recv_x .. recv_topk_weights are unused.
+    void* const* peer_recv_x = nullptr;
+    float* const* peer_recv_scales = nullptr;
+    int32_t* const* peer_recv_topk_idx = nullptr;
+    float* const* peer_recv_topk_weights = nullptr;
+    const int32_t* peer_offset = nullptr;  // [E]; NULL: one local buffer
+    int64_t peer_rows = 0;                 // rows of every rank's receive buffers
 };
 // Launched programmatically dependent on the preceding layout kernel.
 cudaError_t launch_dispatch_fp8(const DispatchParams& p, cudaStream_t stream);
@@ -89,8 +98,30 @@ struct CombineParams {
     float* grad_w;
     uint32_t* status;
     int32_t sparse = 0;         // about half the slots empty (one slot per partition)
+    // Peer mode (partitions are ranks): the row of (t, k) is row_of[t, k] +
+    // peer_offset[e], e = topk_idx[t, k], in peer_out[e / experts_per_partition];
+    // expert_out is unused and expert_out_rows bounds every rank's rows.
+    const void* const* peer_out = nullptr;
+    const int64_t* topk_idx = nullptr;
+    const int32_t* peer_offset = nullptr;
+    int32_t experts_per_partition = 1;
+    int32_t num_experts = 0;
 };
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+
+// Destination offsets of one rank's rows in the owners' receive buffers, from every
+// rank's per-expert counts (one CTA).
+struct PeerPlanParams {
+    int32_t world, rank, num_experts;
+    const int32_t* counts;         // [world, E]: num_tokens_per_expert of every rank
+    const int32_t* expert_offset;  // [E + 1]: this rank's layout
+    int64_t capacity;              // rows of every rank's receive buffers
+    int32_t* dst_offset;           // [E]
+    int32_t* recv_count;           // [E / world]: rows this rank receives per local expert
+    int32_t* recv_offset;          // [E / world + 1]
+    uint32_t* status;
+};
+cudaError_t launch_peer_plan(const PeerPlanParams& p, cudaStream_t stream);
 
 struct CombineBackwardParams {
     int64_t T;

@@ -1,30 +1,41 @@
 """Expert parallelism across processes: partitions are ranks.
 
-The DeepEP pages describe dispatch and combine as an all-to-all between the
-ranks of an EP group ("DeepSeek 开源周第二弹：DeepEP", section "DeepEP 的常规内核和低延迟
-内核": normal kernels over NVLink and RDMA; "deepseek-ai/DeepEP", section "典型工作流程":
-dispatch, expert GEMM, combine back to the source ranks).  ``EpGroup`` builds that
-exchange from this library's one-GPU kernels and ``torch.distributed``:
+The DeepEP pages describe dispatch and combine as an exchange between the ranks of
+an EP group ("DeepSeek 开源周第二弹：DeepEP", section "DeepEP 的常规内核和低延迟内核":
+normal kernels over NVLink and RDMA; "deepseek-ai/DeepEP", section "典型工作流程":
+dispatch, expert GEMM, combine back to the source ranks).  ``EpGroup`` offers two
+transports, one process per GPU; rank r owns experts [r * E / W, (r + 1) * E / W).
 
-dispatch (on every rank, for its own tokens)
-  1. layout + FP8 (or BF16) dispatch with P = group size: the rows for rank p are
-     one contiguous, expert-major slice of the send buffer (partition p);
-  2. the per-rank row counts (from the layout's expert offsets) are exchanged;
-  3. rows, scales, local expert ids and weights go to their owner ranks with
-     ``all_to_all_single`` (NCCL on GPUs; other backends through host memory).
-  Each rank receives, per source rank in rank order, that source's rows for its
-  own experts (expert-major within a source), plus per-(source, local expert)
-  counts for the expert computation.
-combine
-  4. the expert outputs go back along the same splits, so each row lands where
-     it left the sender's send buffer;
-  5. the one-GPU combine kernel reduces them with the sender's handle.
+``transport="peer"`` (GPUs of one node, NVLink / NVSwitch): every rank allocates one
+IPC-shareable region (receive payload, scales, local ids, weights, expert outputs)
+and maps every other rank's.  Per step:
 
-The exchange is the plain collective; the kernels are the library's.
+  1. layout of this rank's tokens with P = W (one kernel);
+  2. all-gather of every rank's per-expert counts (W x E int32);
+  3. plan: where this rank's rows go in the owners' buffers (one kernel);
+  4. dispatch: the FP8 (or BF16) rows, scales, local ids and weights are stored by
+     the dispatch kernel straight into the owners' receive buffers over NVLink;
+  5. a barrier (one-element all-reduce on the stream); the caller computes its
+     experts into ``expert_out_buffer`` ...
+  6. ... and combine: a barrier, then the combine kernel reads each token's expert
+     outputs straight from the owners' buffers and reduces them in fixed k order.
+
+  A rank receives its rows expert-major, then by source rank, then by source token
+  and k: partition r's rows of the one-GPU dispatch of all ranks' tokens
+  concatenated in rank order.
+
+``transport="nccl"`` (any backend): the one-GPU dispatch with P = W fills a send
+buffer whose rank-p rows are one contiguous slice; the rows, scales, local ids and
+weights go to their owners with ``all_to_all_single`` (through host memory when the
+backend is not NCCL), and the expert outputs come back the same way before the
+one-GPU combine.  A rank receives its rows grouped by source rank, then expert.
+
+Both return ``recv_counts_per_expert`` [W, E/W]: rows received from each source
+rank for each local expert.
 """
 from __future__ import annotations
 
-from dataclasses import dataclass
+from dataclasses import dataclass, field
 from typing import List, Optional
 
 import torch
@@ -34,6 +45,8 @@ from . import _lib
 from ._lib import EP_QUANT_FP8_E4M3_1X128, EP_QUANT_NONE, Layout
 
 __all__ = ["EpGroup", "EpContext"]
+
+_ALIGN = 256
 
 
 @dataclass
@@ -45,21 +58,34 @@ class EpContext:
     recv_counts: List[int]       # rows this rank received from each rank
     num_tokens: int
     hidden: int
+    # peer transport only
+    topk_idx: Optional[torch.Tensor] = None
+    dst_offset: Optional[torch.Tensor] = None
+    recv_rows: int = 0
+    order: str = field(default="source_major")
 
 
 class EpGroup:
     """Dispatch / combine across the ranks of ``group`` (default: the world).
 
-    Rank r owns experts [r * E / W, (r + 1) * E / W).  One process per GPU.
+    transport: "nccl" (all-to-all collectives) or "peer" (the dispatch and combine
+    kernels store to and load from the other GPUs' buffers; needs ``hidden``).
+    capacity: rows of each rank's receive buffers in peer mode (default
+    max_tokens * W * 8, every token of every rank routed here with top-8).
+    Call :meth:`close` before destroying the process group.
     """
 
     def __init__(self, num_experts: int, group=None, max_tokens: int = 4096,
-                 device: Optional[torch.device] = None):
+                 device: Optional[torch.device] = None, *, transport: str = "nccl",
+                 hidden: Optional[int] = None, capacity: Optional[int] = None):
         self.group = group if group is not None else dist.group.WORLD
         self.world = dist.get_world_size(self.group)
         self.rank = dist.get_rank(self.group)
         if num_experts % self.world:
             raise ValueError("num_experts must be a multiple of the group size")
+        if transport not in ("nccl", "peer"):
+            raise ValueError(f"unknown transport {transport!r}")
+        self.transport = transport
         self.num_experts = num_experts
         self.experts_per_rank = num_experts // self.world
         self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
@@ -67,12 +93,83 @@ class EpGroup:
         self.max_tokens = max_tokens
         self.workspace = self._new_workspace(max_tokens)
         self.via_host = dist.get_backend(self.group) != "nccl"
+        self._peer = None
+        if transport == "peer":
+            if hidden is None:
+                raise ValueError("the peer transport needs `hidden` to size the receive buffers")
+            self._open_peers(int(hidden), int(capacity if capacity is not None
+                                                  else max_tokens * self.world * 8))
 
     def _new_workspace(self, tokens: int) -> torch.Tensor:
         ws = torch.empty(_lib.ep_workspace_bytes(max(tokens, 1), self.num_experts, self.world),
                          dtype=torch.uint8, device=self.device)
         _lib.ep_workspace_init(ws)
         return ws
+
+    # ---------------------------------------------------------- peer buffers --
+    def _open_peers(self, hidden: int, capacity: int) -> None:
+        """One IPC region per rank: recv_x (room for BF16 rows) | recv_scales |
+        recv_topk_idx | recv_topk_weights | expert_out, each 256-byte aligned."""
+        if hidden % 128:
+            raise ValueError("hidden must be a multiple of 128")
+        sizes = [("recv_x", capacity * hidden * 2), ("recv_scales", capacity * (hidden // 128) * 4),
+                 ("recv_topk_idx", capacity * 4), ("recv_topk_weights", capacity * 4),
+                 ("expert_out", capacity * hidden * 2)]
+        offsets, total = {}, 0
+        for name, n in sizes:
+            offsets[name] = total
+            total += (n + _ALIGN - 1) // _ALIGN * _ALIGN
+        base, handle = _lib.ep_ipc_alloc(max(total, _ALIGN))
+        handles: List[bytes] = [b""] * self.world
+        dist.all_gather_object(handles, handle, group=self.group)
+        bases, opened = [], []
+        try:
+            for q, h in enumerate(handles):
+                if q == self.rank:
+                    bases.append(base)
+                else:
+                    ptr = _lib.ep_ipc_open(h)
+                    opened.append(ptr)
+                    bases.append(ptr)
+        except Exception:
+            for ptr in opened:
+                _lib.ep_ipc_close(ptr)
+            _lib.ep_ipc_free(base)
+            raise
+        self._peer = dict(base=base, opened=opened, hidden=hidden, capacity=capacity,
+                          region=_lib.device_bytes(base, max(total, _ALIGN), self.device),
+                          offsets=offsets, sizes=dict(sizes))
+        self.tables = _lib.PeerTables.from_addresses(
+            self.device, capacity, *[[b + offsets[n] for b in bases] for n, _ in sizes])
+        self._flag = torch.zeros(1, dtype=torch.int32, device=self.device)
+
+    def _view(self, name: str, dtype, shape) -> torch.Tensor:
+        pr = self._peer
+        n = pr["sizes"][name]
+        return pr["region"][pr["offsets"][name]:pr["offsets"][name] + n].view(dtype).view(*shape)
+
+    def expert_out_buffer(self, ctx: EpContext) -> torch.Tensor:
+        """Peer transport: the BF16 [recv rows, H] buffer the expert outputs go into
+        (row i answers received row i); the other ranks' combine kernels read it."""
+        if self._peer is None:
+            raise RuntimeError("expert_out_buffer belongs to the peer transport")
+        cap, H = self._peer["capacity"], self._peer["hidden"]
+        return self._view("expert_out", torch.bfloat16, (cap, H))[:ctx.recv_rows]
+
+    def close(self) -> None:
+        """Unmap the peers' regions and free this rank's (a collective: every rank
+        calls it, after its last combine)."""
+        if self._peer is None:
+            return
+        if self.device.type == "cuda":
+            torch.cuda.synchronize(self.device)
+        self._barrier()
+        for ptr in self._peer["opened"]:
+            _lib.ep_ipc_close(ptr)
+        self._barrier()  # nobody maps this rank's region any more
+        self._peer["region"] = None
+        _lib.ep_ipc_free(self._peer["base"])
+        self._peer = None
 
     # --------------------------------------------------------------- exchange --
     def _a2a(self, inp: torch.Tensor, out_rows: int, out_splits: List[int],
@@ -88,6 +185,25 @@ class EpGroup:
                                group=self.group)
         return out.to(inp.device)
 
+    def _all_gather_rows(self, t: torch.Tensor) -> torch.Tensor:
+        """[n] on every rank -> [W, n] in rank order."""
+        if not self.via_host:
+            out = torch.empty((self.world,) + tuple(t.shape), dtype=t.dtype, device=t.device)
+            dist.all_gather_into_tensor(out, t.contiguous(), group=self.group)
+            return out
+        parts = [torch.empty_like(t, device="cpu") for _ in range(self.world)]
+        dist.all_gather(parts, t.contiguous().cpu(), group=self.group)
+        return torch.stack(parts).to(t.device)
+
+    def _barrier(self) -> None:
+        """Every rank's preceding work on the stream is done before anything after."""
+        if not self.via_host:
+            dist.all_reduce(self._flag, group=self.group)  # ordered on the current stream
+        else:
+            if self.device.type == "cuda":
+                torch.cuda.synchronize(self.device)
+            dist.barrier(group=self.group)
+
     # --------------------------------------------------------------- dispatch --
     def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
                  use_fp8: bool = True):
@@ -96,15 +212,21 @@ class EpGroup:
         recv_x: ``(float8_e4m3fn [Rr, H], float32 [Rr, H/128])`` or BF16 ``[Rr, H]``;
         recv_local_idx: int32 [Rr] (expert id minus this rank's first expert);
         recv_weights: float32 [Rr]; recv_counts_per_expert: int32 [W, E/W] rows
-        received from each source rank for each local expert (rows are grouped by
-        source rank, then local expert, then source token).
+        received from each source rank for each local expert.  Row order: see the
+        module docstring (``ctx.order``).
         """
-        T, H = x.shape
-        K = topk_idx.shape[1]
-        W, E, epp = self.world, self.num_experts, self.experts_per_rank
+        T = x.shape[0]
         if T > self.max_tokens:
             self.max_tokens = T
             self.workspace = self._new_workspace(T)
+        if self.transport == "peer":
+            return self._dispatch_peer(x, topk_idx, topk_weights, use_fp8)
+        return self._dispatch_nccl(x, topk_idx, topk_weights, use_fp8)
+
+    def _dispatch_nccl(self, x, topk_idx, topk_weights, use_fp8):
+        T, H = x.shape
+        K = topk_idx.shape[1]
+        W, E, epp = self.world, self.num_experts, self.experts_per_rank
         rows = max(T * K, 1)
         dev = self.device
         lay = Layout.empty(T, K, E, W, dev)
@@ -131,19 +253,66 @@ class EpGroup:
         recv_i = self._a2a(ri[:Rs], Rr, recv_counts, send_counts)
         recv_w = self._a2a(rw[:Rs], Rr, recv_counts, send_counts)
         per_expert = self._a2a(lay.num_tokens_per_expert.view(W, epp), W, [1] * W, [1] * W)
-        ctx = EpContext(lay, send_counts, recv_counts, T, H)
+        ctx = EpContext(lay, send_counts, recv_counts, T, H, recv_rows=Rr)
         recv_x = (recv_q.view(torch.float8_e4m3fn), recv_s) if use_fp8 else recv_q
         return recv_x, recv_i, recv_w, per_expert, ctx
+
+    def _dispatch_peer(self, x, topk_idx, topk_weights, use_fp8):
+        T, H = x.shape
+        K = topk_idx.shape[1]
+        W, E, epp, r = self.world, self.num_experts, self.experts_per_rank, self.rank
+        pr = self._peer
+        if H != pr["hidden"]:
+            raise ValueError(f"hidden {H} differs from the receive buffers' {pr['hidden']}")
+        cap, dev = pr["capacity"], self.device
+        lay = Layout.empty(T, K, E, W, dev)
+        _lib.ep_get_dispatch_layout(topk_idx, E, W, lay, self.workspace)
+        counts = self._all_gather_rows(lay.num_tokens_per_expert)  # [W, E]
+        # every rank reads the same counts: all of them raise, or none
+        totals = counts.view(W, W, epp).sum(dim=(0, 2)).to("cpu").tolist()
+        if max(totals) > cap:
+            raise ValueError(f"a rank would receive {max(totals)} rows; capacity is {cap}")
+        dst = torch.empty(E, dtype=torch.int32, device=dev)
+        rc = torch.empty(epp, dtype=torch.int32, device=dev)
+        ro = torch.empty(epp + 1, dtype=torch.int32, device=dev)
+        _lib.ep_peer_plan(counts, r, lay.expert_offset, cap, dst, rc, ro, self.workspace)
+        quant = EP_QUANT_FP8_E4M3_1X128 if use_fp8 else EP_QUANT_NONE
+        _lib.ep_peer_dispatch(x, topk_idx, topk_weights, E, W, quant, lay, dst, self.tables,
+                              self.workspace)
+        self._barrier()  # every rank's rows have landed in their owners' buffers
+        Rr = int(totals[r])
+        per_expert = counts[:, r * epp:(r + 1) * epp]
+        send = counts.view(W, W, epp)[r].sum(dim=1).to("cpu").tolist()
+        recv = per_expert.sum(dim=1).to("cpu").tolist()
+        ctx = EpContext(lay, send, recv, T, H, topk_idx=topk_idx, dst_offset=dst, recv_rows=Rr,
+                        order="expert_major")
+        ri = self._view("recv_topk_idx", torch.int32, (cap,))[:Rr]
+        rw = self._view("recv_topk_weights", torch.float32, (cap,))[:Rr]
+        if use_fp8:
+            q = self._view("recv_x", torch.uint8, (-1,))[:cap * H].view(cap, H)[:Rr]
+            s = self._view("recv_scales", torch.float32, (cap, H // 128))[:Rr]
+            recv_x = (q.view(torch.float8_e4m3fn), s)
+        else:
+            recv_x = self._view("recv_x", torch.bfloat16, (cap, H))[:Rr]
+        return recv_x, ri, rw, per_expert, ctx
 
     # ---------------------------------------------------------------- combine --
     def combine(self, expert_out: torch.Tensor, ctx: EpContext,
                 topk_weights: torch.Tensor) -> torch.Tensor:
-        """expert_out: BF16 [sum(recv_counts), H] in the received row order.
-        Returns y: BF16 [T, H], the weighted sum of each token's expert outputs."""
+        """expert_out: BF16 [recv rows, H] in the received row order (peer transport:
+        the tensor from :meth:`expert_out_buffer`).  Returns y: BF16 [T, H], the
+        weighted sum of each token's expert outputs."""
+        y = torch.empty((ctx.num_tokens, ctx.hidden), dtype=torch.bfloat16, device=self.device)
+        if self.transport == "peer":
+            if ctx.recv_rows and expert_out.data_ptr() != self.expert_out_buffer(ctx).data_ptr():
+                raise ValueError("write the expert outputs into expert_out_buffer(ctx)")
+            self._barrier()  # every rank's expert outputs are complete
+            _lib.ep_peer_combine(self.tables, ctx.handle, ctx.topk_idx, ctx.dst_offset,
+                                 topk_weights, y, self.num_experts, self.world, self.workspace)
+            return y
         Rs = sum(ctx.send_counts)
         back = self._a2a(expert_out, Rs, ctx.send_counts, ctx.recv_counts)
         if Rs == 0:
             back = torch.zeros((1, ctx.hidden), dtype=torch.bfloat16, device=self.device)
-        y = torch.empty((ctx.num_tokens, ctx.hidden), dtype=torch.bfloat16, device=self.device)
         _lib.ep_combine(back, ctx.handle, topk_weights, y, self.workspace)
         return y

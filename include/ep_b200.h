@@ -36,8 +36,9 @@
  * Conventions (every entry point):
  *   - Pointers named as device memory must be device (or managed) memory of
  *     the current CUDA device.  Every buffer is owned and allocated by the
- *     caller; the library allocates nothing and keeps no state between calls
- *     apart from a per-device cache of the SM count and kernel attributes.
+ *     caller; the library allocates nothing (except ep_ipc_alloc, on request)
+ *     and keeps no state between calls apart from a per-device cache of the SM
+ *     count and kernel attributes.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Every call is asynchronous on that stream; host-side argument checks
  *     run before anything is enqueued and return an error synchronously.
@@ -88,7 +89,8 @@ typedef enum ep_status {
 /* Sticky device status bits (ep_read_status). */
 #define EP_DEV_INDEX_RANGE 0x1u /* an expert id outside [-1, E) or a row outside the buffer: skipped */
 #define EP_DEV_TIMEOUT 0x2u     /* a bounded device wait gave up; the kernel stopped early */
-#define EP_DEV_CAPACITY 0x4u    /* a low-latency row did not fit num_max_tokens: dropped */
+#define EP_DEV_CAPACITY 0x4u    /* a low-latency row did not fit num_max_tokens, or a rank's
+                                   receive buffer was too small (peer mode): dropped */
 
 /* Dispatch payload format. */
 typedef enum ep_quant {
@@ -389,6 +391,102 @@ EP_API ep_status ep_lb_prefetch_weights(int32_t num_slots, int64_t bytes_per_slo
 EP_API ep_status ep_lb_reduce_grads(int32_t num_slots, int64_t n, const int32_t* primary_of,
                                     float* grads, void* workspace, size_t workspace_bytes,
                                     void* stream);
+
+/* ---- expert parallelism across GPUs (partitions are ranks) ------------------
+ * "DeepSeek 开源周第二弹：DeepEP", section "DeepEP 的常规内核和低延迟内核": the
+ * normal kernels move tokens between the GPUs of a node over NVLink;
+ * "deepseek-ai/DeepEP", section "典型工作流程": dispatch to the ranks that hold the
+ * experts, expert computation, combine back to where the tokens came from.
+ *
+ * With W ranks (one process per GPU), rank p owns experts [p*E/W, (p+1)*E/W).
+ * Every rank maps every rank's receive buffers (CUDA IPC, ep_ipc_*), and the
+ * dispatch kernel stores each row straight into its owner's buffer; the combine
+ * kernel reads the expert outputs straight from the owners' buffers.  Rank p's
+ * receive rows are ordered expert (ascending), then source rank, then source
+ * (token, k): exactly partition p's rows of the one-GPU dispatch of all ranks'
+ * tokens concatenated in rank order.  One step on rank s:
+ *   1. ep_get_dispatch_layout with num_partitions = W (handle, per-expert counts);
+ *   2. the caller gathers every rank's num_tokens_per_expert into counts[W, E]
+ *      (e.g. an all-gather; a few KB);
+ *   3. ep_peer_plan: destination offsets of this rank's rows, and this rank's
+ *      receive counts / offsets;
+ *   4. the caller makes sure every rank is past its use of the buffers this step
+ *      overwrites (step 2's collective does that for the receive buffers);
+ *   5. ep_peer_dispatch: rows, scales, local ids and weights into the owners;
+ *   6. a barrier across the ranks (e.g. a one-element all-reduce on the stream),
+ *      then each rank computes its experts into its expert-output buffer;
+ *   7. a barrier, then ep_peer_combine on every rank.
+ * Tables of peer pointers are device arrays of W device addresses (rank order),
+ * each 16-byte aligned; this rank's own entry is its local buffer.  All ranks'
+ * buffers have `capacity` rows.  A partition that would receive more than
+ * `capacity` rows receives none: its rows are dropped and EP_DEV_CAPACITY is set
+ * on every sender (ep_peer_plan), and its rows are skipped by ep_peer_combine.
+ * Nothing here waits on another rank inside a kernel; the ordering comes from the
+ * caller's collectives on the same stream. */
+
+/* Bytes of a CUDA IPC memory handle (cudaIpcMemHandle_t). */
+#define EP_IPC_HANDLE_BYTES 64
+
+/* Allocate `bytes` of device memory that other processes can map, and its handle.
+ * The one allocation the library makes: memory shared by IPC must be a whole
+ * allocation of its own (a caching allocator's pool block would expose its
+ * neighbours).  ptr: out, 256-byte aligned; handle: out, EP_IPC_HANDLE_BYTES. */
+EP_API ep_status ep_ipc_alloc(size_t bytes, void** ptr, void* handle);
+/* Free memory from ep_ipc_alloc (after every peer has closed its mapping). */
+EP_API ep_status ep_ipc_free(void* ptr);
+/* Map another process's ep_ipc_alloc memory into this one (peer access enabled). */
+EP_API ep_status ep_ipc_open(const void* handle, void** ptr);
+/* Unmap memory from ep_ipc_open. */
+EP_API ep_status ep_ipc_close(void* ptr);
+
+/* Step 3.  counts: device int32 [W, E], row s = rank s's num_tokens_per_expert;
+ * expert_offset: device int32 [E+1] of this rank's layout.  Writes (device):
+ *   dst_offset[E]        row_of[t, k] + dst_offset[e] is (t, k)'s row in rank e/(E/W)
+ *   recv_count[E/W]      rows this rank receives for each of its experts
+ *   recv_offset[E/W + 1] their offsets in its receive buffer (last = total rows)
+ * (zeros for this rank, and EP_DEV_CAPACITY, if it would exceed `capacity`).
+ * 1 <= W <= 64 dividing E; 0 <= rank < W; 0 <= capacity < 2^31.  The workspace
+ * carries the status word (workspace_bytes >= 256). */
+EP_API ep_status ep_peer_plan(int32_t world, int32_t rank, int32_t num_experts, const int32_t* counts,
+                              const int32_t* expert_offset, int64_t capacity, int32_t* dst_offset,
+                              int32_t* recv_count, int32_t* recv_offset, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Receive buffers of every rank, as tables of W device pointers (device arrays). */
+typedef struct ep_peer_buffers {
+    void* const* recv_x;               /* [capacity, H] E4M3 or BF16 */
+    float* const* recv_scales;         /* [capacity, H/128] fp32 row-major; NULL for BF16 */
+    int32_t* const* recv_topk_idx;     /* [capacity] local expert id */
+    float* const* recv_topk_weights;   /* [capacity] */
+    int64_t capacity;                  /* rows of each rank's arrays, < 2^31 */
+} ep_peer_buffers;
+
+/* Step 5: ep_dispatch's payload, scales and metadata for every valid (t, k),
+ * written to row row_of[t, k] + dst_offset[e] of the owner's buffers (peers).
+ * handle: this rank's layout from ep_get_dispatch_layout with W partitions
+ * (row_of is read); quant as for ep_dispatch except EP_QUANT_SCALES_MN_MAJOR
+ * (EP_ERR_INVALID_ARG).  The workspace needs only its 256-byte header (the
+ * ticket counter and status word) and must not be used by another call at the
+ * same time. */
+EP_API ep_status ep_peer_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                  int32_t num_experts, int32_t world, int32_t quant, const void* x,
+                                  const int64_t* topk_idx, const float* topk_weights,
+                                  const ep_layout* handle, const int32_t* dst_offset,
+                                  const ep_peer_buffers* peers, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* Step 7: ep_combine with the rows read from the owners' expert outputs:
+ *   acc = +0.0f; for k = 0..K-1 with row_of[t, k] >= 0:
+ *       e = topk_idx[t, k]; row = row_of[t, k] + dst_offset[e];
+ *       acc = fmaf(topk_weights[t, k], float(expert_out[e / (E/W)][row, i]), acc)
+ *   y[t, i] = bf16_round_to_nearest_even(acc)
+ * expert_out: device table of W pointers to BF16 [capacity, H]; a row outside
+ * [0, capacity) is skipped and sets EP_DEV_INDEX_RANGE.  y: BF16 [T, H]. */
+EP_API ep_status ep_peer_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                 int32_t num_experts, int32_t world, const void* const* expert_out,
+                                 int64_t capacity, const ep_layout* handle, const int64_t* topk_idx,
+                                 const int32_t* dst_offset, const float* topk_weights, void* y,
+                                 void* workspace, size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

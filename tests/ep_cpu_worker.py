@@ -102,3 +102,186 @@ def run(rank: int, world: int, port: int, out_dir: str) -> None:
         with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
             f.write(status)
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------------ peer transport --
+
+def _peer_stand_ins(oracle, torch):
+    """CPU stand-ins for the peer transport: IPC regions are POSIX shared memory
+    (the handle is its name), pointer tables hold host addresses, and the plan,
+    dispatch and combine move bytes through those addresses."""
+    import ctypes
+    from multiprocessing import resource_tracker, shared_memory
+
+    regions = {}
+
+    def addr(shm):
+        obj = ctypes.c_char.from_buffer(shm.buf)
+        a = ctypes.addressof(obj)
+        del obj
+        return a
+
+    def ipc_alloc(n):
+        shm = shared_memory.SharedMemory(create=True, size=n)
+        a = addr(shm)
+        regions[a] = shm
+        return a, shm.name.encode().ljust(64, b"\0")
+
+    def ipc_open(h):
+        shm = shared_memory.SharedMemory(name=h.rstrip(b"\0").decode())
+        resource_tracker.unregister(shm._name, "shared_memory")  # the owner unlinks it
+        a = addr(shm)
+        regions[a] = shm
+        return a
+
+    def ipc_close(a):
+        regions.pop(a).close()
+
+    def ipc_free(a):
+        shm = regions.pop(a)
+        shm.close()
+        shm.unlink()
+
+    def device_bytes(ptr, n, device):
+        return torch.frombuffer((ctypes.c_uint8 * n).from_address(ptr), dtype=torch.uint8)
+
+    def layout(idx, E, P, lay, ws, stream=None):
+        d = oracle.layout(idx.numpy(), E, P)
+        for name in ("num_tokens_per_expert", "num_tokens_per_partition",
+                     "is_token_in_partition", "expert_offset", "row_of", "num_recv"):
+            t = getattr(lay, name)
+            t.copy_(torch.from_numpy(np.ascontiguousarray(d[name])).view(t.shape))
+        lay.src_of[:len(d["src_of"])] = torch.from_numpy(d["src_of"])
+
+    def plan(counts, rank, expert_offset, cap, dst, rc, ro, ws, stream=None):
+        c = counts.numpy().astype(np.int64)
+        W, E = c.shape
+        epp = E // W
+        tot, before = c.sum(0), c[:rank].sum(0)
+        base = np.zeros(E, np.int64)
+        for q in range(W):
+            seg = tot[q * epp:(q + 1) * epp]
+            base[q * epp:(q + 1) * epp] = np.concatenate([[0], np.cumsum(seg)[:-1]])
+        dst.copy_(torch.from_numpy((base + before - expert_offset.numpy()[:E]).astype(np.int32)))
+        mine = tot[rank * epp:(rank + 1) * epp]
+        rc.copy_(torch.from_numpy(mine.astype(np.int32)))
+        ro.copy_(torch.from_numpy(np.concatenate([[0], np.cumsum(mine)]).astype(np.int32)))
+
+    def put(address, arr):
+        arr = np.ascontiguousarray(arr)
+        ctypes.memmove(int(address), arr.ctypes.data, arr.nbytes)
+
+    def get(address, n):
+        return np.frombuffer((ctypes.c_uint8 * n).from_address(int(address)), np.uint8).copy()
+
+    def dispatch(x, idx, w, E, W, quant, lay, dst, tables, ws, stream=None):
+        xs = x.view(torch.int16).numpy().view(np.uint16)
+        ids = idx.numpy()
+        K = ids.shape[1]
+        d = oracle.dispatch(xs, ids, w.numpy(), E, W, quant="fp8" if quant else "none")
+        epp, H = E // W, xs.shape[1]
+        off = dst.numpy()
+        for r, src in enumerate(d["src_of"]):
+            t, k = divmod(int(src), K)
+            e = int(ids[t, k])
+            p, row = e // epp, r + int(off[e])
+            rx = d["recv_x"][r]
+            put(tables.recv_x[p] + row * rx.nbytes, rx)
+            if quant:
+                put(tables.recv_scales[p] + row * (H // 128) * 4, d["recv_scales"][r])
+            put(tables.recv_topk_idx[p] + row * 4, d["recv_topk_idx"][r:r + 1])
+            put(tables.recv_topk_weights[p] + row * 4, d["recv_topk_weights"][r:r + 1])
+
+    def combine(tables, lay, idx, dst, w, y, E, W, ws, stream=None):
+        ids, ro = idx.numpy(), lay.row_of.numpy()
+        T, K = ids.shape
+        H = y.shape[1]
+        epp, off = E // W, dst.numpy()
+        rows = np.zeros((max(T * K, 1), H), np.uint16)
+        row_of = np.full((T, K), -1, np.int32)
+        for t in range(T):
+            for k in range(K):
+                if ro[t, k] >= 0:
+                    e = int(ids[t, k])
+                    a = tables.expert_out[e // epp] + (int(ro[t, k]) + int(off[e])) * H * 2
+                    rows[t * K + k] = get(a, H * 2).view(np.uint16)
+                    row_of[t, k] = t * K + k
+        yb, _ = oracle.combine(rows, row_of, w.numpy())
+        y.copy_(torch.from_numpy(yb.view(np.int16)).view(torch.bfloat16))
+
+    return dict(ep_ipc_alloc=ipc_alloc, ep_ipc_open=ipc_open, ep_ipc_close=ipc_close,
+                ep_ipc_free=ipc_free, device_bytes=device_bytes, ep_get_dispatch_layout=layout,
+                ep_peer_plan=plan, ep_peer_dispatch=dispatch, ep_peer_combine=combine,
+                ep_workspace_init=lambda ws, stream=None: None)
+
+
+def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for p in (root, os.path.join(root, "tests")):
+        if p not in sys.path:
+            sys.path.insert(0, p)
+    import torch
+    import torch.distributed as dist
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    status = "failed"
+    g = None
+    try:
+        import oracle
+        from combine_get_dispatch_05_b200 import ep_group
+        from workloads import make_custom
+
+        for name, fn in _peer_stand_ins(oracle, torch).items():
+            setattr(ep_group._lib, name, fn)
+
+        E, H, K = 24, 256, 4
+        epp = E // world
+        tokens = [0 if r == world - 1 and world > 2 else 70 + 29 * r for r in range(world)]
+        loads = [make_custom(tokens[r], H, K, E, world, seed=300 + r, mask_frac=0.1)
+                 for r in range(world)]
+        x_all = np.concatenate([w.x for w in loads])
+        idx_all = np.concatenate([w.topk_idx for w in loads])
+        w_all = np.concatenate([w.topk_weights for w in loads])
+        t0 = sum(tokens[:rank])
+        w = loads[rank]
+        g = ep_group.EpGroup(E, device="cpu", transport="peer", hidden=H, max_tokens=128)
+        x = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16)
+        idx = torch.from_numpy(w.topk_idx)
+        wts = torch.from_numpy(w.topk_weights)
+        for quant in ("fp8", "none", "fp8"):  # the buffers are reused across steps
+            recv_x, ri, rw, per_expert, ctx = g.dispatch(x, idx, wts, use_fp8=quant == "fp8")
+            d = oracle.dispatch(x_all, idx_all, w_all, E, world, quant=quant)
+            lo, hi = d["expert_offset"][rank * epp], d["expert_offset"][(rank + 1) * epp]
+            if quant == "fp8":
+                got = recv_x[0].view(torch.uint8).numpy()
+                assert np.array_equal(recv_x[1].numpy().view(np.uint32),
+                                      d["recv_scales"][lo:hi].view(np.uint32))
+            else:
+                got = recv_x.view(torch.int16).numpy().view(np.uint16)
+            assert np.array_equal(got, d["recv_x"][lo:hi]), quant
+            assert np.array_equal(ri.numpy(), d["recv_topk_idx"][lo:hi]), quant
+            assert np.array_equal(rw.numpy().view(np.uint32),
+                                  d["recv_topk_weights"][lo:hi].view(np.uint32)), quant
+            want_cnt = np.stack([oracle.layout(l.topk_idx, E, world)["num_tokens_per_expert"]
+                                 [rank * epp:(rank + 1) * epp] for l in loads])
+            assert np.array_equal(per_expert.numpy(), want_cnt), quant
+            assert ctx.recv_counts == want_cnt.sum(1).tolist()
+            eo_all = oracle.identity_expert(d["recv_x"], d["recv_scales"], quant=quant)
+            buf = g.expert_out_buffer(ctx)
+            buf.copy_(torch.from_numpy(eo_all[lo:hi].view(np.int16)).view(torch.bfloat16))
+            y = g.combine(buf, ctx, wts)
+            y_all, _ = oracle.combine(eo_all, d["row_of"], w_all)
+            assert np.array_equal(y.view(torch.int16).numpy().view(np.uint16),
+                                  y_all[t0:t0 + tokens[rank]]), quant
+        status = "ok"
+    finally:
+        try:
+            if g is not None:
+                g.close()
+        finally:
+            with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
+                f.write(status)
+            dist.destroy_process_group()

@@ -52,7 +52,7 @@ def test_built_for_sm100a_only():
 
 
 def test_version_and_strings(ep):
-    assert ep.lib.ep_abi_version() == 1
+    assert ep.lib.ep_abi_version() == 2
     assert ep.status_string(ep.EP_ERR_SHAPE) == "unsupported size"
     assert ep.status_string(99) == "unknown status"
 
@@ -226,3 +226,59 @@ def test_lb_host_checks(ep):
     assert red(4, -4, f, f, f, 4096, None) == 2
     assert red(4, 8, f, f + 4, f, 4096, None) == 1       # grads not 16-byte aligned
     assert red(4, 0, f, None, f, 4096, None) == 0        # nothing to reduce
+
+
+def test_peer_host_checks(ep):
+    f = _Fake.P
+    lay = _layout_struct(ep)
+    L = ep.lib
+    plan = L.ep_peer_plan
+    assert plan(0, 0, 8, f, f, 64, f, f, f, f, 4096, None) == 2         # no ranks
+    assert plan(65, 0, 130, f, f, 64, f, f, f, f, 4096, None) == 2      # too many ranks
+    assert plan(3, 0, 8, f, f, 64, f, f, f, f, 4096, None) == 2         # E % W
+    assert plan(2, 2, 8, f, f, 64, f, f, f, f, 4096, None) == 2         # rank >= W
+    assert plan(2, 0, 8, f, f, -1, f, f, f, f, 4096, None) == 2         # capacity < 0
+    assert plan(2, 0, 8, f, f, 1 << 31, f, f, f, f, 4096, None) == 2    # capacity >= 2^31
+    assert plan(2, 0, 8, None, f, 64, f, f, f, f, 4096, None) == 1
+    assert plan(2, 0, 8, f, f, 64, f, None, f, f, 4096, None) == 1
+    assert plan(2, 0, 8, f, f, 64, f, f, f, f, 64, None) == 1          # workspace too small
+
+    peers = ep._lib.ep_peer_buffers(f, f, f, f, 64)
+
+    def disp(T=16, H=256, K=4, E=8, W=2, quant=1, x=f, dst=f, pb=peers, ws=f):
+        return L.ep_peer_dispatch(T, H, K, E, W, quant, x, f, f, ctypes.byref(lay), dst,
+                                  ctypes.byref(pb) if pb is not None else None, ws, 4096, None)
+
+    assert disp(quant=0x101) == 1       # block-major scales are not offered
+    assert disp(quant=4) == 1
+    assert disp(E=7) == 2
+    assert disp(H=136) == 2             # FP8 needs H % 128 == 0
+    assert disp(pb=None) == 2
+    assert disp(pb=ep._lib.ep_peer_buffers(f, f, f, f, 1 << 31)) == 2
+    assert disp(pb=ep._lib.ep_peer_buffers(f, None, f, f, 64)) == 1     # FP8 needs scales
+    assert disp(pb=ep._lib.ep_peer_buffers(None, f, f, f, 64)) == 1
+    assert disp(x=f + 8) == 1
+    assert disp(dst=None) == 1
+    assert disp(ws=f + 8) == 1
+    assert disp(T=0, x=None, dst=None) == 0   # an empty batch touches nothing
+
+    comb = L.ep_peer_combine
+    assert comb(4, 100, 2, 8, 2, f, 64, ctypes.byref(lay), f, f, f, f, f, 4096, None) == 2  # H % 8
+    assert comb(4, 128, 2, 8, 3, f, 64, ctypes.byref(lay), f, f, f, f, f, 4096, None) == 2  # E % W
+    assert comb(4, 128, 2, 8, 2, f, -1, ctypes.byref(lay), f, f, f, f, f, 4096, None) == 2
+    assert comb(4, 128, 2, 8, 2, None, 64, ctypes.byref(lay), f, f, f, f, f, 4096, None) == 1
+    assert comb(4, 128, 2, 8, 2, f, 64, ctypes.byref(lay), None, f, f, f, f, 4096, None) == 1
+    assert comb(4, 128, 2, 8, 2, f, 64, ctypes.byref(lay), f, f, f, f + 4, f, 4096, None) == 1
+    assert comb(4, 128, 2, 8, 2, f, 64, None, f, f, f, f, f, 4096, None) == 1
+    assert comb(0, 128, 2, 8, 2, None, 64, ctypes.byref(lay), None, None, None, None, f, 4096,
+                None) == 0
+
+    ptr = ctypes.c_void_p()
+    handle = ctypes.create_string_buffer(ep.EP_IPC_HANDLE_BYTES)
+    assert L.ep_ipc_alloc(0, ctypes.byref(ptr), handle) == 1
+    assert L.ep_ipc_alloc(256, None, handle) == 1
+    assert L.ep_ipc_alloc(256, ctypes.byref(ptr), None) == 1
+    assert L.ep_ipc_free(None) == 1
+    assert L.ep_ipc_open(None, ctypes.byref(ptr)) == 1
+    assert L.ep_ipc_open(handle, None) == 1
+    assert L.ep_ipc_close(None) == 1

@@ -1,7 +1,10 @@
-"""EpGroup's exchange on the CPU: 2 and 3 gloo ranks as processes, the one-GPU
-kernels replaced by oracle-based stand-ins (so no GPU is needed), one rank with an
-empty batch.  Checks the rows each rank receives, the per-(source, expert) counts
-and the combine results against the oracle, for FP8 and BF16 payloads."""
+"""EpGroup's exchange on the CPU: 2 and 3 gloo ranks as processes, the kernels
+replaced by oracle-based stand-ins (so no GPU is needed), one rank with an empty
+batch.  Checks the rows each rank receives, the per-(source, expert) counts and the
+combine results against the oracle, for FP8 and BF16 payloads, for both transports:
+the all-to-all one, and the peer one (receive buffers in POSIX shared memory stand
+for IPC-mapped GPU memory; the stand-in kernels store and load through the pointer
+tables)."""
 import multiprocessing as mp
 import socket
 
@@ -14,13 +17,15 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
+@pytest.mark.parametrize("transport", ["nccl", "peer"])
 @pytest.mark.parametrize("world", [2, 3])
-def test_ep_group_exchange_on_cpu(tmp_path, world):
+def test_ep_group_exchange_on_cpu(tmp_path, world, transport):
     import ep_cpu_worker
 
+    target = ep_cpu_worker.run if transport == "nccl" else ep_cpu_worker.run_peer
     ctx = mp.get_context("spawn")
     port = _free_port()
-    procs = [ctx.Process(target=ep_cpu_worker.run, args=(r, world, port, str(tmp_path)))
+    procs = [ctx.Process(target=target, args=(r, world, port, str(tmp_path)))
              for r in range(world)]
     for p in procs:
         p.start()
