@@ -554,6 +554,93 @@ def time_dedup(ep, w, dev, steps):
     return out
 
 
+def time_peer(ep, w, dev, steps):
+    """The peer-memory (multi-GPU) kernels on workload w with every owner's buffers on
+    this GPU: rank 0 of W = w.num_partitions holds all tokens, the other ranks none.
+    Dispatch = layout + the count copy that stands for the all-gather + plan + peer
+    dispatch (rows stored into the W owners' buffers); combine = peer combine (rows
+    loaded from them).  Same algorithmic bytes as the one-GPU step; the stores and
+    loads stay in this GPU's HBM, so this measures the kernels, not NVLink."""
+    import numpy as np
+    import torch
+
+    T, H, K, E, W = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
+    fp8 = w.quant == "fp8"
+    epp = E // W
+    x = torch.from_numpy(w.x.view(np.int16)).to(dev).view(torch.bfloat16)
+    idx = torch.from_numpy(w.topk_idx).to(dev)
+    wts = torch.from_numpy(w.topk_weights).to(dev)
+    lay = ep.Layout.empty(T, K, E, W, dev)
+    ws = torch.empty(ep.ep_workspace_bytes(T, E, W), dtype=torch.uint8, device=dev)
+    ep.ep_workspace_init(ws)
+    ep.ep_get_dispatch_layout(idx, E, W, lay, ws)
+    torch.cuda.synchronize()
+    per_part = lay.num_tokens_per_expert.view(W, epp).sum(dim=1)
+    cap = int(per_part.max().item()) + 16
+    R = int(lay.num_recv.item())
+    bufs = [dict(x=torch.empty((cap, H), dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev),
+                 s=torch.empty((cap, H // 128), dtype=torch.float32, device=dev),
+                 i=torch.empty(cap, dtype=torch.int32, device=dev),
+                 w=torch.empty(cap, dtype=torch.float32, device=dev),
+                 eo=torch.empty((cap, H), dtype=torch.bfloat16, device=dev)) for _ in range(W)]
+    tables = ep.PeerTables.from_addresses(dev, cap, *[[b[k].data_ptr() for b in bufs]
+                                                      for k in ("x", "s", "i", "w", "eo")])
+    counts = torch.zeros((W, E), dtype=torch.int32, device=dev)
+    dst = torch.empty(E, dtype=torch.int32, device=dev)
+    rc = torch.empty(epp, dtype=torch.int32, device=dev)
+    ro = torch.empty(epp + 1, dtype=torch.int32, device=dev)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    quant = ep.EP_QUANT_FP8_E4M3_1X128 if fp8 else ep.EP_QUANT_NONE
+
+    def disp():
+        ep.ep_get_dispatch_layout(idx, E, W, lay, ws)
+        counts[0].copy_(lay.num_tokens_per_expert)  # stands for the all-gather
+        ep.ep_peer_plan(counts, 0, lay.expert_offset, cap, dst, rc, ro, ws)
+        ep.ep_peer_dispatch(x, idx, wts, E, W, quant, lay, dst, tables, ws)
+
+    def comb():
+        ep.ep_peer_combine(tables, lay, idx, dst, wts, y, E, W, ws)
+
+    disp()
+    torch.cuda.synchronize()
+    for b, n in zip(bufs, per_part.tolist()):  # identity experts on the received rows
+        if fp8:
+            v = b["x"][:n].view(torch.float8_e4m3fn).to(torch.float32)
+            b["eo"][:n] = (v * b["s"][:n].repeat_interleave(128, dim=1)).to(torch.bfloat16)
+        else:
+            b["eo"][:n] = b["x"][:n]
+    bytes_d, bytes_c = algorithmic_bytes(T, H, K, E, W, R, fp8)
+    out = {"ranks": W, "tokens": T, "recv_rows": R, "capacity": cap}
+    for name, fn, nbytes in (("dispatch", disp, bytes_d), ("combine", comb, bytes_c)):
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            fn()
+            fn()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        evs[0].record()
+        for i in range(steps):
+            g.replay()
+            evs[i + 1].record()
+        torch.cuda.synchronize()
+        us = statistics.mean(evs[i].elapsed_time(evs[i + 1]) for i in range(steps)) * 1e3
+        out[name + "_us"] = round(us, 2)
+        out[name + "_gbs"] = round(nbytes / (us * 1e-6) / 1e9, 1)
+    if ep.ep_read_status(ws) != 0:
+        raise RuntimeError("device status set in the peer-memory run")
+    del bufs, tables
+    torch.cuda.empty_cache()
+    return out
+
+
 def time_e2e(ep, runner, steps):
     """The same step through the public API with host buffers, pipelined the way a
     serving loop would run it: every step copies its inputs (x, topk_idx,
@@ -785,6 +872,11 @@ def run_ours(args):
             extra["dedup"]["workload"] = args.workload
         except Exception as exc:
             extra["dedup"] = {"error": repr(exc)}
+        try:
+            extra["peer"] = time_peer(ep, w, dev, args.extra_steps)
+            extra["peer"]["workload"] = args.workload
+        except Exception as exc:  # report, do not hide
+            extra["peer"] = {"error": repr(exc)}
         try:
             extra["lb"] = time_lb(ep, dev, min(args.extra_steps, 20), args.seed, args.lb_scale)
         except Exception as exc:  # report, do not hide
