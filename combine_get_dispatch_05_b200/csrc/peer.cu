@@ -17,7 +17,10 @@
 // by the caller), with this rank's receive counts and offsets.  If a partition
 // receives more rows than `capacity`, every offset of its experts is set so that
 // all their rows fall outside the buffer (the dispatch and combine kernels then
-// skip them) and EP_DEV_CAPACITY is raised.
+// skip them) and EP_DEV_CAPACITY is raised.  The plan is a programmatic dependent
+// of what precedes it and, once that is complete, lets the dispatch kernel start:
+// the dispatch loads and quantises its rows while the plan runs, and only its storer
+// waits for the offsets.
 #include "ep_device.cuh"
 #include "ep_internal.h"
 
@@ -32,6 +35,8 @@ constexpr int32_t kNoRoom = 0x7fffffff;  // offset that puts every row past any 
 // (rows of e from ranks < rank) | base[E] (offset of e's segment in its owner's
 // buffer) as int64.
 __global__ void __launch_bounds__(kPlanThreads) peer_plan_kernel(PeerPlanParams p) {
+    pdl_wait();               // the counts and the layout are complete and visible
+    pdl_launch_dependents();  // the dispatch may start loading and quantising its rows
     extern __shared__ int64_t psm[];
     const int E = p.num_experts, W = p.world;
     const int epp = E / W;
@@ -87,8 +92,18 @@ cudaError_t launch_peer_plan(const PeerPlanParams& p, cudaStream_t stream) {
     cudaError_t err = cudaFuncSetAttribute(peer_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    peer_plan_kernel<<<1, kPlanThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    // programmatic dependent of the previous kernel; it waits for it before reading
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(kPlanThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, peer_plan_kernel, p);
 }
 
 }  // namespace ep

@@ -161,12 +161,10 @@ class EpGroup:
         calls it, after its last combine)."""
         if self._peer is None:
             return
-        if self.device.type == "cuda":
-            torch.cuda.synchronize(self.device)
-        self._barrier()
+        self._host_barrier()  # no rank's kernels touch any region any more
         for ptr in self._peer["opened"]:
             _lib.ep_ipc_close(ptr)
-        self._barrier()  # nobody maps this rank's region any more
+        self._host_barrier()  # every rank has closed its mappings of this rank's region
         self._peer["region"] = None
         _lib.ep_ipc_free(self._peer["base"])
         self._peer = None
@@ -196,13 +194,23 @@ class EpGroup:
         return torch.stack(parts).to(t.device)
 
     def _barrier(self) -> None:
-        """Every rank's preceding work on the stream is done before anything after."""
+        """Every rank's preceding work on the stream is done before anything after it
+        on the stream (NCCL: asynchronous for the host)."""
         if not self.via_host:
             dist.all_reduce(self._flag, group=self.group)  # ordered on the current stream
         else:
             if self.device.type == "cuda":
                 torch.cuda.synchronize(self.device)
             dist.barrier(group=self.group)
+
+    def _host_barrier(self) -> None:
+        """As _barrier, and the host waits for it: when it returns, every rank's host
+        has reached this point and every rank's preceding device work is done."""
+        if self.device.type == "cuda":
+            torch.cuda.synchronize(self.device)
+        self._barrier()
+        if self.device.type == "cuda":
+            torch.cuda.synchronize(self.device)
 
     # --------------------------------------------------------------- dispatch --
     def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,

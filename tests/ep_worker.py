@@ -86,3 +86,68 @@ def run(rank: int, world: int, port: int, out_dir: str) -> None:
         with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
             f.write(status)
         dist.destroy_process_group()
+
+
+def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
+    """EpGroup(transport="peer") with every kernel real.  With one rank the region the
+    rank allocates (ep_ipc_alloc) is the only one, so no peer mapping is opened: this
+    runs the allocation, the views over it, the tables, layout, count gather, plan,
+    peer dispatch, barriers, peer combine and close() on the GPU."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for p in (root, os.path.join(root, "tests")):
+        if p not in sys.path:
+            sys.path.insert(0, p)
+    import torch
+    import torch.distributed as dist
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    status = "failed"
+    g = None
+    try:
+        import combine_get_dispatch_05_b200 as ep
+        import oracle
+        from gpu_path import bf16_to_u16, dev_u16_as_bf16
+        from workloads import make_custom
+
+        E, H, K = 32, 512, 4
+        w = make_custom(333, H, K, E, world, seed=120 + rank, mask_frac=0.1)
+        g = ep.EpGroup(E, transport="peer", hidden=H, max_tokens=512)
+        x = dev_u16_as_bf16(w.x)
+        idx = torch.from_numpy(w.topk_idx).cuda()
+        wts = torch.from_numpy(w.topk_weights).cuda()
+        for quant in ("fp8", "none", "fp8"):  # the region is reused across steps
+            recv_x, ri, rw, per_expert, ctx = g.dispatch(x, idx, wts, use_fp8=quant == "fp8")
+            d = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, E, world, quant=quant)
+            R = int(d["num_recv"][0])
+            assert ctx.recv_rows == R
+            if quant == "fp8":
+                assert np.array_equal(recv_x[0].view(torch.uint8).cpu().numpy(), d["recv_x"])
+                assert np.array_equal(recv_x[1].cpu().numpy().view(np.uint32),
+                                      d["recv_scales"].view(np.uint32))
+            else:
+                assert np.array_equal(bf16_to_u16(recv_x), d["recv_x"])
+            assert np.array_equal(ri.cpu().numpy(), d["recv_topk_idx"])
+            assert np.array_equal(rw.cpu().numpy().view(np.uint32),
+                                  d["recv_topk_weights"].view(np.uint32))
+            assert np.array_equal(per_expert.cpu().numpy().reshape(-1),
+                                  d["num_tokens_per_expert"])
+            eo = oracle.identity_expert(d["recv_x"], d["recv_scales"], quant=quant)
+            out = g.expert_out_buffer(ctx)
+            out.copy_(dev_u16_as_bf16(eo))
+            y = g.combine(out, ctx, wts)
+            y_ref, _ = oracle.combine(eo, d["row_of"], w.topk_weights)
+            assert np.array_equal(bf16_to_u16(y), y_ref), quant
+        assert ep.ep_read_status(g.workspace) == 0
+        status = "ok"
+    finally:
+        try:
+            if g is not None:
+                g.close()
+        finally:
+            with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
+                f.write(status)
+            dist.destroy_process_group()

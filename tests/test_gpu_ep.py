@@ -40,3 +40,19 @@ def test_ep_group_dispatch_combine(tmp_path, world):
                else "missing" for r in range(world)]
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
     assert results == ["ok"] * world, results
+
+
+def test_ep_group_peer_transport_one_rank(tmp_path):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import ep_worker
+
+    ctx = mp.get_context("spawn")
+    p = ctx.Process(target=ep_worker.run_peer, args=(0, 1, _free_port(), str(tmp_path)))
+    p.start()
+    p.join(timeout=240)
+    if p.is_alive():  # only our own child
+        p.kill()
+        p.join()
+    assert p.exitcode == 0
+    assert (tmp_path / "rank0.txt").read_text() == "ok"
