@@ -560,7 +560,8 @@ def time_peer(ep, w, dev, steps):
     Dispatch = layout + the count copy that stands for the all-gather + plan + peer
     dispatch (rows stored into the W owners' buffers); combine = peer combine (rows
     loaded from them).  Same algorithmic bytes as the one-GPU step; the stores and
-    loads stay in this GPU's HBM, so this measures the kernels, not NVLink."""
+    loads stay in this GPU's HBM, so this measures the kernels, not NVLink.  Then
+    the same for deduplicated rows (one per token and owner rank)."""
     import numpy as np
     import torch
 
@@ -634,9 +635,64 @@ def time_peer(ep, w, dev, steps):
         us = statistics.mean(evs[i].elapsed_time(evs[i + 1]) for i in range(steps)) * 1e3
         out[name + "_us"] = round(us, 2)
         out[name + "_gbs"] = round(nbytes / (us * 1e-6) / 1e9, 1)
+    # deduplicated rows: one per (token, owner rank), [K] id / weight lists
+    dlay = ep.Layout.empty(T, W, W, W, dev)
+    ep.ep_get_dispatch_layout_dedup(idx, E, W, dlay, ws)
+    torch.cuda.synchronize()
+    dper = dlay.num_tokens_per_expert.clone()
+    dcap = int(dper.max().item()) + 16
+    Rd = int(dlay.num_recv.item())
+    dbufs = [dict(x=b["x"], s=b["s"], eo=b["eo"],
+                  i=torch.empty((dcap, K), dtype=torch.int32, device=dev),
+                  w=torch.empty((dcap, K), dtype=torch.float32, device=dev)) for b in bufs]
+    assert dcap <= cap
+    dtables = ep.PeerTables.from_addresses(dev, dcap, *[[b[k].data_ptr() for b in dbufs]
+                                                        for k in ("x", "s", "i", "w", "eo")])
+    dcounts = torch.zeros((W, W), dtype=torch.int32, device=dev)
+    ddst = torch.empty(W, dtype=torch.int32, device=dev)
+    drc = torch.empty(1, dtype=torch.int32, device=dev)
+    dro = torch.empty(2, dtype=torch.int32, device=dev)
+
+    def ddisp():
+        ep.ep_get_dispatch_layout_dedup(idx, E, W, dlay, ws)
+        dcounts[0].copy_(dlay.num_tokens_per_expert)  # stands for the all-gather
+        ep.ep_peer_plan(dcounts, 0, dlay.expert_offset, dcap, ddst, drc, dro, ws)
+        ep.ep_peer_dispatch_dedup(x, idx, wts, E, W, quant, dlay, ddst, dtables, ws)
+
+    def dcomb():
+        ep.ep_peer_combine_dedup(dtables, dlay, ddst, y, W, ws)
+
+    payload = Rd * H * (1 if fp8 else 2) + (Rd * (H // 128) * 4 if fp8 else 0)
+    bytes_dd = (T * H * 2 + payload + T * K * 12 + Rd * K * 8 + Rd * 4 + T * W * 4
+                + (W + 1) * 4 + 2 * W * 4 + T * W)
+    bytes_dc = Rd * H * 2 + T * H * 2 + T * W * 4
+    out["dedup_rows"] = Rd
+    for name, fn, nbytes in (("dedup_dispatch", ddisp, bytes_dd), ("dedup_combine", dcomb, bytes_dc)):
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            fn()
+            fn()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        evs[0].record()
+        for i in range(steps):
+            g.replay()
+            evs[i + 1].record()
+        torch.cuda.synchronize()
+        us = statistics.mean(evs[i].elapsed_time(evs[i + 1]) for i in range(steps)) * 1e3
+        out[name + "_us"] = round(us, 2)
+        out[name + "_gbs"] = round(nbytes / (us * 1e-6) / 1e9, 1)
     if ep.ep_read_status(ws) != 0:
         raise RuntimeError("device status set in the peer-memory run")
-    del bufs, tables
+    del bufs, tables, dbufs, dtables
     torch.cuda.empty_cache()
     return out
 

@@ -21,6 +21,7 @@ from ._lib import (  # noqa: F401
     ep_low_latency_dispatch, ep_read_status, ep_workspace_bytes, ep_workspace_init, lib,
     status_string, EP_IPC_HANDLE_BYTES, PeerTables, device_bytes, ep_ipc_alloc, ep_ipc_close,
     ep_ipc_free, ep_ipc_open, ep_peer_combine, ep_peer_dispatch, ep_peer_plan,
+    ep_get_dispatch_layout_dedup, ep_peer_combine_dedup, ep_peer_dispatch_dedup,
 )
 from .buffer import Buffer  # noqa: F401
 from .ep_group import EpContext, EpGroup  # noqa: F401

@@ -38,7 +38,8 @@ EXPORTED = (
     "ep_get_dispatch_layout_static", "ep_dispatch_backward", "ep_combine_backward",
     "ep_dispatch_dedup", "ep_combine_dedup", "ep_lb_prefetch_weights", "ep_lb_reduce_grads",
     "ep_ipc_alloc", "ep_ipc_free", "ep_ipc_open", "ep_ipc_close", "ep_peer_plan",
-    "ep_peer_dispatch", "ep_peer_combine",
+    "ep_peer_dispatch", "ep_peer_combine", "ep_get_dispatch_layout_dedup",
+    "ep_peer_dispatch_dedup", "ep_peer_combine_dedup",
 )
 EP_IPC_HANDLE_BYTES = 64
 
@@ -126,6 +127,14 @@ def _load() -> ctypes.CDLL:
     L.ep_peer_combine.argtypes = [i64, i64, i32, i32, i32, vp, i64, ctypes.POINTER(ep_layout), vp,
                                   vp, vp, vp, vp, sz, vp]
     L.ep_peer_combine.restype = st
+    L.ep_get_dispatch_layout_dedup.argtypes = [i64, i32, i32, i32, vp, ctypes.POINTER(ep_layout),
+                                               vp, sz, vp]
+    L.ep_get_dispatch_layout_dedup.restype = st
+    L.ep_peer_dispatch_dedup.argtypes = L.ep_peer_dispatch.argtypes
+    L.ep_peer_dispatch_dedup.restype = st
+    L.ep_peer_combine_dedup.argtypes = [i64, i64, i32, vp, i64, ctypes.POINTER(ep_layout), vp, vp,
+                                        vp, sz, vp]
+    L.ep_peer_combine_dedup.restype = st
     return L
 
 
@@ -602,3 +611,68 @@ def ep_peer_combine(tables: PeerTables, handle: Layout, topk_idx: torch.Tensor,
         T, H, K, num_experts, world, tables.expert_out.data_ptr(), tables.capacity,
         ctypes.byref(c), topk_idx.data_ptr(), dst_offset.data_ptr(), topk_weights.data_ptr(),
         y.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_get_dispatch_layout_dedup(topk_idx: torch.Tensor, num_experts: int, num_partitions: int,
+                                 layout: Layout, workspace: torch.Tensor, stream=None) -> None:
+    """The deduplicated layout; layout = Layout.empty(T, P, P, P) (partition-sized)."""
+    _need(topk_idx, "topk_idx", torch.int64)
+    T, K = topk_idx.shape
+    P = num_partitions
+    _need(layout.row_of, "layout.row_of", torch.int32, shape=(T, P))
+    _need(layout.num_tokens_per_expert, "layout.num_tokens_per_expert", torch.int32, shape=(P,))
+    _need(layout.num_tokens_per_partition, "layout.num_tokens_per_partition", torch.int32,
+          shape=(P,))
+    _need(layout.is_token_in_partition, "layout.is_token_in_partition", torch.uint8, shape=(T, P))
+    _need(layout.expert_offset, "layout.expert_offset", torch.int32, shape=(P + 1,))
+    _need(layout.src_of, "layout.src_of", torch.int32, numel_at_least=T * min(P, K))
+    _need(workspace, "workspace", torch.uint8)
+    c = layout.c()
+    _check("ep_get_dispatch_layout_dedup", lib.ep_get_dispatch_layout_dedup(
+        T, K, num_experts, P, topk_idx.data_ptr(), ctypes.byref(c), workspace.data_ptr(),
+        workspace.numel(), _stream(stream)))
+
+
+def ep_peer_dispatch_dedup(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
+                           num_experts: int, world: int, quant: int, handle: Layout,
+                           dst_offset: torch.Tensor, tables: PeerTables, workspace: torch.Tensor,
+                           stream=None) -> None:
+    """Rows per (token, rank); the id / weight tables point to [capacity, K] arrays."""
+    _need(x, "x", torch.bfloat16)
+    T, H = x.shape
+    K = topk_idx.shape[1]
+    _need(topk_idx, "topk_idx", torch.int64, shape=(T, K))
+    _need(topk_weights, "topk_weights", torch.float32, shape=(T, K))
+    _need(handle.row_of, "handle.row_of", torch.int32, shape=(T, world))
+    _need(dst_offset, "dst_offset", torch.int32, shape=(world,))
+    for name in ("recv_x", "recv_scales", "recv_topk_idx", "recv_topk_weights"):
+        _need(getattr(tables, name), "tables." + name, torch.int64, shape=(world,))
+    _need(workspace, "workspace", torch.uint8)
+    c = ep_layout(row_of=handle.row_of.data_ptr())
+    fp8 = quant != EP_QUANT_NONE
+    b = ep_peer_buffers(tables.recv_x.data_ptr(),
+                        tables.recv_scales.data_ptr() if fp8 else None,
+                        tables.recv_topk_idx.data_ptr(), tables.recv_topk_weights.data_ptr(),
+                        tables.capacity)
+    _check("ep_peer_dispatch_dedup", lib.ep_peer_dispatch_dedup(
+        T, H, K, num_experts, world, quant, x.data_ptr(), topk_idx.data_ptr(),
+        topk_weights.data_ptr(), ctypes.byref(c), dst_offset.data_ptr(), ctypes.byref(b),
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_peer_combine_dedup(tables: PeerTables, handle: Layout, dst_offset: torch.Tensor,
+                          y: torch.Tensor, world: int, workspace: torch.Tensor,
+                          stream=None) -> None:
+    """y[t] = sum over ranks q (in order) of rank q's partition output for (t, q);
+    the outputs are read through tables.expert_out."""
+    _need(y, "y", torch.bfloat16)
+    T, H = y.shape
+    _need(handle.row_of, "handle.row_of", torch.int32, shape=(T, world))
+    _need(dst_offset, "dst_offset", torch.int32, shape=(world,))
+    _need(tables.expert_out, "tables.expert_out", torch.int64, shape=(world,))
+    _need(workspace, "workspace", torch.uint8)
+    c = ep_layout(row_of=handle.row_of.data_ptr())
+    _check("ep_peer_combine_dedup", lib.ep_peer_combine_dedup(
+        T, H, world, tables.expert_out.data_ptr(), tables.capacity, ctypes.byref(c),
+        dst_offset.data_ptr(), y.data_ptr(), workspace.data_ptr(), workspace.numel(),
+        _stream(stream)))

@@ -30,12 +30,15 @@ constexpr int kLoadBatch = 8;  // combine backward: slots handled per batch
 // kBatch: row loads issued per thread before the first FMA.  The token's valid
 // rows are compacted (k order kept) so a batch holds only rows that exist; sparse
 // routings (one slot per partition, about half of them empty) use a batch of 4 and
-// fewer registers, so more threads and more loads are in flight per SM.
+// fewer registers, so more threads and more loads are in flight per SM (the peer
+// variant, which holds row pointers, keeps two CTAs per SM so it does not spill).
 // kPeer: partitions are ranks; slot k's row is row_of[t, k] + peer_offset[e] in the
-// expert outputs of the rank that owns e = topk_idx[t, k] (read over NVLink), and
-// the compaction records a pointer to each valid row instead of its index.
+// expert outputs of the rank that owns e = topk_idx[t, k] (read over NVLink), or,
+// with peer_by_slot (deduplicated rows, slot k = rank k), row_of[t, k] +
+// peer_offset[k] in rank k's outputs; the compaction records a pointer to each
+// valid row instead of its index.
 template <int kBatch, bool kPeer>
-__global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
+__global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 && !kPeer ? 3 : 2)
     combine_kernel(CombineParams p, int64_t vec_per_slice) {
     pdl_wait();               // the previous kernel (e.g. the dispatch) is complete
     pdl_launch_dependents();  // the next kernel may be scheduled
@@ -57,7 +60,8 @@ __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
     if (tid < K && static_cast<int64_t>(blockIdx.x) < T) {
         nrow = p.row_of[static_cast<int64_t>(blockIdx.x) * K + tid];
         if (p.topk_weights) nw = p.topk_weights[static_cast<int64_t>(blockIdx.x) * K + tid];
-        if constexpr (kPeer) ne = p.topk_idx[static_cast<int64_t>(blockIdx.x) * K + tid];
+        if constexpr (kPeer)
+            if (!p.peer_by_slot) ne = p.topk_idx[static_cast<int64_t>(blockIdx.x) * K + tid];
     }
     int buf = 0;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x, buf ^= 1) {
@@ -68,14 +72,20 @@ __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
                 // rows past the owner's buffer (or with an id the handle does not
                 // match) are skipped
                 if (r >= 0) {
-                    const int ei = ne >= 0 && ne < p.num_experts ? static_cast<int>(ne) : -1;
-                    const int64_t pr = ei >= 0 ? static_cast<int64_t>(r) + p.peer_offset[ei] : -1;
+                    int at, part;
+                    if (p.peer_by_slot) {
+                        at = tid;
+                        part = tid;
+                    } else {
+                        at = ne >= 0 && ne < p.num_experts ? static_cast<int>(ne) : -1;
+                        part = at >= 0 ? at / p.experts_per_partition : 0;
+                    }
+                    const int64_t pr = at >= 0 ? static_cast<int64_t>(r) + p.peer_offset[at] : -1;
                     if (pr < 0 || pr >= p.expert_out_rows) {
                         raise_status(p.status, kDevIndexRange);
                         r = -1;
                     } else {
-                        src = static_cast<const uint4*>(p.peer_out[ei / p.experts_per_partition]) +
-                              pr * V;
+                        src = static_cast<const uint4*>(p.peer_out[part]) + pr * V;
                     }
                 }
             } else if (r >= 0 && static_cast<int64_t>(r) >= p.expert_out_rows) {
@@ -99,7 +109,8 @@ __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
                 if (tn < T) {
                     nrow = p.row_of[tn * K + tid];
                     if (p.topk_weights) nw = p.topk_weights[tn * K + tid];
-                    if constexpr (kPeer) ne = p.topk_idx[tn * K + tid];
+                    if constexpr (kPeer)
+                        if (!p.peer_by_slot) ne = p.topk_idx[tn * K + tid];
                 }
             }
         }
@@ -258,7 +269,8 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
     int threads = static_cast<int>((per_slice + 31) / 32 * 32);
     if (threads > kCombineMaxThreads) threads = kCombineMaxThreads;
     const void* kernel =
-        p.peer_out ? reinterpret_cast<const void*>(combine_kernel<8, true>)
+        p.peer_out ? (p.sparse ? reinterpret_cast<const void*>(combine_kernel<4, true>)
+                               : reinterpret_cast<const void*>(combine_kernel<8, true>))
         : p.sparse ? reinterpret_cast<const void*>(combine_kernel<4, false>)
                    : reinterpret_cast<const void*>(combine_kernel<8, false>);
     int per_sm = 0;
@@ -280,6 +292,7 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (p.peer_out && p.sparse) return cudaLaunchKernelEx(&cfg, combine_kernel<4, true>, p, per_slice);
     if (p.peer_out) return cudaLaunchKernelEx(&cfg, combine_kernel<8, true>, p, per_slice);
     if (p.sparse) return cudaLaunchKernelEx(&cfg, combine_kernel<4, false>, p, per_slice);
     return cudaLaunchKernelEx(&cfg, combine_kernel<8, false>, p, per_slice);

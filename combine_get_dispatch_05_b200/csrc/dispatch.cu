@@ -147,18 +147,26 @@ struct Dest {
 };
 
 // Peer mode (partitions are ranks): slot k's row goes to the rank that owns its
-// expert, at row_of[t, k] + peer_offset[e] there.  A row outside the owner's
-// buffers (the owner receives more rows than it has room for) is dropped and
-// reported.  Lane k < K holds both the row and the id of slot k.
-__device__ __forceinline__ int peer_dest(const DispatchParams& p, int row, int64_t e, Dest& d) {
+// expert, at row_of[t, k] + peer_offset[e] there (lane k < K holds both the row
+// and the id of slot k).  Deduplicated rows: lane q's row goes to rank q, at
+// row_of[t, q] + peer_offset[q].  A row outside the owner's buffers (the owner
+// receives more rows than it has room for) is dropped and reported.
+__device__ __forceinline__ int peer_dest(const DispatchParams& p, int lane, int row, int64_t e,
+                                         Dest& d) {
     if (row < 0) return -1;
-    if (e < 0 || e >= p.num_experts) {  // a handle that does not match topk_idx
-        raise_status(p.status, kDevIndexRange);
-        return -1;
+    int part, at;
+    if (p.dedup) {
+        part = lane;
+        at = lane;
+    } else {
+        if (e < 0 || e >= p.num_experts) {  // a handle that does not match topk_idx
+            raise_status(p.status, kDevIndexRange);
+            return -1;
+        }
+        at = static_cast<int>(e);
+        part = at / p.experts_per_partition;
     }
-    const int ei = static_cast<int>(e);
-    const int part = ei / p.experts_per_partition;
-    const int64_t r = static_cast<int64_t>(row) + p.peer_offset[ei];
+    const int64_t r = static_cast<int64_t>(row) + p.peer_offset[at];
     if (r < 0 || r >= p.peer_rows) {
         raise_status(p.status, kDevCapacity);
         return -1;
@@ -172,10 +180,11 @@ __device__ __forceinline__ int peer_dest(const DispatchParams& p, int row, int64
 
 // Metadata of one token's receive rows, written by the storer warp.  Per-expert
 // rows: lane k owns slot k and writes the local id and weight of its row into
-// ri / rw (its own buffers in peer mode).
+// ri / rw (its own destination's arrays in peer mode).
 // Deduplicated rows (one per partition): lane p owns partition p's row and writes
-// its K-entry lists, reading every slot's id and weight from the id lanes by
-// shuffle (all lanes take part in the shuffles).
+// its K-entry lists into ri / rw, reading every slot's id and weight from the id
+// lanes by shuffle (all lanes take part in the shuffles).
+template <bool kPeer>
 __device__ __forceinline__ void write_row_metadata(const DispatchParams& p, int lane, int row,
                                                    int64_t e, float wt, int32_t* ri, float* rw) {
     // lane k < K: partition and partition-local id of routing entry k, one 32-bit
@@ -198,8 +207,10 @@ __device__ __forceinline__ void write_row_metadata(const DispatchParams& p, int 
         const float wk = __shfl_sync(0xffffffffu, wt, k);
         if (lane < p.slots && row >= 0) {
             const bool in = pk == lane;
-            p.recv_topk_idx[static_cast<int64_t>(row) * p.K + k] = in ? lk : -1;
-            p.recv_topk_weights[static_cast<int64_t>(row) * p.K + k] = in ? wk : 0.0f;
+            int32_t* li = kPeer ? ri : p.recv_topk_idx;
+            float* lw = kPeer ? rw : p.recv_topk_weights;
+            li[static_cast<int64_t>(row) * p.K + k] = in ? lk : -1;
+            lw[static_cast<int64_t>(row) * p.K + k] = in ? wk : 0.0f;
         }
     }
 }
@@ -332,7 +343,7 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
             const int64_t e = cur.e;
             const float wt = cur.wt;
             Dest d{recv_x, p.recv_scales, p.recv_topk_idx, p.recv_topk_weights};
-            if constexpr (kPeer) row = peer_dest(p, row, e, d);
+            if constexpr (kPeer) row = peer_dest(p, lane, row, e, d);
             uint8_t* out_q = sm + L.off_out + o * L.out_bytes;
             const float* out_s = reinterpret_cast<const float*>(out_q + L.q_bytes);
             if (slot_lane) {
@@ -345,7 +356,7 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
                 bulk_commit();
                 rows_sm[o * 32 + lane] = row;
             }
-            write_row_metadata(p, lane, row, e, wt, d.i, d.w);
+            write_row_metadata<kPeer>(p, lane, row, e, wt, d.i, d.w);
             if constexpr (kPeer) {
                 if (!scale_bulk && slot_lane && row >= 0)  // row-major: the lane's own row
                     for (int b = 0; b < nb; ++b) d.s[static_cast<int64_t>(row) * nb + b] = out_s[b];
@@ -461,14 +472,14 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
             const int64_t e = cur.e;
             const float wt = cur.wt;
             Dest d{recv_x, nullptr, p.recv_topk_idx, p.recv_topk_weights};
-            if constexpr (kPeer) row = peer_dest(p, row, e, d);
+            if constexpr (kPeer) row = peer_dest(p, lane, row, e, d);
             if (slot_lane) {
                 if (row >= 0)
                     bulk_store(d.x + static_cast<int64_t>(row) * row_bytes, sm + s * row_bytes,
                                row_bytes);
                 bulk_commit();
             }
-            write_row_metadata(p, lane, row, e, wt, d.i, d.w);
+            write_row_metadata<kPeer>(p, lane, row, e, wt, d.i, d.w);
             if (slot_lane) bulk_wait_read<1>();  // the previous token's stores have read their stage
             __syncwarp();
             if (lane == 0 && i >= 1) mbar_arrive(&empty[(i - 1) % kBf16Stages]);

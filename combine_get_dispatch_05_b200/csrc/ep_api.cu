@@ -615,6 +615,119 @@ ep_status ep_peer_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk,
     return cuda_status(launch_combine(p, static_cast<cudaStream_t>(stream)));
 }
 
+ep_status ep_get_dispatch_layout_dedup(int64_t num_tokens, int32_t num_topk, int32_t num_experts,
+                                       int32_t num_partitions, const int64_t* topk_idx,
+                                       const ep_layout* layout, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+    ep_status st = check_routing(num_tokens, num_topk, num_experts, num_partitions);
+    if (st != EP_OK) return st;
+    if (num_partitions > 32) return EP_ERR_SHAPE;
+    if (num_tokens * static_cast<int64_t>(num_partitions) >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    if ((st = check_layout_ptrs(layout, num_tokens)) != EP_OK) return st;
+    if (!workspace || !aligned16(workspace) || (num_tokens > 0 && !topk_idx))
+        return EP_ERR_INVALID_ARG;
+    if (workspace_bytes < ep_workspace_bytes(num_tokens, num_experts, num_partitions))
+        return EP_ERR_WORKSPACE;
+    if ((st = check_layout_size(num_tokens, num_topk, num_experts, num_partitions, true)) != EP_OK)
+        return st;
+    const Workspace ws = carve_workspace(workspace, num_tokens, num_partitions);
+    return cuda_status(launch_layout(num_tokens, num_topk, num_experts, num_partitions, topk_idx,
+                                     *layout, ws, static_cast<cudaStream_t>(stream),
+                                     /*by_partition=*/true));
+}
+
+ep_status ep_peer_dispatch_dedup(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                 int32_t num_experts, int32_t world, int32_t quant, const void* x,
+                                 const int64_t* topk_idx, const float* topk_weights,
+                                 const ep_layout* handle, const int32_t* dst_offset,
+                                 const ep_peer_buffers* peers, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    if (quant != EP_QUANT_NONE && quant != EP_QUANT_FP8_E4M3_1X128 &&
+        quant != EP_QUANT_FP8_E4M3_1X128_POW2)
+        return EP_ERR_INVALID_ARG;
+    const bool fp8 = quant != EP_QUANT_NONE;
+    ep_status st = check_routing(num_tokens, num_topk, num_experts, world);
+    if (st != EP_OK) return st;
+    if (world > 32) return EP_ERR_SHAPE;  // one storer lane per rank
+    if ((st = check_hidden(hidden, fp8)) != EP_OK) return st;
+    if (!peers || peers->capacity < 0 || peers->capacity >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    if (!handle || !workspace || !aligned16(workspace) || workspace_bytes < kWsHeader)
+        return EP_ERR_INVALID_ARG;
+    if (num_tokens == 0) return EP_OK;
+    if (!handle->row_of || !x || !topk_idx || !topk_weights || !dst_offset || !peers->recv_x ||
+        !peers->recv_topk_idx || !peers->recv_topk_weights || (fp8 && !peers->recv_scales) ||
+        !aligned16(x))
+        return EP_ERR_INVALID_ARG;
+    const Workspace ws = carve_workspace(workspace, 0, 1);
+    DispatchParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = num_topk;
+    p.slots = world;
+    p.dedup = 1;
+    p.pow2_scales = quant == EP_QUANT_FP8_E4M3_1X128_POW2 ? 1 : 0;
+    p.scales_mn = 0;
+    p.scales_ld = 0;
+    p.num_experts = num_experts;
+    p.experts_per_partition = num_experts / world;
+    p.x = x;
+    p.topk_idx = topk_idx;
+    p.topk_weights = topk_weights;
+    p.row_of = handle->row_of;
+    p.recv_x = nullptr;
+    p.recv_scales = nullptr;
+    p.recv_topk_idx = nullptr;
+    p.recv_topk_weights = nullptr;
+    p.status = ws.status;
+    p.ticket = ws.ticket;
+    p.done = ws.done;
+    p.timeout_ns = kDefaultTimeoutNs;
+    p.peer_recv_x = peers->recv_x;
+    p.peer_recv_scales = fp8 ? peers->recv_scales : nullptr;
+    p.peer_recv_topk_idx = peers->recv_topk_idx;
+    p.peer_recv_topk_weights = peers->recv_topk_weights;
+    p.peer_offset = dst_offset;
+    p.peer_rows = peers->capacity;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return cuda_status(fp8 ? launch_dispatch_fp8(p, s) : launch_dispatch_bf16(p, s));
+}
+
+ep_status ep_peer_combine_dedup(int64_t num_tokens, int64_t hidden, int32_t world,
+                                const void* const* partition_out, int64_t capacity,
+                                const ep_layout* handle, const int32_t* dst_offset, void* y,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    if (num_tokens < 0 || world < 1 || world > 32 || capacity < 0 ||
+        capacity >= (int64_t(1) << 31))
+        return EP_ERR_SHAPE;
+    if (num_tokens * static_cast<int64_t>(world) >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    ep_status st = check_hidden(hidden, false);
+    if (st != EP_OK) return st;
+    if (!handle || !workspace || workspace_bytes < kWsHeader) return EP_ERR_INVALID_ARG;
+    if (num_tokens == 0) return EP_OK;
+    if (!handle->row_of || !partition_out || !dst_offset || !y || !aligned16(y))
+        return EP_ERR_INVALID_ARG;
+    CombineParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = world;  // slots are ranks
+    p.expert_out = nullptr;
+    p.expert_out_rows = capacity;
+    p.row_of = handle->row_of;
+    p.topk_weights = nullptr;  // partitions return weighted rows: a plain sum
+    p.y = y;
+    p.grad_recv_w = nullptr;
+    p.grad_w = nullptr;
+    p.status = carve_workspace(workspace, 0, 1).status;
+    p.sparse = 1;
+    p.peer_out = partition_out;
+    p.topk_idx = nullptr;
+    p.peer_offset = dst_offset;
+    p.experts_per_partition = 1;
+    p.num_experts = world;
+    p.peer_by_slot = 1;
+    return cuda_status(launch_combine(p, static_cast<cudaStream_t>(stream)));
+}
+
 ep_status ep_debug_wait_probe(uint64_t timeout_ns, void* workspace, size_t workspace_bytes,
                               void* stream) {
     if (!workspace || workspace_bytes < kWsHeader) return EP_ERR_INVALID_ARG;

@@ -71,9 +71,10 @@ struct DispatchParams {
     int32_t* ticket;  // token counter (zero on entry; the last CTA to finish re-zeroes it)
     uint32_t* done;
     uint64_t timeout_ns;
-    // Peer mode (partitions are ranks; per-expert rows only): the row of (t, k) is
-    // row_of[t, k] + peer_offset[e] in the buffers of rank e / experts_per_partition,
-    // whose base pointers the tables hold; recv_x .. recv_topk_weights are unused.
+    // Peer mode (partitions are ranks): the row of (t, k) is row_of[t, k] +
+    // peer_offset[e] in the buffers of rank e / experts_per_partition (deduplicated
+    // rows: the row of (t, q) is row_of[t, q] + peer_offset[q] in rank q's), whose
+    // base pointers the tables hold; recv_x .. recv_topk_weights are unused.
     void* const* peer_recv_x = nullptr;
     float* const* peer_recv_scales = nullptr;
     int32_t* const* peer_recv_topk_idx = nullptr;
@@ -106,6 +107,7 @@ struct CombineParams {
     const int32_t* peer_offset = nullptr;
     int32_t experts_per_partition = 1;
     int32_t num_experts = 0;
+    int32_t peer_by_slot = 0;  // deduplicated rows: slot k is rank k (topk_idx unused)
 };
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 

@@ -24,6 +24,13 @@ and maps every other rank's.  Per step:
   and k: partition r's rows of the one-GPU dispatch of all ranks' tokens
   concatenated in rank order.
 
+  ``dispatch(..., dedup=True)`` sends each token once to each rank that holds any of
+  its experts (DeepEP's normal-kernel semantics; under group-limited routing about
+  half the rows of the per-expert form cross NVLink): rows by source rank, then
+  token, each with [K] local-id / weight lists (-1 / 0 for experts elsewhere); the
+  caller writes one BF16 row per received row (its experts' weighted sum) into
+  ``expert_out_buffer`` and combine sums the ranks' rows per token.
+
 ``transport="nccl"`` (any backend): the one-GPU dispatch with P = W fills a send
 buffer whose rank-p rows are one contiguous slice; the rows, scales, local ids and
 weights go to their owners with ``all_to_all_single`` (through host memory when the
@@ -63,6 +70,7 @@ class EpContext:
     dst_offset: Optional[torch.Tensor] = None
     recv_rows: int = 0
     order: str = field(default="source_major")
+    dedup: bool = False
 
 
 class EpGroup:
@@ -72,12 +80,14 @@ class EpGroup:
     kernels store to and load from the other GPUs' buffers; needs ``hidden``).
     capacity: rows of each rank's receive buffers in peer mode (default
     max_tokens * W * 8, every token of every rank routed here with top-8).
+    num_topk: the largest K the peer buffers' id / weight lists hold (dedup rows).
     Call :meth:`close` before destroying the process group.
     """
 
     def __init__(self, num_experts: int, group=None, max_tokens: int = 4096,
                  device: Optional[torch.device] = None, *, transport: str = "nccl",
-                 hidden: Optional[int] = None, capacity: Optional[int] = None):
+                 hidden: Optional[int] = None, capacity: Optional[int] = None,
+                 num_topk: int = 8):
         self.group = group if group is not None else dist.group.WORLD
         self.world = dist.get_world_size(self.group)
         self.rank = dist.get_rank(self.group)
@@ -98,7 +108,8 @@ class EpGroup:
             if hidden is None:
                 raise ValueError("the peer transport needs `hidden` to size the receive buffers")
             self._open_peers(int(hidden), int(capacity if capacity is not None
-                                                  else max_tokens * self.world * 8))
+                                                  else max_tokens * self.world * 8),
+                             int(num_topk))
 
     def _new_workspace(self, tokens: int) -> torch.Tensor:
         ws = torch.empty(_lib.ep_workspace_bytes(max(tokens, 1), self.num_experts, self.world),
@@ -107,13 +118,14 @@ class EpGroup:
         return ws
 
     # ---------------------------------------------------------- peer buffers --
-    def _open_peers(self, hidden: int, capacity: int) -> None:
+    def _open_peers(self, hidden: int, capacity: int, topk: int) -> None:
         """One IPC region per rank: recv_x (room for BF16 rows) | recv_scales |
-        recv_topk_idx | recv_topk_weights | expert_out, each 256-byte aligned."""
+        recv_topk_idx | recv_topk_weights (room for [K] lists) | expert_out, each
+        256-byte aligned."""
         if hidden % 128:
             raise ValueError("hidden must be a multiple of 128")
         sizes = [("recv_x", capacity * hidden * 2), ("recv_scales", capacity * (hidden // 128) * 4),
-                 ("recv_topk_idx", capacity * 4), ("recv_topk_weights", capacity * 4),
+                 ("recv_topk_idx", capacity * topk * 4), ("recv_topk_weights", capacity * topk * 4),
                  ("expert_out", capacity * hidden * 2)]
         offsets, total = {}, 0
         for name, n in sizes:
@@ -136,7 +148,7 @@ class EpGroup:
                 _lib.ep_ipc_close(ptr)
             _lib.ep_ipc_free(base)
             raise
-        self._peer = dict(base=base, opened=opened, hidden=hidden, capacity=capacity,
+        self._peer = dict(base=base, opened=opened, hidden=hidden, capacity=capacity, topk=topk,
                           region=_lib.device_bytes(base, max(total, _ALIGN), self.device),
                           offsets=offsets, sizes=dict(sizes))
         self.tables = _lib.PeerTables.from_addresses(
@@ -145,8 +157,12 @@ class EpGroup:
 
     def _view(self, name: str, dtype, shape) -> torch.Tensor:
         pr = self._peer
-        n = pr["sizes"][name]
-        return pr["region"][pr["offsets"][name]:pr["offsets"][name] + n].view(dtype).view(*shape)
+        n = 1
+        for d in shape:
+            n *= d
+        n *= torch.empty(0, dtype=dtype).element_size()
+        o = pr["offsets"][name]
+        return pr["region"][o:o + n].view(dtype).view(*shape)
 
     def expert_out_buffer(self, ctx: EpContext) -> torch.Tensor:
         """Peer transport: the BF16 [recv rows, H] buffer the expert outputs go into
@@ -214,7 +230,7 @@ class EpGroup:
 
     # --------------------------------------------------------------- dispatch --
     def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
-                 use_fp8: bool = True):
+                 use_fp8: bool = True, dedup: bool = False):
         """Returns ``(recv_x, recv_local_idx, recv_weights, recv_counts_per_expert, ctx)``.
 
         recv_x: ``(float8_e4m3fn [Rr, H], float32 [Rr, H/128])`` or BF16 ``[Rr, H]``;
@@ -222,11 +238,18 @@ class EpGroup:
         recv_weights: float32 [Rr]; recv_counts_per_expert: int32 [W, E/W] rows
         received from each source rank for each local expert.  Row order: see the
         module docstring (``ctx.order``).
+
+        dedup (peer transport): one row per (token, rank); recv_local_idx and
+        recv_weights are [Rr, K] lists and the counts are [W, 1] rows per source.
         """
         T = x.shape[0]
         if T > self.max_tokens:
             self.max_tokens = T
             self.workspace = self._new_workspace(T)
+        if dedup:
+            if self.transport != "peer":
+                raise NotImplementedError("deduplicated rows are offered by the peer transport")
+            return self._dispatch_peer_dedup(x, topk_idx, topk_weights, use_fp8)
         if self.transport == "peer":
             return self._dispatch_peer(x, topk_idx, topk_weights, use_fp8)
         return self._dispatch_nccl(x, topk_idx, topk_weights, use_fp8)
@@ -297,12 +320,54 @@ class EpGroup:
         ri = self._view("recv_topk_idx", torch.int32, (cap,))[:Rr]
         rw = self._view("recv_topk_weights", torch.float32, (cap,))[:Rr]
         if use_fp8:
-            q = self._view("recv_x", torch.uint8, (-1,))[:cap * H].view(cap, H)[:Rr]
+            q = self._view("recv_x", torch.uint8, (cap, H))[:Rr]
             s = self._view("recv_scales", torch.float32, (cap, H // 128))[:Rr]
             recv_x = (q.view(torch.float8_e4m3fn), s)
         else:
             recv_x = self._view("recv_x", torch.bfloat16, (cap, H))[:Rr]
         return recv_x, ri, rw, per_expert, ctx
+
+    def _dispatch_peer_dedup(self, x, topk_idx, topk_weights, use_fp8):
+        T, H = x.shape
+        K = topk_idx.shape[1]
+        W, E, r = self.world, self.num_experts, self.rank
+        pr = self._peer
+        if H != pr["hidden"]:
+            raise ValueError(f"hidden {H} differs from the receive buffers' {pr['hidden']}")
+        if K > pr["topk"]:
+            raise ValueError(f"top-k {K} exceeds the buffers' lists of {pr['topk']}")
+        if W > 32:
+            raise ValueError("deduplicated rows support at most 32 ranks")
+        cap, dev = pr["capacity"], self.device
+        lay = Layout.empty(T, W, W, W, dev)  # partition-sized handle
+        _lib.ep_get_dispatch_layout_dedup(topk_idx, E, W, lay, self.workspace)
+        counts = self._all_gather_rows(lay.num_tokens_per_expert)  # [W sources, W owners]
+        totals = counts.sum(dim=0).to("cpu").tolist()
+        if max(totals) > cap:
+            raise ValueError(f"a rank would receive {max(totals)} rows; capacity is {cap}")
+        dst = torch.empty(W, dtype=torch.int32, device=dev)
+        rc = torch.empty(1, dtype=torch.int32, device=dev)
+        ro = torch.empty(2, dtype=torch.int32, device=dev)
+        _lib.ep_peer_plan(counts, r, lay.expert_offset, cap, dst, rc, ro, self.workspace)
+        quant = EP_QUANT_FP8_E4M3_1X128 if use_fp8 else EP_QUANT_NONE
+        _lib.ep_peer_dispatch_dedup(x, topk_idx, topk_weights, E, W, quant, lay, dst, self.tables,
+                                    self.workspace)
+        self._barrier()  # every rank's rows have landed in their owners' buffers
+        Rr = int(totals[r])
+        per_source = counts[:, r:r + 1]
+        send = counts[r].to("cpu").tolist()
+        recv = per_source.reshape(-1).to("cpu").tolist()
+        ctx = EpContext(lay, send, recv, T, H, dst_offset=dst, recv_rows=Rr, order="source_major",
+                        dedup=True)
+        ri = self._view("recv_topk_idx", torch.int32, (cap, K))[:Rr]
+        rw = self._view("recv_topk_weights", torch.float32, (cap, K))[:Rr]
+        if use_fp8:
+            q = self._view("recv_x", torch.uint8, (cap, H))[:Rr]
+            s = self._view("recv_scales", torch.float32, (cap, H // 128))[:Rr]
+            recv_x = (q.view(torch.float8_e4m3fn), s)
+        else:
+            recv_x = self._view("recv_x", torch.bfloat16, (cap, H))[:Rr]
+        return recv_x, ri, rw, per_source, ctx
 
     # ---------------------------------------------------------------- combine --
     def combine(self, expert_out: torch.Tensor, ctx: EpContext,
@@ -315,8 +380,13 @@ class EpGroup:
             if ctx.recv_rows and expert_out.data_ptr() != self.expert_out_buffer(ctx).data_ptr():
                 raise ValueError("write the expert outputs into expert_out_buffer(ctx)")
             self._barrier()  # every rank's expert outputs are complete
-            _lib.ep_peer_combine(self.tables, ctx.handle, ctx.topk_idx, ctx.dst_offset,
-                                 topk_weights, y, self.num_experts, self.world, self.workspace)
+            if ctx.dedup:  # partition outputs are already weighted: a plain sum
+                _lib.ep_peer_combine_dedup(self.tables, ctx.handle, ctx.dst_offset, y, self.world,
+                                           self.workspace)
+            else:
+                _lib.ep_peer_combine(self.tables, ctx.handle, ctx.topk_idx, ctx.dst_offset,
+                                     topk_weights, y, self.num_experts, self.world,
+                                     self.workspace)
             return y
         Rs = sum(ctx.send_counts)
         back = self._a2a(expert_out, Rs, ctx.send_counts, ctx.recv_counts)

@@ -488,6 +488,55 @@ EP_API ep_status ep_peer_combine(int64_t num_tokens, int64_t hidden, int32_t num
                                  const int32_t* dst_offset, const float* topk_weights, void* y,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- deduplicated rows across GPUs -------------------------------------------
+ * DeepEP's normal kernels send a token once to each rank that holds any of its
+ * experts ("deepseek.csdn.net/67bd3eb22e30c863900615cc", "使用示例": recv_topk_idx /
+ * recv_topk_weights list each received token's local experts; "DeepSeek 开源周第二弹：
+ * DeepEP", "DeepEP 的常规内核和低延迟内核": top-4 groups of top-8 experts), which under
+ * group-limited routing roughly halves the rows that cross NVLink.  The peer form of
+ * ep_dispatch_dedup / ep_combine_dedup, with W = number of ranks = partitions:
+ *   1. ep_get_dispatch_layout_dedup (partition-sized handle);
+ *   2. the caller gathers every rank's handle.num_tokens_per_expert[W] (rows per
+ *      rank) into counts[W, W];
+ *   3. ep_peer_plan(world = W, num_experts = W, counts, handle.expert_offset, ...):
+ *      dst_offset[W], this rank's recv_count[1] and recv_offset[2];
+ *   5. ep_peer_dispatch_dedup; 6. barrier, each rank computes its partition outputs
+ *      (one BF16 row per received row: the weighted sum over its listed experts);
+ *   7. barrier, ep_peer_combine_dedup.
+ * Rank q receives its rows source rank first, then token ascending: partition q's
+ * rows of the one-GPU ep_dispatch_dedup of all ranks' tokens concatenated in rank
+ * order.  recv_topk_idx / recv_topk_weights tables point to [capacity, K] arrays. */
+
+/* The deduplicated layout of ep_dispatch_dedup on its own (partition-sized handle:
+ * num_tokens_per_expert[P] = rows per partition, expert_offset[P+1], row_of[T, P],
+ * src_of[T*min(P, K)] = token of each row).  1 <= P <= 32. */
+EP_API ep_status ep_get_dispatch_layout_dedup(int64_t num_tokens, int32_t num_topk,
+                                              int32_t num_experts, int32_t num_partitions,
+                                              const int64_t* topk_idx, const ep_layout* layout,
+                                              void* workspace, size_t workspace_bytes,
+                                              void* stream);
+
+/* Step 5: ep_dispatch_dedup's rows (payload, scales, [K] local-id and weight lists)
+ * written to row row_of[t, q] + dst_offset[q] of rank q's buffers.  handle: from
+ * ep_get_dispatch_layout_dedup with W partitions; quant as for ep_peer_dispatch.
+ * 1 <= W <= 32.  The workspace needs only its 256-byte header. */
+EP_API ep_status ep_peer_dispatch_dedup(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                        int32_t num_experts, int32_t world, int32_t quant,
+                                        const void* x, const int64_t* topk_idx,
+                                        const float* topk_weights, const ep_layout* handle,
+                                        const int32_t* dst_offset, const ep_peer_buffers* peers,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Step 7: y[t, i] = bf16_rne(sum over q = 0..W-1 with row_of[t, q] >= 0, in q order, of
+ * float(partition_out[q][row_of[t, q] + dst_offset[q], i])) (fp32 adds from +0.0f).
+ * partition_out: device table of W pointers to BF16 [capacity, H]; a row outside
+ * [0, capacity) is skipped and sets EP_DEV_INDEX_RANGE. */
+EP_API ep_status ep_peer_combine_dedup(int64_t num_tokens, int64_t hidden, int32_t world,
+                                       const void* const* partition_out, int64_t capacity,
+                                       const ep_layout* handle, const int32_t* dst_offset,
+                                       void* y, void* workspace, size_t workspace_bytes,
+                                       void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -209,9 +209,54 @@ def _peer_stand_ins(oracle, torch):
         yb, _ = oracle.combine(rows, row_of, w.numpy())
         y.copy_(torch.from_numpy(yb.view(np.int16)).view(torch.bfloat16))
 
+    def layout_dedup(idx, E, P, lay, ws, stream=None):
+        ids = idx.numpy()
+        d = oracle.dispatch_dedup(np.zeros((ids.shape[0], 128), np.uint16), ids,
+                                  np.zeros(ids.shape, np.float32), E, P, quant="none")
+        lay.num_tokens_per_expert.copy_(torch.from_numpy(d["part_count"]))
+        lay.num_tokens_per_partition.copy_(torch.from_numpy(d["part_count"]))
+        lay.expert_offset.copy_(torch.from_numpy(d["part_offset"]))
+        lay.row_of.copy_(torch.from_numpy(d["prow_of"]))
+        lay.is_token_in_partition.copy_(torch.from_numpy((d["prow_of"] >= 0).astype(np.uint8)))
+        lay.src_of[:len(d["src_tok"])] = torch.from_numpy(d["src_tok"])
+        lay.num_recv.fill_(int(d["num_rows"][0]))
+
+    def dispatch_dedup(x, idx, w, E, W, quant, lay, dst, tables, ws, stream=None):
+        xs = x.view(torch.int16).numpy().view(np.uint16)
+        H = xs.shape[1]
+        d = oracle.dispatch_dedup(xs, idx.numpy(), w.numpy(), E, W, quant="fp8" if quant else "none")
+        off, po = dst.numpy(), d["part_offset"]
+        for q in range(W):
+            for r in range(int(po[q]), int(po[q + 1])):
+                row = r + int(off[q])
+                rx = d["recv_x"][r]
+                put(tables.recv_x[q] + row * rx.nbytes, rx)
+                if quant:
+                    put(tables.recv_scales[q] + row * (H // 128) * 4, d["recv_scales"][r])
+                put(tables.recv_topk_idx[q] + row * d["recv_topk_idx"][r].nbytes,
+                    d["recv_topk_idx"][r])
+                put(tables.recv_topk_weights[q] + row * d["recv_topk_weights"][r].nbytes,
+                    d["recv_topk_weights"][r])
+
+    def combine_dedup(tables, lay, dst, y, W, ws, stream=None):
+        pr, off = lay.row_of.numpy(), dst.numpy()
+        T, H = y.shape
+        rows = np.zeros((max(T * W, 1), H), np.uint16)
+        prow = np.full((T, W), -1, np.int32)
+        for t in range(T):
+            for q in range(W):
+                if pr[t, q] >= 0:
+                    a = tables.expert_out[q] + (int(pr[t, q]) + int(off[q])) * H * 2
+                    rows[t * W + q] = get(a, H * 2).view(np.uint16)
+                    prow[t, q] = t * W + q
+        yb, _ = oracle.combine_dedup(rows, prow)
+        y.copy_(torch.from_numpy(yb.view(np.int16)).view(torch.bfloat16))
+
     return dict(ep_ipc_alloc=ipc_alloc, ep_ipc_open=ipc_open, ep_ipc_close=ipc_close,
                 ep_ipc_free=ipc_free, device_bytes=device_bytes, ep_get_dispatch_layout=layout,
                 ep_peer_plan=plan, ep_peer_dispatch=dispatch, ep_peer_combine=combine,
+                ep_get_dispatch_layout_dedup=layout_dedup, ep_peer_dispatch_dedup=dispatch_dedup,
+                ep_peer_combine_dedup=combine_dedup,
                 ep_workspace_init=lambda ws, stream=None: None)
 
 
@@ -276,6 +321,32 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
             y_all, _ = oracle.combine(eo_all, d["row_of"], w_all)
             assert np.array_equal(y.view(torch.int16).numpy().view(np.uint16),
                                   y_all[t0:t0 + tokens[rank]]), quant
+        for quant in ("fp8", "none"):  # one row per (token, rank)
+            recv_x, ri, rw, per_source, ctx = g.dispatch(x, idx, wts, use_fp8=quant == "fp8",
+                                                         dedup=True)
+            d = oracle.dispatch_dedup(x_all, idx_all, w_all, E, world, quant=quant)
+            lo, hi = d["part_offset"][rank], d["part_offset"][rank + 1]
+            if quant == "fp8":
+                got = recv_x[0].view(torch.uint8).numpy()
+                assert np.array_equal(recv_x[1].numpy().view(np.uint32),
+                                      d["recv_scales"][lo:hi].view(np.uint32))
+            else:
+                got = recv_x.view(torch.int16).numpy().view(np.uint16)
+            assert np.array_equal(got, d["recv_x"][lo:hi]), quant
+            assert np.array_equal(ri.numpy(), d["recv_topk_idx"][lo:hi]), quant
+            assert np.array_equal(rw.numpy().view(np.uint32),
+                                  d["recv_topk_weights"][lo:hi].view(np.uint32)), quant
+            want = [int(oracle.dispatch_dedup(l.x, l.topk_idx, l.topk_weights, E, world,
+                                              quant=quant)["part_count"][rank]) for l in loads]
+            assert per_source.reshape(-1).tolist() == want and ctx.recv_counts == want
+            po_all = oracle.partition_identity(d["recv_x"], d["recv_scales"], d["recv_topk_idx"],
+                                               d["recv_topk_weights"], quant=quant)
+            buf = g.expert_out_buffer(ctx)
+            buf.copy_(torch.from_numpy(po_all[lo:hi].view(np.int16)).view(torch.bfloat16))
+            y = g.combine(buf, ctx, wts)
+            y_all, _ = oracle.combine_dedup(po_all, d["prow_of"])
+            assert np.array_equal(y.view(torch.int16).numpy().view(np.uint16),
+                                  y_all[t0:t0 + tokens[rank]]), "dedup " + quant
         status = "ok"
     finally:
         try:

@@ -141,6 +141,28 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
             y = g.combine(out, ctx, wts)
             y_ref, _ = oracle.combine(eo, d["row_of"], w.topk_weights)
             assert np.array_equal(bf16_to_u16(y), y_ref), quant
+        for quant in ("fp8", "none"):  # one row per (token, rank), [K] expert lists
+            recv_x, ri, rw, per_source, ctx = g.dispatch(x, idx, wts, use_fp8=quant == "fp8",
+                                                         dedup=True)
+            d = oracle.dispatch_dedup(w.x, w.topk_idx, w.topk_weights, E, world, quant=quant)
+            R = int(d["num_rows"][0])
+            assert ctx.recv_rows == R and per_source.reshape(-1).tolist() == [R]
+            if quant == "fp8":
+                assert np.array_equal(recv_x[0].view(torch.uint8).cpu().numpy(), d["recv_x"])
+                assert np.array_equal(recv_x[1].cpu().numpy().view(np.uint32),
+                                      d["recv_scales"].view(np.uint32))
+            else:
+                assert np.array_equal(bf16_to_u16(recv_x), d["recv_x"])
+            assert np.array_equal(ri.cpu().numpy(), d["recv_topk_idx"])
+            assert np.array_equal(rw.cpu().numpy().view(np.uint32),
+                                  d["recv_topk_weights"].view(np.uint32))
+            po = oracle.partition_identity(d["recv_x"], d["recv_scales"], d["recv_topk_idx"],
+                                           d["recv_topk_weights"], quant=quant)
+            out = g.expert_out_buffer(ctx)
+            out.copy_(dev_u16_as_bf16(po))
+            y = g.combine(out, ctx, wts)
+            y_ref, _ = oracle.combine_dedup(po, d["prow_of"])
+            assert np.array_equal(bf16_to_u16(y), y_ref), "dedup " + quant
         assert ep.ep_read_status(g.workspace) == 0
         status = "ok"
     finally:

@@ -282,3 +282,33 @@ def test_peer_host_checks(ep):
     assert L.ep_ipc_open(None, ctypes.byref(ptr)) == 1
     assert L.ep_ipc_open(handle, None) == 1
     assert L.ep_ipc_close(None) == 1
+
+
+def test_peer_dedup_host_checks(ep):
+    f = _Fake.P
+    lay = _layout_struct(ep)
+    L = ep.lib
+    lo = L.ep_get_dispatch_layout_dedup
+    assert lo(4, 2, 64, 33, f, ctypes.byref(lay), f, 1 << 20, None) == 2   # P > 32
+    assert lo(4, 2, 60, 8, f, ctypes.byref(lay), f, 1 << 20, None) == 2    # E % P
+    assert lo(4, 2, 64, 8, None, ctypes.byref(lay), f, 1 << 20, None) == 1
+    assert lo(4, 2, 64, 8, f, ctypes.byref(lay), f, 16, None) == 3          # workspace
+    peers = ep._lib.ep_peer_buffers(f, f, f, f, 64)
+
+    def disp(T=16, H=256, K=4, E=64, W=8, quant=1, pb=peers):
+        return L.ep_peer_dispatch_dedup(T, H, K, E, W, quant, f, f, f, ctypes.byref(lay), f,
+                                        ctypes.byref(pb) if pb is not None else None, f, 4096,
+                                        None)
+
+    assert disp(W=64, E=128) == 2       # one storer lane per rank: W <= 32
+    assert disp(quant=0x101) == 1
+    assert disp(H=136) == 2
+    assert disp(pb=None) == 2
+    assert disp(pb=ep._lib.ep_peer_buffers(f, None, f, f, 64)) == 1
+    assert disp(T=0) == 0
+    comb = L.ep_peer_combine_dedup
+    assert comb(4, 128, 33, f, 64, ctypes.byref(lay), f, f, f, 4096, None) == 2
+    assert comb(4, 100, 8, f, 64, ctypes.byref(lay), f, f, f, 4096, None) == 2
+    assert comb(4, 128, 8, None, 64, ctypes.byref(lay), f, f, f, 4096, None) == 1
+    assert comb(4, 128, 8, f, 64, ctypes.byref(lay), None, f, f, 4096, None) == 1
+    assert comb(0, 128, 8, None, 64, ctypes.byref(lay), None, None, f, 4096, None) == 0

@@ -189,3 +189,121 @@ def test_peer_capacity_overflow_drops_one_rank(ep):
     rows1 = int(d["expert_offset"][8] - d["expert_offset"][4])
     assert rows0 > rows1
     _check(ep, loads, 8, 2, "fp8", capacity=rows1, drop=(0,))
+
+
+# ------------------------------------------------------- deduplicated rows --
+
+def _check_dedup(ep, loads, E, W, quant, capacity=None, drop=()):
+    H, K = loads[0].hidden, loads[0].num_topk
+    fp8 = quant != "none"
+    x, idx, wts = _concat(loads)
+    d = oracle.dispatch_dedup(x, idx, wts, E, W, quant=quant)
+    off = d["part_offset"]
+    part_rows = [int(off[q + 1] - off[q]) for q in range(W)]
+    cap = capacity if capacity is not None else max(max(part_rows), 1) + 5
+    bufs = [dict(x=Guarded((cap, H), torch.uint8 if fp8 else torch.bfloat16),
+                 s=Guarded((cap, H // 128), torch.float32) if fp8 else None,
+                 i=Guarded((cap, K), torch.int32), w=Guarded((cap, K), torch.float32),
+                 eo=Guarded((cap, H), torch.bfloat16)) for _ in range(W)]
+    tables = ep.PeerTables.from_addresses(
+        "cuda", cap, [b["x"].t.data_ptr() for b in bufs],
+        [b["s"].t.data_ptr() if fp8 else 0 for b in bufs],
+        [b["i"].t.data_ptr() for b in bufs], [b["w"].t.data_ptr() for b in bufs],
+        [b["eo"].t.data_ptr() for b in bufs])
+    ranks = []
+    for w in loads:
+        T = w.num_tokens
+        r = dict(x=dev_u16_as_bf16(w.x), idx=torch.from_numpy(w.topk_idx).cuda(),
+                 wts=torch.from_numpy(w.topk_weights).cuda(),
+                 lay=ep.Layout.empty(T, W, W, W, "cuda"), ws=new_workspace(ep, T, E, W),
+                 dst=torch.empty(W, dtype=torch.int32, device="cuda"),
+                 rc=torch.empty(1, dtype=torch.int32, device="cuda"),
+                 ro=torch.empty(2, dtype=torch.int32, device="cuda"))
+        ep.ep_get_dispatch_layout_dedup(r["idx"], E, W, r["lay"], r["ws"])
+        ranks.append(r)
+    counts = torch.stack([r["lay"].num_tokens_per_expert for r in ranks]).contiguous()
+    for s, r in enumerate(ranks):
+        ep.ep_peer_plan(counts, s, r["lay"].expert_offset, cap, r["dst"], r["rc"], r["ro"], r["ws"])
+    for r in ranks:
+        ep.ep_peer_dispatch_dedup(r["x"], r["idx"], r["wts"], E, W, quant_code(ep, quant),
+                                  r["lay"], r["dst"], tables, r["ws"])
+    torch.cuda.synchronize()
+    status = [ep.ep_read_status(r["ws"]) for r in ranks]
+    if drop:
+        assert all(st & ep.EP_DEV_CAPACITY for st in status), status
+    else:
+        assert status == [0] * W, status
+
+    row_bytes = H * (1 if fp8 else 2)
+    for q in range(W):
+        lo, n = int(off[q]), part_rows[q]
+        b = bufs[q]
+        if q in drop:
+            assert bool((b["x"].raw == CANARY).all().item()), f"rank {q} was written"
+            n = 0
+        else:
+            if fp8:
+                assert np.array_equal(b["x"].t[:n].cpu().numpy(), d["recv_x"][lo:lo + n]), q
+                assert np.array_equal(b["s"].t[:n].cpu().numpy().view(np.uint32),
+                                      d["recv_scales"][lo:lo + n].view(np.uint32)), q
+            else:
+                assert np.array_equal(bf16_to_u16(b["x"].t[:n]), d["recv_x"][lo:lo + n]), q
+            assert np.array_equal(b["i"].t[:n].cpu().numpy(), d["recv_topk_idx"][lo:lo + n]), q
+            assert np.array_equal(b["w"].t[:n].cpu().numpy().view(np.uint32),
+                                  d["recv_topk_weights"][lo:lo + n].view(np.uint32)), q
+            assert int(ranks[q]["rc"].item()) == n
+            assert ranks[q]["ro"].cpu().tolist() == [0, n]
+        assert bool((b["x"].raw[n * row_bytes:] == CANARY).all().item()), q
+        assert all(g.canary_ok() for g in (b["x"], b["i"], b["w"]) + ((b["s"],) if fp8 else ()))
+
+    # partition outputs (each received row reduced over its listed experts), then combine
+    po_all = oracle.partition_identity(d["recv_x"], d["recv_scales"], d["recv_topk_idx"],
+                                       d["recv_topk_weights"], quant="none" if not fp8 else "fp8")
+    for q in range(W):
+        lo, n = int(off[q]), part_rows[q]
+        if q not in drop and n:
+            bufs[q]["eo"].t[:n].copy_(dev_u16_as_bf16(po_all[lo:lo + n]))
+    torch.cuda.synchronize()
+    prow = d["prow_of"].copy()
+    for q in drop:
+        prow[:, q] = -1
+    y_all, _ = oracle.combine_dedup(po_all, prow)
+    t0 = 0
+    for s, (w, r) in enumerate(zip(loads, ranks)):
+        T = w.num_tokens
+        y = Guarded((T, H), torch.bfloat16)
+        ep.ep_peer_combine_dedup(tables, r["lay"], r["dst"], y.t, W, r["ws"])
+        torch.cuda.synchronize()
+        assert np.array_equal(bf16_to_u16(y.t), y_all[t0:t0 + T]), s
+        assert y.canary_ok()
+        st = ep.ep_read_status(r["ws"])
+        dropped_here = bool(drop) and bool((d["prow_of"][t0:t0 + T][:, list(drop)] >= 0).any())
+        assert bool(st & ep.EP_DEV_INDEX_RANGE) == dropped_here, (s, st)
+        t0 += T
+
+
+@pytest.mark.parametrize("quant", ["fp8", "none"])
+def test_peer_dedup_two_ranks_ragged(ep, quant):
+    loads = [make_custom(T, 256, 6, 16, 2, seed=90 + s, mask_frac=0.05)
+             for s, T in enumerate([241, 130])]
+    _check_dedup(ep, loads, 16, 2, quant)
+
+
+def test_peer_dedup_four_ranks_empty_rank_pow2(ep):
+    loads = [make_custom(T, 512, 8, 32, 4, seed=95 + s, duplicates=True)
+             for s, T in enumerate([77, 0, 190, 33])]
+    _check_dedup(ep, loads, 32, 4, "fp8_pow2")
+
+
+def test_peer_dedup_eight_ranks_normal_routing(ep):
+    loads = [make_workload("normal", seed=110 + s, num_tokens=512) for s in range(8)]
+    _check_dedup(ep, loads, 256, 8, "fp8")
+
+
+def test_peer_dedup_capacity_overflow_drops_one_rank(ep):
+    loads = [make_custom(T, 512, 2, 8, 2, seed=120 + s, hot_expert=1) for s, T in enumerate([90, 70])]
+    x, idx, wts = _concat(loads)
+    d = oracle.dispatch_dedup(x, idx, wts, 8, 2, quant="fp8")
+    rows1 = int(d["part_offset"][2] - d["part_offset"][1])
+    assert int(d["part_offset"][1]) > rows1
+    _check_dedup(ep, loads, 8, 2, "fp8", capacity=rows1, drop=(0,))
