@@ -16,7 +16,9 @@
 // source rows are contiguous 14 KB rows (hidden 7168), so every warp reads whole
 // 512-byte runs: the reads are coalesced and the traffic is the algorithmic
 // minimum (K rows read once, one row written).  The rows and weights of the
-// next token are prefetched while the current one is reduced.
+// next token are prefetched while the current one is reduced.  In peer mode
+// (partitions are the ranks of a node) the rows are read from the owner ranks'
+// IPC-mapped expert outputs; the arithmetic and its order are the same.
 #include "ep_device.cuh"
 #include "ep_internal.h"
 

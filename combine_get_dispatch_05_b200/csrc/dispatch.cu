@@ -20,6 +20,11 @@
 // traffic is the algorithmic minimum.  The x loads of the first stages are
 // issued before waiting on the layout kernels (x is an input of the call), so
 // they overlap the layout.
+//
+// Peer mode (template parameter kPeer; partitions are the ranks of a node): the
+// storer lane of each row resolves the owner rank and the row there (peer_dest)
+// and its bulk stores go to that rank's IPC-mapped receive buffer; everything
+// else is the one-GPU pipeline.
 #include "ep_device.cuh"
 #include "ep_internal.h"
 #include "ep_quant.cuh"

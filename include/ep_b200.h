@@ -31,7 +31,10 @@
  * On one GPU the EP "ranks" are logical partitions of one HBM buffer:
  * partition p owns experts [p*E/P, (p+1)*E/P) and, because the receive buffer
  * is expert-major, one contiguous slice of rows.  The exchange is a
- * device-local permutation; there is no inter-GPU traffic.
+ * device-local permutation; there is no inter-GPU traffic.  Across the GPUs of
+ * a node (partitions = ranks, one process per GPU) the ep_peer_* calls at the
+ * end of this header store the rows straight into the owner ranks' receive
+ * buffers and read the expert outputs back from them (CUDA IPC mappings).
  *
  * Conventions (every entry point):
  *   - Pointers named as device memory must be device (or managed) memory of
