@@ -379,6 +379,41 @@ def time_low_latency(ep, w, dev, reps=200, per_graph=20):
     if ep.ep_read_status(ws) != 0:
         raise RuntimeError("device status set in the low-latency run")
     out["config"] = f"{T} tokens x hidden {H}, top-{K} of {E} experts, capacity {cap}, FP8"
+
+    # the peer-memory form: rank 0 of W = w.num_partitions sends the same batch into
+    # the W owners' padded blocks [E/W, W*cap, H] (all on this GPU), and its combine
+    # reads the rows back from them
+    W = w.num_partitions
+    epp = E // W
+    owners = [dict(x=torch.empty((epp, W * cap, H), dtype=torch.uint8, device=dev),
+                   s=torch.empty((epp, W * cap, H // 128), dtype=torch.float32, device=dev),
+                   c=torch.empty((epp, W), dtype=torch.int32, device=dev),
+                   eo=torch.empty((epp, W * cap, H), dtype=torch.bfloat16, device=dev))
+              for _ in range(W)]
+    tab = {k: torch.tensor([o[k].data_ptr() for o in owners], dtype=torch.int64, device=dev)
+           for k in ("x", "s", "c", "eo")}
+    for q, o in enumerate(owners):  # rank 0's block of each owner: the rows it would receive
+        o["eo"][:, :cap] = eo[q * epp:(q + 1) * epp]
+
+    def pdisp():
+        ep.ep_peer_low_latency_dispatch(x, idx, cap, E, W, 0, tab["x"], tab["s"], tab["c"], h, ws)
+
+    def pcomb():
+        ep.ep_peer_low_latency_combine(tab["eo"], idx, h, wts, y, E, W, 0, ws)
+
+    for name, fn in (("peer_dispatch", pdisp), ("peer_combine", pcomb)):
+        gn = capture(fn, per_graph)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(10):
+            gn.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = {"gpu_us": round(e0.elapsed_time(e1) * 1e3 / (10 * per_graph), 2),
+                     "ranks": W}
+    if ep.ep_read_status(ws) != 0:
+        raise RuntimeError("device status set in the peer low-latency run")
+    del owners, tab
     return out
 
 

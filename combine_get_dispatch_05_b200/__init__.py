@@ -22,6 +22,7 @@ from ._lib import (  # noqa: F401
     status_string, EP_IPC_HANDLE_BYTES, PeerTables, device_bytes, ep_ipc_alloc, ep_ipc_close,
     ep_ipc_free, ep_ipc_open, ep_peer_combine, ep_peer_dispatch, ep_peer_plan,
     ep_get_dispatch_layout_dedup, ep_peer_combine_dedup, ep_peer_dispatch_dedup,
+    ep_peer_low_latency_combine, ep_peer_low_latency_dispatch,
 )
 from .buffer import Buffer  # noqa: F401
 from .ep_group import EpContext, EpGroup  # noqa: F401

@@ -39,7 +39,8 @@ EXPORTED = (
     "ep_dispatch_dedup", "ep_combine_dedup", "ep_lb_prefetch_weights", "ep_lb_reduce_grads",
     "ep_ipc_alloc", "ep_ipc_free", "ep_ipc_open", "ep_ipc_close", "ep_peer_plan",
     "ep_peer_dispatch", "ep_peer_combine", "ep_get_dispatch_layout_dedup",
-    "ep_peer_dispatch_dedup", "ep_peer_combine_dedup",
+    "ep_peer_dispatch_dedup", "ep_peer_combine_dedup", "ep_peer_low_latency_dispatch",
+    "ep_peer_low_latency_combine",
 )
 EP_IPC_HANDLE_BYTES = 64
 
@@ -135,6 +136,12 @@ def _load() -> ctypes.CDLL:
     L.ep_peer_combine_dedup.argtypes = [i64, i64, i32, vp, i64, ctypes.POINTER(ep_layout), vp, vp,
                                         vp, sz, vp]
     L.ep_peer_combine_dedup.restype = st
+    L.ep_peer_low_latency_dispatch.argtypes = [i64, i64, i32, i32, i32, i32, i32, vp, vp, vp, vp,
+                                               vp, ctypes.POINTER(ep_ll_handle), vp, sz, vp]
+    L.ep_peer_low_latency_dispatch.restype = st
+    L.ep_peer_low_latency_combine.argtypes = [i64, i64, i32, i32, i32, i32, i32, vp, vp,
+                                              ctypes.POINTER(ep_ll_handle), vp, vp, vp, sz, vp]
+    L.ep_peer_low_latency_combine.restype = st
     return L
 
 
@@ -676,3 +683,47 @@ def ep_peer_combine_dedup(tables: PeerTables, handle: Layout, dst_offset: torch.
         T, H, world, tables.expert_out.data_ptr(), tables.capacity, ctypes.byref(c),
         dst_offset.data_ptr(), y.data_ptr(), workspace.data_ptr(), workspace.numel(),
         _stream(stream)))
+
+
+def ep_peer_low_latency_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, num_max_tokens: int,
+                                 num_experts: int, world: int, rank: int, recv_x: torch.Tensor,
+                                 recv_scales: torch.Tensor, recv_expert_count: torch.Tensor,
+                                 handle: LowLatencyHandle, workspace: torch.Tensor,
+                                 stream=None) -> None:
+    """recv_x / recv_scales / recv_expert_count: int64 [W] device tables of every rank's
+    [E/W, W*cap, H] E4M3, [E/W, W*cap, H/128] fp32 and [E/W, W] int32 buffers."""
+    _need(x, "x", torch.bfloat16)
+    T, H = x.shape
+    K = topk_idx.shape[1]
+    _need(topk_idx, "topk_idx", torch.int64, shape=(T, K))
+    for name, t in (("recv_x", recv_x), ("recv_scales", recv_scales),
+                    ("recv_expert_count", recv_expert_count)):
+        _need(t, name, torch.int64, shape=(world,))
+    _need(handle.row_of, "handle.row_of", torch.int32, shape=(T, K))
+    _need(handle.src_of, "handle.src_of", torch.int32, shape=(num_experts, num_max_tokens))
+    _need(workspace, "workspace", torch.uint8)
+    c = handle.c()
+    _check("ep_peer_low_latency_dispatch", lib.ep_peer_low_latency_dispatch(
+        T, H, K, num_experts, world, rank, num_max_tokens, x.data_ptr(), topk_idx.data_ptr(),
+        recv_x.data_ptr(), recv_scales.data_ptr(), recv_expert_count.data_ptr(), ctypes.byref(c),
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))
+
+
+def ep_peer_low_latency_combine(expert_out: torch.Tensor, topk_idx: torch.Tensor,
+                                handle: LowLatencyHandle, topk_weights: torch.Tensor,
+                                y: torch.Tensor, num_experts: int, world: int, rank: int,
+                                workspace: torch.Tensor, stream=None) -> None:
+    """expert_out: int64 [W] device table of every rank's BF16 [E/W, W*cap, H] outputs."""
+    _need(y, "y", torch.bfloat16)
+    T, H = y.shape
+    K = topk_idx.shape[1]
+    _need(topk_idx, "topk_idx", torch.int64, shape=(T, K))
+    _need(topk_weights, "topk_weights", torch.float32, shape=(T, K))
+    _need(expert_out, "expert_out", torch.int64, shape=(world,))
+    _need(handle.row_of, "handle.row_of", torch.int32, shape=(T, K))
+    _need(workspace, "workspace", torch.uint8)
+    c = handle.c()
+    _check("ep_peer_low_latency_combine", lib.ep_peer_low_latency_combine(
+        T, H, K, num_experts, world, rank, handle.num_max_tokens, expert_out.data_ptr(),
+        topk_idx.data_ptr(), ctypes.byref(c), topk_weights.data_ptr(), y.data_ptr(),
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))

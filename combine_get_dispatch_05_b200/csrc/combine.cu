@@ -37,8 +37,9 @@ constexpr int kLoadBatch = 8;  // combine backward: slots handled per batch
 // kPeer: partitions are ranks; slot k's row is row_of[t, k] + peer_offset[e] in the
 // expert outputs of the rank that owns e = topk_idx[t, k] (read over NVLink), or,
 // with peer_by_slot (deduplicated rows, slot k = rank k), row_of[t, k] +
-// peer_offset[k] in rank k's outputs; the compaction records a pointer to each
-// valid row instead of its index.
+// peer_offset[k] in rank k's outputs, or, for low-latency rows (row_of = e * cap +
+// j), row ((e % Epp) * W + rank) * cap + j of rank e / Epp's padded outputs; the
+// compaction records a pointer to each valid row instead of its index.
 template <int kBatch, bool kPeer>
 __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 && !kPeer ? 3 : 2)
     combine_kernel(CombineParams p, int64_t vec_per_slice) {
@@ -82,7 +83,15 @@ __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 && !kPeer ? 3 
                         at = ne >= 0 && ne < p.num_experts ? static_cast<int>(ne) : -1;
                         part = at >= 0 ? at / p.experts_per_partition : 0;
                     }
-                    const int64_t pr = at >= 0 ? static_cast<int64_t>(r) + p.peer_offset[at] : -1;
+                    int64_t pr = -1;
+                    if (at >= 0 && p.peer_ll_cap > 0) {
+                        const int64_t c = p.peer_ll_cap;
+                        const int64_t j = static_cast<int64_t>(r) - static_cast<int64_t>(at) * c;
+                        const int64_t el = at - part * p.experts_per_partition;
+                        if (j >= 0 && j < c) pr = (el * p.peer_world + p.peer_rank) * c + j;
+                    } else if (at >= 0) {
+                        pr = static_cast<int64_t>(r) + p.peer_offset[at];
+                    }
                     if (pr < 0 || pr >= p.expert_out_rows) {
                         raise_status(p.status, kDevIndexRange);
                         r = -1;

@@ -728,6 +728,86 @@ ep_status ep_peer_combine_dedup(int64_t num_tokens, int64_t hidden, int32_t worl
     return cuda_status(launch_combine(p, static_cast<cudaStream_t>(stream)));
 }
 
+ep_status ep_peer_low_latency_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                       int32_t num_experts, int32_t world, int32_t rank,
+                                       int32_t num_max_tokens, const void* x,
+                                       const int64_t* topk_idx, void* const* recv_x,
+                                       float* const* recv_scales, int32_t* const* recv_expert_count,
+                                       const ep_ll_handle* handle, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+    ep_status st = check_routing(num_tokens, num_topk, num_experts, world);
+    if (st != EP_OK) return st;
+    if ((st = check_hidden(hidden, true)) != EP_OK) return st;
+    if (rank < 0 || rank >= world) return EP_ERR_SHAPE;
+    if (num_max_tokens < 1 || num_tokens > num_max_tokens) return EP_ERR_SHAPE;
+    if (static_cast<int64_t>(num_experts) * num_max_tokens >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    if (!handle || !workspace || !recv_x || !recv_scales || !recv_expert_count ||
+        workspace_bytes < kWsHeader)
+        return EP_ERR_INVALID_ARG;
+    if (num_tokens > 0 && (!x || !topk_idx || !handle->row_of || !handle->src_of || !aligned16(x)))
+        return EP_ERR_INVALID_ARG;
+    LowLatencyDispatchParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = num_topk;
+    p.E = num_experts;
+    p.cap = num_max_tokens;
+    p.x = x;
+    p.topk_idx = topk_idx;
+    p.recv_x = nullptr;
+    p.recv_scales = nullptr;
+    p.recv_expert_count = nullptr;
+    p.row_of = handle->row_of;
+    p.src_of = handle->src_of;
+    p.status = carve_workspace(workspace, 0, 1).status;
+    p.timeout_ns = kDefaultTimeoutNs;
+    p.peer_recv_x = recv_x;
+    p.peer_recv_scales = recv_scales;
+    p.peer_recv_count = recv_expert_count;
+    p.world = world;
+    p.rank = rank;
+    p.epp = num_experts / world;
+    return cuda_status(launch_ll_dispatch(p, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status ep_peer_low_latency_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                      int32_t num_experts, int32_t world, int32_t rank,
+                                      int32_t num_max_tokens, const void* const* expert_out,
+                                      const int64_t* topk_idx, const ep_ll_handle* handle,
+                                      const float* topk_weights, void* y, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+    ep_status st = check_routing(num_tokens, num_topk, num_experts, world);
+    if (st != EP_OK) return st;
+    if ((st = check_hidden(hidden, false)) != EP_OK) return st;
+    if (rank < 0 || rank >= world || num_max_tokens < 1) return EP_ERR_SHAPE;
+    if (static_cast<int64_t>(num_experts) * num_max_tokens >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
+    if (!handle || !workspace || workspace_bytes < kWsHeader) return EP_ERR_INVALID_ARG;
+    if (num_tokens == 0) return EP_OK;
+    if (!handle->row_of || !expert_out || !topk_idx || !topk_weights || !y || !aligned16(y))
+        return EP_ERR_INVALID_ARG;
+    CombineParams p;
+    p.T = num_tokens;
+    p.H = hidden;
+    p.K = num_topk;
+    p.expert_out = nullptr;
+    p.expert_out_rows = static_cast<int64_t>(num_experts / world) * world * num_max_tokens;
+    p.row_of = handle->row_of;
+    p.topk_weights = topk_weights;
+    p.y = y;
+    p.grad_recv_w = nullptr;
+    p.grad_w = nullptr;
+    p.status = carve_workspace(workspace, 0, 1).status;
+    p.peer_out = expert_out;
+    p.topk_idx = topk_idx;
+    p.peer_offset = nullptr;
+    p.experts_per_partition = num_experts / world;
+    p.num_experts = num_experts;
+    p.peer_ll_cap = num_max_tokens;
+    p.peer_world = world;
+    p.peer_rank = rank;
+    return cuda_status(launch_combine(p, static_cast<cudaStream_t>(stream)));
+}
+
 ep_status ep_debug_wait_probe(uint64_t timeout_ns, void* workspace, size_t workspace_bytes,
                               void* stream) {
     if (!workspace || workspace_bytes < kWsHeader) return EP_ERR_INVALID_ARG;

@@ -108,6 +108,9 @@ struct CombineParams {
     int32_t experts_per_partition = 1;
     int32_t num_experts = 0;
     int32_t peer_by_slot = 0;  // deduplicated rows: slot k is rank k (topk_idx unused)
+    // low-latency rows (row_of = e * cap + j): the row is ((e % epp) * peer_world +
+    // peer_rank) * peer_ll_cap + j in rank e / epp's outputs (peer_offset unused)
+    int32_t peer_ll_cap = 0, peer_world = 1, peer_rank = 0;
 };
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 
@@ -155,6 +158,14 @@ struct LowLatencyDispatchParams {
     int32_t* src_of;
     uint32_t* status;
     uint64_t timeout_ns;
+    // Peer mode (partitions are the ranks of a node): slot j of expert e goes to row
+    // ((e % epp) * world + rank) * cap + j of rank e / epp's buffers, and the count of
+    // e to entry (e % epp) * world + rank of its count table; recv_x, recv_scales and
+    // recv_expert_count are unused (row_of / src_of stay local: e * cap + j).
+    void* const* peer_recv_x = nullptr;
+    float* const* peer_recv_scales = nullptr;
+    int32_t* const* peer_recv_count = nullptr;
+    int32_t world = 1, rank = 0, epp = 1;
 };
 cudaError_t launch_ll_dispatch(const LowLatencyDispatchParams& p, cudaStream_t stream);
 

@@ -18,6 +18,12 @@
 //   - CTA 0 also histograms all T*K ids into recv_expert_count;
 //   - quantise the slice (same arithmetic as the normal FP8 path) and bulk-store it
 //     into slot e * num_max_tokens + j of each destination expert.
+// Peer mode (template parameter kPeer; partitions are the ranks of a node, as in
+// DeepEP's low-latency kernels, whose receive buffer is [local experts, ranks *
+// num_max_tokens, hidden]): source rank s stores slot j of expert e into row
+// ((e % Epp) * W + s) * num_max_tokens + j of rank e / Epp's buffer and its count of
+// e into entry (e % Epp) * W + s of that rank's count table, so no counts have to be
+// exchanged first.  The handle stays local (e * num_max_tokens + j).
 #include "ep_device.cuh"
 #include "ep_internal.h"
 #include "ep_quant.cuh"
@@ -53,10 +59,29 @@ __host__ __device__ inline LLSmem ll_smem(int nbs, int32_t E) {
     return s;
 }
 
+// Where slot row (= e * cap + j) of expert e goes: the local padded buffer, or in peer
+// mode rank e / epp's buffer at ((e % epp) * world + rank) * cap + j.
+template <bool kPeer>
+__device__ __forceinline__ int64_t ll_dest(const LowLatencyDispatchParams& p, int row, int64_t e,
+                                           uint8_t*& x, float*& s) {
+    if constexpr (kPeer) {
+        const int q = static_cast<int>(e) / p.epp;
+        const int64_t j = row - e * p.cap;
+        x = static_cast<uint8_t*>(p.peer_recv_x[q]);
+        s = p.peer_recv_scales[q];
+        return (static_cast<int64_t>(static_cast<int>(e) - q * p.epp) * p.world + p.rank) * p.cap + j;
+    } else {
+        x = static_cast<uint8_t*>(p.recv_x);
+        s = p.recv_scales;
+        return row;
+    }
+}
+
 // grid = (T, S): CTA (t, y) handles token t's 128-channel blocks
 // [y * nbs, min(nb, (y + 1) * nbs)).  Every slice computes the token's slots (the
 // prefix is short and L2-hot); slice 0 also writes the handle; CTA (0, 0) writes
 // recv_expert_count.
+template <bool kPeer>
 __global__ void __launch_bounds__(kLLMaxThreads) ll_dispatch_kernel(LowLatencyDispatchParams p,
                                                                     int nbs) {
     extern __shared__ __align__(128) uint8_t sm[];
@@ -139,8 +164,14 @@ __global__ void __launch_bounds__(kLLMaxThreads) ll_dispatch_kernel(LowLatencyDi
             if (row >= 0) p.src_of[row] = static_cast<int32_t>(base + tid);
         }
     }
-    if (all)
-        for (int e = tid; e < E; e += blockDim.x) p.recv_expert_count[e] = min(hist[e], cap);
+    if (all) {
+        for (int e = tid; e < E; e += blockDim.x) {
+            if constexpr (kPeer)
+                p.peer_recv_count[e / p.epp][(e % p.epp) * p.world + p.rank] = min(hist[e], cap);
+            else
+                p.recv_expert_count[e] = min(hist[e], cap);
+        }
+    }
 
     const bool ok = mbar_wait_bounded(bar, 0, p.timeout_ns);
     if (!__syncthreads_and(ok)) {
@@ -153,26 +184,38 @@ __global__ void __launch_bounds__(kLLMaxThreads) ll_dispatch_kernel(LowLatencyDi
     quantize_row_fp8(sm, out_q, out_s, nbl, warp, nwarps, lane);
     fence_proxy_async_smem();
     __syncthreads();
-    uint8_t* recv_x = static_cast<uint8_t*>(p.recv_x);
     if (warp == 0 && lane < K) {
         const int row = rows_sm[lane];
         if (row >= 0) {
-            bulk_store(recv_x + static_cast<int64_t>(row) * H + static_cast<int64_t>(b0) * 128,
-                       out_q, static_cast<uint32_t>(nbl) * 128u);
+            uint8_t* dx;
+            float* ds;
+            const int64_t r = ll_dest<kPeer>(p, row, eid_sm[lane], dx, ds);
+            bulk_store(dx + r * H + static_cast<int64_t>(b0) * 128, out_q,
+                       static_cast<uint32_t>(nbl) * 128u);
             if (scale_bulk)
-                bulk_store(p.recv_scales + static_cast<int64_t>(row) * nb + b0, out_s,
-                           static_cast<uint32_t>(nbl) * 4u);
+                bulk_store(ds + r * nb + b0, out_s, static_cast<uint32_t>(nbl) * 4u);
         }
         bulk_commit();
     }
     if (!scale_bulk) {
         for (int idx = tid; idx < K * nbl; idx += blockDim.x) {
             const int k = idx / nbl, b = idx - k * nbl;
-            const int r = rows_sm[k];
-            if (r >= 0) p.recv_scales[static_cast<int64_t>(r) * nb + b0 + b] = out_s[b];
+            const int row = rows_sm[k];
+            if (row >= 0) {
+                uint8_t* dx;
+                float* ds;
+                const int64_t r = ll_dest<kPeer>(p, row, eid_sm[k], dx, ds);
+                ds[r * nb + b0 + b] = out_s[b];
+            }
         }
     }
     if (warp == 0 && lane < K) bulk_wait_all<0>();
+}
+
+// Peer mode with no tokens: this rank's count of every expert is zero.
+__global__ void ll_peer_zero_counts_kernel(LowLatencyDispatchParams p) {
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x)
+        p.peer_recv_count[e / p.epp][(e % p.epp) * p.world + p.rank] = 0;
 }
 
 __global__ void wait_probe_kernel(uint32_t* status, const volatile uint32_t* flag,
@@ -197,6 +240,10 @@ __global__ void wait_probe_kernel(uint32_t* status, const volatile uint32_t* fla
 cudaError_t launch_ll_dispatch(const LowLatencyDispatchParams& p, cudaStream_t stream) {
     if (p.T == 0) {
         // no tokens: every expert received nothing
+        if (p.peer_recv_x) {
+            ll_peer_zero_counts_kernel<<<1, 256, 0, stream>>>(p);
+            return cudaGetLastError();
+        }
         return cudaMemsetAsync(p.recv_expert_count, 0, sizeof(int32_t) * p.E, stream);
     }
     DeviceInfo dev;
@@ -214,14 +261,18 @@ cudaError_t launch_ll_dispatch(const LowLatencyDispatchParams& p, cudaStream_t s
     if (S > 65535) return cudaErrorInvalidValue;
     const LLSmem L = ll_smem(nbs, p.E);
     if (L.total > dev.max_smem_optin) return cudaErrorInvalidValue;
-    err = cudaFuncSetAttribute(ll_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(L.total));
+    const bool peer = p.peer_recv_x != nullptr;
+    err = cudaFuncSetAttribute(peer ? ll_dispatch_kernel<true> : ll_dispatch_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
     if (err != cudaSuccess) return err;
     const int pairs = (nbs + 1) / 2;
     int threads = 32 * (pairs < 2 ? 2 : pairs);
     if (threads > kLLMaxThreads) threads = kLLMaxThreads;
-    ll_dispatch_kernel<<<dim3(static_cast<unsigned>(p.T), static_cast<unsigned>(S)), threads, L.total,
-                         stream>>>(p, nbs);
+    const dim3 grid(static_cast<unsigned>(p.T), static_cast<unsigned>(S));
+    if (peer)
+        ll_dispatch_kernel<true><<<grid, threads, L.total, stream>>>(p, nbs);
+    else
+        ll_dispatch_kernel<false><<<grid, threads, L.total, stream>>>(p, nbs);
     return cudaGetLastError();
 }
 

@@ -81,13 +81,15 @@ class EpGroup:
     capacity: rows of each rank's receive buffers in peer mode (default
     max_tokens * W * 8, every token of every rank routed here with top-8).
     num_topk: the largest K the peer buffers' id / weight lists hold (dedup rows).
+    ll_max_tokens: peer transport, low-latency calls: the most tokens a rank sends
+    per call (each rank's buffer holds E/W experts x W ranks x ll_max_tokens rows).
     Call :meth:`close` before destroying the process group.
     """
 
     def __init__(self, num_experts: int, group=None, max_tokens: int = 4096,
                  device: Optional[torch.device] = None, *, transport: str = "nccl",
                  hidden: Optional[int] = None, capacity: Optional[int] = None,
-                 num_topk: int = 8):
+                 num_topk: int = 8, ll_max_tokens: int = 0):
         self.group = group if group is not None else dist.group.WORLD
         self.world = dist.get_world_size(self.group)
         self.rank = dist.get_rank(self.group)
@@ -109,7 +111,7 @@ class EpGroup:
                 raise ValueError("the peer transport needs `hidden` to size the receive buffers")
             self._open_peers(int(hidden), int(capacity if capacity is not None
                                                   else max_tokens * self.world * 8),
-                             int(num_topk))
+                             int(num_topk), int(ll_max_tokens))
 
     def _new_workspace(self, tokens: int) -> torch.Tensor:
         ws = torch.empty(_lib.ep_workspace_bytes(max(tokens, 1), self.num_experts, self.world),
@@ -118,20 +120,16 @@ class EpGroup:
         return ws
 
     # ---------------------------------------------------------- peer buffers --
-    def _open_peers(self, hidden: int, capacity: int, topk: int) -> None:
-        """One IPC region per rank: recv_x (room for BF16 rows) | recv_scales |
-        recv_topk_idx | recv_topk_weights (room for [K] lists) | expert_out, each
-        256-byte aligned."""
-        if hidden % 128:
-            raise ValueError("hidden must be a multiple of 128")
-        sizes = [("recv_x", capacity * hidden * 2), ("recv_scales", capacity * (hidden // 128) * 4),
-                 ("recv_topk_idx", capacity * topk * 4), ("recv_topk_weights", capacity * topk * 4),
-                 ("expert_out", capacity * hidden * 2)]
+    def _map_region(self, sizes) -> dict:
+        """Allocate this rank's IPC region holding the named arrays (each 256-byte
+        aligned), exchange the handles and map every other rank's region.  Returns
+        the region's description with every rank's array addresses."""
         offsets, total = {}, 0
         for name, n in sizes:
             offsets[name] = total
             total += (n + _ALIGN - 1) // _ALIGN * _ALIGN
-        base, handle = _lib.ep_ipc_alloc(max(total, _ALIGN))
+        total = max(total, _ALIGN)
+        base, handle = _lib.ep_ipc_alloc(total)
         handles: List[bytes] = [b""] * self.world
         dist.all_gather_object(handles, handle, group=self.group)
         bases, opened = [], []
@@ -148,15 +146,39 @@ class EpGroup:
                 _lib.ep_ipc_close(ptr)
             _lib.ep_ipc_free(base)
             raise
-        self._peer = dict(base=base, opened=opened, hidden=hidden, capacity=capacity, topk=topk,
-                          region=_lib.device_bytes(base, max(total, _ALIGN), self.device),
-                          offsets=offsets, sizes=dict(sizes))
-        self.tables = _lib.PeerTables.from_addresses(
-            self.device, capacity, *[[b + offsets[n] for b in bases] for n, _ in sizes])
-        self._flag = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self._regions.append(dict(base=base, opened=opened))
+        return dict(region=_lib.device_bytes(base, total, self.device), offsets=offsets,
+                    sizes=dict(sizes),
+                    addrs={n: [b + offsets[n] for b in bases] for n, _ in sizes})
 
-    def _view(self, name: str, dtype, shape) -> torch.Tensor:
-        pr = self._peer
+    def _open_peers(self, hidden: int, capacity: int, topk: int, ll_max_tokens: int) -> None:
+        """The normal region: recv_x (room for BF16 rows) | recv_scales | recv_topk_idx |
+        recv_topk_weights (room for [K] lists) | expert_out; and, with ll_max_tokens,
+        the low-latency region: [E/W, W*cap] rows of E4M3 payload, scales and BF16
+        outputs, and the [E/W, W] counts."""
+        if hidden % 128:
+            raise ValueError("hidden must be a multiple of 128")
+        self._regions = []
+        self._flag = torch.zeros(1, dtype=torch.int32, device=self.device)
+        sizes = [("recv_x", capacity * hidden * 2), ("recv_scales", capacity * (hidden // 128) * 4),
+                 ("recv_topk_idx", capacity * topk * 4), ("recv_topk_weights", capacity * topk * 4),
+                 ("expert_out", capacity * hidden * 2)]
+        reg = self._map_region(sizes)
+        self._peer = dict(reg, hidden=hidden, capacity=capacity, topk=topk, ll=None)
+        self.tables = _lib.PeerTables.from_addresses(
+            self.device, capacity, *[reg["addrs"][n] for n, _ in sizes])
+        if ll_max_tokens > 0:
+            rows = self.experts_per_rank * self.world * ll_max_tokens
+            ll = self._map_region([("x", rows * hidden), ("scales", rows * (hidden // 128) * 4),
+                                   ("count", self.experts_per_rank * self.world * 4),
+                                   ("expert_out", rows * hidden * 2)])
+            ll["cap"] = ll_max_tokens
+            ll["tables"] = {n: torch.tensor(a, dtype=torch.int64, device=self.device)
+                            for n, a in ll["addrs"].items()}
+            self._peer["ll"] = ll
+
+    def _view(self, name: str, dtype, shape, region=None) -> torch.Tensor:
+        pr = self._peer if region is None else region
         n = 1
         for d in shape:
             n *= d
@@ -178,12 +200,14 @@ class EpGroup:
         if self._peer is None:
             return
         self._host_barrier()  # no rank's kernels touch any region any more
-        for ptr in self._peer["opened"]:
-            _lib.ep_ipc_close(ptr)
-        self._host_barrier()  # every rank has closed its mappings of this rank's region
-        self._peer["region"] = None
-        _lib.ep_ipc_free(self._peer["base"])
+        for reg in self._regions:
+            for ptr in reg["opened"]:
+                _lib.ep_ipc_close(ptr)
+        self._host_barrier()  # every rank has closed its mappings of this rank's regions
         self._peer = None
+        for reg in self._regions:
+            _lib.ep_ipc_free(reg["base"])
+        self._regions = []
 
     # --------------------------------------------------------------- exchange --
     def _a2a(self, inp: torch.Tensor, out_rows: int, out_splits: List[int],
@@ -368,6 +392,57 @@ class EpGroup:
         else:
             recv_x = self._view("recv_x", torch.bfloat16, (cap, H))[:Rr]
         return recv_x, ri, rw, per_source, ctx
+
+    # ------------------------------------------------------------ low latency --
+    def low_latency_dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor):
+        """Peer transport (constructed with ll_max_tokens): DeepEP's low-latency
+        dispatch across the ranks.  Every rank's FP8 rows go straight into padded
+        per-expert blocks of their owners' buffers, with no count exchange first.
+
+        Returns ``((recv_x, recv_scales), recv_count, ctx)``: recv_x E4M3
+        [E/W, W*cap, H] and recv_scales [E/W, W*cap, H/128] (rows [s*cap, s*cap + n)
+        of local expert el come from rank s, n = recv_count[el, s]), recv_count int32
+        [E/W, W]."""
+        ll = self._peer["ll"] if self._peer is not None else None
+        if ll is None:
+            raise RuntimeError("low-latency calls need the peer transport and ll_max_tokens")
+        T, H = x.shape
+        K = topk_idx.shape[1]
+        cap, E, W, epp = ll["cap"], self.num_experts, self.world, self.experts_per_rank
+        if T > cap:
+            raise ValueError(f"{T} tokens exceed ll_max_tokens = {cap}")
+        h = _lib.LowLatencyHandle.empty(T, K, E, cap, self.device)
+        t = ll["tables"]
+        _lib.ep_peer_low_latency_dispatch(x, topk_idx, cap, E, W, self.rank, t["x"], t["scales"],
+                                          t["count"], h, self.workspace)
+        self._barrier()  # every rank's rows and counts have landed
+        rows = epp * W * cap
+        q = self._view("x", torch.uint8, (epp, W * cap, H), ll).view(torch.float8_e4m3fn)
+        s = self._view("scales", torch.float32, (epp, W * cap, H // 128), ll)
+        count = self._view("count", torch.int32, (epp, W), ll)
+        ctx = EpContext(h, [], [], T, H, topk_idx=topk_idx, recv_rows=rows, order="low_latency")
+        return (q, s), count, ctx
+
+    def ll_expert_out_buffer(self) -> torch.Tensor:
+        """BF16 [E/W, W*cap, H]: where a rank's low-latency expert outputs go (row i of
+        a block answers received row i); the other ranks' combines read it."""
+        ll = self._peer["ll"]
+        return self._view("expert_out", torch.bfloat16,
+                          (self.experts_per_rank, self.world * ll["cap"], self._peer["hidden"]), ll)
+
+    def low_latency_combine(self, expert_out: torch.Tensor, ctx: EpContext,
+                            topk_weights: torch.Tensor) -> torch.Tensor:
+        """expert_out: the tensor from :meth:`ll_expert_out_buffer`.  Returns y BF16
+        [T, H]: each token's expert outputs, read from their owners and reduced in
+        fixed k order with its weights."""
+        if expert_out.data_ptr() != self.ll_expert_out_buffer().data_ptr():
+            raise ValueError("write the expert outputs into ll_expert_out_buffer()")
+        y = torch.empty((ctx.num_tokens, ctx.hidden), dtype=torch.bfloat16, device=self.device)
+        self._barrier()  # every rank's expert outputs are complete
+        _lib.ep_peer_low_latency_combine(self._peer["ll"]["tables"]["expert_out"], ctx.topk_idx,
+                                         ctx.handle, topk_weights, y, self.num_experts, self.world,
+                                         self.rank, self.workspace)
+        return y
 
     # ---------------------------------------------------------------- combine --
     def combine(self, expert_out: torch.Tensor, ctx: EpContext,

@@ -540,6 +540,44 @@ EP_API ep_status ep_peer_combine_dedup(int64_t num_tokens, int64_t hidden, int32
                                        void* y, void* workspace, size_t workspace_bytes,
                                        void* stream);
 
+/* ---- low-latency rows across GPUs ---------------------------------------------
+ * deepseek.csdn.net/67bd3eb22e30c863900615cc, "推理解码阶段的应用":
+ * low_latency_dispatch(hidden_states, topk_idx, num_max_tokens, num_experts) with a
+ * buffer of num_max_tokens rows per expert; "DeepSeek 开源周第二弹：DeepEP",
+ * "DeepEP 的常规内核和低延迟内核": low-latency kernels for decode.  The peer form,
+ * in the layout of DeepEP's low-latency receive buffer: rank q holds, for each of
+ * its Epp = E/W experts, W * cap rows, source rank s owning rows [s*cap, (s+1)*cap).
+ * Source rank `rank` writes slot j of expert e (the slot ep_low_latency_dispatch
+ * would use) to row ((e % Epp) * W + rank) * cap + j of rank e/Epp's buffer, and
+ * its row count of e to entry (e % Epp) * W + rank of that rank's count table, so
+ * nothing is exchanged before the dispatch.  Steps: ep_peer_low_latency_dispatch
+ * on every rank; barrier; each rank computes its experts over the first
+ * count[el][s] rows of each (local expert el, source s) block; barrier;
+ * ep_peer_low_latency_combine on every rank.  cap = num_max_tokens >= T on every
+ * rank; the handle (local: e * cap + j) is what ep_low_latency_dispatch returns. */
+
+/* recv_x: device table of W pointers to E4M3 [E/W, W*cap, H]; recv_scales: to fp32
+ * [E/W, W*cap, H/128]; recv_expert_count: to int32 [E/W, W].  Unused rows are not
+ * written.  Errors as for ep_low_latency_dispatch; 0 <= rank < W, W divides E. */
+EP_API ep_status ep_peer_low_latency_dispatch(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                              int32_t num_experts, int32_t world, int32_t rank,
+                                              int32_t num_max_tokens, const void* x,
+                                              const int64_t* topk_idx, void* const* recv_x,
+                                              float* const* recv_scales,
+                                              int32_t* const* recv_expert_count,
+                                              const ep_ll_handle* handle, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+
+/* ep_low_latency_combine with slot row e * cap + j of (t, k) read from row
+ * ((e % Epp) * W + rank) * cap + j of expert_out[e / Epp] (device table of W
+ * pointers to BF16 [E/W, W*cap, H]).  topk_idx: the ids the dispatch used. */
+EP_API ep_status ep_peer_low_latency_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk,
+                                             int32_t num_experts, int32_t world, int32_t rank,
+                                             int32_t num_max_tokens, const void* const* expert_out,
+                                             const int64_t* topk_idx, const ep_ll_handle* handle,
+                                             const float* topk_weights, void* y, void* workspace,
+                                             size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -252,7 +252,40 @@ def _peer_stand_ins(oracle, torch):
         yb, _ = oracle.combine_dedup(rows, prow)
         y.copy_(torch.from_numpy(yb.view(np.int16)).view(torch.bfloat16))
 
+    def ll_dispatch(x, idx, cap, E, W, rank, tx, ts, tc, h, ws, stream=None):
+        xs = x.view(torch.int16).numpy().view(np.uint16)
+        H = xs.shape[1]
+        o = oracle.ll_dispatch(xs, idx.numpy(), E, cap)
+        epp = E // W
+        for e in range(E):
+            q, el, n = e // epp, e % epp, int(o["recv_expert_count"][e])
+            put(tc[q] + (el * W + rank) * 4, np.array([n], np.int32))
+            for j in range(n):
+                row = (el * W + rank) * cap + j
+                put(tx[q] + row * H, o["recv_x"][e, j])
+                put(ts[q] + row * (H // 128) * 4, o["recv_scales"][e, j])
+        h.row_of.copy_(torch.from_numpy(o["ll_row_of"]))
+        h.src_of.copy_(torch.from_numpy(o["ll_src_of"]))
+
+    def ll_combine(te, idx, h, w, y, E, W, rank, ws, stream=None):
+        ids, ro = idx.numpy(), h.row_of.numpy()
+        T, K = ids.shape
+        H, cap, epp = y.shape[1], h.num_max_tokens, E // W
+        rows = np.zeros((max(T * K, 1), H), np.uint16)
+        row_of = np.full((T, K), -1, np.int32)
+        for t in range(T):
+            for k in range(K):
+                if ro[t, k] >= 0:
+                    e = int(ids[t, k])
+                    j = int(ro[t, k]) - e * cap
+                    a = te[e // epp] + (((e % epp) * W + rank) * cap + j) * H * 2
+                    rows[t * K + k] = get(a, H * 2).view(np.uint16)
+                    row_of[t, k] = t * K + k
+        yb, _ = oracle.combine(rows, row_of, w.numpy())
+        y.copy_(torch.from_numpy(yb.view(np.int16)).view(torch.bfloat16))
+
     return dict(ep_ipc_alloc=ipc_alloc, ep_ipc_open=ipc_open, ep_ipc_close=ipc_close,
+                ep_peer_low_latency_dispatch=ll_dispatch, ep_peer_low_latency_combine=ll_combine,
                 ep_ipc_free=ipc_free, device_bytes=device_bytes, ep_get_dispatch_layout=layout,
                 ep_peer_plan=plan, ep_peer_dispatch=dispatch, ep_peer_combine=combine,
                 ep_get_dispatch_layout_dedup=layout_dedup, ep_peer_dispatch_dedup=dispatch_dedup,
@@ -292,7 +325,9 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
         w_all = np.concatenate([w.topk_weights for w in loads])
         t0 = sum(tokens[:rank])
         w = loads[rank]
-        g = ep_group.EpGroup(E, device="cpu", transport="peer", hidden=H, max_tokens=128)
+        cap = 128
+        g = ep_group.EpGroup(E, device="cpu", transport="peer", hidden=H, max_tokens=128,
+                             ll_max_tokens=cap)
         x = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16)
         idx = torch.from_numpy(w.topk_idx)
         wts = torch.from_numpy(w.topk_weights)
@@ -347,6 +382,29 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
             y_all, _ = oracle.combine_dedup(po_all, d["prow_of"])
             assert np.array_equal(y.view(torch.int16).numpy().view(np.uint16),
                                   y_all[t0:t0 + tokens[rank]]), "dedup " + quant
+        for _ in range(2):  # low-latency rows: padded per-expert blocks, one per source rank
+            (q, s), count, ctx = g.low_latency_dispatch(x, idx)
+            got_q, got_s, got_c = q.view(torch.uint8).numpy(), s.numpy(), count.numpy()
+            for src, l in enumerate(loads):
+                o = oracle.ll_dispatch(l.x, l.topk_idx, E, cap)
+                for el in range(epp):
+                    e = rank * epp + el
+                    n = int(o["recv_expert_count"][e])
+                    assert got_c[el, src] == n
+                    blk = slice(src * cap, src * cap + n)
+                    assert np.array_equal(got_q[el, blk], o["recv_x"][e, :n])
+                    assert np.array_equal(got_s[el, blk].view(np.uint32),
+                                          o["recv_scales"][e, :n].view(np.uint32))
+                eo = oracle.identity_expert(o["recv_x"].reshape(E * cap, H),
+                                            o["recv_scales"].reshape(E * cap, H // 128))
+                eo = eo.reshape(E, cap, H)
+                buf = g.ll_expert_out_buffer()
+                buf[:, src * cap:(src + 1) * cap].copy_(torch.from_numpy(
+                    eo[rank * epp:(rank + 1) * epp].view(np.int16)).view(torch.bfloat16))
+                if src == rank:
+                    y_ref, _ = oracle.ll_combine(eo, o["ll_row_of"], w.topk_weights)
+            y = g.low_latency_combine(g.ll_expert_out_buffer(), ctx, wts)
+            assert np.array_equal(y.view(torch.int16).numpy().view(np.uint16), y_ref), "ll"
         status = "ok"
     finally:
         try:

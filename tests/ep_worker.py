@@ -115,7 +115,7 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
 
         E, H, K = 32, 512, 4
         w = make_custom(333, H, K, E, world, seed=120 + rank, mask_frac=0.1)
-        g = ep.EpGroup(E, transport="peer", hidden=H, max_tokens=512)
+        g = ep.EpGroup(E, transport="peer", hidden=H, max_tokens=512, ll_max_tokens=384)
         x = dev_u16_as_bf16(w.x)
         idx = torch.from_numpy(w.topk_idx).cuda()
         wts = torch.from_numpy(w.topk_weights).cuda()
@@ -163,6 +163,23 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
             y = g.combine(out, ctx, wts)
             y_ref, _ = oracle.combine_dedup(po, d["prow_of"])
             assert np.array_equal(bf16_to_u16(y), y_ref), "dedup " + quant
+        for _ in range(2):  # low-latency rows (padded per-expert blocks)
+            (q, s), count, ctx = g.low_latency_dispatch(x, idx)
+            o = oracle.ll_dispatch(w.x, w.topk_idx, E, 384)
+            assert np.array_equal(count.cpu().numpy().reshape(-1), o["recv_expert_count"])
+            gq, gs = q.view(torch.uint8).cpu().numpy(), s.cpu().numpy()
+            for e in range(E):
+                n = int(o["recv_expert_count"][e])
+                assert np.array_equal(gq[e, :n], o["recv_x"][e, :n]), e
+                assert np.array_equal(gs[e, :n].view(np.uint32),
+                                      o["recv_scales"][e, :n].view(np.uint32)), e
+            eo = oracle.identity_expert(o["recv_x"].reshape(E * 384, H),
+                                        o["recv_scales"].reshape(E * 384, H // 128))
+            buf = g.ll_expert_out_buffer()
+            buf.copy_(dev_u16_as_bf16(eo).view(E, 384, H))
+            y = g.low_latency_combine(buf, ctx, wts)
+            y_ref, _ = oracle.ll_combine(eo.reshape(E, 384, H), o["ll_row_of"], w.topk_weights)
+            assert np.array_equal(bf16_to_u16(y), y_ref), "ll"
         assert ep.ep_read_status(g.workspace) == 0
         status = "ok"
     finally:

@@ -312,3 +312,31 @@ def test_peer_dedup_host_checks(ep):
     assert comb(4, 128, 8, None, 64, ctypes.byref(lay), f, f, f, 4096, None) == 1
     assert comb(4, 128, 8, f, 64, ctypes.byref(lay), None, f, f, 4096, None) == 1
     assert comb(0, 128, 8, None, 64, ctypes.byref(lay), None, None, f, 4096, None) == 0
+
+
+def test_peer_low_latency_host_checks(ep):
+    f = _Fake.P
+    h = ep._lib.ep_ll_handle(f, f)
+    L = ep.lib
+
+    def disp(T=8, H=256, K=4, E=16, W=2, rank=0, cap=8, x=f, tx=f):
+        return L.ep_peer_low_latency_dispatch(T, H, K, E, W, rank, cap, x, f, tx, f, f,
+                                              ctypes.byref(h), f, 4096, None)
+
+    assert disp(T=9) == 2           # more tokens than capacity
+    assert disp(rank=2) == 2        # rank >= W
+    assert disp(E=15) == 2          # E % W
+    assert disp(H=136) == 2         # FP8 needs H % 128 == 0
+    assert disp(tx=None) == 1
+    assert disp(x=f + 8) == 1
+    comb = L.ep_peer_low_latency_combine
+
+    def cmb(T=8, H=256, K=4, E=16, W=2, rank=0, cap=8, eo=f, y=f):
+        return comb(T, H, K, E, W, rank, cap, eo, f, ctypes.byref(h), f, y, f, 4096, None)
+
+    assert cmb(rank=-1) == 2
+    assert cmb(cap=0) == 2
+    assert cmb(H=100) == 2
+    assert cmb(eo=None) == 1
+    assert cmb(y=f + 2) == 1
+    assert cmb(T=0, eo=None, y=None) == 0

@@ -307,3 +307,94 @@ def test_peer_dedup_capacity_overflow_drops_one_rank(ep):
     rows1 = int(d["part_offset"][2] - d["part_offset"][1])
     assert int(d["part_offset"][1]) > rows1
     _check_dedup(ep, loads, 8, 2, "fp8", capacity=rows1, drop=(0,))
+
+
+# ------------------------------------------------------ low-latency rows --
+
+def _check_ll(ep, loads, E, W, cap):
+    """Every rank's padded receive buffer [E/W, W*cap, H]: source s's block of local
+    expert el must equal, byte for byte, the oracle's one-GPU low-latency dispatch of
+    s's tokens for expert q*Epp + el (unwritten slots keep the 0xA5 fill on both
+    sides); the counts and the local handle likewise; then each rank's combine."""
+    H, K = loads[0].hidden, loads[0].num_topk
+    epp = E // W
+    bufs = [dict(x=Guarded((epp, W * cap, H), torch.uint8),
+                 s=Guarded((epp, W * cap, H // 128), torch.float32),
+                 c=Guarded((epp, W), torch.int32),
+                 eo=Guarded((epp, W * cap, H), torch.bfloat16)) for _ in range(W)]
+
+    def table(key):
+        return torch.tensor([b[key].t.data_ptr() for b in bufs], dtype=torch.int64, device="cuda")
+
+    tx, ts, tc, te = table("x"), table("s"), table("c"), table("eo")
+    ranks, want = [], []
+    for s, w in enumerate(loads):
+        T = w.num_tokens
+        r = dict(x=dev_u16_as_bf16(w.x), idx=torch.from_numpy(w.topk_idx).cuda(),
+                 wts=torch.from_numpy(w.topk_weights).cuda(),
+                 h=ep.LowLatencyHandle.empty(T, K, E, cap, "cuda"), ws=new_workspace(ep, T, E, W))
+        ep.ep_peer_low_latency_dispatch(r["x"], r["idx"], cap, E, W, s, tx, ts, tc, r["h"], r["ws"])
+        ranks.append(r)
+        want.append(oracle.ll_dispatch(w.x, w.topk_idx, E, cap, fill=CANARY))
+    torch.cuda.synchronize()
+    assert [ep.ep_read_status(r["ws"]) for r in ranks] == [0] * W
+    for q in range(W):
+        b = bufs[q]
+        gx, gs, gc = b["x"].t.cpu().numpy(), b["s"].t.cpu().numpy(), b["c"].t.cpu().numpy()
+        for s in range(W):
+            o = want[s]
+            blk = slice(s * cap, (s + 1) * cap)
+            assert np.array_equal(gx[:, blk], o["recv_x"][q * epp:(q + 1) * epp]), (q, s)
+            cnt = o["recv_expert_count"][q * epp:(q + 1) * epp]
+            assert np.array_equal(gc[:, s], cnt), (q, s)
+            for el in range(epp):
+                n = int(cnt[el])
+                assert np.array_equal(gs[el, s * cap:s * cap + n].view(np.uint32),
+                                      o["recv_scales"][q * epp + el, :n].view(np.uint32)), (q, s, el)
+        assert all(g.canary_ok() for g in (b["x"], b["s"], b["c"]))
+    for s, r in enumerate(ranks):
+        assert np.array_equal(r["h"].row_of.cpu().numpy(), want[s]["ll_row_of"]), s
+        so = r["h"].src_of.cpu().numpy()
+        for e in range(E):  # the local handle: slot j of e holds (t, k) = src_of[e, j]
+            n = int(want[s]["recv_expert_count"][e])
+            assert np.array_equal(so[e, :n], want[s]["ll_src_of"][e, :n]), (s, e)
+
+    # expert outputs: identity experts on each source's rows, placed in the owners'
+    # blocks; then every rank's combine reads them back
+    y_refs = []
+    for s, w in enumerate(loads):
+        o = want[s]
+        eo = oracle.identity_expert(o["recv_x"].reshape(E * cap, H),
+                                    o["recv_scales"].reshape(E * cap, H // 128)).reshape(E, cap, H)
+        for q in range(W):
+            bufs[q]["eo"].t[:, s * cap:(s + 1) * cap].copy_(
+                dev_u16_as_bf16(eo[q * epp:(q + 1) * epp].reshape(-1, H)).view(epp, cap, H))
+        y_refs.append(oracle.ll_combine(eo, o["ll_row_of"], w.topk_weights)[0])
+        del eo
+        want[s] = None
+    torch.cuda.synchronize()
+    for s, (w, r) in enumerate(zip(loads, ranks)):
+        y = Guarded((w.num_tokens, H), torch.bfloat16)
+        ep.ep_peer_low_latency_combine(te, r["idx"], r["h"], r["wts"], y.t, E, W, s, r["ws"])
+        torch.cuda.synchronize()
+        assert np.array_equal(bf16_to_u16(y.t), y_refs[s]), s
+        assert y.canary_ok()
+        assert ep.ep_read_status(r["ws"]) == 0
+
+
+def test_peer_ll_two_ranks(ep):
+    loads = [make_custom(T, 512, 4, 16, 2, seed=130 + s, mask_frac=0.05)
+             for s, T in enumerate([40, 64])]
+    _check_ll(ep, loads, 16, 2, 64)
+
+
+def test_peer_ll_four_ranks_empty_rank(ep):
+    # H = 384: 3 scale blocks per row (the per-element scale stores)
+    loads = [make_custom(T, 384, 8, 32, 4, seed=140 + s) for s, T in enumerate([128, 0, 77, 128])]
+    _check_ll(ep, loads, 32, 4, 128)
+
+
+def test_peer_ll_eight_ranks_decode_batches(ep):
+    # the low-latency workload on each of 8 ranks: 128 tokens, hidden 7168, top-8 of 256
+    loads = [make_workload("ll", seed=150 + s) for s in range(8)]
+    _check_ll(ep, loads, 256, 8, 128)
