@@ -254,7 +254,7 @@ class EpGroup:
 
     # --------------------------------------------------------------- dispatch --
     def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
-                 use_fp8: bool = True, dedup: bool = False):
+                 use_fp8: bool = True, dedup: bool = False, return_recv_hook: bool = False):
         """Returns ``(recv_x, recv_local_idx, recv_weights, recv_counts_per_expert, ctx)``.
 
         recv_x: ``(float8_e4m3fn [Rr, H], float32 [Rr, H/128])`` or BF16 ``[Rr, H]``;
@@ -265,7 +265,16 @@ class EpGroup:
 
         dedup (peer transport): one row per (token, rank); recv_local_idx and
         recv_weights are [Rr, K] lists and the counts are [W, 1] rows per source.
+
+        return_recv_hook (peer transport): return as soon as this rank's rows are on
+        their way, with a ``hook`` appended to the result; calling it (every rank, a
+        collective) waits until every rank's rows have landed.  Work enqueued
+        between the two overlaps the transfer; the received tensors are valid after
+        the hook.  As DeepEP's receive hook ("deepseek.csdn.net/67bd3eb22e30c863900615cc",
+        "推理解码阶段的应用": low_latency_dispatch returns a hook).
         """
+        if return_recv_hook and self.transport != "peer":
+            raise NotImplementedError("the receive hook belongs to the peer transport")
         T = x.shape[0]
         if T > self.max_tokens:
             self.max_tokens = T
@@ -273,9 +282,11 @@ class EpGroup:
         if dedup:
             if self.transport != "peer":
                 raise NotImplementedError("deduplicated rows are offered by the peer transport")
-            return self._dispatch_peer_dedup(x, topk_idx, topk_weights, use_fp8)
+            return self._deliver(self._dispatch_peer_dedup(x, topk_idx, topk_weights, use_fp8),
+                                 return_recv_hook)
         if self.transport == "peer":
-            return self._dispatch_peer(x, topk_idx, topk_weights, use_fp8)
+            return self._deliver(self._dispatch_peer(x, topk_idx, topk_weights, use_fp8),
+                                 return_recv_hook)
         return self._dispatch_nccl(x, topk_idx, topk_weights, use_fp8)
 
     def _dispatch_nccl(self, x, topk_idx, topk_weights, use_fp8):
@@ -334,7 +345,6 @@ class EpGroup:
         quant = EP_QUANT_FP8_E4M3_1X128 if use_fp8 else EP_QUANT_NONE
         _lib.ep_peer_dispatch(x, topk_idx, topk_weights, E, W, quant, lay, dst, self.tables,
                               self.workspace)
-        self._barrier()  # every rank's rows have landed in their owners' buffers
         Rr = int(totals[r])
         per_expert = counts[:, r * epp:(r + 1) * epp]
         send = counts.view(W, W, epp)[r].sum(dim=1).to("cpu").tolist()
@@ -376,7 +386,6 @@ class EpGroup:
         quant = EP_QUANT_FP8_E4M3_1X128 if use_fp8 else EP_QUANT_NONE
         _lib.ep_peer_dispatch_dedup(x, topk_idx, topk_weights, E, W, quant, lay, dst, self.tables,
                                     self.workspace)
-        self._barrier()  # every rank's rows have landed in their owners' buffers
         Rr = int(totals[r])
         per_source = counts[:, r:r + 1]
         send = counts[r].to("cpu").tolist()
@@ -394,7 +403,23 @@ class EpGroup:
         return recv_x, ri, rw, per_source, ctx
 
     # ------------------------------------------------------------ low latency --
-    def low_latency_dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor):
+    def _deliver(self, result, return_recv_hook: bool):
+        """The receive side of a peer dispatch: a barrier after which every rank's
+        rows have landed in their owners' buffers, now or when the hook is called."""
+        if not return_recv_hook:
+            self._barrier()
+            return result
+        done = []
+
+        def hook() -> None:
+            if not done:  # once
+                done.append(True)
+                self._barrier()
+
+        return result + (hook,)
+
+    def low_latency_dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor,
+                             return_recv_hook: bool = False):
         """Peer transport (constructed with ll_max_tokens): DeepEP's low-latency
         dispatch across the ranks.  Every rank's FP8 rows go straight into padded
         per-expert blocks of their owners' buffers, with no count exchange first.
@@ -402,7 +427,7 @@ class EpGroup:
         Returns ``((recv_x, recv_scales), recv_count, ctx)``: recv_x E4M3
         [E/W, W*cap, H] and recv_scales [E/W, W*cap, H/128] (rows [s*cap, s*cap + n)
         of local expert el come from rank s, n = recv_count[el, s]), recv_count int32
-        [E/W, W]."""
+        [E/W, W]; with return_recv_hook, a ``hook`` as for :meth:`dispatch`."""
         ll = self._peer["ll"] if self._peer is not None else None
         if ll is None:
             raise RuntimeError("low-latency calls need the peer transport and ll_max_tokens")
@@ -415,13 +440,12 @@ class EpGroup:
         t = ll["tables"]
         _lib.ep_peer_low_latency_dispatch(x, topk_idx, cap, E, W, self.rank, t["x"], t["scales"],
                                           t["count"], h, self.workspace)
-        self._barrier()  # every rank's rows and counts have landed
         rows = epp * W * cap
         q = self._view("x", torch.uint8, (epp, W * cap, H), ll).view(torch.float8_e4m3fn)
         s = self._view("scales", torch.float32, (epp, W * cap, H // 128), ll)
         count = self._view("count", torch.int32, (epp, W), ll)
         ctx = EpContext(h, [], [], T, H, topk_idx=topk_idx, recv_rows=rows, order="low_latency")
-        return (q, s), count, ctx
+        return self._deliver(((q, s), count, ctx), return_recv_hook)
 
     def ll_expert_out_buffer(self) -> torch.Tensor:
         """BF16 [E/W, W*cap, H]: where a rank's low-latency expert outputs go (row i of

@@ -331,9 +331,16 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
         x = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16)
         idx = torch.from_numpy(w.topk_idx)
         wts = torch.from_numpy(w.topk_weights)
-        for quant in ("fp8", "none", "fp8"):  # the buffers are reused across steps
-            recv_x, ri, rw, per_expert, ctx = g.dispatch(x, idx, wts, use_fp8=quant == "fp8")
-            d = oracle.dispatch(x_all, idx_all, w_all, E, world, quant=quant)
+        for step, quant in enumerate(("fp8", "none", "fp8")):  # the buffers are reused
+            if step == 2:  # through the receive hook: the oracle runs while rows travel
+                recv_x, ri, rw, per_expert, ctx, hook = g.dispatch(
+                    x, idx, wts, use_fp8=quant == "fp8", return_recv_hook=True)
+                d = oracle.dispatch(x_all, idx_all, w_all, E, world, quant=quant)
+                hook()
+                hook()  # a second call is a no-op
+            else:
+                recv_x, ri, rw, per_expert, ctx = g.dispatch(x, idx, wts, use_fp8=quant == "fp8")
+                d = oracle.dispatch(x_all, idx_all, w_all, E, world, quant=quant)
             lo, hi = d["expert_offset"][rank * epp], d["expert_offset"][(rank + 1) * epp]
             if quant == "fp8":
                 got = recv_x[0].view(torch.uint8).numpy()
@@ -382,8 +389,12 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
             y_all, _ = oracle.combine_dedup(po_all, d["prow_of"])
             assert np.array_equal(y.view(torch.int16).numpy().view(np.uint16),
                                   y_all[t0:t0 + tokens[rank]]), "dedup " + quant
-        for _ in range(2):  # low-latency rows: padded per-expert blocks, one per source rank
-            (q, s), count, ctx = g.low_latency_dispatch(x, idx)
+        for step in range(2):  # low-latency rows: padded per-expert blocks, one per source
+            if step == 0:
+                (q, s), count, ctx, hook = g.low_latency_dispatch(x, idx, return_recv_hook=True)
+                hook()
+            else:
+                (q, s), count, ctx = g.low_latency_dispatch(x, idx)
             got_q, got_s, got_c = q.view(torch.uint8).numpy(), s.numpy(), count.numpy()
             for src, l in enumerate(loads):
                 o = oracle.ll_dispatch(l.x, l.topk_idx, E, cap)
