@@ -25,7 +25,7 @@ a no-op callable: on one GPU there is no receive phase to defer.
 """
 from __future__ import annotations
 
-from typing import Optional, Tuple, Union
+from typing import Optional, Union
 
 import torch
 

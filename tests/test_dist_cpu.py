@@ -7,7 +7,6 @@ reduction of the device times, which these tests exercise with gloo.
 import os
 import socket
 
-import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp

@@ -9,7 +9,6 @@ has already run every other test.  It also passes when run alone.
 """
 import ctypes
 
-import numpy as np
 import pytest
 
 from workloads import make_custom, make_workload
