@@ -476,7 +476,8 @@ class EpGroup:
         weighted sum of each token's expert outputs."""
         y = torch.empty((ctx.num_tokens, ctx.hidden), dtype=torch.bfloat16, device=self.device)
         if self.transport == "peer":
-            if ctx.recv_rows and expert_out.data_ptr() != self.expert_out_buffer(ctx).data_ptr():
+            # checked on every rank alike (also with no rows), before the barrier
+            if expert_out.data_ptr() != self.expert_out_buffer(ctx).data_ptr():
                 raise ValueError("write the expert outputs into expert_out_buffer(ctx)")
             self._barrier()  # every rank's expert outputs are complete
             if ctx.dedup:  # partition outputs are already weighted: a plain sum

@@ -416,6 +416,30 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
                     y_ref, _ = oracle.ll_combine(eo, o["ll_row_of"], w.topk_weights)
             y = g.low_latency_combine(g.ll_expert_out_buffer(), ctx, wts)
             assert np.array_equal(y.view(torch.int16).numpy().view(np.uint16), y_ref), "ll"
+
+        # error paths: each raises on every rank alike, and the group stays usable
+        def raises(exc, fn):
+            try:
+                fn()
+            except exc:
+                return True
+            return False
+
+        assert raises(ValueError, lambda: g.dispatch(x[:, :128].contiguous(), idx, wts))  # hidden
+        recv_x, ri, rw, per_expert, ctx = g.dispatch(x, idx, wts)
+        assert raises(ValueError, lambda: g.combine(torch.empty_like(g.expert_out_buffer(ctx)),
+                                                    ctx, wts))
+        g.combine(g.expert_out_buffer(ctx), ctx, wts)  # the step completes normally
+        small = ep_group.EpGroup(E, device="cpu", transport="peer", hidden=H, max_tokens=128,
+                                 capacity=8)
+        try:
+            assert raises(ValueError, lambda: small.dispatch(x, idx, wts))  # over capacity
+            assert raises(ValueError, lambda: small.dispatch(x, idx, wts, dedup=True))
+            assert raises(RuntimeError, lambda: small.low_latency_dispatch(x, idx))
+        finally:
+            small.close()
+        (q, s), count, ctx = g.low_latency_dispatch(x, idx)  # still usable
+        g.low_latency_combine(g.ll_expert_out_buffer(), ctx, wts)
         status = "ok"
     finally:
         try:
