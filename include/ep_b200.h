@@ -503,6 +503,7 @@ EP_API ep_status ep_peer_combine(int64_t num_tokens, int64_t hidden, int32_t num
  *      rank) into counts[W, W];
  *   3. ep_peer_plan(world = W, num_experts = W, counts, handle.expert_offset, ...):
  *      dst_offset[W], this rank's recv_count[1] and recv_offset[2];
+ *   4. as above (the buffers this step overwrites are free);
  *   5. ep_peer_dispatch_dedup; 6. barrier, each rank computes its partition outputs
  *      (one BF16 row per received row: the weighted sum over its listed experts);
  *   7. barrier, ep_peer_combine_dedup.
