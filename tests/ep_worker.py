@@ -190,3 +190,106 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
             with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
                 f.write(status)
             dist.destroy_process_group()
+
+
+def run_peer_multi(rank: int, world: int, port: int, out_dir: str) -> None:
+    """One process per GPU, NCCL: EpGroup(transport="peer") across real GPUs (IPC
+    mappings, stores and loads over NVLink).  Per-expert, deduplicated and
+    low-latency rows, each checked bit for bit against the oracle's one-GPU result on
+    all ranks' tokens concatenated in rank order."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for p in (root, os.path.join(root, "tests")):
+        if p not in sys.path:
+            sys.path.insert(0, p)
+    os.environ["NCCL_NVLS_ENABLE"] = "0"
+    import torch
+    import torch.distributed as dist
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.cuda.set_device(rank)
+    dist.init_process_group("nccl", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", rank))
+    status = "failed"
+    g = None
+    try:
+        import combine_get_dispatch_05_b200 as ep
+        import oracle
+        from gpu_path import bf16_to_u16, dev_u16_as_bf16
+        from workloads import make_custom
+
+        E, H, K, cap = 8 * world, 1024, 6, 96
+        epp = E // world
+        tokens = [96 - 17 * (r % 3) for r in range(world)]
+        loads = [make_custom(tokens[r], H, K, E, world, seed=160 + r, mask_frac=0.05)
+                 for r in range(world)]
+        x_all = np.concatenate([l.x for l in loads])
+        idx_all = np.concatenate([l.topk_idx for l in loads])
+        w_all = np.concatenate([l.topk_weights for l in loads])
+        t0 = sum(tokens[:rank])
+        w = loads[rank]
+        g = ep.EpGroup(E, transport="peer", hidden=H, max_tokens=128, ll_max_tokens=cap)
+        x = dev_u16_as_bf16(w.x)
+        idx = torch.from_numpy(w.topk_idx).cuda()
+        wts = torch.from_numpy(w.topk_weights).cuda()
+
+        # per-expert rows
+        (q, s), ri, rw, per_expert, ctx = g.dispatch(x, idx, wts)
+        d = oracle.dispatch(x_all, idx_all, w_all, E, world)
+        lo, hi = d["expert_offset"][rank * epp], d["expert_offset"][(rank + 1) * epp]
+        assert np.array_equal(q.view(torch.uint8).cpu().numpy(), d["recv_x"][lo:hi])
+        assert np.array_equal(s.cpu().numpy().view(np.uint32),
+                              d["recv_scales"][lo:hi].view(np.uint32))
+        assert np.array_equal(ri.cpu().numpy(), d["recv_topk_idx"][lo:hi])
+        eo_all = oracle.identity_expert(d["recv_x"], d["recv_scales"])
+        out = g.expert_out_buffer(ctx)
+        out.copy_(dev_u16_as_bf16(eo_all[lo:hi]))
+        y = g.combine(out, ctx, wts)
+        y_all, _ = oracle.combine(eo_all, d["row_of"], w_all)
+        assert np.array_equal(bf16_to_u16(y), y_all[t0:t0 + tokens[rank]])
+
+        # deduplicated rows
+        (q, s), ri, rw, per_source, ctx = g.dispatch(x, idx, wts, dedup=True)
+        d = oracle.dispatch_dedup(x_all, idx_all, w_all, E, world)
+        lo, hi = d["part_offset"][rank], d["part_offset"][rank + 1]
+        assert np.array_equal(q.view(torch.uint8).cpu().numpy(), d["recv_x"][lo:hi])
+        assert np.array_equal(ri.cpu().numpy(), d["recv_topk_idx"][lo:hi])
+        po_all = oracle.partition_identity(d["recv_x"], d["recv_scales"], d["recv_topk_idx"],
+                                           d["recv_topk_weights"])
+        out = g.expert_out_buffer(ctx)
+        out.copy_(dev_u16_as_bf16(po_all[lo:hi]))
+        y = g.combine(out, ctx, wts)
+        y_all, _ = oracle.combine_dedup(po_all, d["prow_of"])
+        assert np.array_equal(bf16_to_u16(y), y_all[t0:t0 + tokens[rank]])
+
+        # low-latency rows
+        (q, s), count, ctx = g.low_latency_dispatch(x, idx)
+        gq, gc = q.view(torch.uint8).cpu().numpy(), count.cpu().numpy()
+        buf = g.ll_expert_out_buffer()
+        for src, l in enumerate(loads):
+            o = oracle.ll_dispatch(l.x, l.topk_idx, E, cap)
+            for el in range(epp):
+                e = rank * epp + el
+                n = int(o["recv_expert_count"][e])
+                assert gc[el, src] == n
+                assert np.array_equal(gq[el, src * cap:src * cap + n], o["recv_x"][e, :n])
+            eo = oracle.identity_expert(o["recv_x"].reshape(E * cap, H),
+                                        o["recv_scales"].reshape(E * cap, H // 128))
+            eo = eo.reshape(E, cap, H)
+            buf[:, src * cap:(src + 1) * cap].copy_(
+                dev_u16_as_bf16(eo[rank * epp:(rank + 1) * epp].reshape(-1, H)).view(epp, cap, H))
+            if src == rank:
+                y_ref, _ = oracle.ll_combine(eo, o["ll_row_of"], w.topk_weights)
+        y = g.low_latency_combine(buf, ctx, wts)
+        assert np.array_equal(bf16_to_u16(y), y_ref)
+        assert ep.ep_read_status(g.workspace) == 0
+        status = "ok"
+    finally:
+        try:
+            if g is not None:
+                g.close()
+        finally:
+            with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
+                f.write(status)
+            dist.destroy_process_group()

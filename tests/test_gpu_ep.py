@@ -56,3 +56,27 @@ def test_ep_group_peer_transport_one_rank(tmp_path):
         p.join()
     assert p.exitcode == 0
     assert (tmp_path / "rank0.txt").read_text() == "ok"
+
+
+@pytest.mark.skipif(not torch.cuda.is_available() or torch.cuda.device_count() < 2,
+                    reason="needs two or more GPUs (one process per GPU)")
+def test_ep_group_peer_transport_across_gpus(tmp_path):
+    import ep_worker
+
+    world = min(torch.cuda.device_count(), 4)
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=ep_worker.run_peer_multi, args=(r, world, port, str(tmp_path)))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+    for p in procs:
+        if p.is_alive():  # only our own children
+            p.kill()
+            p.join()
+    results = [(tmp_path / f"rank{r}.txt").read_text() if (tmp_path / f"rank{r}.txt").exists()
+               else "missing" for r in range(world)]
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    assert results == ["ok"] * world, results
