@@ -31,6 +31,15 @@ and maps every other rank's.  Per step:
   caller writes one BF16 row per received row (its experts' weighted sum) into
   ``expert_out_buffer`` and combine sums the ranks' rows per token.
 
+  ``low_latency_dispatch`` / ``low_latency_combine`` (constructed with
+  ``ll_max_tokens``) use DeepEP's low-latency layout: per local expert, W blocks of
+  ``ll_max_tokens`` rows, one per source rank, so the source writes each row and its
+  counts straight to the owner with no exchange before the dispatch.
+
+  ``return_recv_hook=True`` returns from a peer dispatch as soon as the rows are on
+  their way, with a hook appended: the receive barrier, called when the rows are
+  needed (work enqueued in between overlaps the transfer).
+
 ``transport="nccl"`` (any backend): the one-GPU dispatch with P = W fills a send
 buffer whose rank-p rows are one contiguous slice; the rows, scales, local ids and
 weights go to their owners with ``all_to_all_single`` (through host memory when the
