@@ -340,3 +340,22 @@ def test_peer_low_latency_host_checks(ep):
     assert cmb(eo=None) == 1
     assert cmb(y=f + 2) == 1
     assert cmb(T=0, eo=None, y=None) == 0
+
+
+def test_plain_c_client(ep, tmp_path):
+    """The header compiles as C11 (warnings as errors), a C program links the library
+    and its host-side checks answer the same as through the binding."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(ep.LIB_PATH)
+    exe = tmp_path / "abi_c_check"
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "abi_c_check.c"), "-L", lib_dir, "-lep_b200",
+                    f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == "ok"
