@@ -8,6 +8,7 @@
 // recv_x, recv_topk_idx, recv_topk_weights, handle).
 //
 // CTA c owns a contiguous chunk of tokens:
+//   0. before waiting for the preceding kernel, prefetch the chunk's ids into L2;
 //   1. load the chunk's expert ids into shared memory (many loads in flight per
 //      thread), histogram them and OR each token's partition bits (shared-memory
 //      atomics: neither depends on the order they land in);
@@ -109,6 +110,20 @@ __device__ __forceinline__ bool grid_wait(const unsigned long long* word, unsign
         if (globaltimer_ns() - t0 > timeout_ns) return false;
     }
     return true;
+}
+
+// L2 prefetch of the ids of tokens [t0, t1), issued before the kernel waits for its
+// predecessor: a prefetch has no result, so it may run before the producer of
+// topk_idx is done (that producer's stores reach L2, where the loads after the wait
+// read), and it takes the ids' DRAM latency off the layout's critical path.
+__device__ __forceinline__ void prefetch_ids(const LayoutArgs& a, int64_t t0, int64_t t1) {
+    if (t1 <= t0) return;
+    const int64_t per_tok = a.by_partition ? a.K_src : a.K;
+    const char* src = reinterpret_cast<const char*>(a.topk_idx + t0 * per_tok);
+    const int64_t bytes = (t1 - t0) * per_tok * 8;
+    for (int64_t off = static_cast<int64_t>(threadIdx.x) * 128; off < bytes;
+         off += static_cast<int64_t>(blockDim.x) * 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(src + off));
 }
 
 // The low 8 bits of m as eight 0/1 bytes (bit i -> byte i).
@@ -416,6 +431,7 @@ __device__ __forceinline__ int run_length(int n, int W) {
 
 // The whole batch in one CTA: the chunk's counts are the totals.
 __global__ void __launch_bounds__(kSingleThreads, 1) layout_single_kernel(LayoutArgs a) {
+    prefetch_ids(a, 0, a.T);
     pdl_wait();               // the previous kernel (e.g. the one writing topk_idx) is complete
     pdl_launch_dependents();  // the dispatch kernel may start loading x
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -437,6 +453,10 @@ __global__ void __launch_bounds__(kSingleThreads, 1) layout_single_kernel(Layout
 // ------------------------------------------------------------ grid kernel --
 
 __global__ void __launch_bounds__(kLayoutThreads, 1) layout_kernel(LayoutArgs a) {
+    const int64_t c = blockIdx.x;
+    const int64_t t0 = c * a.chunk_tokens;
+    const int64_t t1 = min(a.T, t0 + a.chunk_tokens);
+    prefetch_ids(a, t0, t1);
     pdl_wait();               // the previous kernel (e.g. the one writing topk_idx) is complete
     pdl_launch_dependents();  // the dispatch kernel may start loading x
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -444,9 +464,6 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_kernel(LayoutArgs a)
     const int E = a.E, P = a.P;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    const int64_t c = blockIdx.x;
-    const int64_t t0 = c * a.chunk_tokens;
-    const int64_t t1 = min(a.T, t0 + a.chunk_tokens);
     const int n = t1 > t0 ? static_cast<int>((t1 - t0) * a.K) : 0;
 
     count_chunk(a, s, t0, t1, n);
