@@ -21,16 +21,21 @@ DeviceInfo g_info[kMaxDevices];
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+ep_status check_hidden(int64_t H, bool fp8) {
+    if (H <= 0 || H > 16384) return EP_ERR_SHAPE;
+    if (fp8 ? (H % 128 != 0) : (H % 8 != 0)) return EP_ERR_SHAPE;
+    return EP_OK;
+}
+
+inline ep_status cuda_status(cudaError_t e) { return e == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
+
+}  // namespace
+
+// Argument checks shared by every layout entry point (ep_internal.h).
 ep_status check_routing(int64_t T, int32_t K, int32_t E, int32_t P) {
     if (T < 0 || K < 1 || K > 32 || E < 1 || E > 4096 || P < 1 || P > 64 || E % P != 0)
         return EP_ERR_SHAPE;
     if (T * static_cast<int64_t>(K) >= (int64_t(1) << 31)) return EP_ERR_SHAPE;
-    return EP_OK;
-}
-
-ep_status check_hidden(int64_t H, bool fp8) {
-    if (H <= 0 || H > 16384) return EP_ERR_SHAPE;
-    if (fp8 ? (H % 128 != 0) : (H % 8 != 0)) return EP_ERR_SHAPE;
     return EP_OK;
 }
 
@@ -43,16 +48,12 @@ ep_status check_layout_ptrs(const ep_layout* lay, int64_t T) {
     return EP_OK;
 }
 
-inline ep_status cuda_status(cudaError_t e) { return e == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
-
 // EP_ERR_SHAPE if the batch is too large for the layout kernels.
 ep_status check_layout_size(int64_t T, int32_t K, int32_t E, int32_t P, bool by_partition) {
     bool fits = true;
     if (layout_fits(T, K, E, P, by_partition, &fits) != cudaSuccess) return EP_ERR_CUDA;
     return fits ? EP_OK : EP_ERR_SHAPE;
 }
-
-}  // namespace
 
 cudaError_t device_info(DeviceInfo* out) {
     int dev = 0;

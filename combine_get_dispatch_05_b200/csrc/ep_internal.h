@@ -18,6 +18,15 @@ struct DeviceInfo {
 };
 cudaError_t device_info(DeviceInfo* out);
 
+// Host-side argument checks of the layout entry points (the workspace and the
+// no-workspace forms validate alike).  check_routing: sizes in range
+// (EP_ERR_SHAPE); check_layout_ptrs: the arrays a batch of T tokens needs are set
+// (EP_ERR_INVALID_ARG); check_layout_size: the batch fits the layout kernel's
+// shared memory (EP_ERR_SHAPE; EP_ERR_CUDA if the device cannot be queried).
+ep_status check_routing(int64_t T, int32_t K, int32_t E, int32_t P);
+ep_status check_layout_ptrs(const ep_layout* lay, int64_t T);
+ep_status check_layout_size(int64_t T, int32_t K, int32_t E, int32_t P, bool by_partition);
+
 // Upper bound on the layout kernel's CTAs (chunks) for a batch of num_tokens.
 int64_t max_layout_chunks(int64_t num_tokens);
 

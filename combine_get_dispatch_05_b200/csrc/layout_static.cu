@@ -6,7 +6,7 @@
 // whose enqueue step must not allocate, or a latency-critical path where the
 // implicit device synchronisation of cudaMalloc would stall other streams.  This
 // entry point gives them the same layout as ep_get_dispatch_layout, with its
-// scratch (status word, grid-barrier words, per-chunk expert and partition counts) in
+// scratch (status word, grid-barrier word, per-chunk expert and partition counts) in
 // a fixed array compiled into the library instead of a workspace.
 //
 // The array below is EP_STATIC_SCRATCH_BYTES (1 MiB) per GPU; every GPU that
@@ -15,10 +15,11 @@
 // streams, or different host threads on one device) race; calls in one stream
 // are ordered and safe.  Nothing here allocates: no cudaMalloc, no cudaFree, no
 // allocating library routine.
+#include <cuda.h>  // CUcontext / CUresult types only: the driver is reached through
+                   // the runtime's entry-point query, not linked
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include <atomic>
 #include <mutex>
 
 #include "ep_b200.h"
@@ -31,30 +32,61 @@ namespace {
 static __device__ __align__(256) uint8_t g_layout_scratch[EP_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxStaticDevices = 64;
-std::mutex g_setup_mutex;
-std::atomic<int> g_ready[kMaxStaticDevices];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+std::mutex g_mutex;  // guards everything below
+bool g_have_fns = false;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+unsigned long long g_ctx_id[kMaxStaticDevices];  // context the cached address belongs to (0: none)
 void* g_scratch_ptr[kMaxStaticDevices];
 
-// Device address of g_layout_scratch on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once per
-// device with that device current, and cached.
+// Unique id of the calling thread's current context, 0 if there is none yet.
+cudaError_t current_context_id(unsigned long long* id) {
+    *id = 0;
+    if (!g_have_fns) {
+        cudaDriverEntryPointQueryResult q1 = cudaDriverEntryPointSymbolNotFound, q2 = q1;
+        cudaError_t err = cudaGetDriverEntryPointByVersion(
+            "cuCtxGetCurrent", reinterpret_cast<void**>(&g_ctx_get_current), 12000,
+            cudaEnableDefault, &q1);
+        if (err != cudaSuccess) return err;
+        err = cudaGetDriverEntryPointByVersion("cuCtxGetId", reinterpret_cast<void**>(&g_ctx_get_id),
+                                               12000, cudaEnableDefault, &q2);
+        if (err != cudaSuccess) return err;
+        if (q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess ||
+            !g_ctx_get_current || !g_ctx_get_id)
+            return cudaErrorNotSupported;
+        g_have_fns = true;
+    }
+    CUcontext ctx = nullptr;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
+    if (ctx == nullptr) return cudaSuccess;
+    return g_ctx_get_id(ctx, id) == CUDA_SUCCESS ? cudaSuccess : cudaErrorUnknown;
+}
+
+// Device address of g_layout_scratch in the current context.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up with the
+// device current and cached together with the id of the context it belongs to;
+// a different current context (a device reset re-creates it, and the array may
+// move) makes the next call look it up again.
 cudaError_t scratch_address(void** out) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev < 0 || dev >= kMaxStaticDevices) return cudaErrorInvalidDevice;
-    if (g_ready[dev].load(std::memory_order_acquire)) {
-        *out = g_scratch_ptr[dev];
-        return cudaSuccess;
-    }
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_ready[dev].load(std::memory_order_relaxed)) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    unsigned long long id = 0;
+    if ((err = current_context_id(&id)) != cudaSuccess) return err;
+    if (id == 0 || g_ctx_id[dev] != id) {
         void* ptr = nullptr;
-        err = cudaGetSymbolAddress(&ptr, g_layout_scratch);
+        err = cudaGetSymbolAddress(&ptr, g_layout_scratch);  // makes the context current
         if (err != cudaSuccess) return err;
         if (ptr == nullptr) return cudaErrorInvalidSymbol;
+        if ((err = current_context_id(&id)) != cudaSuccess) return err;
         g_scratch_ptr[dev] = ptr;
-        g_ready[dev].store(1, std::memory_order_release);
+        g_ctx_id[dev] = id;
     }
     *out = g_scratch_ptr[dev];
     return cudaSuccess;
@@ -69,25 +101,16 @@ extern "C" ep_status ep_get_dispatch_layout_static(int64_t num_tokens, int32_t n
                                                    int32_t num_experts, int32_t num_partitions,
                                                    const int64_t* topk_idx,
                                                    const ep_layout* layout, void* stream) {
-    if (num_tokens < 0 || num_topk < 1 || num_topk > 32 || num_experts < 1 ||
-        num_experts > 4096 || num_partitions < 1 || num_partitions > 64 ||
-        num_experts % num_partitions != 0 ||
-        num_tokens * static_cast<int64_t>(num_topk) >= (int64_t(1) << 31))
-        return EP_ERR_SHAPE;
-    if (!layout || !layout->num_tokens_per_expert || !layout->num_tokens_per_partition ||
-        !layout->expert_offset || !layout->num_recv)
-        return EP_ERR_INVALID_ARG;
-    if (num_tokens > 0 &&
-        (!topk_idx || !layout->is_token_in_partition || !layout->row_of || !layout->src_of))
-        return EP_ERR_INVALID_ARG;
+    // the same checks as ep_get_dispatch_layout, in the same order
+    ep_status st = check_routing(num_tokens, num_topk, num_experts, num_partitions);
+    if (st != EP_OK) return st;
+    if ((st = check_layout_ptrs(layout, num_tokens)) != EP_OK) return st;
+    if (num_tokens > 0 && !topk_idx) return EP_ERR_INVALID_ARG;
     // the batch must fit the built-in scratch
     if (ep_workspace_bytes(num_tokens, num_experts, num_partitions) > EP_STATIC_SCRATCH_BYTES)
         return EP_ERR_WORKSPACE;
-
-    bool fits = true;
-    if (layout_fits(num_tokens, num_topk, num_experts, num_partitions, false, &fits) != cudaSuccess)
-        return EP_ERR_CUDA;
-    if (!fits) return EP_ERR_SHAPE;
+    if ((st = check_layout_size(num_tokens, num_topk, num_experts, num_partitions, false)) != EP_OK)
+        return st;
     void* scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return EP_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -155,8 +155,8 @@ EP_API const char* ep_status_string(int32_t status);
 
 /* Bytes of device workspace the calls need for a batch of num_tokens tokens
  * (status word, grid-barrier word, the dispatch kernels' token ticket counter,
- * per-chunk expert counts).  The same workspace serves every entry point for
- * batches up to that size. */
+ * per-chunk expert and partition counts).  The same workspace serves every entry
+ * point for batches up to that size. */
 EP_API size_t ep_workspace_bytes(int64_t num_tokens, int32_t num_experts, int32_t num_partitions);
 
 /* Zero a workspace (once, after allocating it) on `stream`.  Every call leaves
@@ -175,6 +175,14 @@ EP_API ep_status ep_read_status(void* workspace, size_t workspace_bytes, void* s
  * arrays written).  Per-expert counts, per-partition distinct-token counts and
  * flags, expert offsets, and the stable row of every (t, k).  An id outside
  * [-1, E) is treated as masked and sets EP_DEV_INDEX_RANGE.
+ * Source: the `handle` that dispatch returns and combine takes back
+ * (deepseek.csdn.net/67bd3eb22e30c863900615cc, "使用示例": dispatch(x,
+ * topk_idx, topk_weights, num_experts) -> recv_x, recv_topk_idx,
+ * recv_topk_weights, handle, event).  The pages name the handle but not its
+ * contents; what it holds here -- per-expert and per-partition counts, a
+ * warp-ranked prefix scan into expert offsets and a stable slot per (t, k) by
+ * token index -- is this library's reading of that handle, the layout a
+ * DeepEP-style dispatch needs before it can place any row.
  */
 EP_API ep_status ep_get_dispatch_layout(int64_t num_tokens, int32_t num_topk, int32_t num_experts,
                                  int32_t num_partitions, const int64_t* topk_idx,
@@ -203,8 +211,15 @@ EP_API ep_status ep_get_dispatch_layout(int64_t num_tokens, int32_t num_topk, in
  *   - Every call shares the one array and it keeps the last call's contents:
  *     each call clears the part that must start at zero, and calls that overlap
  *     on the GPU (other streams or host threads on the same device) race.
- *   - Ids outside [-1, E) are skipped as masked; this variant has no status word
- *     the caller can read, so they are not reported.
+ *   - Ids outside [-1, E) are skipped as masked.  This variant keeps its status
+ *     word inside the private array, so nothing it would report reaches the
+ *     caller: neither such ids nor a grid barrier that gave up after its bounded
+ *     wait (a layout that then stops early, leaving row_of partly written).
+ *     Callers that must see either use ep_get_dispatch_layout and
+ *     ep_read_status.
+ *   - The cached address belongs to the CUDA context current at the first
+ *     call; it is looked up again whenever the device's current context
+ *     changes (after cudaDeviceReset, for instance).
  */
 EP_API ep_status ep_get_dispatch_layout_static(int64_t num_tokens, int32_t num_topk,
                                                int32_t num_experts, int32_t num_partitions,
@@ -345,8 +360,13 @@ EP_API ep_status ep_low_latency_dispatch(int64_t num_tokens, int64_t hidden, int
                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Low-latency combine: the combine reduce above over
- * expert_out BF16 [E, num_max_tokens, H] addressed by handle->row_of.
+ * Low-latency combine ("DeepSeek 开源周第二弹：DeepEP", "DeepEP 的常规内核和低延迟
+ * 内核": the low-latency kernels serve decode with FP8 dispatch and BF16 result
+ * merge): the combine reduce above, with the same fixed k order and fp32 fmaf
+ * chain, over expert_out BF16 [E, num_max_tokens, H] addressed by
+ * handle->row_of (row e * num_max_tokens + slot).  Only handle->row_of is read;
+ * a row outside [0, E * num_max_tokens) is skipped and sets EP_DEV_INDEX_RANGE.
+ * y: BF16 [T, H].  Errors as for ep_combine.
  */
 EP_API ep_status ep_low_latency_combine(int64_t num_tokens, int64_t hidden, int32_t num_topk,
                                  int32_t num_experts, int32_t num_max_tokens,

@@ -41,10 +41,14 @@ def test_static_layout_matches_workspace_layout_twice(ep):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     stream = torch.cuda.current_stream()
-    # two calls in a row with different batches: the second must not see the
-    # first call's leftovers in the shared scratch
+    # calls in a row with different batches: none may see an earlier call's
+    # leftovers in the shared scratch.  The first and third take the multi-CTA
+    # layout (per-chunk counts and the grid-barrier word live in the scratch; the
+    # third has fewer tokens and other E / P than the first), the second the
+    # one-CTA layout (header only).
     batches = [make_workload("normal", seed=31, num_tokens=1000, hidden=128),
-               make_custom(300, 128, 6, 64, 16, seed=32, mask_frac=0.1)]
+               make_custom(300, 128, 6, 64, 16, seed=32, mask_frac=0.1),
+               make_custom(700, 128, 6, 64, 16, seed=33, mask_frac=0.1)]
     for w in batches:
         T, K, E, P = w.num_tokens, w.num_topk, w.num_experts, w.num_partitions
         idx = torch.from_numpy(w.topk_idx).cuda()
