@@ -5,7 +5,10 @@ times (same calls, same shapes), on sampled tokens the oracle computes one by on
 * dispatch: for 48 sampled tokens, every destination row's E4M3 bytes and scale
   bits (or BF16 bits) against the oracle's quantisation of that token's row;
 * combine (identity experts): for the same tokens, y bit for bit against the
-  oracle's fmaf chain over that token's K dequantised rows.
+  oracle's fmaf chain over that token's K dequantised rows;
+* combine on random expert outputs (every row different, the workload's
+  weights): sampled tokens of the normal and stress batches, and every token of
+  the 128-token low-latency batch, bit for bit against the oracle.
 """
 import numpy as np
 import pytest
@@ -106,3 +109,78 @@ def test_layout_many_chunks_and_rank_rounds(ep):
         assert np.array_equal(lay.num_tokens_per_partition.cpu().numpy(),
                               want["num_tokens_per_partition"])
     assert ep.ep_read_status(ws) == 0
+
+
+# ---- combine on random expert outputs, at the benchmark's launch geometry ---------
+
+def _random_bf16(shape, seed):
+    """Seeded N(0, 1) rows drawn on the device by torch (an input, like x)."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    return torch.randn(shape, generator=g, device="cuda", dtype=torch.float32).to(torch.bfloat16)
+
+
+def _oracle_y(eo_rows: torch.Tensor, row_of: np.ndarray, weights: np.ndarray, tokens):
+    """The oracle's combine of `tokens`, from the rows their slots name (gathered from
+    the device tensor eo_rows by torch and brought to the host)."""
+    ro = row_of[tokens]
+    used = np.unique(ro[ro >= 0])
+    rows = bf16_to_u16(eo_rows[torch.from_numpy(used).long().cuda()]) if used.size else \
+        np.zeros((1, eo_rows.shape[1]), np.uint16)
+    local = np.where(ro >= 0, np.searchsorted(used, np.where(ro >= 0, ro, 0)), -1).astype(np.int32)
+    y, st = oracle.combine(rows, local, weights[tokens])
+    assert st == 0
+    return y
+
+
+@pytest.mark.parametrize("name", ["normal", "stress"])
+def test_full_size_combine_random_rows_sampled(ep, name):
+    # every row of every token differs, so a slip in pairing a row with its weight
+    # at the benchmark's geometry (persistent CTAs striding over the tokens with the
+    # next token's rows prefetched) changes y
+    w = make_workload(name, seed=0)
+    T, H, K = w.num_tokens, w.hidden, w.num_topk
+    lay, _, _, _ = _run(ep, w)
+    want = oracle.layout(w.topk_idx, w.num_experts, w.num_partitions)
+    assert np.array_equal(lay.row_of.cpu().numpy(), want["row_of"])
+    R = int(want["num_recv"][0])
+    eo = _random_bf16((R, H), seed=1000 + T)
+    wts = torch.from_numpy(w.topk_weights).cuda()
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(ep.ep_workspace_bytes(T, w.num_experts, w.num_partitions), dtype=torch.uint8,
+                     device="cuda")
+    ep.ep_workspace_init(ws)
+    ep.ep_combine(eo, lay, wts, y, ws)
+    torch.cuda.synchronize()
+    assert ep.ep_read_status(ws) == 0
+    rng = np.random.default_rng(7)
+    sample = np.unique(np.concatenate([[0, 1, T // 2, T - 2, T - 1], rng.choice(T, 48, replace=False)]))
+    y_ref = _oracle_y(eo, want["row_of"], w.topk_weights, sample)
+    got = bf16_to_u16(y[torch.from_numpy(sample).long().cuda()])
+    assert np.array_equal(got, y_ref)
+
+
+def test_ll_full_batch_combine_random_rows(ep):
+    # the whole 128-token decode batch at hidden 7168 into capacity 128 per expert,
+    # every expert output row random: all of y against the oracle
+    w = make_workload("ll", seed=0)
+    T, H, K, E, cap = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_max_tokens
+    x = torch.from_numpy(w.x.view(np.int16)).cuda().view(torch.bfloat16)
+    idx = torch.from_numpy(w.topk_idx).cuda()
+    recv_x = torch.empty((E, cap, H), dtype=torch.uint8, device="cuda")
+    recv_s = torch.empty((E, cap, H // 128), dtype=torch.float32, device="cuda")
+    cnt = torch.empty(E, dtype=torch.int32, device="cuda")
+    handle = ep.LowLatencyHandle.empty(T, K, E, cap, "cuda")
+    ws = torch.empty(ep.ep_workspace_bytes(T, E, 1), dtype=torch.uint8, device="cuda")
+    ep.ep_workspace_init(ws)
+    ep.ep_low_latency_dispatch(x, idx, cap, E, recv_x, recv_s, cnt, handle, ws)
+    eo = _random_bf16((E, cap, H), seed=2024)
+    wts = torch.from_numpy(w.topk_weights).cuda()
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    ep.ep_low_latency_combine(eo, handle, wts, y, ws)
+    torch.cuda.synchronize()
+    assert ep.ep_read_status(ws) == 0
+    want = oracle.ll_dispatch(w.x, w.topk_idx, E, cap)
+    assert np.array_equal(handle.row_of.cpu().numpy(), want["ll_row_of"])
+    y_ref = _oracle_y(eo.view(E * cap, H), want["ll_row_of"], w.topk_weights, np.arange(T))
+    assert np.array_equal(bf16_to_u16(y), y_ref)
