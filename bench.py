@@ -18,7 +18,8 @@ to back: every step reads 529 MB of inputs (x and the expert outputs) and
 writes 294 MB, several times the 126 MB L2, so nothing a step reads is still in
 L2 from the step before.  `--l2-flush write|read` instead flushes L2 with a
 256 MiB buffer before every step (outside the events).
-`--impl reference` times the CPU oracle on a bounded sample instead.
+`--impl reference` times the CPU oracle on the host's cores instead (the same
+workload, or a bounded prefix of it when the host is slow).
 """
 from __future__ import annotations
 
@@ -375,7 +376,8 @@ def time_low_latency(ep, w, dev, reps=200, per_graph=20):
             torch.cuda.synchronize()
             walls.append((time.perf_counter() - t0) * 1e6)
         out[name] = {"gpu_us": round(gpu_us, 2), "graph_replay_us": round(replay_us, 2),
-                     "eager_call_us": round(statistics.median(walls), 2)}
+                     "eager_call_us": round(statistics.median(walls), 2),
+                     "tokens_per_s": round(T / (gpu_us * 1e-6))}
     if ep.ep_read_status(ws) != 0:
         raise RuntimeError("device status set in the low-latency run")
     out["config"] = f"{T} tokens x hidden {H}, top-{K} of {E} experts, capacity {cap}, FP8"
@@ -798,9 +800,64 @@ def time_e2e(ep, runner, steps):
     return ms, h2d, d2h
 
 
-def cpu_baseline(w, min_seconds=10.0):
-    """The oracle, as it stands (single-threaded C), on the same batch."""
+def host_cores():
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class ShardedOracle:
+    """The oracle, unchanged, on the host's cores: the layout of the batch runs
+    serially (every row depends on all tokens), then dispatch and combine run over
+    contiguous token shards, one per thread (the oracle is C behind ctypes, which
+    releases the GIL for each call).  A shard's dispatch lays out and quantises its
+    own tokens (the same per-token work as in the whole batch; the rows land in a
+    shard-local buffer); the combine of a shard reads the batch's expert outputs
+    through the batch's layout."""
+
+    def __init__(self, w, threads):
+        import concurrent.futures
+        import oracle
+
+        self.oracle, self.w = oracle, w
+        self.threads = max(1, threads)
+        T = w.num_tokens
+        bounds = [T * i // self.threads for i in range(self.threads + 1)]
+        self.shards = [(a, b) for a, b in zip(bounds[:-1], bounds[1:]) if b > a]
+        self.pool = concurrent.futures.ThreadPoolExecutor(max_workers=self.threads)
+        d = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, w.num_experts, w.num_partitions,
+                            quant=w.quant)
+        self.R = int(d["num_recv"][0])
+        self.eo = oracle.identity_expert(d["recv_x"], d["recv_scales"], quant=w.quant)
+
+    def one_pass(self):
+        """(layout s, dispatch s, combine s) of one pass over the batch."""
+        o, w = self.oracle, self.w
+        E, P = w.num_experts, w.num_partitions
+        t0 = time.perf_counter()
+        lay = o.layout(w.topk_idx, E, P)
+        t1 = time.perf_counter()
+        list(self.pool.map(lambda ab: o.dispatch(w.x[ab[0]:ab[1]], w.topk_idx[ab[0]:ab[1]],
+                                                 w.topk_weights[ab[0]:ab[1]], E, P,
+                                                 quant=w.quant), self.shards))
+        t2 = time.perf_counter()
+        list(self.pool.map(lambda ab: o.combine(self.eo, lay["row_of"][ab[0]:ab[1]],
+                                                w.topk_weights[ab[0]:ab[1]]), self.shards))
+        t3 = time.perf_counter()
+        return t1 - t0, t2 - t1, t3 - t2
+
+    def close(self):
+        self.pool.shutdown()
+
+
+def cpu_baseline(w, min_seconds=10.0, configs=True):
+    """The oracle, as it stands, on the same batch: single-threaded C (the reported
+    value), then the same work spread over the host's cores, and per-workload
+    layout / dispatch / combine medians of the spread-out form."""
     import oracle
+    from workloads import make_workload
 
     T, H, K, E, P = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
     d = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, E, P, quant=w.quant)
@@ -813,10 +870,90 @@ def cpu_baseline(w, min_seconds=10.0):
         oracle.combine(eo, dd["row_of"], w.topk_weights)
         t += time.perf_counter() - t0
         passes += 1
-    return {"value": round((bd + bc) * passes / t / 1e9, 3), "unit": "GB/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"the full {T}-token batch (layout + dispatch + combine), {passes} passes, "
-                      f"{t:.1f} s, single-threaded C"}
+    cores = host_cores()
+    out = {"value": round((bd + bc) * passes / t / 1e9, 3), "unit": "GB/s", "cores": 1,
+           "kind": "oracle", "host_cores": cores,
+           "sample": f"the full {T}-token batch (layout + dispatch + combine), {passes} passes, "
+                     f"{t:.1f} s, single-threaded C"}
+    so = ShardedOracle(w, cores)
+    try:
+        so.one_pass()
+        runs = [so.one_pass() for _ in range(5)]
+    finally:
+        so.close()
+    tt = statistics.median([sum(r) for r in runs])
+    out["threaded"] = {
+        "value": round((bd + bc) / tt / 1e9, 3), "unit": "GB/s", "cores": so.threads,
+        "ms_per_step": round(tt * 1e3, 2),
+        "sample": f"the full {T}-token batch, median of 5 passes: layout serial, dispatch and "
+                  f"combine over {len(so.shards)} token shards in {so.threads} threads"}
+    if configs:
+        per = {}
+        try:  # the low-latency batch through the oracle's padded layout, one thread
+            wl = make_workload("ll", seed=w.seed)
+            dl = oracle.ll_dispatch(wl.x, wl.topk_idx, wl.num_experts, wl.num_max_tokens)
+            eol = oracle.identity_expert(
+                dl["recv_x"].reshape(-1, wl.hidden),
+                dl["recv_scales"].reshape(-1, wl.hidden // 128)).reshape(
+                    wl.num_experts, wl.num_max_tokens, wl.hidden)
+            rl = []
+            for _ in range(4):
+                t0 = time.perf_counter()
+                oracle.ll_dispatch(wl.x, wl.topk_idx, wl.num_experts, wl.num_max_tokens)
+                t1 = time.perf_counter()
+                oracle.ll_combine(eol, dl["ll_row_of"], wl.topk_weights)
+                rl.append((t1 - t0, time.perf_counter() - t1))
+            dm, cm = (statistics.median(r[i] for r in rl[1:]) for i in range(2))
+            per["ll"] = {"tokens": wl.num_tokens, "dispatch_ms": round(dm * 1e3, 3),
+                         "combine_ms": round(cm * 1e3, 3),
+                         "dispatch_tokens_per_s": round(wl.num_tokens / dm),
+                         "combine_tokens_per_s": round(wl.num_tokens / cm),
+                         "sample": "padded low-latency layout (layout fused into the dispatch), "
+                                   "single-threaded, median of 3 passes"}
+        except Exception as exc:  # report, do not hide
+            per["ll"] = {"error": repr(exc)}
+        for name in ("normal", "skew", "bf16", "stress"):
+            try:
+                n = 4096 if name == "stress" else None  # a bounded sample of the largest batch
+                wx = make_workload(name, seed=w.seed, num_tokens=n)
+                sx = ShardedOracle(wx, cores)
+                try:
+                    sx.one_pass()
+                    rr = [sx.one_pass() for _ in range(3)]
+                finally:
+                    sx.close()
+                lm, dm, cm = (statistics.median(r[i] for r in rr) for i in range(3))
+                per[name] = {"tokens": wx.num_tokens, "layout_ms": round(lm * 1e3, 3),
+                             "dispatch_ms": round(dm * 1e3, 3), "combine_ms": round(cm * 1e3, 3),
+                             "dispatch_tokens_per_s": round(wx.num_tokens / (lm + dm)),
+                             "combine_tokens_per_s": round(wx.num_tokens / cm)}
+                if n is not None:
+                    per[name]["sample"] = f"the stress recipe drawn at {n} tokens"
+            except Exception as exc:  # report, do not hide
+                per[name] = {"error": repr(exc)}
+        out["configs"] = per
+        out["configs_note"] = (f"oracle over {cores} threads (layout serial, dispatch and combine "
+                               "sharded over tokens), medians of 3 passes; dispatch tokens/s "
+                               "includes the layout")
+    return out
+
+
+L2_TEXT = ("inputs larger than L2: each step reads 529 MB (x + expert outputs) and writes "
+           "294 MB, steps back to back, no flush")
+
+
+def workload_config(name, w, R, step_bytes, seed, world, l2_flush="none"):
+    """The `config` object of the JSON line: what the workload is, identical in
+    both arms for the same workload and seed."""
+    return {
+        "workload": WORKLOAD_TEXT[name],
+        "tokens_per_gpu": w.num_tokens, "hidden": w.hidden, "topk": w.num_topk,
+        "experts": w.num_experts, "partitions": w.num_partitions, "recv_rows": R,
+        "bytes_per_step": step_bytes, "seed": seed,
+        "l2": L2_TEXT if l2_flush == "none"
+        else f"flushed before every step by a 256 MiB {l2_flush} (outside the events)",
+        "parallelism": f"replicas x{world} (independent batches, no exchange)",
+    }
 
 
 def make_flush(mode, dev):
@@ -915,25 +1052,19 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": DTYPE_TEXT[runner.fp8],
         "data": "synthetic",
-        "config": {
-            "workload": WORKLOAD_TEXT[args.workload],
-            "tokens_per_gpu": w.num_tokens, "hidden": w.hidden, "topk": w.num_topk,
-            "experts": w.num_experts, "partitions": w.num_partitions, "recv_rows": runner.R,
-            "bytes_per_step": step_bytes, "seed": args.seed,
-            "l2": ("inputs larger than L2: each step reads 529 MB (x + expert outputs) and "
-                   "writes 294 MB, steps back to back, no flush") if args.l2_flush == "none"
-            else f"flushed before every step by a 256 MiB {args.l2_flush} (outside the events)",
-            "launch": "CUDA graphs (dispatch: layout + dispatch kernels, programmatic dependent launch; "
-                      "combine: 1 kernel)" if not args.eager else "eager",
-            "parallelism": f"replicas x{world} (independent batches, no exchange)",
-        },
+        "config": workload_config(args.workload, w, runner.R, step_bytes, args.seed, world,
+                                  args.l2_flush),
+        "launch": "CUDA graphs (dispatch: layout + dispatch kernels, programmatic dependent launch; "
+                  "combine: 1 kernel)" if not args.eager else "eager",
         "breakdown": {
             "dispatch": {"us": round(disp_us, 2), "bytes": runner.bytes_dispatch,
                          "gbs": round(disp_gbs, 1), "frac": round(disp_gbs / peak, 4),
+                         "tokens_per_s": round(w.num_tokens / (disp_us * 1e-6)),
                          "kernels": "layout (cooperative) + dispatch_%s (programmatic dependent "
                                     "launch)" % ("fp8" if runner.fp8 else "bf16")},
             "combine": {"us": round(comb_us, 2), "bytes": runner.bytes_combine,
                         "gbs": round(comb_gbs, 1), "frac": round(comb_gbs / peak, 4),
+                        "tokens_per_s": round(w.num_tokens / (comb_us * 1e-6)),
                         "kernels": "combine"},
         },
         "roofline": {
@@ -988,8 +1119,10 @@ def run_ours(args):
                     "quant": wx.quant, "recv_rows": r.R,
                     "dispatch_us": round(du, 2),
                     "dispatch_gbs": round(r.bytes_dispatch / (du * 1e-6) / 1e9, 1),
+                    "dispatch_tokens_per_s": round(wx.num_tokens / (du * 1e-6)),
                     "combine_us": round(cu, 2),
                     "combine_gbs": round(r.bytes_combine / (cu * 1e-6) / 1e9, 1),
+                    "combine_tokens_per_s": round(wx.num_tokens / (cu * 1e-6)),
                     "status": ep.ep_read_status(r.ws)}
                 del r
                 torch.cuda.empty_cache()
@@ -1001,8 +1134,19 @@ def run_ours(args):
 
 # -------------------------------------------------------- reference arm -----
 
+def token_prefix(w, n):
+    """The first n tokens of a workload (a bounded sample of it)."""
+    import dataclasses
+
+    if n >= w.num_tokens:
+        return w
+    return dataclasses.replace(w, num_tokens=n, x=w.x[:n], topk_idx=w.topk_idx[:n],
+                               topk_weights=w.topk_weights[:n])
+
+
 def run_reference(args):
-    """The CPU oracle as it stands, on bounded samples of the same workload."""
+    """The CPU oracle as it stands, on the host's cores (layout serial, dispatch and
+    combine over token shards), on the same workload or a bounded prefix of it."""
     rank, world, _ = env_rank()
     if rank != 0:
         return
@@ -1012,51 +1156,44 @@ def run_reference(args):
     w = make_workload(args.workload, seed=args.seed)
     T, H, K, E, P = w.num_tokens, w.hidden, w.num_topk, w.num_experts, w.num_partitions
     fp8 = w.quant == "fp8"
-
-    def make_step(n):
-        xs, idxs, wts = w.x[:n], w.topk_idx[:n], w.topk_weights[:n]
-        ds = oracle.dispatch(xs, idxs, wts, E, P, quant=w.quant)
-        eos = oracle.identity_expert(ds["recv_x"], ds.get("recv_scales"), quant=w.quant)
-
-        def step():
-            dx = oracle.dispatch(xs, idxs, wts, E, P, quant=w.quant)
-            oracle.combine(eos, dx["row_of"], wts)
-        return step, int(ds["num_recv"][0])
+    R_full = int(oracle.layout(w.topk_idx, E, P)["num_recv"][0])
+    bd_full, bc_full = algorithmic_bytes(T, H, K, E, P, R_full, fp8)
+    cores = host_cores()
 
     # calibrate seconds per token, then size each step's sample so the whole run
     # stays near two minutes
-    n_cal = 64
-    cal, _ = make_step(n_cal)
-    t0 = time.perf_counter()
-    cal()
-    per_tok = (time.perf_counter() - t0) / n_cal
+    n_cal = min(T, 256)
+    cal = ShardedOracle(token_prefix(w, n_cal), cores)
+    try:
+        cal.one_pass()
+        per_tok = sum(cal.one_pass()) / n_cal
+    finally:
+        cal.close()
     budget = 120.0 / max(1, args.steps + args.warmup)
-    S = int(max(1, min(T, budget / per_tok)))
-    step, R = make_step(S)
-    bd, bc = algorithmic_bytes(S, H, K, E, P, R, fp8)
-
-    for _ in range(args.warmup):
-        step()
-    times = []
-    for _ in range(args.steps):
-        t = time.perf_counter()
-        step()
-        times.append(time.perf_counter() - t)
+    S = int(max(1, min(T, budget / max(per_tok, 1e-12))))
+    so = ShardedOracle(token_prefix(w, S), cores)
+    try:
+        bd, bc = algorithmic_bytes(S, H, K, E, P, so.R, fp8)
+        for _ in range(args.warmup):
+            so.one_pass()
+        times = [sum(so.one_pass()) for _ in range(args.steps)]
+    finally:
+        so.close()
     ms = statistics.mean(times) * 1e3
     value = (bd + bc) / (ms * 1e-3) / 1e9
-    sample = (f"first {S} of {T} tokens of the {args.workload} workload per step (layout + "
-              f"{'FP8' if fp8 else 'BF16'} dispatch + combine), single-threaded C oracle")
+    sample = (f"{'all' if S == T else 'the first'} {S} of {T} tokens of the {args.workload} "
+              f"workload per step: layout serial, {'FP8' if fp8 else 'BF16'} dispatch and "
+              f"combine over {len(so.shards)} token shards in {so.threads} threads (C oracle)")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": DTYPE_TEXT[fp8],
         "data": "synthetic",
-        "config": {"workload": WORKLOAD_TEXT[args.workload], "tokens_per_gpu": T, "hidden": H,
-                   "topk": K, "experts": E, "partitions": P, "seed": args.seed,
-                   "sample_tokens": S},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "config": workload_config(args.workload, w, R_full, bd_full + bc_full, args.seed, world),
+        "sample_tokens": S,
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": so.threads,
+                         "host_cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }), flush=True)

@@ -66,5 +66,13 @@ def test_reference_arm_json_line():
     assert line["steps"] == 3 and line["warmup"] == 3 and line["n_gpus"] == 1
     assert line["value"] > 0 and line["higher_is_better"] is True
     assert line["config"]["workload"].startswith("normal")
+    # the same config object as the GPU arm prints for this workload: what the work is,
+    # not how this arm samples it
+    assert set(line["config"]) == {"workload", "tokens_per_gpu", "hidden", "topk", "experts",
+                                   "partitions", "recv_rows", "bytes_per_step", "seed", "l2",
+                                   "parallelism"}
+    assert line["config"]["tokens_per_gpu"] == 4096 and line["config"]["recv_rows"] == 32768
+    assert 1 <= line["sample_tokens"] <= 4096
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["host_cores"] >= 1
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
