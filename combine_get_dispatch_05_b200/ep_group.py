@@ -51,7 +51,6 @@ rank for each local expert.
 """
 from __future__ import annotations
 
-from dataclasses import dataclass, field
 from typing import List, Optional
 
 import torch
@@ -65,21 +64,55 @@ __all__ = ["EpGroup", "EpContext"]
 _ALIGN = 256
 
 
-@dataclass
 class EpContext:
-    """What combine needs from the dispatch that preceded it."""
+    """What combine needs from the dispatch that preceded it.
 
-    handle: Layout               # the sender-side layout (P = group size)
-    send_counts: List[int]       # rows this rank sent to each rank
-    recv_counts: List[int]       # rows this rank received from each rank
-    num_tokens: int
-    hidden: int
-    # peer transport only
-    topk_idx: Optional[torch.Tensor] = None
-    dst_offset: Optional[torch.Tensor] = None
-    recv_rows: int = 0
-    order: str = field(default="source_major")
-    dedup: bool = False
+    The row counts are lists (and ``recv_rows`` an int) after a dispatch that
+    synchronised with the host; after a peer dispatch with ``sync_sizes=False`` they
+    stay on the device and the first read of ``send_counts``, ``recv_counts`` or
+    ``recv_rows`` copies them to the host (one device synchronisation)."""
+
+    def __init__(self, handle: Layout, send_counts, recv_counts, num_tokens: int, hidden: int,
+                 topk_idx: Optional[torch.Tensor] = None,
+                 dst_offset: Optional[torch.Tensor] = None, recv_rows=0,
+                 order: str = "source_major", dedup: bool = False):
+        self.handle = handle            # the sender-side layout (P = group size)
+        self._send = send_counts        # rows this rank sent to each rank
+        self._recv = recv_counts        # rows this rank received from each rank
+        self.num_tokens = num_tokens
+        self.hidden = hidden
+        self.topk_idx = topk_idx        # peer transport only
+        self.dst_offset = dst_offset
+        self._recv_rows = recv_rows
+        self.order = order
+        self.dedup = dedup
+        # True when the received tensors were cut to the received rows
+        self.sizes_synced = not isinstance(recv_rows, torch.Tensor)
+
+    @staticmethod
+    def _host(v):
+        return v.to("cpu").tolist() if isinstance(v, torch.Tensor) else v
+
+    @property
+    def send_counts(self) -> List[int]:
+        self._send = self._host(self._send)
+        return self._send
+
+    @property
+    def recv_counts(self) -> List[int]:
+        self._recv = self._host(self._recv)
+        return self._recv
+
+    @property
+    def recv_rows(self) -> int:
+        if isinstance(self._recv_rows, torch.Tensor):
+            self._recv_rows = int(self._recv_rows.item())
+        return self._recv_rows
+
+    @property
+    def recv_rows_device(self) -> Optional[torch.Tensor]:
+        """The received row count as a device scalar (a no-sync peer dispatch), else None."""
+        return self._recv_rows if isinstance(self._recv_rows, torch.Tensor) else None
 
 
 class EpGroup:
@@ -197,11 +230,14 @@ class EpGroup:
 
     def expert_out_buffer(self, ctx: EpContext) -> torch.Tensor:
         """Peer transport: the BF16 [recv rows, H] buffer the expert outputs go into
-        (row i answers received row i); the other ranks' combine kernels read it."""
+        (row i answers received row i); the other ranks' combine kernels read it.
+        After a dispatch with sync_sizes=False: all [capacity, H] rows (the first
+        ctx.recv_rows_device of them are read)."""
         if self._peer is None:
             raise RuntimeError("expert_out_buffer belongs to the peer transport")
         cap, H = self._peer["capacity"], self._peer["hidden"]
-        return self._view("expert_out", torch.bfloat16, (cap, H))[:ctx.recv_rows]
+        full = self._view("expert_out", torch.bfloat16, (cap, H))
+        return full[:ctx.recv_rows] if ctx.sizes_synced else full
 
     def close(self) -> None:
         """Unmap the peers' regions and free this rank's (a collective: every rank
@@ -263,7 +299,8 @@ class EpGroup:
 
     # --------------------------------------------------------------- dispatch --
     def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
-                 use_fp8: bool = True, dedup: bool = False, return_recv_hook: bool = False):
+                 use_fp8: bool = True, dedup: bool = False, return_recv_hook: bool = False,
+                 sync_sizes: bool = True):
         """Returns ``(recv_x, recv_local_idx, recv_weights, recv_counts_per_expert, ctx)``.
 
         recv_x: ``(float8_e4m3fn [Rr, H], float32 [Rr, H/128])`` or BF16 ``[Rr, H]``;
@@ -275,6 +312,14 @@ class EpGroup:
         dedup (peer transport): one row per (token, rank); recv_local_idx and
         recv_weights are [Rr, K] lists and the counts are [W, 1] rows per source.
 
+        sync_sizes=False (peer transport): nothing waits on the host.  The counts stay
+        on the device (the all-gather, the plan and the dispatch are all enqueued on
+        the stream), the received tensors are [capacity, ...] views of which the first
+        ``ctx.recv_rows_device`` rows are this step's, and a receiver over capacity is
+        not raised on the host: its rows are dropped by the dispatch kernel and
+        reported as EP_DEV_CAPACITY in the workspace status.  (DeepEP likewise returns
+        exact-size tensors only after a host wait.)
+
         return_recv_hook (peer transport): return as soon as this rank's rows are on
         their way, with a ``hook`` appended to the result; calling it (every rank, a
         collective) waits until every rank's rows have landed.  Work enqueued
@@ -284,6 +329,8 @@ class EpGroup:
         """
         if return_recv_hook and self.transport != "peer":
             raise NotImplementedError("the receive hook belongs to the peer transport")
+        if not sync_sizes and self.transport != "peer":
+            raise NotImplementedError("the all-to-all needs its splits on the host")
         T = x.shape[0]
         if T > self.max_tokens:
             self.max_tokens = T
@@ -291,10 +338,11 @@ class EpGroup:
         if dedup:
             if self.transport != "peer":
                 raise NotImplementedError("deduplicated rows are offered by the peer transport")
-            return self._deliver(self._dispatch_peer_dedup(x, topk_idx, topk_weights, use_fp8),
-                                 return_recv_hook)
+            return self._deliver(
+                self._dispatch_peer_dedup(x, topk_idx, topk_weights, use_fp8, sync_sizes),
+                return_recv_hook)
         if self.transport == "peer":
-            return self._deliver(self._dispatch_peer(x, topk_idx, topk_weights, use_fp8),
+            return self._deliver(self._dispatch_peer(x, topk_idx, topk_weights, use_fp8, sync_sizes),
                                  return_recv_hook)
         return self._dispatch_nccl(x, topk_idx, topk_weights, use_fp8)
 
@@ -332,7 +380,7 @@ class EpGroup:
         recv_x = (recv_q.view(torch.float8_e4m3fn), recv_s) if use_fp8 else recv_q
         return recv_x, recv_i, recv_w, per_expert, ctx
 
-    def _dispatch_peer(self, x, topk_idx, topk_weights, use_fp8):
+    def _dispatch_peer(self, x, topk_idx, topk_weights, use_fp8, sync_sizes=True):
         T, H = x.shape
         K = topk_idx.shape[1]
         W, E, epp, r = self.world, self.num_experts, self.experts_per_rank, self.rank
@@ -343,10 +391,12 @@ class EpGroup:
         lay = Layout.empty(T, K, E, W, dev)
         _lib.ep_get_dispatch_layout(topk_idx, E, W, lay, self.workspace)
         counts = self._all_gather_rows(lay.num_tokens_per_expert)  # [W, E]
-        # every rank reads the same counts: all of them raise, or none
-        totals = counts.view(W, W, epp).sum(dim=(0, 2)).to("cpu").tolist()
-        if max(totals) > cap:
-            raise ValueError(f"a rank would receive {max(totals)} rows; capacity is {cap}")
+        totals = counts.view(W, W, epp).sum(dim=(0, 2))  # rows each rank receives
+        if sync_sizes:
+            # every rank reads the same counts: all of them raise, or none
+            totals = totals.to("cpu").tolist()
+            if max(totals) > cap:
+                raise ValueError(f"a rank would receive {max(totals)} rows; capacity is {cap}")
         dst = torch.empty(E, dtype=torch.int32, device=dev)
         rc = torch.empty(epp, dtype=torch.int32, device=dev)
         ro = torch.empty(epp + 1, dtype=torch.int32, device=dev)
@@ -354,23 +404,26 @@ class EpGroup:
         quant = EP_QUANT_FP8_E4M3_1X128 if use_fp8 else EP_QUANT_NONE
         _lib.ep_peer_dispatch(x, topk_idx, topk_weights, E, W, quant, lay, dst, self.tables,
                               self.workspace)
-        Rr = int(totals[r])
         per_expert = counts[:, r * epp:(r + 1) * epp]
-        send = counts.view(W, W, epp)[r].sum(dim=1).to("cpu").tolist()
-        recv = per_expert.sum(dim=1).to("cpu").tolist()
+        send = counts.view(W, W, epp)[r].sum(dim=1)
+        recv = per_expert.sum(dim=1)
+        Rr = int(totals[r]) if sync_sizes else totals[r]
+        n = Rr if sync_sizes else cap
+        if sync_sizes:
+            send, recv = send.to("cpu").tolist(), recv.to("cpu").tolist()
         ctx = EpContext(lay, send, recv, T, H, topk_idx=topk_idx, dst_offset=dst, recv_rows=Rr,
                         order="expert_major")
-        ri = self._view("recv_topk_idx", torch.int32, (cap,))[:Rr]
-        rw = self._view("recv_topk_weights", torch.float32, (cap,))[:Rr]
+        ri = self._view("recv_topk_idx", torch.int32, (cap,))[:n]
+        rw = self._view("recv_topk_weights", torch.float32, (cap,))[:n]
         if use_fp8:
-            q = self._view("recv_x", torch.uint8, (cap, H))[:Rr]
-            s = self._view("recv_scales", torch.float32, (cap, H // 128))[:Rr]
+            q = self._view("recv_x", torch.uint8, (cap, H))[:n]
+            s = self._view("recv_scales", torch.float32, (cap, H // 128))[:n]
             recv_x = (q.view(torch.float8_e4m3fn), s)
         else:
-            recv_x = self._view("recv_x", torch.bfloat16, (cap, H))[:Rr]
+            recv_x = self._view("recv_x", torch.bfloat16, (cap, H))[:n]
         return recv_x, ri, rw, per_expert, ctx
 
-    def _dispatch_peer_dedup(self, x, topk_idx, topk_weights, use_fp8):
+    def _dispatch_peer_dedup(self, x, topk_idx, topk_weights, use_fp8, sync_sizes=True):
         T, H = x.shape
         K = topk_idx.shape[1]
         W, E, r = self.world, self.num_experts, self.rank
@@ -385,9 +438,11 @@ class EpGroup:
         lay = Layout.empty(T, W, W, W, dev)  # partition-sized handle
         _lib.ep_get_dispatch_layout_dedup(topk_idx, E, W, lay, self.workspace)
         counts = self._all_gather_rows(lay.num_tokens_per_expert)  # [W sources, W owners]
-        totals = counts.sum(dim=0).to("cpu").tolist()
-        if max(totals) > cap:
-            raise ValueError(f"a rank would receive {max(totals)} rows; capacity is {cap}")
+        totals = counts.sum(dim=0)
+        if sync_sizes:
+            totals = totals.to("cpu").tolist()
+            if max(totals) > cap:
+                raise ValueError(f"a rank would receive {max(totals)} rows; capacity is {cap}")
         dst = torch.empty(W, dtype=torch.int32, device=dev)
         rc = torch.empty(1, dtype=torch.int32, device=dev)
         ro = torch.empty(2, dtype=torch.int32, device=dev)
@@ -395,20 +450,22 @@ class EpGroup:
         quant = EP_QUANT_FP8_E4M3_1X128 if use_fp8 else EP_QUANT_NONE
         _lib.ep_peer_dispatch_dedup(x, topk_idx, topk_weights, E, W, quant, lay, dst, self.tables,
                                     self.workspace)
-        Rr = int(totals[r])
         per_source = counts[:, r:r + 1]
-        send = counts[r].to("cpu").tolist()
-        recv = per_source.reshape(-1).to("cpu").tolist()
+        send, recv = counts[r], per_source.reshape(-1)
+        Rr = int(totals[r]) if sync_sizes else totals[r]
+        n = Rr if sync_sizes else cap
+        if sync_sizes:
+            send, recv = send.to("cpu").tolist(), recv.to("cpu").tolist()
         ctx = EpContext(lay, send, recv, T, H, dst_offset=dst, recv_rows=Rr, order="source_major",
                         dedup=True)
-        ri = self._view("recv_topk_idx", torch.int32, (cap, K))[:Rr]
-        rw = self._view("recv_topk_weights", torch.float32, (cap, K))[:Rr]
+        ri = self._view("recv_topk_idx", torch.int32, (cap, K))[:n]
+        rw = self._view("recv_topk_weights", torch.float32, (cap, K))[:n]
         if use_fp8:
-            q = self._view("recv_x", torch.uint8, (cap, H))[:Rr]
-            s = self._view("recv_scales", torch.float32, (cap, H // 128))[:Rr]
+            q = self._view("recv_x", torch.uint8, (cap, H))[:n]
+            s = self._view("recv_scales", torch.float32, (cap, H // 128))[:n]
             recv_x = (q.view(torch.float8_e4m3fn), s)
         else:
-            recv_x = self._view("recv_x", torch.bfloat16, (cap, H))[:Rr]
+            recv_x = self._view("recv_x", torch.bfloat16, (cap, H))[:n]
         return recv_x, ri, rw, per_source, ctx
 
     # ------------------------------------------------------------ low latency --

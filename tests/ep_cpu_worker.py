@@ -363,6 +363,36 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
             y_all, _ = oracle.combine(eo_all, d["row_of"], w_all)
             assert np.array_equal(y.view(torch.int16).numpy().view(np.uint16),
                                   y_all[t0:t0 + tokens[rank]]), quant
+        # sync_sizes=False: nothing waits on the host; capacity-sized views whose first
+        # recv_rows_device rows are this step's, counts read on request
+        for dedup in (False, True):
+            recv_x, ri, rw, per, ctx = g.dispatch(x, idx, wts, dedup=dedup, sync_sizes=False)
+            assert not ctx.sizes_synced and ri.shape[0] == g._peer["capacity"]
+            if dedup:
+                d = oracle.dispatch_dedup(x_all, idx_all, w_all, E, world, quant="fp8")
+                lo, hi = d["part_offset"][rank], d["part_offset"][rank + 1]
+            else:
+                d = oracle.dispatch(x_all, idx_all, w_all, E, world, quant="fp8")
+                lo, hi = d["expert_offset"][rank * epp], d["expert_offset"][(rank + 1) * epp]
+            n = int(ctx.recv_rows_device.item())
+            assert n == hi - lo and ctx.recv_rows == n
+            assert np.array_equal(recv_x[0][:n].view(torch.uint8).numpy(), d["recv_x"][lo:hi])
+            assert np.array_equal(ri[:n].numpy(), d["recv_topk_idx"][lo:hi])
+            assert sum(ctx.recv_counts) == n and len(ctx.send_counts) == world
+            buf = g.expert_out_buffer(ctx)
+            assert buf.shape[0] == g._peer["capacity"]
+            if dedup:
+                po_all = oracle.partition_identity(d["recv_x"], d["recv_scales"],
+                                                   d["recv_topk_idx"], d["recv_topk_weights"])
+                buf[:n].copy_(torch.from_numpy(po_all[lo:hi].view(np.int16)).view(torch.bfloat16))
+                y_all, _ = oracle.combine_dedup(po_all, d["prow_of"])
+            else:
+                eo_all = oracle.identity_expert(d["recv_x"], d["recv_scales"])
+                buf[:n].copy_(torch.from_numpy(eo_all[lo:hi].view(np.int16)).view(torch.bfloat16))
+                y_all, _ = oracle.combine(eo_all, d["row_of"], w_all)
+            y = g.combine(buf, ctx, wts)
+            assert np.array_equal(y.view(torch.int16).numpy().view(np.uint16),
+                                  y_all[t0:t0 + tokens[rank]]), f"no-sync dedup={dedup}"
         for quant in ("fp8", "none"):  # one row per (token, rank)
             recv_x, ri, rw, per_source, ctx = g.dispatch(x, idx, wts, use_fp8=quant == "fp8",
                                                          dedup=True)

@@ -141,6 +141,27 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
             y = g.combine(out, ctx, wts)
             y_ref, _ = oracle.combine(eo, d["row_of"], w.topk_weights)
             assert np.array_equal(bf16_to_u16(y), y_ref), quant
+        # sync_sizes=False: the whole step without a host wait; then a receiver over
+        # capacity, reported by the kernels instead of raised on the host
+        recv_x, ri, rw, per_expert, ctx = g.dispatch(x, idx, wts, sync_sizes=False)
+        d = oracle.dispatch(w.x, w.topk_idx, w.topk_weights, E, world, quant="fp8")
+        R = int(d["num_recv"][0])
+        assert int(ctx.recv_rows_device.item()) == R and ri.shape[0] == g._peer["capacity"]
+        assert np.array_equal(recv_x[0][:R].view(torch.uint8).cpu().numpy(), d["recv_x"])
+        assert np.array_equal(ri[:R].cpu().numpy(), d["recv_topk_idx"])
+        eo = oracle.identity_expert(d["recv_x"], d["recv_scales"])
+        out = g.expert_out_buffer(ctx)
+        out[:R].copy_(dev_u16_as_bf16(eo))
+        y = g.combine(out, ctx, wts)
+        y_ref, _ = oracle.combine(eo, d["row_of"], w.topk_weights)
+        assert np.array_equal(bf16_to_u16(y), y_ref), "no-sync"
+        assert ep.ep_read_status(g.workspace) == 0
+        small = ep.EpGroup(E, transport="peer", hidden=H, max_tokens=512, capacity=64)
+        try:
+            small.dispatch(x, idx, wts, sync_sizes=False)  # 1k+ rows for 64 slots: dropped
+            assert ep.ep_read_status(small.workspace) == ep.EP_DEV_CAPACITY
+        finally:
+            small.close()
         for quant in ("fp8", "none"):  # one row per (token, rank), [K] expert lists
             recv_x, ri, rw, per_source, ctx = g.dispatch(x, idx, wts, use_fp8=quant == "fp8",
                                                          dedup=True)
