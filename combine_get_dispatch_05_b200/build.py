@@ -65,7 +65,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     objs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [nvcc, *ARCH, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-dc" if False else "-c",
+        cmd = [nvcc, *ARCH, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c",
                src, "-o", obj]
         if ptxas_verbose:
             cmd.insert(1, "-Xptxas=-v")
