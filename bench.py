@@ -170,6 +170,13 @@ def source_hash(paths):
 
 COMBINE_SOURCES = ["combine_get_dispatch_05_b200/csrc/combine.cu",
                    "combine_get_dispatch_05_b200/csrc/ep_device.cuh"]
+DISPATCH_SOURCES = ["combine_get_dispatch_05_b200/csrc/dispatch.cu",
+                    "combine_get_dispatch_05_b200/csrc/ep_quant.cuh",
+                    "combine_get_dispatch_05_b200/csrc/ep_device.cuh",
+                    "combine_get_dispatch_05_b200/csrc/ep_internal.h"]
+LAYOUT_SOURCES = ["combine_get_dispatch_05_b200/csrc/layout.cu",
+                  "combine_get_dispatch_05_b200/csrc/ep_device.cuh",
+                  "combine_get_dispatch_05_b200/csrc/ep_internal.h"]
 
 
 def profiled_traffic(summary: str, sources):
@@ -416,6 +423,104 @@ def time_low_latency(ep, w, dev, reps=200, per_graph=20):
     if ep.ep_read_status(ws) != 0:
         raise RuntimeError("device status set in the peer low-latency run")
     del owners, tab
+    return out
+
+
+def time_epgroup(ep, w, dev, steps):
+    """EpGroup(transport="peer") as whole calls through the Python API at one rank
+    (workload w): dispatch = layout + count all-gather (NCCL) + plan + peer dispatch +
+    receive barrier; combine = barrier + peer combine.  Per call: device time between
+    CUDA events around the call (it includes any time the GPU waits for the host) and
+    host time to return.  sync_sizes=True returns exact-size tensors, which needs the
+    received counts on the host; sync_sizes=False keeps them on the device."""
+    import socket
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    own = not dist.is_initialized()
+    if own:
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    T, H, K, E = w.num_tokens, w.hidden, w.num_topk, w.num_experts
+    g = ep.EpGroup(E, transport="peer", hidden=H, max_tokens=T, num_topk=K,
+                   capacity=T * K + 16, device=dev)
+    out = {"ranks": 1, "tokens": T}
+    try:
+        x = torch.from_numpy(w.x.view(np.int16)).to(dev).view(torch.bfloat16)
+        idx = torch.from_numpy(w.topk_idx).to(dev)
+        wts = torch.from_numpy(w.topk_weights).to(dev)
+        for sync in (True, False):
+            rec = {}
+            d_dev, d_host, c_dev, c_host = [], [], [], []
+            for i in range(steps + 3):
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                e[0].record()
+                t0 = time.perf_counter()
+                res = g.dispatch(x, idx, wts, sync_sizes=sync)
+                t1 = time.perf_counter()
+                e[1].record()
+                ctx = res[4]
+                t2 = time.perf_counter()
+                g.combine(g.expert_out_buffer(ctx), ctx, wts)
+                t3 = time.perf_counter()
+                e[2].record()
+                torch.cuda.synchronize()
+                if i >= 3:
+                    d_dev.append(e[0].elapsed_time(e[1]) * 1e3)
+                    c_dev.append(e[1].elapsed_time(e[2]) * 1e3)
+                    d_host.append((t1 - t0) * 1e6)
+                    c_host.append((t3 - t2) * 1e6)
+            rec["dispatch_us"] = round(statistics.median(d_dev), 2)
+            rec["dispatch_call_host_us"] = round(statistics.median(d_host), 1)
+            rec["combine_us"] = round(statistics.median(c_dev), 2)
+            rec["combine_call_host_us"] = round(statistics.median(c_host), 1)
+            out["sync_sizes" if sync else "no_sync"] = rec
+        # with sync_sizes=False nothing in a step waits on the host, so the whole step
+        # (NCCL collectives included) can be captured in a CUDA graph and replayed
+        try:
+            cs = torch.cuda.Stream(device=dev)
+            cs.wait_stream(torch.cuda.current_stream())
+
+            def step():
+                res = g.dispatch(x, idx, wts, sync_sizes=False)
+                g.combine(g.expert_out_buffer(res[4]), res[4], wts)
+
+            with torch.cuda.stream(cs):
+                step()
+                step()
+            torch.cuda.current_stream().wait_stream(cs)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=cs):
+                step()
+            for _ in range(3):
+                graph.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            out["no_sync_graph_step_us"] = round(e0.elapsed_time(e1) * 1e3 / steps, 2)
+            del graph
+        except Exception as exc:  # report, do not hide
+            out["no_sync_graph_error"] = repr(exc)
+        if ep.ep_read_status(g.workspace) != 0:
+            raise RuntimeError("device status set in the EpGroup run")
+    finally:
+        g.close()
+        if own:
+            dist.destroy_process_group()
+    out["note"] = ("one rank: the owner's buffers are this GPU's, so no NVLink traffic; "
+                   "the expert outputs are whatever the buffer holds (the time does not "
+                   "depend on them)")
     return out
 
 
@@ -1061,7 +1166,13 @@ def run_ours(args):
                          "gbs": round(disp_gbs, 1), "frac": round(disp_gbs / peak, 4),
                          "tokens_per_s": round(w.num_tokens / (disp_us * 1e-6)),
                          "kernels": "layout (cooperative) + dispatch_%s (programmatic dependent "
-                                    "launch)" % ("fp8" if runner.fp8 else "bf16")},
+                                    "launch)" % ("fp8" if runner.fp8 else "bf16"),
+                         "traffic": {
+                             "layout_kernel": profiled_traffic(
+                                 "layout_kernel_normal_4096x7168.md", LAYOUT_SOURCES),
+                             "dispatch_fp8_kernel": profiled_traffic(
+                                 "dispatch_fp8_kernel_normal_4096x7168.md", DISPATCH_SOURCES)}
+                         if args.workload == "normal" and runner.fp8 else None},
             "combine": {"us": round(comb_us, 2), "bytes": runner.bytes_combine,
                         "gbs": round(comb_gbs, 1), "frac": round(comb_gbs / peak, 4),
                         "tokens_per_s": round(w.num_tokens / (comb_us * 1e-6)),
@@ -1072,7 +1183,8 @@ def run_ours(args):
             "peak": peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
             if peak_kind == "measured" else "fallback 6.65 TB/s",
             "unit": "GB/s", "frac": round(comb_gbs / peak, 4),
-            "traffic": profiled_traffic("combine_kernel_normal_4096x7168.md", COMBINE_SOURCES),
+            "traffic": profiled_traffic("combine_kernel_normal_4096x7168.md", COMBINE_SOURCES)
+            if args.workload == "normal" else None,
         },
         "gpu_launches": 3 * args.steps,
         "device_status": status,
@@ -1099,6 +1211,12 @@ def run_ours(args):
             extra["peer"]["workload"] = args.workload
         except Exception as exc:  # report, do not hide
             extra["peer"] = {"error": repr(exc)}
+        if world == 1:
+            try:
+                extra["epgroup"] = time_epgroup(ep, w, dev, min(args.extra_steps, 20))
+                extra["epgroup"]["workload"] = args.workload
+            except Exception as exc:  # report, do not hide
+                extra["epgroup"] = {"error": repr(exc)}
         try:
             extra["lb"] = time_lb(ep, dev, min(args.extra_steps, 20), args.seed, args.lb_scale)
         except Exception as exc:  # report, do not hide

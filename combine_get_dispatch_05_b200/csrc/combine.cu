@@ -32,8 +32,9 @@ constexpr int kLoadBatch = 8;  // combine backward: slots handled per batch
 // kBatch: row loads issued per thread before the first FMA.  The token's valid
 // rows are compacted (k order kept) so a batch holds only rows that exist; sparse
 // routings (one slot per partition, about half of them empty) use a batch of 4 and
-// fewer registers, so more threads and more loads are in flight per SM (the peer
-// variant, which holds row pointers, keeps two CTAs per SM so it does not spill).
+// fewer registers, so three CTAs per SM and more loads in flight (the peer variant
+// then spills a few bytes of its per-slot set-up; measured 57.3 -> 53.0 us on the
+// deduplicated normal workload against two CTAs per SM without spills).
 // kPeer: partitions are ranks; slot k's row is row_of[t, k] + peer_offset[e] in the
 // expert outputs of the rank that owns e = topk_idx[t, k] (read over NVLink), or,
 // with peer_by_slot (deduplicated rows, slot k = rank k), row_of[t, k] +
@@ -41,7 +42,7 @@ constexpr int kLoadBatch = 8;  // combine backward: slots handled per batch
 // j), row ((e % Epp) * W + rank) * cap + j of rank e / Epp's padded outputs; the
 // compaction records a pointer to each valid row instead of its index.
 template <int kBatch, bool kPeer>
-__global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 && !kPeer ? 3 : 2)
+__global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
     combine_kernel(CombineParams p, int64_t vec_per_slice) {
     pdl_wait();               // the previous kernel (e.g. the dispatch) is complete
     pdl_launch_dependents();  // the next kernel may be scheduled

@@ -87,10 +87,12 @@ class EpContext:
         self.order = order
         self.dedup = dedup
         # True when the received tensors were cut to the received rows
-        self.sizes_synced = not isinstance(recv_rows, torch.Tensor)
+        self.sizes_synced = isinstance(recv_rows, int)
 
     @staticmethod
     def _host(v):
+        if callable(v):  # computed on first use (no-sync dispatch)
+            v = v()
         return v.to("cpu").tolist() if isinstance(v, torch.Tensor) else v
 
     @property
@@ -105,13 +107,16 @@ class EpContext:
 
     @property
     def recv_rows(self) -> int:
-        if isinstance(self._recv_rows, torch.Tensor):
-            self._recv_rows = int(self._recv_rows.item())
+        if not isinstance(self._recv_rows, int):
+            self._recv_rows = int(self.recv_rows_device.item())
         return self._recv_rows
 
     @property
     def recv_rows_device(self) -> Optional[torch.Tensor]:
-        """The received row count as a device scalar (a no-sync peer dispatch), else None."""
+        """The received row count as a device scalar (a no-sync peer dispatch; computed
+        on the stream at the first read), else None."""
+        if callable(self._recv_rows):
+            self._recv_rows = self._recv_rows()
         return self._recv_rows if isinstance(self._recv_rows, torch.Tensor) else None
 
 
@@ -391,10 +396,9 @@ class EpGroup:
         lay = Layout.empty(T, K, E, W, dev)
         _lib.ep_get_dispatch_layout(topk_idx, E, W, lay, self.workspace)
         counts = self._all_gather_rows(lay.num_tokens_per_expert)  # [W, E]
-        totals = counts.view(W, W, epp).sum(dim=(0, 2))  # rows each rank receives
         if sync_sizes:
             # every rank reads the same counts: all of them raise, or none
-            totals = totals.to("cpu").tolist()
+            totals = counts.view(W, W, epp).sum(dim=(0, 2)).to("cpu").tolist()
             if max(totals) > cap:
                 raise ValueError(f"a rank would receive {max(totals)} rows; capacity is {cap}")
         dst = torch.empty(E, dtype=torch.int32, device=dev)
@@ -405,12 +409,15 @@ class EpGroup:
         _lib.ep_peer_dispatch(x, topk_idx, topk_weights, E, W, quant, lay, dst, self.tables,
                               self.workspace)
         per_expert = counts[:, r * epp:(r + 1) * epp]
-        send = counts.view(W, W, epp)[r].sum(dim=1)
-        recv = per_expert.sum(dim=1)
-        Rr = int(totals[r]) if sync_sizes else totals[r]
-        n = Rr if sync_sizes else cap
         if sync_sizes:
-            send, recv = send.to("cpu").tolist(), recv.to("cpu").tolist()
+            Rr = int(totals[r])
+            send = counts.view(W, W, epp)[r].sum(dim=1).to("cpu").tolist()
+            recv = per_expert.sum(dim=1).to("cpu").tolist()
+        else:  # reductions launched only if the caller reads them
+            Rr = lambda: per_expert.sum()  # noqa: E731
+            send = lambda: counts.view(W, W, epp)[r].sum(dim=1)  # noqa: E731
+            recv = lambda: per_expert.sum(dim=1)  # noqa: E731
+        n = Rr if sync_sizes else cap
         ctx = EpContext(lay, send, recv, T, H, topk_idx=topk_idx, dst_offset=dst, recv_rows=Rr,
                         order="expert_major")
         ri = self._view("recv_topk_idx", torch.int32, (cap,))[:n]
@@ -438,9 +445,8 @@ class EpGroup:
         lay = Layout.empty(T, W, W, W, dev)  # partition-sized handle
         _lib.ep_get_dispatch_layout_dedup(topk_idx, E, W, lay, self.workspace)
         counts = self._all_gather_rows(lay.num_tokens_per_expert)  # [W sources, W owners]
-        totals = counts.sum(dim=0)
         if sync_sizes:
-            totals = totals.to("cpu").tolist()
+            totals = counts.sum(dim=0).to("cpu").tolist()
             if max(totals) > cap:
                 raise ValueError(f"a rank would receive {max(totals)} rows; capacity is {cap}")
         dst = torch.empty(W, dtype=torch.int32, device=dev)
@@ -452,10 +458,12 @@ class EpGroup:
                                     self.workspace)
         per_source = counts[:, r:r + 1]
         send, recv = counts[r], per_source.reshape(-1)
-        Rr = int(totals[r]) if sync_sizes else totals[r]
-        n = Rr if sync_sizes else cap
         if sync_sizes:
+            Rr = int(totals[r])
             send, recv = send.to("cpu").tolist(), recv.to("cpu").tolist()
+        else:  # the reduction is launched only if the caller reads it
+            Rr = lambda: per_source.sum()  # noqa: E731
+        n = Rr if sync_sizes else cap
         ctx = EpContext(lay, send, recv, T, H, dst_offset=dst, recv_rows=Rr, order="source_major",
                         dedup=True)
         ri = self._view("recv_topk_idx", torch.int32, (cap, K))[:n]
