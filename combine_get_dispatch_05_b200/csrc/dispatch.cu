@@ -383,7 +383,9 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
             if (lane == 0 && prev >= 0) mbar_arrive(&out_empty[prev]);
             prev = o;
         }
-        if (slot_lane) bulk_wait_all<0>();
+        // the CTA may exit once its stores have read their stages; the grid completes
+        // only when the writes have landed
+        if (slot_lane) bulk_wait_read<0>();
     }
     __syncthreads();
     if (tid == 0) {
@@ -489,7 +491,7 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
             __syncwarp();
             if (lane == 0 && i >= 1) mbar_arrive(&empty[(i - 1) % kBf16Stages]);
         }
-        if (slot_lane) bulk_wait_all<0>();
+        if (slot_lane) bulk_wait_read<0>();  // stages read: the CTA may exit
     }
     __syncthreads();
     if (tid == 0) {
