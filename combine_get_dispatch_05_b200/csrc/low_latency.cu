@@ -33,7 +33,7 @@ namespace ep {
 namespace {
 
 constexpr int kLLMaxThreads = 256;
-constexpr int kPrefixBatch = 4;  // topk_idx loads in flight per thread
+constexpr int kPrefixBatch = 8;  // topk_idx loads in flight per thread
 
 // Shared memory of one (token, slice) CTA: the slice's BF16 input, its E4M3 codes
 // and scales, an mbarrier, the token's K rows / slot counters / ids, and (CTA 0
@@ -115,28 +115,35 @@ __global__ void __launch_bounds__(kLLMaxThreads) ll_dispatch_kernel(LowLatencyDi
         bulk_load(sm, static_cast<const uint8_t*>(p.x) + t * H * 2 + static_cast<int64_t>(b0) * 256,
                   static_cast<uint32_t>(nbl) * 256u, bar);
     }
-    if (tid < K) eid_sm[tid] = p.topk_idx[t * K + tid];
-    for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
-    __syncthreads();
-
     // slot of (t, k) = pairs (t', k') < (t, k) in (token, k) order with the same
     // expert: a histogram of the ids of the earlier tokens (shared-memory atomics,
-    // kPrefixBatch loads in flight per thread), plus the equal ids among the
-    // token's own earlier slots.  CTA (0, 0) -- token 0, no earlier tokens --
-    // histograms the whole batch instead, for recv_expert_count.
+    // kPrefixBatch loads in flight per thread; the first batch is issued before the
+    // histogram is cleared, so its latency overlaps the barrier), plus the equal ids
+    // among the token's own earlier slots.  CTA (0, 0) -- token 0, no earlier tokens
+    // -- histograms the whole batch instead, for recv_expert_count.
     const int64_t base = t * K;
     const int64_t upto = all ? p.T * K : base;
     const int64_t stride = static_cast<int64_t>(blockDim.x);
-    for (int64_t j0 = tid; j0 < upto; j0 += kPrefixBatch * stride) {
-        int64_t v[kPrefixBatch];
+    int64_t v[kPrefixBatch];
 #pragma unroll
-        for (int u = 0; u < kPrefixBatch; ++u) {
-            const int64_t j = j0 + u * stride;
-            v[u] = j < upto ? p.topk_idx[j] : -1;
-        }
+    for (int u = 0; u < kPrefixBatch; ++u) {
+        const int64_t j = tid + u * stride;
+        v[u] = j < upto ? p.topk_idx[j] : -1;
+    }
+    if (tid < K) eid_sm[tid] = p.topk_idx[t * K + tid];
+    for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    for (int64_t j0 = tid;; j0 += kPrefixBatch * stride) {
 #pragma unroll
         for (int u = 0; u < kPrefixBatch; ++u)
             if (v[u] >= 0 && v[u] < E) atomicAdd(&hist[v[u]], 1);
+        const int64_t jn = j0 + kPrefixBatch * stride;
+        if (jn >= upto) break;
+#pragma unroll
+        for (int u = 0; u < kPrefixBatch; ++u) {
+            const int64_t j = jn + u * stride;
+            v[u] = j < upto ? p.topk_idx[j] : -1;
+        }
     }
     __syncthreads();
     if (tid < K) {
