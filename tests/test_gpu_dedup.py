@@ -64,6 +64,12 @@ CASES = [
     ("p1", lambda: make_custom(90, 128, 4, 8, 1, seed=11)),
     ("e-eq-p", lambda: make_custom(257, 256, 3, 16, 16, seed=12)),
     ("t1", lambda: make_custom(1, 128, 8, 256, 8, seed=6)),
+    # more than 1024 tokens: the partition layout's multi-CTA form; P = 6 and P = 5 take
+    # its byte-by-byte flag and row stores, P = 32 is the most partitions it takes
+    ("grid-2500", lambda: make_workload("normal", seed=3, num_tokens=2500, hidden=128)),
+    ("grid-p6-3001", lambda: make_custom(3001, 128, 6, 48, 6, seed=14, mask_frac=0.1)),
+    ("grid-p32-2049", lambda: make_custom(2049, 128, 8, 64, 32, seed=15, mask_frac=0.05)),
+    ("p5-1025", lambda: make_custom(1025, 128, 3, 5, 5, seed=16, duplicates=True)),
 ]
 
 
@@ -81,6 +87,9 @@ def test_dispatch_dedup_parity(ep, name, mk):
     assert np.array_equal(got["count"], want["part_count"])
     assert np.array_equal(got["offset"], want["part_offset"])
     assert np.array_equal(got["src_of"] // P, want["src_tok"])
+    # the slot of each row is the partition whose segment holds it
+    part_of_row = np.searchsorted(want["part_offset"], np.arange(got["R"]), side="right") - 1
+    assert np.array_equal(got["src_of"] % P, part_of_row)
     assert np.array_equal(got["itp"], lay["is_token_in_partition"])
     assert np.array_equal(got["ntp"], lay["num_tokens_per_partition"])
     assert np.array_equal(got["recv_x"], want["recv_x"])
@@ -201,3 +210,21 @@ def test_dispatch_dedup_block_major_pow2_scales(ep):
     assert np.all(np.isnan(got[:, R:]))
     assert np.array_equal(rq[:R].cpu().numpy(), want["recv_x"])
     assert ep.ep_read_status(ws) == 0
+
+
+def test_dedup_layout_skips_and_reports_out_of_range_ids(ep):
+    # ids outside [-1, E) count as masked in the deduplicated layout too, and are reported
+    w = make_custom(1500, 128, 8, 64, 8, seed=17)
+    bad = w.topk_idx.copy()
+    bad[3, 2], bad[1200, 0], bad[700, 7] = 64, -5, 1000
+    T, K, E, P = w.num_tokens, w.num_topk, w.num_experts, w.num_partitions
+    idx = torch.from_numpy(bad).cuda()
+    lay = ep.Layout.empty(T, P, P, P, "cuda")
+    ws = new_workspace(ep, T, E, P)
+    ep.ep_get_dispatch_layout_dedup(idx, E, P, lay, ws)
+    torch.cuda.synchronize()
+    clean = np.where((bad >= 0) & (bad < E), bad, -1)
+    want = oracle.dispatch_dedup(w.x, clean, w.topk_weights, E, P, quant="none")
+    assert np.array_equal(lay.row_of.cpu().numpy(), want["prow_of"])
+    assert np.array_equal(lay.expert_offset.cpu().numpy(), want["part_offset"])
+    assert ep.ep_read_status(ws) == ep.EP_DEV_INDEX_RANGE
