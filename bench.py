@@ -12,10 +12,12 @@ dispatched rows dequantised, i.e. identity experts).
 
 Prints ONE JSON line (rank 0).  `value` is algorithmic HBM GB/s of the whole
 step (bytes the method must move / device time, summed over ranks' batches,
-max time over ranks).  Each step is captured as one CUDA graph (the layout,
-dispatch and combine kernels) and timed with CUDA events on the launching stream
-around each replay; a second pass times the dispatch and the combine apart (two
-graphs, events between them) for the breakdown.  Steps run back
+max time over ranks).  Steps are captured in CUDA graphs, ten whole steps (the
+layout, dispatch and combine kernels of each) per graph by default
+(`--steps-per-graph`), and timed with CUDA events on the launching stream around
+each replay; a second pass times the dispatch and the combine apart (two graphs,
+events between them) for the breakdown, and a third the whole step as one graph
+per step.  Steps run back
 to back: every step reads 529 MB of inputs (x and the expert outputs) and
 writes 294 MB, several times the 126 MB L2, so nothing a step reads is still in
 L2 from the step before.  `--l2-flush write|read` instead flushes L2 with a
@@ -243,6 +245,7 @@ class PathRunner:
             raise RuntimeError("device status set during setup")
         self.bytes_dispatch, self.bytes_combine = algorithmic_bytes(T, H, K, E, P, self.R, self.fp8)
         self.graphs = None
+        self._step_graphs = {}
         if use_graphs:
             self.graphs = self._capture()
 
@@ -287,33 +290,59 @@ class PathRunner:
         else:
             self.combine()
 
-    def time_whole_steps(self, steps, warmup, flush=None):
-        """Per-step ms of the whole step as one launch (one CUDA graph holding the
-        layout, dispatch and combine kernels; eagerly the two calls); `flush` (if
-        given) runs before each step, outside the events."""
+    def step_graph(self, n):
+        """A CUDA graph of n whole steps back to back (cached per n)."""
         import torch
 
-        def run():
-            if self.graphs:
-                self.graphs[2].replay()
-            else:
-                self.dispatch()
-                self.combine()
+        if n not in self._step_graphs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for _ in range(n):
+                    self.dispatch()
+                    self.combine()
+            torch.cuda.synchronize()
+            self._step_graphs[n] = g
+        return self._step_graphs[n]
 
+    def time_whole_steps(self, steps, warmup, flush=None, per_graph=1):
+        """Per-step ms of whole steps (layout, dispatch and combine kernels) replayed
+        back to back, `per_graph` steps per CUDA graph (a last, shorter graph makes the
+        count exactly `steps`); eagerly the two calls per step.  `flush` (if given) runs
+        before each step, outside the events, and implies one step per graph.  Returns
+        one time per step (a graph's time divided among its steps)."""
+        import torch
+
+        if flush is not None or not self.graphs:
+            per_graph = 1
+
+        def run(n):
+            if self.graphs:
+                (self.graphs[2] if n == 1 else self.step_graph(n)).replay()
+            else:
+                for _ in range(n):
+                    self.dispatch()
+                    self.combine()
+
+        sizes = [per_graph] * (steps // per_graph) + ([steps % per_graph] if steps % per_graph else [])
+        for n in sorted(set(sizes)):  # capture (and warm) every graph before timing
+            run(n)
         for _ in range(warmup):
             if flush is not None:
                 flush()
-            run()
+            run(1)
         torch.cuda.synchronize()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
-        for i in range(steps):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in sizes]
+        for i, n in enumerate(sizes):
             if flush is not None:
                 flush()
             evs[i][0].record()
-            run()
+            run(n)
             evs[i][1].record()
         torch.cuda.synchronize()
-        return [e[0].elapsed_time(e[1]) for e in evs]
+        out = []
+        for e, n in zip(evs, sizes):
+            out += [e[0].elapsed_time(e[1]) / n] * n
+        return out
 
     def time_steps(self, steps, warmup, flush=None):
         """Per-step (dispatch ms, combine ms); `flush` (if given) runs before each step,
@@ -1142,19 +1171,21 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
     t0 = time.time()
-    s_ms = runner.time_whole_steps(args.steps, args.warmup, flush)
+    s_ms = runner.time_whole_steps(args.steps, args.warmup, flush, per_graph=args.steps_per_graph)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     t1 = time.time()
     sampler.mark(t0, t1)
     # breakdown: the same steps again with the dispatch and the combine launched as two
-    # graphs, events between them (the boundary costs the step a few us)
+    # graphs, events between them (the boundary costs the step a few us); and the
+    # whole step as one graph per step, for reference
     d_ms, c_ms = runner.time_steps(args.steps, 3, flush)
+    one_ms = runner.time_whole_steps(args.steps, 3, flush, per_graph=1)
     torch.cuda.synchronize()
     status = ep.ep_read_status(runner.ws)
 
-    tot = reduce_max_over_ranks([sum(s_ms), sum(c_ms), sum(d_ms)], world, dev)
+    tot = reduce_max_over_ranks([sum(s_ms), sum(c_ms), sum(d_ms), sum(one_ms)], world, dev)
     total_ms = tot[0]
     ms_step = total_ms / args.steps
     step_bytes = runner.bytes_dispatch + runner.bytes_combine
@@ -1196,9 +1227,12 @@ def run_ours(args):
         "data": "synthetic",
         "config": workload_config(args.workload, w, runner.R, step_bytes, args.seed, world,
                                   args.l2_flush),
-        "launch": "one CUDA graph per step: layout, dispatch (a programmatic dependent of the "
-                  "layout) and combine kernels; steps replayed back to back" if not args.eager
-        else "eager",
+        "launch": (f"CUDA graphs of {min(args.steps_per_graph, args.steps)} whole steps each "
+                   "(layout, dispatch as a programmatic dependent of the layout, combine; the next "
+                   "step's layout a programmatic dependent of the combine), replayed back to back; "
+                   "one graph per step: %.2f us per step" % (tot[3] / args.steps * 1e3))
+        if not args.eager and args.l2_flush == "none" else
+        ("one CUDA graph per step (L2 flushed between steps)" if not args.eager else "eager"),
         "breakdown_note": "dispatch and combine intervals from a second pass of the same steps "
                           "with the two calls captured as separate graphs and events between "
                           "them; their sum exceeds the whole-step time by the graph boundary",
@@ -1270,7 +1304,7 @@ def run_ours(args):
             try:
                 wx = make_workload(name, seed=args.seed)
                 r = PathRunner(ep, wx, dev, use_graphs=not args.eager)
-                ss = r.time_whole_steps(args.extra_steps, 3, flush)
+                ss = r.time_whole_steps(args.extra_steps, 3, flush, per_graph=args.steps_per_graph)
                 dd, cc = r.time_steps(args.extra_steps, 3, flush)
                 du, cu = statistics.mean(dd) * 1e3, statistics.mean(cc) * 1e3
                 su = statistics.mean(ss) * 1e3
@@ -1372,6 +1406,8 @@ def main():
     ap.add_argument("--extra-steps", type=int, default=50)
     ap.add_argument("--eager", action="store_true", help="launch eagerly instead of CUDA graphs")
     ap.add_argument("--l2-flush", choices=("none", "write", "read"), default="none")
+    ap.add_argument("--steps-per-graph", type=int, default=10,
+                    help="whole steps captured in one CUDA graph for the headline timing")
     ap.add_argument("--workload", choices=("normal", "skew", "bf16", "stress"), default="normal",
                     help="workload of the timed step (the headline metric is quoted on normal)")
     ap.add_argument("--no-extra", action="store_true", help="skip the ll/skew/bf16/stress configs")
@@ -1382,6 +1418,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.steps_per_graph < 1:
+        ap.error("--steps-per-graph must be at least 1")
     rank, world, _ = env_rank()
     if world != args.gpus and not (world == 1 and args.gpus == 1):
         if world == 1 and args.gpus > 1:
