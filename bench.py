@@ -494,7 +494,9 @@ def time_epgroup(ep, w, dev, steps):
     receive barrier; combine = barrier + peer combine.  Per call: device time between
     CUDA events around the call (it includes any time the GPU waits for the host) and
     host time to return.  sync_sizes=True returns exact-size tensors, which needs the
-    received counts on the host; sync_sizes=False keeps them on the device."""
+    received counts on the host; sync_sizes=False keeps them on the device, and its
+    whole steps are also timed launched back to back (step_us: device time per step;
+    step_host_us: the host's time to issue one) and captured in a CUDA graph."""
     import socket
 
     import numpy as np
@@ -542,6 +544,20 @@ def time_epgroup(ep, w, dev, steps):
             rec["dispatch_call_host_us"] = round(statistics.median(d_host), 1)
             rec["combine_us"] = round(statistics.median(c_dev), 2)
             rec["combine_call_host_us"] = round(statistics.median(c_host), 1)
+            if not sync:
+                # whole steps launched back to back, as a training loop does: the host
+                # runs ahead of the device unless its calls take longer than the kernels
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                e[0].record()
+                t0 = time.perf_counter()
+                for _ in range(steps):
+                    res = g.dispatch(x, idx, wts, sync_sizes=False)
+                    g.combine(g.expert_out_buffer(res[4]), res[4], wts)
+                t1 = time.perf_counter()
+                e[1].record()
+                torch.cuda.synchronize()
+                rec["step_us"] = round(e[0].elapsed_time(e[1]) * 1e3 / steps, 2)
+                rec["step_host_us"] = round((t1 - t0) * 1e6 / steps, 1)
             out["sync_sizes" if sync else "no_sync"] = rec
         # with sync_sizes=False nothing in a step waits on the host, so the whole step
         # (NCCL collectives included) can be captured in a CUDA graph and replayed

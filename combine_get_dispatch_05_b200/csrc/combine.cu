@@ -286,10 +286,7 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
                                : reinterpret_cast<const void*>(combine_kernel<8, true>))
         : p.sparse ? reinterpret_cast<const void*>(combine_kernel<4, false>)
                    : reinterpret_cast<const void*>(combine_kernel<8, false>);
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
+    const int per_sm = blocks_per_sm(kernel, dev.device, threads, 0);
     int64_t gx = (static_cast<int64_t>(per_sm) * dev.num_sms + slices - 1) / slices;
     if (gx > p.T) gx = p.T;
     if (gx < 1) gx = 1;
@@ -328,11 +325,8 @@ cudaError_t launch_combine_backward(const CombineBackwardParams& p, cudaStream_t
     const int64_t V = p.H / 8;
     int threads = static_cast<int>((V + 31) / 32 * 32);
     if (threads > kBwdThreads) threads = kBwdThreads;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_backward_kernel, threads,
-                                                      0) != cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
+    const int per_sm =
+        blocks_per_sm(reinterpret_cast<const void*>(combine_backward_kernel), dev.device, threads, 0);
     int64_t grid = static_cast<int64_t>(per_sm) * dev.num_sms;
     if (grid > p.T) grid = p.T;
     combine_backward_kernel<<<static_cast<unsigned>(grid), threads, 0, stream>>>(p);

@@ -500,13 +500,9 @@ __global__ void __launch_bounds__(64) dispatch_bf16_kernel(DispatchParams p) {
     }
 }
 
-int grid_for(const void* kernel, int threads, size_t smem, int64_t work, int num_sms) {
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) !=
-            cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
-    const int64_t g = static_cast<int64_t>(per_sm) * num_sms;
+int grid_for(const void* kernel, int threads, size_t smem, int64_t work, const DeviceInfo& dev) {
+    const int64_t g = static_cast<int64_t>(blocks_per_sm(kernel, dev.device, threads, smem)) *
+                      dev.num_sms;
     return static_cast<int>(work < g ? (work > 0 ? work : 1) : g);
 }
 
@@ -562,7 +558,7 @@ cudaError_t launch_dispatch_fp8(const DispatchParams& params, cudaStream_t strea
     const int iters = (pairs + kFp8MaxQuantWarps - 1) / kFp8MaxQuantWarps;
     const int nq = (pairs + iters - 1) / iters;
     const int threads = 32 * (nq + 2);
-    const int grid = grid_for(kernel, threads, L.total, p.T, dev.num_sms);
+    const int grid = grid_for(kernel, threads, L.total, p.T, dev);
     return launch_pdl(kernel, dim3(grid), dim3(threads), L.total, stream, p);
 }
 
@@ -579,7 +575,7 @@ cudaError_t launch_dispatch_bf16(const DispatchParams& p, cudaStream_t stream) {
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    const int grid = grid_for(kernel, 64, smem, p.T, dev.num_sms);
+    const int grid = grid_for(kernel, 64, smem, p.T, dev);
     return launch_pdl(kernel, dim3(grid), dim3(64), smem, stream, p);
 }
 

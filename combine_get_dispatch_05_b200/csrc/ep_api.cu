@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "ep_b200.h"
 #include "ep_device.cuh"
@@ -18,6 +19,17 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_have_info[kMaxDevices];
 DeviceInfo g_info[kMaxDevices];
+
+struct OccupancyEntry {
+    const void* kernel;
+    int device, threads;
+    size_t smem;
+    int per_sm;
+};
+constexpr int kOccupancyEntries = 64;
+std::mutex g_occ_mu;
+OccupancyEntry g_occ[kOccupancyEntries];
+int g_occ_n = 0;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -53,6 +65,24 @@ ep_status check_layout_size(int64_t T, int32_t K, int32_t E, int32_t P, bool by_
     bool fits = true;
     if (layout_fits(T, K, E, P, by_partition, &fits) != cudaSuccess) return EP_ERR_CUDA;
     return fits ? EP_OK : EP_ERR_SHAPE;
+}
+
+int blocks_per_sm(const void* kernel, int device, int threads, size_t smem) {
+    std::lock_guard<std::mutex> lock(g_occ_mu);
+    for (int i = 0; i < g_occ_n; ++i) {
+        const OccupancyEntry& o = g_occ[i];
+        if (o.kernel == kernel && o.device == device && o.threads == threads && o.smem == smem)
+            return o.per_sm;
+    }
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) !=
+        cudaSuccess) {
+        cudaGetLastError();  // not sticky; the launch reports any real fault
+        return 1;
+    }
+    if (per_sm < 1) per_sm = 1;
+    if (g_occ_n < kOccupancyEntries) g_occ[g_occ_n++] = {kernel, device, threads, smem, per_sm};
+    return per_sm;
 }
 
 cudaError_t device_info(DeviceInfo* out) {

@@ -18,6 +18,11 @@ struct DeviceInfo {
 };
 cudaError_t device_info(DeviceInfo* out);
 
+// Resident CTAs per SM (at least 1) of `kernel` launched with `threads` threads and
+// `smem` bytes of dynamic shared memory on device `device`.  The answer depends
+// only on the kernel and the device, so each is computed once and kept.
+int blocks_per_sm(const void* kernel, int device, int threads, size_t smem);
+
 // Host-side argument checks of the layout entry points (the workspace and the
 // no-workspace forms validate alike).  check_routing: sizes in range
 // (EP_ERR_SHAPE); check_layout_ptrs: the arrays a batch of T tokens needs are set

@@ -149,6 +149,8 @@ class EpGroup:
         self.experts_per_rank = num_experts // self.world
         self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
             else torch.device(device)
+        if self.device.type == "cuda" and self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
         self.max_tokens = max_tokens
         self.workspace = self._new_workspace(max_tokens)
         self.via_host = dist.get_backend(self.group) != "nccl"
@@ -206,6 +208,7 @@ class EpGroup:
         if hidden % 128:
             raise ValueError("hidden must be a multiple of 128")
         self._regions = []
+        self._views = {}
         self._flag = torch.zeros(1, dtype=torch.int32, device=self.device)
         sizes = [("recv_x", capacity * hidden * 2), ("recv_scales", capacity * (hidden // 128) * 4),
                  ("recv_topk_idx", capacity * topk * 4), ("recv_topk_weights", capacity * topk * 4),
@@ -225,13 +228,32 @@ class EpGroup:
             self._peer["ll"] = ll
 
     def _view(self, name: str, dtype, shape, region=None) -> torch.Tensor:
+        """A typed view of a named array of a region; made once per (array, dtype,
+        shape) and kept, as every call of a step asks for the same views."""
         pr = self._peer if region is None else region
-        n = 1
-        for d in shape:
-            n *= d
-        n *= torch.empty(0, dtype=dtype).element_size()
-        o = pr["offsets"][name]
-        return pr["region"][o:o + n].view(dtype).view(*shape)
+        key = (id(pr), name, dtype, tuple(shape))
+        v = self._views.get(key)
+        if v is None:
+            n = 1
+            for d in shape:
+                n *= d
+            n *= torch.empty(0, dtype=dtype).element_size()
+            o = pr["offsets"][name]
+            v = self._views[key] = pr["region"][o:o + n].view(dtype).view(*shape)
+        return v
+
+    def _stream(self):
+        """The current stream of this group's device, resolved once per call and
+        passed to every library call of it."""
+        if self.device.type != "cuda":
+            return None
+        if _lib._raw_stream is not None:
+            return _lib._raw_stream(self.device.index)
+        return torch.cuda.current_stream(self.device).cuda_stream
+
+    @staticmethod
+    def _rows(t: torch.Tensor, n: int) -> torch.Tensor:
+        return t if n == t.shape[0] else t[:n]
 
     def expert_out_buffer(self, ctx: EpContext) -> torch.Tensor:
         """Peer transport: the BF16 [recv rows, H] buffer the expert outputs go into
@@ -255,6 +277,7 @@ class EpGroup:
                 _lib.ep_ipc_close(ptr)
         self._host_barrier()  # every rank has closed its mappings of this rank's regions
         self._peer = None
+        self._views = {}
         for reg in self._regions:
             _lib.ep_ipc_free(reg["base"])
         self._regions = []
@@ -392,9 +415,9 @@ class EpGroup:
         pr = self._peer
         if H != pr["hidden"]:
             raise ValueError(f"hidden {H} differs from the receive buffers' {pr['hidden']}")
-        cap, dev = pr["capacity"], self.device
+        cap, dev, st = pr["capacity"], self.device, self._stream()
         lay = Layout.empty(T, K, E, W, dev)
-        _lib.ep_get_dispatch_layout(topk_idx, E, W, lay, self.workspace)
+        _lib.ep_get_dispatch_layout(topk_idx, E, W, lay, self.workspace, stream=st)
         counts = self._all_gather_rows(lay.num_tokens_per_expert)  # [W, E]
         if sync_sizes:
             # every rank reads the same counts: all of them raise, or none
@@ -404,10 +427,11 @@ class EpGroup:
         dst = torch.empty(E, dtype=torch.int32, device=dev)
         rc = torch.empty(epp, dtype=torch.int32, device=dev)
         ro = torch.empty(epp + 1, dtype=torch.int32, device=dev)
-        _lib.ep_peer_plan(counts, r, lay.expert_offset, cap, dst, rc, ro, self.workspace)
+        _lib.ep_peer_plan(counts, r, lay.expert_offset, cap, dst, rc, ro, self.workspace,
+                          stream=st)
         quant = EP_QUANT_FP8_E4M3_1X128 if use_fp8 else EP_QUANT_NONE
         _lib.ep_peer_dispatch(x, topk_idx, topk_weights, E, W, quant, lay, dst, self.tables,
-                              self.workspace)
+                              self.workspace, stream=st)
         per_expert = counts[:, r * epp:(r + 1) * epp]
         if sync_sizes:
             Rr = int(totals[r])
@@ -420,14 +444,13 @@ class EpGroup:
         n = Rr if sync_sizes else cap
         ctx = EpContext(lay, send, recv, T, H, topk_idx=topk_idx, dst_offset=dst, recv_rows=Rr,
                         order="expert_major")
-        ri = self._view("recv_topk_idx", torch.int32, (cap,))[:n]
-        rw = self._view("recv_topk_weights", torch.float32, (cap,))[:n]
+        ri = self._rows(self._view("recv_topk_idx", torch.int32, (cap,)), n)
+        rw = self._rows(self._view("recv_topk_weights", torch.float32, (cap,)), n)
         if use_fp8:
-            q = self._view("recv_x", torch.uint8, (cap, H))[:n]
-            s = self._view("recv_scales", torch.float32, (cap, H // 128))[:n]
-            recv_x = (q.view(torch.float8_e4m3fn), s)
+            recv_x = (self._rows(self._view("recv_x", torch.float8_e4m3fn, (cap, H)), n),
+                      self._rows(self._view("recv_scales", torch.float32, (cap, H // 128)), n))
         else:
-            recv_x = self._view("recv_x", torch.bfloat16, (cap, H))[:n]
+            recv_x = self._rows(self._view("recv_x", torch.bfloat16, (cap, H)), n)
         return recv_x, ri, rw, per_expert, ctx
 
     def _dispatch_peer_dedup(self, x, topk_idx, topk_weights, use_fp8, sync_sizes=True):
@@ -441,9 +464,9 @@ class EpGroup:
             raise ValueError(f"top-k {K} exceeds the buffers' lists of {pr['topk']}")
         if W > 32:
             raise ValueError("deduplicated rows support at most 32 ranks")
-        cap, dev = pr["capacity"], self.device
+        cap, dev, st = pr["capacity"], self.device, self._stream()
         lay = Layout.empty(T, W, W, W, dev)  # partition-sized handle
-        _lib.ep_get_dispatch_layout_dedup(topk_idx, E, W, lay, self.workspace)
+        _lib.ep_get_dispatch_layout_dedup(topk_idx, E, W, lay, self.workspace, stream=st)
         counts = self._all_gather_rows(lay.num_tokens_per_expert)  # [W sources, W owners]
         if sync_sizes:
             totals = counts.sum(dim=0).to("cpu").tolist()
@@ -452,10 +475,11 @@ class EpGroup:
         dst = torch.empty(W, dtype=torch.int32, device=dev)
         rc = torch.empty(1, dtype=torch.int32, device=dev)
         ro = torch.empty(2, dtype=torch.int32, device=dev)
-        _lib.ep_peer_plan(counts, r, lay.expert_offset, cap, dst, rc, ro, self.workspace)
+        _lib.ep_peer_plan(counts, r, lay.expert_offset, cap, dst, rc, ro, self.workspace,
+                          stream=st)
         quant = EP_QUANT_FP8_E4M3_1X128 if use_fp8 else EP_QUANT_NONE
         _lib.ep_peer_dispatch_dedup(x, topk_idx, topk_weights, E, W, quant, lay, dst, self.tables,
-                                    self.workspace)
+                                    self.workspace, stream=st)
         per_source = counts[:, r:r + 1]
         send, recv = counts[r], per_source.reshape(-1)
         if sync_sizes:
@@ -466,14 +490,13 @@ class EpGroup:
         n = Rr if sync_sizes else cap
         ctx = EpContext(lay, send, recv, T, H, dst_offset=dst, recv_rows=Rr, order="source_major",
                         dedup=True)
-        ri = self._view("recv_topk_idx", torch.int32, (cap, K))[:n]
-        rw = self._view("recv_topk_weights", torch.float32, (cap, K))[:n]
+        ri = self._rows(self._view("recv_topk_idx", torch.int32, (cap, K)), n)
+        rw = self._rows(self._view("recv_topk_weights", torch.float32, (cap, K)), n)
         if use_fp8:
-            q = self._view("recv_x", torch.uint8, (cap, H))[:n]
-            s = self._view("recv_scales", torch.float32, (cap, H // 128))[:n]
-            recv_x = (q.view(torch.float8_e4m3fn), s)
+            recv_x = (self._rows(self._view("recv_x", torch.float8_e4m3fn, (cap, H)), n),
+                      self._rows(self._view("recv_scales", torch.float32, (cap, H // 128)), n))
         else:
-            recv_x = self._view("recv_x", torch.bfloat16, (cap, H))[:n]
+            recv_x = self._rows(self._view("recv_x", torch.bfloat16, (cap, H)), n)
         return recv_x, ri, rw, per_source, ctx
 
     # ------------------------------------------------------------ low latency --
@@ -513,9 +536,9 @@ class EpGroup:
         h = _lib.LowLatencyHandle.empty(T, K, E, cap, self.device)
         t = ll["tables"]
         _lib.ep_peer_low_latency_dispatch(x, topk_idx, cap, E, W, self.rank, t["x"], t["scales"],
-                                          t["count"], h, self.workspace)
+                                          t["count"], h, self.workspace, stream=self._stream())
         rows = epp * W * cap
-        q = self._view("x", torch.uint8, (epp, W * cap, H), ll).view(torch.float8_e4m3fn)
+        q = self._view("x", torch.float8_e4m3fn, (epp, W * cap, H), ll)
         s = self._view("scales", torch.float32, (epp, W * cap, H // 128), ll)
         count = self._view("count", torch.int32, (epp, W), ll)
         ctx = EpContext(h, [], [], T, H, topk_idx=topk_idx, recv_rows=rows, order="low_latency")
@@ -539,7 +562,7 @@ class EpGroup:
         self._barrier()  # every rank's expert outputs are complete
         _lib.ep_peer_low_latency_combine(self._peer["ll"]["tables"]["expert_out"], ctx.topk_idx,
                                          ctx.handle, topk_weights, y, self.num_experts, self.world,
-                                         self.rank, self.workspace)
+                                         self.rank, self.workspace, stream=self._stream())
         return y
 
     # ---------------------------------------------------------------- combine --
@@ -554,13 +577,14 @@ class EpGroup:
             if expert_out.data_ptr() != self.expert_out_buffer(ctx).data_ptr():
                 raise ValueError("write the expert outputs into expert_out_buffer(ctx)")
             self._barrier()  # every rank's expert outputs are complete
+            st = self._stream()
             if ctx.dedup:  # partition outputs are already weighted: a plain sum
                 _lib.ep_peer_combine_dedup(self.tables, ctx.handle, ctx.dst_offset, y, self.world,
-                                           self.workspace)
+                                           self.workspace, stream=st)
             else:
                 _lib.ep_peer_combine(self.tables, ctx.handle, ctx.topk_idx, ctx.dst_offset,
                                      topk_weights, y, self.num_experts, self.world,
-                                     self.workspace)
+                                     self.workspace, stream=st)
             return y
         Rs = sum(ctx.send_counts)
         back = self._a2a(expert_out, Rs, ctx.send_counts, ctx.recv_counts)
