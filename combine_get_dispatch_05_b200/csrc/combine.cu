@@ -33,18 +33,23 @@ constexpr int kLoadBatch = 8;  // combine backward: slots handled per batch
 // kBatch: row loads issued per thread before the first FMA.  The token's valid
 // rows are compacted (k order kept) so a batch holds only rows that exist; sparse
 // routings (one slot per partition, about half of them empty) use a batch of 4 and
-// fewer registers, so three CTAs per SM and more loads in flight (the peer variant
-// then spills a few bytes of its per-slot set-up; measured 57.3 -> 53.0 us on the
-// deduplicated normal workload against two CTAs per SM without spills).
+// fewer registers, so three CTAs per SM and more loads in flight.
 // kPeer: partitions are ranks; slot k's row is row_of[t, k] + peer_offset[e] in the
 // expert outputs of the rank that owns e = topk_idx[t, k] (read over NVLink), or,
-// with peer_by_slot (deduplicated rows, slot k = rank k), row_of[t, k] +
-// peer_offset[k] in rank k's outputs, or, for low-latency rows (row_of = e * cap +
-// j), row ((e % Epp) * W + rank) * cap + j of rank e / Epp's padded outputs; the
-// compaction records a pointer to each valid row instead of its index.
-template <int kBatch, bool kPeer>
+// for low-latency rows (row_of = e * cap + j), row ((e % Epp) * W + rank) * cap + j
+// of rank e / Epp's padded outputs; the compaction records a pointer to each valid
+// row instead of its index.
+// kBySlot (deduplicated rows, slot k = rank k): slot k's row is row_of[t, k] +
+// peer_offset[k] in rank k's outputs.  Lane k's offset and base address are the
+// same for every token, so they are read once into shared memory, and the variant
+// needs no expert ids: it fits three CTAs per SM without spilling.  Deduplicated
+// normal workload: 57.3 us at two CTAs per SM, 53.0 us at three with a spilling
+// generic peer variant, 51.5 us with the offsets in shared memory, 47.5 us with this
+// variant -- the time of the one-GPU deduplicated combine.
+template <int kBatch, bool kPeer, bool kBySlot = false>
 __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
     combine_kernel(CombineParams p, int64_t vec_per_slice) {
+    static_assert(kPeer || !kBySlot, "slot-indexed rows are a peer layout");
     pdl_wait();               // the previous kernel is complete (a no-op without the attribute)
     pdl_launch_dependents();  // the next kernel may be scheduled
     __shared__ int rows_sm[2][32];
@@ -66,8 +71,19 @@ __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
         nrow = p.row_of[static_cast<int64_t>(blockIdx.x) * K + tid];
         if (p.topk_weights) nw = p.topk_weights[static_cast<int64_t>(blockIdx.x) * K + tid];
         if constexpr (kPeer)
-            if (!p.peer_by_slot) ne = p.topk_idx[static_cast<int64_t>(blockIdx.x) * K + tid];
+            if (!kBySlot) ne = p.topk_idx[static_cast<int64_t>(blockIdx.x) * K + tid];
     }
+    // deduplicated rows (slot k = rank k): lane k's row offset and base address are
+    // the same for every token, so they are read once here instead of per token on
+    // warp 0's set-up path
+    __shared__ const uint4* slot_base_sm[kPeer ? 32 : 1];
+    __shared__ int slot_off_sm[kPeer ? 32 : 1];
+    if constexpr (kPeer)
+        if (kBySlot && tid < K) {
+            slot_off_sm[tid] = p.peer_offset[tid];
+            slot_base_sm[tid] = static_cast<const uint4*>(p.peer_out[tid]);
+        }
+    __syncwarp();
     int buf = 0;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x, buf ^= 1) {
         if (tid < 32) {  // warp 0: lane k < K holds slot k
@@ -76,15 +92,17 @@ __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
             if constexpr (kPeer) {
                 // rows past the owner's buffer (or with an id the handle does not
                 // match) are skipped
-                if (r >= 0) {
-                    int at, part;
-                    if (p.peer_by_slot) {
-                        at = tid;
-                        part = tid;
+                if (kBySlot && r >= 0) {
+                    const int64_t pr = static_cast<int64_t>(r) + slot_off_sm[tid];
+                    if (pr < 0 || pr >= p.expert_out_rows) {
+                        raise_status(p.status, kDevIndexRange);
+                        r = -1;
                     } else {
-                        at = ne >= 0 && ne < p.num_experts ? static_cast<int>(ne) : -1;
-                        part = at >= 0 ? at / p.experts_per_partition : 0;
+                        src = slot_base_sm[tid] + pr * V;
                     }
+                } else if (!kBySlot && r >= 0) {
+                    const int at = ne >= 0 && ne < p.num_experts ? static_cast<int>(ne) : -1;
+                    const int part = at >= 0 ? at / p.experts_per_partition : 0;
                     int64_t pr = -1;
                     if (at >= 0 && p.peer_ll_cap > 0) {
                         const int64_t c = p.peer_ll_cap;
@@ -123,7 +141,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads, kBatch == 4 ? 3 : 2)
                     nrow = p.row_of[tn * K + tid];
                     if (p.topk_weights) nw = p.topk_weights[tn * K + tid];
                     if constexpr (kPeer)
-                        if (!p.peer_by_slot) ne = p.topk_idx[tn * K + tid];
+                        if (!kBySlot) ne = p.topk_idx[tn * K + tid];
                 }
             }
         }
@@ -282,8 +300,8 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
     int threads = static_cast<int>((per_slice + 31) / 32 * 32);
     if (threads > kCombineMaxThreads) threads = kCombineMaxThreads;
     const void* kernel =
-        p.peer_out ? (p.sparse ? reinterpret_cast<const void*>(combine_kernel<4, true>)
-                               : reinterpret_cast<const void*>(combine_kernel<8, true>))
+        p.peer_out ? (p.peer_by_slot ? reinterpret_cast<const void*>(combine_kernel<4, true, true>)
+                                     : reinterpret_cast<const void*>(combine_kernel<8, true>))
         : p.sparse ? reinterpret_cast<const void*>(combine_kernel<4, false>)
                    : reinterpret_cast<const void*>(combine_kernel<8, false>);
     const int per_sm = blocks_per_sm(kernel, dev.device, threads, 0);
@@ -307,7 +325,8 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = p.T * static_cast<int64_t>(p.K) <= kPdlMaxEntries ? 1 : 0;
-    if (p.peer_out && p.sparse) return cudaLaunchKernelEx(&cfg, combine_kernel<4, true>, p, per_slice);
+    if (p.peer_out && p.peer_by_slot)
+        return cudaLaunchKernelEx(&cfg, combine_kernel<4, true, true>, p, per_slice);
     if (p.peer_out) return cudaLaunchKernelEx(&cfg, combine_kernel<8, true>, p, per_slice);
     if (p.sparse) return cudaLaunchKernelEx(&cfg, combine_kernel<4, false>, p, per_slice);
     return cudaLaunchKernelEx(&cfg, combine_kernel<8, false>, p, per_slice);
