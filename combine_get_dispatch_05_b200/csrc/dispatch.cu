@@ -37,7 +37,7 @@ constexpr int kFp8InStages = 4;      // input ring: rows in flight from HBM per 
 constexpr int kFp8MaxOutStages = 40;  // quantised rows staged per CTA, at most
 constexpr int kFp8CtasPerSm = 2;      // the output ring fills this share of an SM
 constexpr int kFp8MaxQuantWarps = 14; // quantiser warps per CTA, at most
-constexpr int kFp8MaxThreads = 32 * (kFp8MaxQuantWarps + 2);
+constexpr int kFp8MaxStorers = 2;     // storer warps per CTA (taking alternate steps), at most
 constexpr int kBf16Stages = 4;        // BF16 rows in flight per CTA
 // Token log: the token of pipeline step i sits in tok[i % kTokLog] from the
 // loader's ticket until the storer has read it; the storer then marks the entry
@@ -46,7 +46,7 @@ constexpr int kBf16Stages = 4;        // BF16 rows in flight per CTA
 // token's routing: a value >= 0 there can only be the next step's token.
 constexpr int kTokFree = -2;
 constexpr int kTokLog = 64;
-static_assert(kTokLog > kFp8InStages + kFp8MaxOutStages + 1, "token log too short");
+static_assert(kTokLog > kFp8InStages + kFp8MaxOutStages + kFp8MaxStorers, "token log too short");
 static_assert(kTokLog > kBf16Stages + 1, "token log too short");
 static_assert((kTokLog & (kTokLog - 1)) == 0, "token log size is a power of two");
 
@@ -183,6 +183,14 @@ __device__ __forceinline__ int peer_dest(const DispatchParams& p, int lane, int 
     return static_cast<int>(r);
 }
 
+// Storer warps of the FP8 kernel.  Issuing a bulk store holds its warp for a few
+// hundred ns, so at about 4 rows per token (deduplicated rows) one warp's issue time
+// per token, not HBM, bounded a single storer (1.0 us of ~2 us per token); two
+// storers issue in parallel (deduplicated normal workload 45.1 -> 41.0 us).  At 8
+// rows per token the kernel is HBM-bound and a second storer only interleaves two
+// tokens' row stores (in the step 60.6 -> 63.5 us): one storer.
+inline int fp8_storers(const DispatchParams& p) { return p.dedup ? 2 : 1; }
+
 // Metadata of one token's receive rows, written by the storer warp.  Per-expert
 // rows: lane k owns slot k and writes the local id and weight of its row into
 // ri / rw (its own destination's arrays in peer mode).
@@ -220,28 +228,33 @@ __device__ __forceinline__ void write_row_metadata(const DispatchParams& p, int 
     }
 }
 
-// Warp-specialised pipeline, one CTA = 1 loader warp + nq quantiser warps + 1 storer
-// warp, coupled only by mbarriers (no CTA-wide barrier between set-up and the end):
+// Warp-specialised pipeline, one CTA = 1 loader warp + nq quantiser warps + kNs storer
+// warps, coupled only by mbarriers (no CTA-wide barrier between set-up and the end):
 //   loader (warp 0, lane 0): takes a ticket, records the token in the token log and
 //       bulk-loads its row into the input ring (in_full[s]: transaction bytes;
 //       waits in_empty[s] before reusing a stage); when the tickets run out it
-//       records -1 and arrives on in_full[s] without a load;
+//       records -1 for one step per storer and arrives on in_full[s] without loads;
 //   quantisers (warps 1..nq): quantise their share of the row's 128-channel blocks
 //       from input stage s into output stage o, then arrive on in_empty[s] and
 //       out_full[o] (waiting out_empty[o] before reusing an output stage); a -1
-//       token is passed on without work and ends the warp;
-//   storer (last warp): lane k bulk-stores the staged row and its scales to row
-//       row_of[t, k], writes recv_topk_idx / recv_topk_weights, and releases the
-//       output stage (out_empty) once its stores have read it; a -1 token ends it.
+//       token is passed on without work, and the last one ends the warp;
+//   storers (the last kNs warps, storer s taking steps s, s + kNs, ...): lane k
+//       bulk-stores the staged row and its scales to row row_of[t, k], writes
+//       recv_topk_idx / recv_topk_weights, and releases the output stage of its
+//       previous step (out_empty) once those stores have read it; a -1 token ends
+//       it.
 // Only the storer reads what the layout kernel wrote, so only it waits on the
 // programmatic dependency; loads and quantisation overlap the layout.
 // kPeer: rows go to the owner ranks' buffers (peer_dest).
-template <bool kPeer>
-__global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchParams p) {
+template <bool kPeer, int kNs>
+__global__ void __launch_bounds__(32 * (kFp8MaxQuantWarps + 1 + kNs), kFp8CtasPerSm)
+    dispatch_fp8_kernel(DispatchParams p) {
+    static_assert(kNs >= 1 && kNs <= kFp8MaxStorers, "storer warps");
     pdl_launch_dependents();  // the next kernel (e.g. the combine) may be scheduled
     extern __shared__ __align__(128) uint8_t sm[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nq = (blockDim.x >> 5) - 2;
+    constexpr int ns = kNs;
+    const int nq = (blockDim.x >> 5) - 1 - ns;
     const int64_t H = p.H;
     const int nb = static_cast<int>(H >> 7);
     const int NI = p.in_stages, NO = p.out_stages;
@@ -277,17 +290,19 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
         if (lane == 0) {
             const uint8_t* x = static_cast<const uint8_t*>(p.x);
             int issued = 0;  // bulk loads issued (steps 0 .. issued-1)
+            int ends = 0;    // end markers recorded
             Ring in;
             for (int i = 0;; ++i, in.next(NI)) {
                 // the ticket's round trip overlaps the wait for a free stage
-                const int t = take_ticket(p);
+                const int t = (ns > 1 && ends) ? -1 : take_ticket(p);
                 if (i >= NI && !wait_or_abort(&in_empty[in.stage], in.parity ^ 1u, p.timeout_ns,
                                               abort_flag))
                     break;
                 tok[i & (kTokLog - 1)] = t;
                 if (t < 0) {
-                    mbar_arrive(&in_full[in.stage]);  // the end marker: no load
-                    break;
+                    mbar_arrive(&in_full[in.stage]);  // an end marker: no load
+                    if (ns == 1 || ++ends == ns) break;
+                    continue;
                 }
                 mbar_arrive_expect_tx(&in_full[in.stage], L.in_bytes);
                 bulk_load(sm + in.stage * L.in_bytes, x + static_cast<int64_t>(t) * H * 2, L.in_bytes,
@@ -305,6 +320,7 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
     } else if (warp <= nq) {
         // ------------------------------------------------------------ quantisers
         const int qw = warp - 1;
+        int ends = 0;
         Ring in, out;
         for (int i = 0;; ++i, in.next(NI), out.next(NO)) {
             if (!wait_or_abort(&in_full[in.stage], in.parity, p.timeout_ns, abort_flag)) break;
@@ -324,26 +340,37 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
                 mbar_arrive(&in_empty[in.stage]);
                 mbar_arrive(&out_full[out.stage]);
             }
-            if (t < 0) break;
+            if (t < 0 && (ns == 1 || ++ends == ns)) break;
         }
     } else {
-        // ---------------------------------------------------------------- storer
+        // --------------------------------------------------------------- storers
         pdl_wait();  // row_of from the layout kernel is complete and visible
         uint8_t* recv_x = static_cast<uint8_t*>(p.recv_x);
         const int S = p.slots;
         const bool slot_lane = lane < S;  // lane s stores slot s's row
+        int prev = -1;  // output stage of this warp's previous step
+        Routing next;   // prefetched routing of this warp's next step's token
         Ring out;
-        int prev = -1;  // output stage of the previous step
-        Routing next;   // prefetched routing of the next step's token
-        for (int i = 0;; ++i, out.next(NO)) {
-            if (!wait_or_abort(&out_full[out.stage], out.parity, p.timeout_ns, abort_flag)) break;
-            const int t = tok[i & (kTokLog - 1)];
-            if (t < 0) break;
+        const int first = ns == 1 ? 0 : warp - 1 - nq;
+        for (int j = 0; j < first; ++j) out.next(NO);
+        for (int i = first;; i += ns) {
             const int o = out.stage;
+            if (!wait_or_abort(&out_full[o], out.parity, p.timeout_ns, abort_flag)) break;
+            const int t = tok[i & (kTokLog - 1)];
+            if (t < 0) {
+                if constexpr (ns > 1) {
+                    // release the previous stage: the quantisers' last end marker may
+                    // be waiting for it (a ring of at least three stages)
+                    if (slot_lane) bulk_wait_read<0>();
+                    __syncwarp();
+                    if (lane == 0 && prev >= 0) mbar_arrive(&out_empty[prev]);
+                }
+                break;
+            }
             const Routing cur = next.token == t ? next : load_routing(p, t, lane);
             __syncwarp();
             if (lane == 0) tok[i & (kTokLog - 1)] = kTokFree;
-            next = peek_routing(p, tok[(i + 1) & (kTokLog - 1)], lane);
+            next = peek_routing(p, tok[(i + ns) & (kTokLog - 1)], lane);
             int row = cur.row;
             const int64_t e = cur.e;
             const float wt = cur.wt;
@@ -382,6 +409,8 @@ __global__ void __launch_bounds__(kFp8MaxThreads) dispatch_fp8_kernel(DispatchPa
             __syncwarp();
             if (lane == 0 && prev >= 0) mbar_arrive(&out_empty[prev]);
             prev = o;
+#pragma unroll
+            for (int j = 0; j < ns; ++j) out.next(NO);
         }
         // the CTA may exit once its stores have read their stages; the grid completes
         // only when the writes have landed
@@ -542,12 +571,17 @@ cudaError_t launch_dispatch_fp8(const DispatchParams& params, cudaStream_t strea
     if (budget > dev.max_smem_optin) budget = dev.max_smem_optin;
     int no = budget >= one.total ? 1 + static_cast<int>((budget - one.total) / per_out) : 1;
     if (no > kFp8MaxOutStages) no = kFp8MaxOutStages;
-    if (no < 2) no = 2;
+    const int ns = fp8_storers(p);
+    // a storer releases a stage at its next step: with two storers, ns + 1 stages
+    if (no < ns + 1) no = ns + 1;
     p.out_stages = no;
     const Fp8Smem L = fp8_smem(p.H, p.in_stages, p.out_stages);
     if (L.total > dev.max_smem_optin) return cudaErrorInvalidValue;
-    const void* kernel = p.peer_offset ? reinterpret_cast<const void*>(dispatch_fp8_kernel<true>)
-                                       : reinterpret_cast<const void*>(dispatch_fp8_kernel<false>);
+    const void* kernel =
+        p.peer_offset ? (ns == 2 ? reinterpret_cast<const void*>(dispatch_fp8_kernel<true, 2>)
+                                 : reinterpret_cast<const void*>(dispatch_fp8_kernel<true, 1>))
+                      : (ns == 2 ? reinterpret_cast<const void*>(dispatch_fp8_kernel<false, 2>)
+                                 : reinterpret_cast<const void*>(dispatch_fp8_kernel<false, 1>));
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(L.total));
     if (err != cudaSuccess) return err;
@@ -557,7 +591,7 @@ cudaError_t launch_dispatch_fp8(const DispatchParams& params, cudaStream_t strea
     const int pairs = static_cast<int>((p.H / 128 + 1) / 2);
     const int iters = (pairs + kFp8MaxQuantWarps - 1) / kFp8MaxQuantWarps;
     const int nq = (pairs + iters - 1) / iters;
-    const int threads = 32 * (nq + 2);
+    const int threads = 32 * (nq + 1 + ns);
     const int grid = grid_for(kernel, threads, L.total, p.T, dev);
     return launch_pdl(kernel, dim3(grid), dim3(threads), L.total, stream, p);
 }
