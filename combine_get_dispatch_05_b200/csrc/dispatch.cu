@@ -40,10 +40,11 @@ constexpr int kFp8MaxQuantWarps = 14; // quantiser warps per CTA, at most
 constexpr int kFp8MaxStorers = 2;     // storer warps per CTA (taking alternate steps), at most
 constexpr int kBf16Stages = 4;        // BF16 rows in flight per CTA
 // Token log: the token of pipeline step i sits in tok[i % kTokLog] from the
-// loader's ticket until the storer has read it; the storer then marks the entry
-// consumed (kTokFree).  The loader runs at most (input stages + output stages)
-// steps ahead of the storer.  The storer peeks at the next entry to prefetch that
-// token's routing: a value >= 0 there can only be the next step's token.
+// loader's ticket until the step's storer has read it; the storer then marks the
+// entry consumed (kTokFree).  The loader runs at most (input stages + output stages
+// + storers) steps ahead of the storers.  A storer peeks at the entry of its next
+// step to prefetch that token's routing: a value >= 0 there can only be that
+// step's token.
 constexpr int kTokFree = -2;
 constexpr int kTokLog = 64;
 static_assert(kTokLog > kFp8InStages + kFp8MaxOutStages + kFp8MaxStorers, "token log too short");
