@@ -64,6 +64,10 @@ CASES = [
     ("p1", lambda: make_custom(90, 128, 4, 8, 1, seed=11)),
     ("e-eq-p", lambda: make_custom(257, 256, 3, 16, 16, seed=12)),
     ("t1", lambda: make_custom(1, 128, 8, 256, 8, seed=6)),
+    # fewer tokens than CTAs (some take none) and a batch with no rows at all: the
+    # pipeline's end markers, one per storer warp, with nothing or little before them
+    ("t5", lambda: make_custom(5, 256, 8, 64, 8, seed=17)),
+    ("all-masked", lambda: make_custom(40, 256, 4, 16, 4, seed=18, mask_frac=1.0)),
     # more than 1024 tokens: the partition layout's multi-CTA form; P = 6 and P = 5 take
     # its byte-by-byte flag and row stores, P = 32 is the most partitions it takes
     ("grid-2500", lambda: make_workload("normal", seed=3, num_tokens=2500, hidden=128)),
