@@ -68,6 +68,8 @@ CASES = [
     # pipeline's end markers, one per storer warp, with nothing or little before them
     ("t5", lambda: make_custom(5, 256, 8, 64, 8, seed=17)),
     ("all-masked", lambda: make_custom(40, 256, 4, 16, 4, seed=18, mask_frac=1.0)),
+    # the largest hidden size: two storers over the smallest output ring they allow
+    ("h16384", lambda: make_custom(150, 16384, 8, 64, 8, seed=19, mask_frac=0.1)),
     # more than 1024 tokens: the partition layout's multi-CTA form; P = 6 and P = 5 take
     # its byte-by-byte flag and row stores, P = 32 is the most partitions it takes
     ("grid-2500", lambda: make_workload("normal", seed=3, num_tokens=2500, hidden=128)),

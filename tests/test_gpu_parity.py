@@ -50,6 +50,9 @@ def _cases():
     yield "masked", make_custom(513, 640, 6, 64, 16, seed=10, mask_frac=0.3)
     yield "hot", make_custom(800, 128, 4, 32, 8, seed=11, hot_expert=5)
     yield "e4096", make_custom(300, 128, 8, 4096, 64, seed=12)
+    # the largest hidden size the calls take: one dispatch CTA per SM, the fewest
+    # staged rows
+    yield "h16384", make_custom(150, 16384, 8, 64, 8, seed=13, mask_frac=0.1)
 
 
 CASES = list(_cases())
