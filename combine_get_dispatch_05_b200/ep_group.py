@@ -229,7 +229,9 @@ class EpGroup:
 
     def _view(self, name: str, dtype, shape, region=None) -> torch.Tensor:
         """A typed view of a named array of a region; made once per (array, dtype,
-        shape) and kept, as every call of a step asks for the same views."""
+        shape) and kept, as every call of a step asks for the same views.  Each call
+        returns a fresh alias of the kept view, so that in-place changes of a
+        returned tensor's shape do not reach later calls."""
         pr = self._peer if region is None else region
         key = (id(pr), name, dtype, tuple(shape))
         v = self._views.get(key)
@@ -240,7 +242,7 @@ class EpGroup:
             n *= torch.empty(0, dtype=dtype).element_size()
             o = pr["offsets"][name]
             v = self._views[key] = pr["region"][o:o + n].view(dtype).view(*shape)
-        return v
+        return v.detach()
 
     def _stream(self):
         """The current stream of this group's device, resolved once per call and

@@ -393,6 +393,16 @@ def run_peer(rank: int, world: int, port: int, out_dir: str) -> None:
             y = g.combine(buf, ctx, wts)
             assert np.array_equal(y.view(torch.int16).numpy().view(np.uint16),
                                   y_all[t0:t0 + tokens[rank]]), f"no-sync dedup={dedup}"
+            # the buffers' views are kept between calls: reshaping a returned tensor in
+            # place must not change what the next call returns
+            shapes = (tuple(recv_x[0].shape), tuple(ri.shape), tuple(buf.shape))
+            recv_x[0].unsqueeze_(0)
+            ri.unsqueeze_(0)
+            buf.unsqueeze_(0)
+            again = g.dispatch(x, idx, wts, dedup=dedup, sync_sizes=False)
+            assert (tuple(again[0][0].shape), tuple(again[1].shape),
+                    tuple(g.expert_out_buffer(again[4]).shape)) == shapes
+            g.combine(g.expert_out_buffer(again[4]), again[4], wts)
         for quant in ("fp8", "none"):  # one row per (token, rank)
             recv_x, ri, rw, per_source, ctx = g.dispatch(x, idx, wts, use_fp8=quant == "fp8",
                                                          dedup=True)
