@@ -76,10 +76,8 @@ int blocks_per_sm(const void* kernel, int device, int threads, size_t smem) {
     }
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) !=
-        cudaSuccess) {
-        cudaGetLastError();  // not sticky; the launch reports any real fault
-        return 1;
-    }
+        cudaSuccess)
+        return 1;  // not kept: the launch that follows reports the error
     if (per_sm < 1) per_sm = 1;
     if (g_occ_n < kOccupancyEntries) g_occ[g_occ_n++] = {kernel, device, threads, smem, per_sm};
     return per_sm;
