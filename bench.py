@@ -1287,60 +1287,56 @@ def run_ours(args):
         result["cpu_baseline"] = cpu_baseline(w)
     if not args.no_extra:
         extra = {}
-        try:
-            extra["backward"] = time_backward(ep, runner, args.extra_steps)
-            extra["backward"]["workload"] = args.workload
-        except Exception as exc:  # report, do not hide
-            extra["backward"] = {"error": repr(exc)}
-        try:
-            extra["dedup"] = time_dedup(ep, w, dev, args.extra_steps)
-            extra["dedup"]["workload"] = args.workload
-        except Exception as exc:
-            extra["dedup"] = {"error": repr(exc)}
-        try:
-            extra["peer"] = time_peer(ep, w, dev, args.extra_steps)
-            extra["peer"]["workload"] = args.workload
-        except Exception as exc:  # report, do not hide
-            extra["peer"] = {"error": repr(exc)}
-        if world == 1:
+        want = set(args.extras.split(",")) if args.extras else None
+
+        def workload_row(name):
+            wx = make_workload(name, seed=args.seed)
+            r = PathRunner(ep, wx, dev, use_graphs=not args.eager)
+            ss = r.time_whole_steps(args.extra_steps, 3, flush, per_graph=args.steps_per_graph)
+            dd, cc = r.time_steps(args.extra_steps, 3, flush)
+            du, cu = statistics.mean(dd) * 1e3, statistics.mean(cc) * 1e3
+            su = statistics.mean(ss) * 1e3
+            row = {
+                "tokens": wx.num_tokens, "hidden": wx.hidden, "topk": wx.num_topk,
+                "experts": wx.num_experts, "partitions": wx.num_partitions,
+                "quant": wx.quant, "recv_rows": r.R,
+                "dispatch_us": round(du, 2),
+                "dispatch_gbs": round(r.bytes_dispatch / (du * 1e-6) / 1e9, 1),
+                "dispatch_tokens_per_s": round(wx.num_tokens / (du * 1e-6)),
+                "combine_us": round(cu, 2),
+                "combine_gbs": round(r.bytes_combine / (cu * 1e-6) / 1e9, 1),
+                "combine_tokens_per_s": round(wx.num_tokens / (cu * 1e-6)),
+                "step_us": round(su, 2),
+                "step_gbs": round((r.bytes_dispatch + r.bytes_combine) / (su * 1e-6) / 1e9, 1),
+                "status": ep.ep_read_status(r.ws)}
+            del r
+            torch.cuda.empty_cache()
+            return row
+
+        def on_workload(fn):
+            def run():
+                out = fn()
+                out["workload"] = args.workload
+                return out
+            return run
+
+        jobs = [
+            ("backward", on_workload(lambda: time_backward(ep, runner, args.extra_steps))),
+            ("dedup", on_workload(lambda: time_dedup(ep, w, dev, args.extra_steps))),
+            ("peer", on_workload(lambda: time_peer(ep, w, dev, args.extra_steps))),
+            # a group of one rank; with more ranks the group would span GPUs
+            ("epgroup", on_workload(lambda: time_epgroup(ep, w, dev, min(args.extra_steps, 20))))
+            if world == 1 else None,
+            ("lb", lambda: time_lb(ep, dev, min(args.extra_steps, 20), args.seed, args.lb_scale)),
+            ("ll", lambda: time_low_latency(ep, make_workload("ll", seed=args.seed), dev)),
+        ] + [(name, lambda name=name: workload_row(name)) for name in ("skew", "bf16", "stress")]
+        for job in jobs:
+            if job is None or (want is not None and job[0] not in want):
+                continue
             try:
-                extra["epgroup"] = time_epgroup(ep, w, dev, min(args.extra_steps, 20))
-                extra["epgroup"]["workload"] = args.workload
+                extra[job[0]] = job[1]()
             except Exception as exc:  # report, do not hide
-                extra["epgroup"] = {"error": repr(exc)}
-        try:
-            extra["lb"] = time_lb(ep, dev, min(args.extra_steps, 20), args.seed, args.lb_scale)
-        except Exception as exc:  # report, do not hide
-            extra["lb"] = {"error": repr(exc)}
-        try:
-            extra["ll"] = time_low_latency(ep, make_workload("ll", seed=args.seed), dev)
-        except Exception as exc:  # report, do not hide
-            extra["ll"] = {"error": repr(exc)}
-        for name in ("skew", "bf16", "stress"):
-            try:
-                wx = make_workload(name, seed=args.seed)
-                r = PathRunner(ep, wx, dev, use_graphs=not args.eager)
-                ss = r.time_whole_steps(args.extra_steps, 3, flush, per_graph=args.steps_per_graph)
-                dd, cc = r.time_steps(args.extra_steps, 3, flush)
-                du, cu = statistics.mean(dd) * 1e3, statistics.mean(cc) * 1e3
-                su = statistics.mean(ss) * 1e3
-                extra[name] = {
-                    "tokens": wx.num_tokens, "hidden": wx.hidden, "topk": wx.num_topk,
-                    "experts": wx.num_experts, "partitions": wx.num_partitions,
-                    "quant": wx.quant, "recv_rows": r.R,
-                    "dispatch_us": round(du, 2),
-                    "dispatch_gbs": round(r.bytes_dispatch / (du * 1e-6) / 1e9, 1),
-                    "dispatch_tokens_per_s": round(wx.num_tokens / (du * 1e-6)),
-                    "combine_us": round(cu, 2),
-                    "combine_gbs": round(r.bytes_combine / (cu * 1e-6) / 1e9, 1),
-                    "combine_tokens_per_s": round(wx.num_tokens / (cu * 1e-6)),
-                    "step_us": round(su, 2),
-                    "step_gbs": round((r.bytes_dispatch + r.bytes_combine) / (su * 1e-6) / 1e9, 1),
-                    "status": ep.ep_read_status(r.ws)}
-                del r
-                torch.cuda.empty_cache()
-            except Exception as exc:
-                extra[name] = {"error": repr(exc)}
+                extra[job[0]] = {"error": repr(exc)}
         result["configs"] = extra
     print(json.dumps(result), flush=True)
 
@@ -1426,7 +1422,10 @@ def main():
                     help="whole steps captured in one CUDA graph for the headline timing")
     ap.add_argument("--workload", choices=("normal", "skew", "bf16", "stress"), default="normal",
                     help="workload of the timed step (the headline metric is quoted on normal)")
-    ap.add_argument("--no-extra", action="store_true", help="skip the ll/skew/bf16/stress configs")
+    ap.add_argument("--no-extra", action="store_true", help="skip the extra configs")
+    ap.add_argument("--extras", default=None,
+                    help="comma-separated subset of the extra configs to run (backward, dedup, "
+                         "peer, epgroup, lb, ll, skew, bf16, stress); all by default")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--lb-scale", type=int, default=1,
