@@ -602,6 +602,45 @@ def time_epgroup(ep, w, dev, steps):
     return out
 
 
+def time_layout_alone(ep, runner, per_graph=20, reps=10):
+    """The layout call by itself (ep_get_dispatch_layout on the runner's routing, with a
+    handle and workspace of its own): per_graph calls captured in one CUDA graph,
+    replayed back to back; device time per call.  In the benchmark step the layout
+    is followed by the dispatch kernel, which starts loading and quantising during it."""
+    import torch
+
+    lay = ep.Layout.empty(runner.T, runner.K, runner.E, runner.P, runner.dev)
+    ws = torch.empty(ep.ep_workspace_bytes(runner.T, runner.E, runner.P), dtype=torch.uint8,
+                     device=runner.dev)
+    ep.ep_workspace_init(ws)
+
+    def call():
+        ep.ep_get_dispatch_layout(runner.idx, runner.E, runner.P, lay, ws)
+
+    s = torch.cuda.Stream(device=runner.dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        call()
+        call()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(per_graph):
+            call()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    if ep.ep_read_status(ws) != 0:
+        raise RuntimeError("device status set in the layout run")
+    return e0.elapsed_time(e1) * 1e3 / (reps * per_graph)
+
+
 def time_backward(ep, runner, steps):
     """Backward pair on the runner's workload: ep_dispatch_backward (row gradients ->
     grad_x, weight-gradient gather) and ep_combine_backward (grad_y -> expert-row
@@ -1198,10 +1237,13 @@ def run_ours(args):
     # whole step as one graph per step, for reference
     d_ms, c_ms = runner.time_steps(args.steps, 3, flush)
     one_ms = runner.time_whole_steps(args.steps, 3, flush, per_graph=1)
+    layout_us = time_layout_alone(ep, runner)
     torch.cuda.synchronize()
     status = ep.ep_read_status(runner.ws)
 
-    tot = reduce_max_over_ranks([sum(s_ms), sum(c_ms), sum(d_ms), sum(one_ms)], world, dev)
+    tot = reduce_max_over_ranks([sum(s_ms), sum(c_ms), sum(d_ms), sum(one_ms), layout_us],
+                                world, dev)
+    layout_us = tot[4]
     total_ms = tot[0]
     ms_step = total_ms / args.steps
     step_bytes = runner.bytes_dispatch + runner.bytes_combine
@@ -1253,6 +1295,10 @@ def run_ours(args):
                           "with the two calls captured as separate graphs and events between "
                           "them; their sum exceeds the whole-step time by the graph boundary",
         "breakdown": {
+            "layout": {"us": round(layout_us, 2),
+                       "note": "the layout call alone, 20 calls per CUDA graph back to back; "
+                               "inside the dispatch interval below it overlaps the dispatch "
+                               "kernel's loads"},
             "dispatch": {"us": round(disp_us, 2), "bytes": runner.bytes_dispatch,
                          "gbs": round(disp_gbs, 1), "frac": round(disp_gbs / peak, 4),
                          "tokens_per_s": round(w.num_tokens / (disp_us * 1e-6)),
